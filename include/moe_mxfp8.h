@@ -1,0 +1,237 @@
+/*
+ * moe_mxfp8.h -- C ABI of the grouped MXFP8 MoE expert MLP for B200 (sm_100a).
+ *
+ * The layer ("Efficient MoE Training for Biological Foundation Models"):
+ *   Challenge 1   tokens grouped by expert with per-expert counts
+ *                 (split_sizes); one grouped GEMM submission per projection;
+ *                 gate_up projection has 2 * intermediate outputs, no bias.
+ *   Challenge 2   MXFP8: 8-bit values, one scale per 32 consecutive values.
+ *   Challenge 3   quantise to MXFP8 before each low-precision GEMM (BF16
+ *                 master weights); GroupedLinear(gate_up) -> ScaledSwiGLU
+ *                 (SwiGLU times the routing probability) -> GroupedLinear
+ *                 (down), fused so the BF16 intermediate is not written;
+ *                 matching fused backward.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.   Every pointer is DEVICE memory owned by the caller unless a
+ *           parameter says "host".  The library never allocates device
+ *           memory; scratch comes from the caller's workspace
+ *           (moe_workspace_size).  Calls are asynchronous on `stream`.
+ * Errors.   Argument errors (null pointer, bad size, misalignment, an
+ *           unsupported shape) are detected on the host before any launch
+ *           and return MOE_ERR_INVALID / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE
+ *           with nothing launched.  CUDA launch failures return MOE_ERR_CUDA.
+ *           Data-dependent errors found by a kernel (an expert id outside
+ *           [0, E), a pipeline wait that ran out) are recorded in a device
+ *           status word and read back by moe_get_device_status().
+ * bf16.     IEEE bfloat16 bit patterns, row-major.
+ * MXFP8 operand ("MX tensor", K-major).  A tensor of `groups` matrices of
+ *           `rows` x `K` values, K a multiple of 32, quantised along K:
+ *             data    uint8 E4M3 codes [groups][rows][K], row-major;
+ *             scales  uint8 E8M0 bytes (2^(b-127)) in the tcgen05 blocked
+ *                     layout: for group g, row r, 32-block kb = k/32,
+ *                       offset = ((g*RT + r/128)*KT + kb/4)*512
+ *                              + (r%32)*16 + ((r%128)/32)*4 + kb%4,
+ *                     RT = ceil(rows/128), KT = ceil(K/128);
+ *                     moe_mx_scale_bytes() gives the size.  Bytes that
+ *                     belong to no (row, block) are written as 0.
+ *           Scale rule: s = smallest integer with amax/2^s <= 448 (448 =
+ *           largest E4M3), clamped to [-127,127]; all-zero block -> s=-127;
+ *           block with NaN/Inf -> scale byte 0xFF.  Codes: E4M3(v * 2^-s),
+ *           round to nearest even, saturating.
+ * Permuted rows.  Routed row (token t, choice j) is slot s = t*k + j.  Rows
+ *           are ordered by (expert, slot) (stable counting sort) and every
+ *           expert's group starts on a multiple of 128 rows in a padded row
+ *           space of capacity moe_padded_rows(T,k,E); padding rows hold zero
+ *           codes and zero scales.
+ */
+#ifndef MOE_MXFP8_H
+#define MOE_MXFP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = 1,      /* null pointer, negative or inconsistent size, misalignment */
+  MOE_ERR_UNSUPPORTED = 2,  /* shape outside what the kernels handle (see each call) */
+  MOE_ERR_WORKSPACE = 3,    /* workspace pointer null or smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE_INDEX = 5, /* device: an expert id outside [0, E) */
+  MOE_ERR_TIMEOUT = 6,      /* device: a bounded pipeline wait ran out */
+  MOE_ERR_NO_DEVICE = 7     /* no sm_100 device current */
+} moe_status_t;
+
+/* Quantisation modes of moe_mlp_quantize_mxfp8. */
+#define MOE_QUANT_ROW 1 /* quantise along the last axis (cols) */
+#define MOE_QUANT_COL 2 /* quantise along rows, store transposed */
+
+/* Workspace sizes for moe_workspace_size(op, ...). */
+#define MOE_OP_PERMUTE 1
+#define MOE_OP_FWD 2
+#define MOE_OP_BWD 3
+
+/* Limits checked on the host. */
+#define MOE_MAX_EXPERTS 256
+
+/* ---------------------------------------------------------------- sizes --- */
+
+/* Bytes of the blocked scale array of an MX tensor of `groups` x `rows` x `k`
+ * (k a multiple of 32).  Returns -1 on invalid sizes. */
+int64_t moe_mx_scale_bytes(int32_t groups, int64_t rows, int64_t k);
+
+/* Capacity of the padded permuted row space for T tokens, top-k, E experts:
+ * the smallest multiple of 128 that holds sum_e roundup(split_sizes[e],128)
+ * for every routing (= roundup(T*k + 127*E, 128)). -1 on invalid sizes. */
+int64_t moe_padded_rows(int32_t T, int32_t k, int32_t E);
+
+/* Workspace bytes for op MOE_OP_PERMUTE / MOE_OP_FWD / MOE_OP_BWD of a layer
+ * (T tokens, top-k, E experts, hidden H, intermediate I).  -1 if invalid. */
+int64_t moe_workspace_size(int32_t op, int32_t T, int32_t k, int32_t E, int32_t H, int32_t I);
+
+/* ----------------------------------------------------------- quantise --- */
+
+/* MXFP8-quantise bf16 matrices (Challenge 2 and 3: one E8M0 scale per 32
+ * consecutive values along the consuming GEMM's K; BF16 master weights are
+ * quantised before each low-precision GEMM).
+ *   src     bf16 [groups][rows][cols], row-major, 16-byte aligned.
+ *   mode    MOE_QUANT_ROW: blocks along cols.  Output MX tensor
+ *             q [groups][rows][cols], scales blocked(groups, rows, cols).
+ *             Needs cols % 32 == 0.
+ *           MOE_QUANT_COL: blocks along rows, stored transposed.  Output MX
+ *             tensor q [groups][cols][rows], scales blocked(groups, cols, rows).
+ *             Needs rows % 32 == 0 and cols % 8 == 0.
+ *   q, sf   outputs, 16-byte aligned; sizes groups*rows*cols and
+ *           moe_mx_scale_bytes(groups, rows|cols, cols|rows).
+ * Weights for the forward: W_gate_up [E][2I][H] as groups=2E, rows=I,
+ * cols=H (gate of expert e is group 2e, up is 2e+1); W_down [E][H][I] as
+ * groups=E, rows=H, cols=I.  For the backward: W_down with MOE_QUANT_COL
+ * (groups=E, rows=H, cols=I) gives W_down^T [E][I][H] along H; W_gate_up
+ * with MOE_QUANT_COL (groups=E, rows=2I, cols=H) gives W_gate_up^T
+ * [E][H][2I] along 2I. */
+moe_status_t moe_mlp_quantize_mxfp8(const void* src, int32_t groups, int64_t rows, int64_t cols,
+                                    int32_t mode, uint8_t* q, uint8_t* sf, moe_stream_t stream);
+
+/* ------------------------------------------------------------ permute --- */
+
+/* Group routed tokens by expert and quantise them (Challenge 1:
+ * split_sizes; Challenge 3: quantise activations before the GEMM).
+ *   x          bf16 [T][H], H % 128 == 0 or H % 32 == 0 (any multiple of 32).
+ *   topk_idx   int32 [T][k] expert ids; topk_prob float [T][k].
+ *   rows_cap   = moe_padded_rows(T,k,E) (or larger, a multiple of 128).
+ * Outputs (all device, caller-owned):
+ *   split_sizes    int32 [E]      tokens per expert.
+ *   group_offsets  int32 [E+1]    padded start of each group (multiples of
+ *                                 128); group_offsets[E] = rows used.
+ *   row_to_slot    int32 [rows_cap]  slot of each padded row, -1 = padding.
+ *   slot_to_row    int32 [T*k]       padded row of each slot.
+ *   prob_perm      float [rows_cap]  routing probability per padded row (0 pad).
+ *   xq, xq_sf      MX tensor (1, rows_cap, H): gathered x, quantised along H.
+ *   xq_col, xq_col_sf  optional (both NULL or both set): MX tensor
+ *                  (1, H, rows_cap) = gathered x^T quantised along tokens
+ *                  (32-token blocks inside each 128-aligned group; padding
+ *                  tokens are zero) -- the weight-gradient operand.
+ *   workspace  >= moe_workspace_size(MOE_OP_PERMUTE, T, k, E, H, 0) bytes.
+ * Expert ids outside [0,E) set MOE_ERR_DEVICE_INDEX in the device status and
+ * are dropped. */
+moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* topk_prob,
+                         int32_t T, int32_t H, int32_t k, int32_t E, int64_t rows_cap,
+                         int32_t* split_sizes, int32_t* group_offsets, int32_t* row_to_slot,
+                         int32_t* slot_to_row, float* prob_perm, uint8_t* xq, uint8_t* xq_sf,
+                         uint8_t* xq_col, uint8_t* xq_col_sf, void* workspace, size_t workspace_bytes,
+                         moe_stream_t stream);
+
+/* ------------------------------------------------------------ forward --- */
+
+/* Fused grouped MLP forward (Challenge 3, GroupedLinear -> ScaledSwiGLU ->
+ * GroupedLinear; Figure 4: one fused kernel before the down projection).
+ *   w1q, w1sf  MX tensor (2E, I, H): W_gate_up quantised along H.
+ *   w2q, w2sf  MX tensor (E, H, I):  W_down quantised along I.
+ *   routing    split_sizes, group_offsets, row_to_slot, prob_perm from moe_permute.
+ *   xq, xq_sf  MX tensor (1, rows_cap, H) from moe_permute.
+ *   out        bf16 [T][H]: out[t] = sum_j y[t*k+j], y = down(h),
+ *              h = prob * silu(gate) * up, gate = A[:, :I], up = A[:, I:],
+ *              A = x W_gate_up^T (fp32 accumulation).
+ *   saved_a    bf16 [rows_cap][2I] or NULL: A rounded to bf16, kept for the
+ *              backward (padding rows are not written).
+ *   hq, hq_sf  optional outputs (both NULL or both set) of the requantised
+ *              intermediate: MX tensor (1, rows_cap, I).  If NULL they live
+ *              in the workspace.
+ *   workspace  >= moe_workspace_size(MOE_OP_FWD, T, k, E, H, I).
+ * Needs H % 32 == 0, I % 64 == 0, E <= MOE_MAX_EXPERTS. */
+moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const uint8_t* w2q,
+                                 const uint8_t* w2sf, int32_t T, int32_t H, int32_t I, int32_t E,
+                                 int32_t k, int64_t rows_cap, const int32_t* split_sizes,
+                                 const int32_t* group_offsets, const int32_t* row_to_slot,
+                                 const float* prob_perm, const uint8_t* xq, const uint8_t* xq_sf,
+                                 void* out, void* saved_a, uint8_t* hq, uint8_t* hq_sf,
+                                 void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* Top-k combine (Challenge 1, index_add back to token order):
+ *   y  bf16 [T*k][H] in slot order -> out bf16 [T][H], out[t] = sum_j y[t*k+j]
+ *   summed in fp32, j ascending. */
+moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* out,
+                         moe_stream_t stream);
+
+/* ----------------------------------------------------------- backward --- */
+
+/* Matching fused backward (Challenge 3).  With dy_r = dY[token(r)]:
+ *   dh  = dy W_down                   (dgrad2; dy, W_down quantised along H)
+ *   g,u = saved_a halves; sig = sigmoid(g); s = g*sig
+ *   dg  = dh*p*u*sig*(1+g*(1-sig)),  du = dh*p*s,  dprob = sum_i dh*s*u
+ *   dW_down_e = dy_e^T h_e, h = p*s*u  (wgrad2; quantised along tokens)
+ *   dx  = [dg,du] W_gate_up           (dgrad1; along 2I)
+ *   dW_gate_up_e = [dg,du]_e^T x_e    (wgrad1; along tokens)
+ *   dX[t] = sum_j dx[row(t,j)].
+ * Inputs:
+ *   w2tq, w2tsf  MX tensor (E, I, H): W_down^T quantised along H
+ *                (moe_mlp_quantize_mxfp8 COL of W_down, groups=E rows=H cols=I).
+ *   w1tq, w1tsf  MX tensor (E, H, 2I): W_gate_up^T quantised along 2I
+ *                (COL of W_gate_up, groups=E rows=2I cols=H).
+ *   routing      as in the forward, plus slot_to_row.
+ *   dY           bf16 [T][H].  saved_a bf16 [rows_cap][2I] from the forward.
+ *   xq_col, xq_col_sf  MX tensor (1, H, rows_cap) from moe_permute.
+ * Outputs: dX bf16 [T][H]; dW1 bf16 [E][2I][H]; dW2 bf16 [E][H][I];
+ *   dprob float [T][k] (slot order).
+ * Needs H % 128 == 0 or H % 32 == 0, I % 64 == 0. */
+moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, const uint8_t* w1tq,
+                                 const uint8_t* w1tsf, int32_t T, int32_t H, int32_t I, int32_t E,
+                                 int32_t k, int64_t rows_cap, const int32_t* split_sizes,
+                                 const int32_t* group_offsets, const int32_t* row_to_slot,
+                                 const int32_t* slot_to_row, const float* prob_perm,
+                                 const void* dY, const void* saved_a, const uint8_t* xq_col,
+                                 const uint8_t* xq_col_sf, void* dX, void* dW1, void* dW2,
+                                 float* dprob, void* workspace, size_t workspace_bytes,
+                                 moe_stream_t stream);
+
+/* ------------------------------------------------------------- status --- */
+
+/* Synchronises `stream`, returns the first data-dependent error recorded by
+ * a kernel of this library on the current device since the last call, and
+ * clears it.  MOE_OK if none. */
+moe_status_t moe_get_device_status(moe_stream_t stream);
+
+/* Static English description of a status code. */
+const char* moe_status_string(moe_status_t status);
+
+/* Number of kernels this library launched from the calling process since
+ * the last reset (host-side counter; for launch accounting in benchmarks). */
+int64_t moe_launch_count(int32_t reset);
+
+/* Self-test of the bounded-wait machinery: launches one CTA that waits on a
+ * pipeline barrier nobody arrives on, with a limit of about `wait_ms`
+ * milliseconds; the kernel gives up, records MOE_ERR_TIMEOUT and exits
+ * normally.  Returns the status read back (MOE_ERR_TIMEOUT when working). */
+moe_status_t moe_selftest_wait_timeout(int32_t wait_ms, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_MXFP8_H */

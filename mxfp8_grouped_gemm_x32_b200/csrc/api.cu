@@ -1,0 +1,372 @@
+// C ABI of the grouped MXFP8 MoE expert MLP (declared in include/moe_mxfp8.h):
+// argument checks, workspace carving and the launch sequence of each call.
+#include <atomic>
+
+#include "gemm.cuh"
+#include "permute.cuh"
+#include "quant.cuh"
+#include "swiglu_bwd.cuh"
+
+namespace moe {
+
+static std::atomic<int64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+namespace {
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t align256(int64_t v) { return (v + 255) / 256 * 256; }
+
+inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+int64_t mx_scale_bytes(int64_t groups, int64_t rows, int64_t k) {
+  return groups * cdiv(rows, 128) * cdiv(k, 128) * 512;
+}
+
+// Carves a workspace into 256-byte aligned pieces.
+struct Carver {
+  uint8_t* base;
+  int64_t off = 0;
+  uint8_t* take(int64_t bytes) {
+    uint8_t* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  }
+};
+
+struct FwdWs {
+  uint8_t *hq, *hq_sf, *y;
+};
+FwdWs carve_fwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t rows_cap, bool need_h) {
+  FwdWs w{};
+  if (need_h) {
+    w.hq = c.take(rows_cap * I);
+    w.hq_sf = c.take(mx_scale_bytes(1, rows_cap, I));
+  }
+  w.y = c.take(T * k * H * 4);
+  return w;
+}
+
+struct BwdWs {
+  uint8_t *dyq, *dyq_sf, *dyc, *dyc_sf, *dh, *daq, *daq_sf, *dac, *dac_sf, *hc, *hc_sf, *dx;
+};
+BwdWs carve_bwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t rows_cap) {
+  BwdWs w{};
+  w.dyq = c.take(rows_cap * H);
+  w.dyq_sf = c.take(mx_scale_bytes(1, rows_cap, H));
+  w.dyc = c.take(H * rows_cap);
+  w.dyc_sf = c.take(mx_scale_bytes(1, H, rows_cap));
+  w.dh = c.take(rows_cap * I * 4);
+  w.daq = c.take(rows_cap * 2 * I);
+  w.daq_sf = c.take(mx_scale_bytes(1, rows_cap, 2 * I));
+  w.dac = c.take(2 * I * rows_cap);
+  w.dac_sf = c.take(mx_scale_bytes(1, 2 * I, rows_cap));
+  w.hc = c.take(I * rows_cap);
+  w.hc_sf = c.take(mx_scale_bytes(1, I, rows_cap));
+  w.dx = c.take(T * k * H * 4);
+  return w;
+}
+
+bool layer_dims_ok(int32_t T, int32_t H, int32_t I, int32_t E, int32_t k) {
+  return T >= 0 && H > 0 && I > 0 && E > 0 && k > 0 && k <= E && E <= MOE_MAX_EXPERTS &&
+         H % 32 == 0 && I % 64 == 0 && int64_t(T) * k < (int64_t(1) << 30);
+}
+
+bool device_ok() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  return major == 10;
+}
+
+// Bounded-wait self test: one thread waits on a barrier nobody arrives on.
+__global__ void wait_timeout_kernel(long long limit_cycles) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, limit_cycles);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int64_t moe_mx_scale_bytes(int32_t groups, int64_t rows, int64_t k) {
+  if (groups < 0 || rows < 0 || k < 0 || k % 32) return -1;
+  return mx_scale_bytes(groups, rows, k);
+}
+
+int64_t moe_padded_rows(int32_t T, int32_t k, int32_t E) {
+  if (T < 0 || k <= 0 || E <= 0) return -1;
+  return cdiv(int64_t(T) * k + 127 * int64_t(E), 128) * 128;
+}
+
+int64_t moe_workspace_size(int32_t op, int32_t T, int32_t k, int32_t E, int32_t H, int32_t I) {
+  const int64_t rows_cap = moe_padded_rows(T, k, E);
+  if (rows_cap < 0) return -1;
+  Carver c{nullptr};
+  switch (op) {
+    case MOE_OP_PERMUTE:
+      return align256(permute_workspace_bytes(int64_t(T) * k, E));
+    case MOE_OP_FWD:
+      if (H <= 0 || I <= 0) return -1;
+      carve_fwd(c, T, k, H, I, rows_cap, true);
+      return c.off;
+    case MOE_OP_BWD:
+      if (H <= 0 || I <= 0) return -1;
+      carve_bwd(c, T, k, H, I, rows_cap);
+      return c.off;
+  }
+  return -1;
+}
+
+moe_status_t moe_mlp_quantize_mxfp8(const void* src, int32_t groups, int64_t rows, int64_t cols,
+                                    int32_t mode, uint8_t* q, uint8_t* sf, moe_stream_t stream) {
+  if (!src || !q || !sf || groups < 0 || rows < 0 || cols < 0) return MOE_ERR_INVALID;
+  if (!al16(src) || !al16(q) || !al16(sf)) return MOE_ERR_INVALID;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (mode == MOE_QUANT_ROW) {
+    if (cols % 32) return MOE_ERR_UNSUPPORTED;
+    QuantRowsArgs a{static_cast<const uint8_t*>(src), cols, nullptr, 1, groups, rows, cols, q, sf};
+    return cuda_status(launch_quant_rows(a, st));
+  }
+  if (mode == MOE_QUANT_COL) {
+    if (rows % 32 || cols % 8) return MOE_ERR_UNSUPPORTED;
+    QuantColsArgs a{static_cast<const uint8_t*>(src), cols, nullptr, 1, groups, rows, cols, q, sf};
+    return cuda_status(launch_quant_cols(a, st));
+  }
+  return MOE_ERR_INVALID;
+}
+
+moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* topk_prob, int32_t T,
+                         int32_t H, int32_t k, int32_t E, int64_t rows_cap, int32_t* split_sizes,
+                         int32_t* group_offsets, int32_t* row_to_slot, int32_t* slot_to_row,
+                         float* prob_perm, uint8_t* xq, uint8_t* xq_sf, uint8_t* xq_col,
+                         uint8_t* xq_col_sf, void* workspace, size_t workspace_bytes,
+                         moe_stream_t stream) {
+  if (!x || !topk_idx || !topk_prob || !split_sizes || !group_offsets || !row_to_slot ||
+      !slot_to_row || !prob_perm || !xq || !xq_sf)
+    return MOE_ERR_INVALID;
+  if ((xq_col == nullptr) != (xq_col_sf == nullptr)) return MOE_ERR_INVALID;
+  if (T < 0 || H <= 0 || k <= 0 || E <= 0 || k > E) return MOE_ERR_INVALID;
+  if (E > MOE_MAX_EXPERTS || H % 32) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
+  if (!al16(x) || !al16(xq) || !al16(xq_sf) || (xq_col && (!al16(xq_col) || !al16(xq_col_sf))))
+    return MOE_ERR_INVALID;
+  const int64_t need = moe_workspace_size(MOE_OP_PERMUTE, T, k, E, H, 0);
+  if (!workspace || int64_t(workspace_bytes) < need) return MOE_ERR_WORKSPACE;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t R = int64_t(T) * k;
+  cudaError_t e = launch_permute_index(topk_idx, topk_prob, R, E, rows_cap, split_sizes, group_offsets,
+                                       row_to_slot, slot_to_row, prob_perm, workspace, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq, xq_sf};
+  if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (xq_col) {
+    QuantColsArgs qc{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq_col, xq_col_sf};
+    if ((e = launch_quant_cols(qc, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* out, moe_stream_t stream) {
+  if (!y || !out || T < 0 || k <= 0 || H <= 0 || H % 8) return MOE_ERR_INVALID;
+  if (!al16(y) || !al16(out)) return MOE_ERR_INVALID;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  return cuda_status(launch_combine(y, false, T, k, H, out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const uint8_t* w2q,
+                                 const uint8_t* w2sf, int32_t T, int32_t H, int32_t I, int32_t E,
+                                 int32_t k, int64_t rows_cap, const int32_t* split_sizes,
+                                 const int32_t* group_offsets, const int32_t* row_to_slot,
+                                 const float* prob_perm, const uint8_t* xq, const uint8_t* xq_sf,
+                                 void* out, void* saved_a, uint8_t* hq, uint8_t* hq_sf, void* workspace,
+                                 size_t workspace_bytes, moe_stream_t stream) {
+  if (!w1q || !w1sf || !w2q || !w2sf || !split_sizes || !group_offsets || !row_to_slot || !prob_perm ||
+      !xq || !xq_sf || !out)
+    return MOE_ERR_INVALID;
+  if ((hq == nullptr) != (hq_sf == nullptr)) return MOE_ERR_INVALID;
+  if (!layer_dims_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
+  for (const void* p : {(const void*)w1q, (const void*)w1sf, (const void*)w2q, (const void*)w2sf,
+                        (const void*)xq, (const void*)xq_sf, (const void*)out})
+    if (!al16(p)) return MOE_ERR_INVALID;
+  if ((saved_a && !al16(saved_a)) || (hq && (!al16(hq) || !al16(hq_sf)))) return MOE_ERR_INVALID;
+  Carver c{static_cast<uint8_t*>(workspace)};
+  FwdWs w = carve_fwd(c, T, k, H, I, rows_cap, hq == nullptr);
+  if (!workspace || int64_t(workspace_bytes) < c.off) return MOE_ERR_WORKSPACE;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  if (hq) { w.hq = hq; w.hq_sf = hq_sf; }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) return MOE_OK;
+
+  // gate_up grouped GEMM + ScaledSwiGLU + requantisation of h
+  GemmMaps m1;
+  cudaError_t e;
+  if ((e = make_map_2d(&m1.a, xq, H, rows_cap, 128)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((e = make_map_3d(&m1.b, w1q, H, I, 2 * int64_t(E), 128)) != cudaSuccess) return MOE_ERR_CUDA;
+  GemmArgs g1{};
+  g1.mode = 0; g1.E = E; g1.N = I; g1.num_kt = int32_t(cdiv(H, 128)); g1.n_tiles = int32_t(cdiv(I, 128));
+  g1.group_offsets = group_offsets; g1.split_sizes = split_sizes;
+  g1.sfa = xq_sf; g1.a_KT = int32_t(cdiv(H, 128));
+  g1.sfb = w1sf; g1.b_RT = int32_t(cdiv(I, 128)); g1.b_KT = int32_t(cdiv(H, 128));
+  g1.prob = prob_perm; g1.row_to_slot = row_to_slot;
+  g1.out2 = static_cast<uint8_t*>(saved_a);
+  g1.q_out = w.hq; g1.sf_out = w.hq_sf; g1.q_KT = int32_t(cdiv(I, 128));
+  if ((e = launch_grouped_gemm(EPI_SWIGLU, m1, g1, st)) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // down grouped GEMM, rows scattered to slot order
+  GemmMaps m2;
+  if ((e = make_map_2d(&m2.a, w.hq, I, rows_cap, 128)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((e = make_map_3d(&m2.b, w2q, I, H, E, 256)) != cudaSuccess) return MOE_ERR_CUDA;
+  GemmArgs g2{};
+  g2.mode = 0; g2.E = E; g2.N = H; g2.num_kt = int32_t(cdiv(I, 128)); g2.n_tiles = int32_t(cdiv(H, 256));
+  g2.group_offsets = group_offsets; g2.split_sizes = split_sizes;
+  g2.sfa = w.hq_sf; g2.a_KT = int32_t(cdiv(I, 128));
+  g2.sfb = w2sf; g2.b_RT = int32_t(cdiv(H, 128)); g2.b_KT = int32_t(cdiv(I, 128));
+  g2.row_to_slot = row_to_slot; g2.out = w.y; g2.ld_out = H;
+  if ((e = launch_grouped_gemm(EPI_F32_SCATTER, m2, g2, st)) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // top-k combine back to token order
+  return cuda_status(launch_combine(w.y, true, T, k, H, out, st));
+}
+
+moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, const uint8_t* w1tq,
+                                 const uint8_t* w1tsf, int32_t T, int32_t H, int32_t I, int32_t E,
+                                 int32_t k, int64_t rows_cap, const int32_t* split_sizes,
+                                 const int32_t* group_offsets, const int32_t* row_to_slot,
+                                 const int32_t* slot_to_row, const float* prob_perm, const void* dY,
+                                 const void* saved_a, const uint8_t* xq_col, const uint8_t* xq_col_sf,
+                                 void* dX, void* dW1, void* dW2, float* dprob, void* workspace,
+                                 size_t workspace_bytes, moe_stream_t stream) {
+  if (!w2tq || !w2tsf || !w1tq || !w1tsf || !split_sizes || !group_offsets || !row_to_slot ||
+      !slot_to_row || !prob_perm || !dY || !saved_a || !xq_col || !xq_col_sf || !dX || !dW1 || !dW2 ||
+      !dprob)
+    return MOE_ERR_INVALID;
+  if (!layer_dims_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
+  for (const void* p : {(const void*)w2tq, (const void*)w2tsf, (const void*)w1tq, (const void*)w1tsf,
+                        dY, saved_a, (const void*)xq_col, (const void*)xq_col_sf, (const void*)dX,
+                        (const void*)dW1, (const void*)dW2})
+    if (!al16(p)) return MOE_ERR_INVALID;
+  Carver c{static_cast<uint8_t*>(workspace)};
+  BwdWs w = carve_bwd(c, T, k, H, I, rows_cap);
+  if (!workspace || int64_t(workspace_bytes) < c.off) return MOE_ERR_WORKSPACE;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+
+  // dy rows gathered to permuted order, quantised along H and along tokens
+  QuantRowsArgs qr{static_cast<const uint8_t*>(dY), H, row_to_slot, k, 1, rows_cap, H, w.dyq, w.dyq_sf};
+  if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  QuantColsArgs qc{static_cast<const uint8_t*>(dY), H, row_to_slot, k, 1, rows_cap, H, w.dyc, w.dyc_sf};
+  if ((e = launch_quant_cols(qc, st)) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // dgrad2: dh = dy W_down (contraction over H)
+  GemmMaps m;
+  if (make_map_2d(&m.a, w.dyq, H, rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m.b, w2tq, H, I, E, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  GemmArgs g{};
+  g.mode = 0; g.E = E; g.N = I; g.num_kt = int32_t(cdiv(H, 128)); g.n_tiles = int32_t(cdiv(I, 256));
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes;
+  g.sfa = w.dyq_sf; g.a_KT = int32_t(cdiv(H, 128));
+  g.sfb = w2tsf; g.b_RT = int32_t(cdiv(I, 128)); g.b_KT = int32_t(cdiv(H, 128));
+  g.out = w.dh; g.ld_out = I;
+  if (launch_grouped_gemm(EPI_F32_ROWS, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // ScaledSwiGLU backward + quantisation of da (both ways) and h (along tokens)
+  SwigluBwdArgs sb{I, E, rows_cap, group_offsets, row_to_slot, prob_perm, w.dh,
+                   static_cast<const uint8_t*>(saved_a), w.daq, w.daq_sf, w.dac, w.dac_sf, w.hc, w.hc_sf,
+                   dprob};
+  if (launch_swiglu_bwd(sb, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // wgrad2: dW_down_e = dy_e^T h_e (contraction over the group's tokens)
+  if (make_map_2d(&m.a, w.dyc, rows_cap, H, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_2d(&m.b, w.hc, rows_cap, I, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  g = GemmArgs{};
+  g.mode = 1; g.E = E; g.N = I; g.n_tiles = int32_t(cdiv(I, 256));
+  g.m_tiles = int32_t(cdiv(H, 128)); g.M_out = H;
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes;
+  g.sfa = w.dyc_sf; g.a_KT = int32_t(rows_cap / 128);
+  g.sfb = w.hc_sf; g.b_RT = int32_t(cdiv(I, 128)); g.b_KT = int32_t(rows_cap / 128);
+  g.out = static_cast<uint8_t*>(dW2); g.ld_out = I; g.out_group_stride = int64_t(H) * I;
+  if (launch_grouped_gemm(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // dgrad1: dx = da W_gate_up (contraction over 2I), rows scattered to slots
+  if (make_map_2d(&m.a, w.daq, 2 * int64_t(I), rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m.b, w1tq, 2 * int64_t(I), H, E, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  g = GemmArgs{};
+  g.mode = 0; g.E = E; g.N = H; g.num_kt = int32_t(cdiv(2 * int64_t(I), 128));
+  g.n_tiles = int32_t(cdiv(H, 256));
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes;
+  g.sfa = w.daq_sf; g.a_KT = int32_t(cdiv(2 * int64_t(I), 128));
+  g.sfb = w1tsf; g.b_RT = int32_t(cdiv(H, 128)); g.b_KT = int32_t(cdiv(2 * int64_t(I), 128));
+  g.row_to_slot = row_to_slot; g.out = w.dx; g.ld_out = H;
+  if (launch_grouped_gemm(EPI_F32_SCATTER, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_combine(w.dx, true, T, k, H, dX, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // wgrad1: dW_gate_up_e = da_e^T x_e (contraction over the group's tokens)
+  if (make_map_2d(&m.a, w.dac, rows_cap, 2 * int64_t(I), 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_2d(&m.b, xq_col, rows_cap, H, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  g = GemmArgs{};
+  g.mode = 1; g.E = E; g.N = H; g.n_tiles = int32_t(cdiv(H, 256));
+  g.m_tiles = int32_t(cdiv(2 * int64_t(I), 128)); g.M_out = 2 * I;
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes;
+  g.sfa = w.dac_sf; g.a_KT = int32_t(rows_cap / 128);
+  g.sfb = xq_col_sf; g.b_RT = int32_t(cdiv(H, 128)); g.b_KT = int32_t(rows_cap / 128);
+  g.out = static_cast<uint8_t*>(dW1); g.ld_out = H; g.out_group_stride = 2 * int64_t(I) * H;
+  if (launch_grouped_gemm(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  (void)slot_to_row;
+  return MOE_OK;
+}
+
+moe_status_t moe_get_device_status(moe_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  return static_cast<moe_status_t>(v);
+}
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID: return "invalid argument (null pointer, size or alignment)";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_DEVICE_INDEX: return "device: expert id out of range";
+    case MOE_ERR_TIMEOUT: return "device: bounded pipeline wait timed out";
+    case MOE_ERR_NO_DEVICE: return "no sm_100 CUDA device current";
+  }
+  return "unknown status";
+}
+
+int64_t moe_launch_count(int32_t reset) {
+  return reset ? g_launches.exchange(0) : g_launches.load();
+}
+
+moe_status_t moe_selftest_wait_timeout(int32_t wait_ms, moe_stream_t stream) {
+  if (wait_ms <= 0 || wait_ms > 10000) return MOE_ERR_INVALID;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  moe_status_t prev = moe_get_device_status(stream);  // clear any earlier record
+  (void)prev;
+  wait_timeout_kernel<<<1, 32, 0, st>>>(static_cast<long long>(wait_ms) * 2000000ll);
+  count_launch();
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  return moe_get_device_status(stream);
+}
+
+}  // extern "C"

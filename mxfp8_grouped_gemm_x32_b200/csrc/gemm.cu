@@ -1,0 +1,448 @@
+// Persistent, warp-specialised grouped MXFP8 GEMM for B200 (sm_100a).
+//
+// "Efficient MoE Training for Biological Foundation Models":
+//   Challenge 1  -- all experts' GEMMs are submitted as one grouped operation
+//                   over ragged per-expert token groups (split_sizes);
+//   Challenge 2  -- MXFP8 operands (E4M3 + one E8M0 scale per 32 values along
+//                   K) on Blackwell's block-scaled tensor-core instructions;
+//   Challenge 3 / Figure 4 -- gate_up GEMM, SwiGLU, routing-probability
+//                   scaling and requantisation fused into one kernel before
+//                   the down projection, so the BF16 intermediate is never
+//                   written.
+//
+// Design (one CTA per SM, 320 threads):
+//   warp 0      TMA producer: A tile 128x128 B, B tile 256x128 B (2-D or
+//               3-D tensor maps, 128-byte swizzle), both scale atoms by bulk
+//               copy, into a 4-stage shared-memory ring (mbarrier pipeline).
+//   warp 1      TMEM owner and MMA issuer: per 128-wide K tile, copies the
+//               scale atoms to TMEM (tcgen05.cp 32x128b.warpx4) and issues
+//               four tcgen05.mma.kind::mxf8f6f4.block_scale (M128 N256 K32)
+//               into an fp32 accumulator of 256 TMEM columns.
+//   warps 2-9   epilogue: drain the accumulator into registers
+//               (tcgen05.ld), release it to the MMA warp at once, then apply
+//               the epilogue and store -- so the next tile's MMAs overlap it.
+// Tiles (128 rows x 256 columns) walk a device-side schedule derived from
+// the group offsets; every CTA strides through them (persistent grid).
+// Every wait is bounded; on time-out the kernel records MOE_ERR_TIMEOUT,
+// stops all roles and still frees its TMEM.
+#include "gemm.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4;
+constexpr int SMEM_A = BM * BK;  // 16 KB
+constexpr int SMEM_B = BN * BK;  // 32 KB
+constexpr int SMEM_SFA = 512;
+constexpr int SMEM_SFB = 1024;
+constexpr uint32_t STAGE_TX = SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB;
+constexpr int NUM_THREADS = 320;
+constexpr int NUM_EPI_WARPS = 8;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 260;
+
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * SMEM_A;
+constexpr int OFF_SFA = OFF_B + STAGES * SMEM_B;
+constexpr int OFF_SFB = OFF_SFA + STAGES * SMEM_SFA;
+constexpr int OFF_BAR = OFF_SFB + STAGES * SMEM_SFB;
+constexpr int NUM_BARS = 2 * STAGES + 2;
+constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem address, abort flag
+constexpr int OFF_GO = OFF_MISC + 16;              // group offsets [E+1]
+constexpr int SMEM_TOTAL = OFF_GO + (MOE_MAX_EXPERTS + 1) * 4;
+constexpr int SMEM_LAUNCH = SMEM_TOTAL + 1024;     // slack for 1 KB alignment
+
+struct Tile {
+  int e, m0, n0, kt0, nkt, row_end;
+};
+
+template <int EPI>
+__device__ __forceinline__ int total_tiles(const GemmArgs& a, const int* go) {
+  if (a.mode == 0) return (go[a.E] >> 7) * a.n_tiles;
+  return a.E * a.m_tiles * a.n_tiles;
+}
+
+template <int EPI>
+__device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, int t) {
+  Tile ti;
+  if (a.mode == 0) {
+    const int nt = a.n_tiles;
+    int lo = 0, hi = a.E - 1;  // last expert whose first tile is <= t
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if ((go[mid] >> 7) * nt <= t) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const int mt = (go[e + 1] - go[e]) >> 7;
+    const int local = t - (go[e] >> 7) * nt;
+    const int n_idx = local / mt, m_idx = local - n_idx * mt;  // rows fastest: B panel reuse
+    ti.e = e;
+    ti.m0 = go[e] + (m_idx << 7);
+    ti.n0 = n_idx * (EPI == EPI_SWIGLU ? 128 : 256);
+    ti.kt0 = 0;
+    ti.nkt = a.num_kt;
+    ti.row_end = go[e] + a.split_sizes[e];
+  } else {
+    const int per = a.m_tiles * a.n_tiles;
+    const int e = t / per;
+    const int local = t - e * per;
+    const int n_idx = local / a.m_tiles, m_idx = local - n_idx * a.m_tiles;
+    ti.e = e;
+    ti.m0 = m_idx << 7;
+    ti.n0 = n_idx << 8;
+    ti.kt0 = go[e] >> 7;
+    ti.nkt = (go[e + 1] - go[e]) >> 7;
+    ti.row_end = a.M_out;
+  }
+  return ti;
+}
+
+__device__ __forceinline__ uint32_t block_amax_bits(const float* f) {
+  uint32_t am = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) am = max(am, __float_as_uint(f[j]) & 0x7FFFFFFFu);
+  return am;
+}
+
+// Quantise 32 fp32 values to E4M3 codes with scale byte sb, store 32 bytes.
+__device__ __forceinline__ void store_block_e4m3(uint8_t* dst, const float* f, uint32_t sb) {
+  const float inv = inv_scale_from_e8m0(sb);
+  uint32_t w[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    w[j] = pack4_e4m3(f[4 * j] * inv, f[4 * j + 1] * inv, f[4 * j + 2] * inv, f[4 * j + 3] * inv);
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// 128 fp32 (as bits) -> bf16, 16 x 16-byte stores, columns >= ncols skipped
+// in units of 8.
+__device__ __forceinline__ void store_row_bf16(uint8_t* dst, const uint32_t* v, int ncols) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (8 * i < ncols)
+      d[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1])),
+                        pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                        pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                        pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+  }
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti, const uint32_t* v,
+                                              int q, int half, int lane) {
+  const int r = ti.m0 + 32 * q + lane;
+  if (r >= ti.row_end) return;
+  if constexpr (EPI == EPI_SWIGLU) {
+    // v[0:64] gate columns nb..nb+63, v[64:128] the matching up columns
+    const int nb = ti.n0 + 64 * half;
+    if (nb >= a.N) return;
+    const int N = a.N;
+    if (a.out2) {
+      uint4* dg = reinterpret_cast<uint4*>(a.out2 + (int64_t(r) * 2 * N + nb) * 2);
+      uint4* du = reinterpret_cast<uint4*>(a.out2 + (int64_t(r) * 2 * N + N + nb) * 2);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t* g = v + 8 * i;
+        const uint32_t* u = v + 64 + 8 * i;
+        dg[i] = make_uint4(pack_bf16x2(__uint_as_float(g[0]), __uint_as_float(g[1])),
+                           pack_bf16x2(__uint_as_float(g[2]), __uint_as_float(g[3])),
+                           pack_bf16x2(__uint_as_float(g[4]), __uint_as_float(g[5])),
+                           pack_bf16x2(__uint_as_float(g[6]), __uint_as_float(g[7])));
+        du[i] = make_uint4(pack_bf16x2(__uint_as_float(u[0]), __uint_as_float(u[1])),
+                           pack_bf16x2(__uint_as_float(u[2]), __uint_as_float(u[3])),
+                           pack_bf16x2(__uint_as_float(u[4]), __uint_as_float(u[5])),
+                           pack_bf16x2(__uint_as_float(u[6]), __uint_as_float(u[7])));
+      }
+    }
+    const float p = a.prob[r];
+    uint32_t sbs = 0;
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      float h[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float g = __uint_as_float(v[32 * b + j]);
+        const float u = __uint_as_float(v[64 + 32 * b + j]);
+        h[j] = p * __fdividef(g, 1.0f + __expf(-g)) * u;
+      }
+      const uint32_t sb = e8m0_from_amax_bits(block_amax_bits(h));
+      store_block_e4m3(a.q_out + int64_t(r) * N + nb + 32 * b, h, sb);
+      sbs |= sb << (8 * b);
+    }
+    const int kb0 = nb >> 5;
+    uint8_t* sfp = a.sf_out + sf_offset(0, r, kb0, 0, a.q_KT);
+    if (nb + 64 == N && (kb0 & 3) == 0)
+      *reinterpret_cast<uint32_t*>(sfp) = sbs;  // also zero the two padding blocks of the K tile
+    else
+      *reinterpret_cast<uint16_t*>(sfp) = uint16_t(sbs);
+  } else {
+    const int nb = ti.n0 + 128 * half;
+    if (nb >= a.N) return;
+    if constexpr (EPI == EPI_F32_SCATTER || EPI == EPI_F32_ROWS) {
+      int64_t orow = r;
+      if constexpr (EPI == EPI_F32_SCATTER) {
+        orow = a.row_to_slot[r];
+        if (orow < 0) return;
+      }
+      uint4* d = reinterpret_cast<uint4*>(a.out + (orow * a.ld_out + nb) * 4);
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (4 * i < a.N - nb) d[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      return;
+    }
+    uint8_t* dst = a.out + (int64_t(ti.e) * a.out_group_stride + int64_t(r) * a.ld_out + nb) * 2;
+    store_row_bf16(dst, v, a.N - nb);
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_mxf8_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB, const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+  int* go = reinterpret_cast<int*>(smem + OFF_GO);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, NUM_EPI_WARPS);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i <= a.E; i += NUM_THREADS) go[i] = a.group_offsets[i];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int ntiles = total_tiles<EPI>(a, go);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const Tile ti = decode_tile<EPI>(a, go, t);
+        for (int kt = 0; kt < ti.nkt; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          uint64_t* bar = &full[stage];
+          mbar_arrive_expect_tx(bar, STAGE_TX);
+          const int kg = ti.kt0 + kt;
+          uint8_t* sa = smem + OFF_A + stage * SMEM_A;
+          uint8_t* sb = smem + OFF_B + stage * SMEM_B;
+          uint8_t* ssfa = smem + OFF_SFA + stage * SMEM_SFA;
+          uint8_t* ssfb = smem + OFF_SFB + stage * SMEM_SFB;
+          tma_load_2d(sa, &tmA, bar, kg * BK, ti.m0);
+          bulk_load(ssfa, a.sfa + (int64_t(ti.m0 >> 7) * a.a_KT + kg) * 512, 512, bar);
+          if constexpr (EPI == EPI_SWIGLU) {
+            tma_load_3d(sb, &tmB, bar, kg * BK, ti.n0, 2 * ti.e);
+            tma_load_3d(sb + SMEM_B / 2, &tmB, bar, kg * BK, ti.n0, 2 * ti.e + 1);
+            const int rb = ti.n0 >> 7;
+            bulk_load(ssfb, a.sfb + ((int64_t(2 * ti.e) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
+            bulk_load(ssfb + 512, a.sfb + ((int64_t(2 * ti.e + 1) * a.b_RT + rb) * a.b_KT + kg) * 512,
+                      512, bar);
+          } else {
+            if (a.mode == 0)
+              tma_load_3d(sb, &tmB, bar, kg * BK, ti.n0, ti.e);
+            else
+              tma_load_2d(sb, &tmB, bar, kg * BK, ti.n0);
+            const int64_t gb = a.mode == 0 ? int64_t(ti.e) * a.b_RT : 0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int rb = min((ti.n0 >> 7) + h, a.b_RT - 1);  // rows past N: any finite atom
+              bulk_load(ssfb + 512 * h, a.sfb + ((gb + rb) * a.b_KT + kg) * 512, 512, bar);
+            }
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int stage = 0;
+      uint32_t phase = 0, acc_it = 0;
+      bool ok = true;
+      const uint32_t sfa_t = tmem + SFA_COL, sfb_t = tmem + SFB_COL;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const Tile ti = decode_tile<EPI>(a, go, t);
+        if (ti.nkt == 0) continue;
+        if (!mbar_wait(acc_empty, (acc_it & 1u) ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        for (int kt = 0; kt < ti.nkt; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + OFF_A + stage * SMEM_A);
+          const uint32_t sb = smem_u32(smem + OFF_B + stage * SMEM_B);
+          const uint32_t ssfa = smem_u32(smem + OFF_SFA + stage * SMEM_SFA);
+          const uint32_t ssfb = smem_u32(smem + OFF_SFB + stage * SMEM_SFB);
+          tc_cp_32x128b_warpx4(sfa_t, make_smem_desc(ssfa, 0, 128, 0));
+          tc_cp_32x128b_warpx4(sfb_t, make_smem_desc(ssfb, 0, 128, 0));
+          tc_cp_32x128b_warpx4(sfb_t + 4, make_smem_desc(ssfb + 512, 0, 128, 0));
+#pragma unroll
+          for (uint32_t kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = make_smem_desc(sa + 32 * kk, 16, 1024, 2);
+            const uint64_t bd = make_smem_desc(sb + 32 * kk, 16, 1024, 2);
+            tc_mma_mxf8(tmem + ACC_COL, ad, bd, make_idesc_mxf8(BM, BN, kk, kk), sfa_t | (kk << 30),
+                        sfb_t | (kk << 30), (kt | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        ++acc_it;
+      }
+    }
+  } else {
+    // ---------------- epilogue warps ----------------
+    const int q = warp & 3;            // TMEM sub-partition this warp may read
+    const int half = (warp - 2) >> 2;  // which half of the tile's columns
+    uint32_t acc_it = 0;
+    uint32_t v[128];
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const Tile ti = decode_tile<EPI>(a, go, t);
+      if (ti.nkt == 0) {
+        if constexpr (EPI == EPI_WGRAD) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) v[i] = 0u;
+          epilogue_tile<EPI>(a, ti, v, q, half, lane);
+        }
+        continue;
+      }
+      if (!mbar_wait(acc_full, acc_it & 1u, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tl = tmem + (uint32_t(32 * q) << 16) + ACC_COL;
+      if constexpr (EPI == EPI_SWIGLU) {
+        tmem_ld32(tl + 64 * half, v);
+        tmem_ld32(tl + 64 * half + 32, v + 32);
+        tmem_ld32(tl + 128 + 64 * half, v + 64);
+        tmem_ld32(tl + 128 + 64 * half + 32, v + 96);
+      } else {
+        tmem_ld32(tl + 128 * half, v);
+        tmem_ld32(tl + 128 * half + 32, v + 32);
+        tmem_ld32(tl + 128 * half + 64, v + 64);
+        tmem_ld32(tl + 128 * half + 96, v + 96);
+      }
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      ++acc_it;
+      epilogue_tile<EPI>(a, ti, v, q, half, lane);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int EPI>
+cudaError_t launch_epi(const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_mxf8_gemm_kernel<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LAUNCH);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  grouped_mxf8_gemm_kernel<EPI><<<sm_count(), NUM_THREADS, SMEM_LAUNCH, st>>>(maps.a, maps.b, a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t groups,
+                        uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {inner, rows, groups};
+  cuuint64_t strides[2] = {inner, inner * rows};
+  cuuint32_t box[3] = {128, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_grouped_gemm(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
+  switch (epi) {
+    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(maps, a, st);
+    case EPI_F32_SCATTER: return launch_epi<EPI_F32_SCATTER>(maps, a, st);
+    case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS>(maps, a, st);
+    case EPI_WGRAD: return launch_epi<EPI_WGRAD>(maps, a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

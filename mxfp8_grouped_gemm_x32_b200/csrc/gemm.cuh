@@ -1,0 +1,61 @@
+// Persistent grouped block-scaled MXFP8 GEMM for sm_100a (tcgen05 + TMA).
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+// Epilogue variants of the grouped GEMM.
+enum EpiKind : int {
+  EPI_SWIGLU = 0,        // gate_up: h = p * silu(gate) * up, requantised to MXFP8 (+ saved A in bf16)
+  EPI_F32_SCATTER = 1,   // down / dgrad1: fp32 rows written to their slot (row_to_slot)
+  EPI_F32_ROWS = 2,      // dgrad2: fp32 rows in permuted order (feeds the requantising SwiGLU backward)
+  EPI_WGRAD = 3          // weight gradients: one bf16 matrix per expert
+};
+
+// One grouped GEMM  D = (A * SFA) (B * SFB)^T  over ragged expert groups.
+//  mode 0: groups along the rows of A (forward, dgrad).  A is the padded
+//          permuted activation [rows_cap][K]; group e owns rows
+//          [group_offsets[e], group_offsets[e+1]) and multiplies B_e.
+//  mode 1: groups along K (wgrad).  A [M_out][rows_cap] and B [N][rows_cap]
+//          are token-major; expert e contracts over its own token range
+//          and writes its own output matrix.
+struct GemmArgs {
+  int32_t mode;
+  int32_t E;
+  int32_t N;        // output columns (EPI_SWIGLU: I, the width of h)
+  int32_t num_kt;   // mode 0: 128-wide K tiles of the contraction
+  int32_t n_tiles;  // tiles along N
+  int32_t m_tiles;  // mode 1: 128-row tiles of the output per expert
+  int32_t M_out;    // mode 1: output rows per expert
+  const int32_t* group_offsets;  // [E+1], multiples of 128
+  const int32_t* split_sizes;    // [E]
+  const uint8_t* sfa;
+  int32_t a_KT;  // K tiles in A's scale layout
+  const uint8_t* sfb;
+  int32_t b_RT, b_KT;  // row tiles per group and K tiles in B's scale layout
+  const float* prob;
+  const int32_t* row_to_slot;
+  uint8_t* out;       // bf16 output
+  int64_t ld_out;     // elements between output rows
+  int64_t out_group_stride;  // mode 1: elements between experts' matrices
+  uint8_t* out2;      // EPI_SWIGLU: saved A, bf16 [rows][2N] (nullable)
+  uint8_t* q_out;     // EPI_SWIGLU: h codes [rows][N]
+  uint8_t* sf_out;    // EPI_SWIGLU: h scales, blocked (1, rows, N)
+  int32_t q_KT;
+};
+
+// Tensor maps: A 2-D {K, rows} with a 128 x 128 box; B either 3-D
+// {K, rows, groups} or 2-D {K, rows} with a 128 x (128|256) box; all uint8
+// with 128-byte swizzle.
+struct GemmMaps {
+  CUtensorMap a, b;
+};
+
+cudaError_t make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                        uint32_t box_rows);
+cudaError_t make_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                        uint64_t groups, uint32_t box_rows);
+
+cudaError_t launch_grouped_gemm(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,20 @@
+// Launch interfaces of the permutation and combine kernels.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+int64_t permute_workspace_bytes(int64_t R, int32_t E);
+
+// Counting sort of R = T*k routed slots by expert into the 128-aligned padded
+// row space (split sizes, group offsets, both index maps, permuted probs).
+cudaError_t launch_permute_index(const int32_t* idx, const float* prob, int64_t R, int32_t E,
+                                 int64_t rows_cap, int32_t* split, int32_t* offs,
+                                 int32_t* row_to_slot, int32_t* slot_to_row, float* prob_perm,
+                                 void* ws, cudaStream_t st);
+
+// out[t] = sum_{j<k} y[t*k+j]  (fp32 or bf16 in, fp32 sum, bf16 out), H % 8 == 0.
+cudaError_t launch_combine(const void* y, bool f32_in, int64_t T, int32_t k, int64_t H, void* out,
+                           cudaStream_t st);
+
+}  // namespace moe

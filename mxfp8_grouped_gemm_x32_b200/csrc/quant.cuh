@@ -1,0 +1,36 @@
+// Launch interfaces of the MXFP8 quantisation kernels.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+// Row mode: out row (g, r) <- src row (g*rows + r), or, with row_map, src row
+// row_map[g*rows + r] / map_div (a negative map entry gives a zero row).
+struct QuantRowsArgs {
+  const uint8_t* src;     // bf16 rows, `ld` elements apart
+  int64_t ld;
+  const int32_t* row_map;  // optional gather map
+  int32_t map_div;
+  int32_t groups;
+  int64_t rows, K;
+  uint8_t* q;   // [groups][rows][K]
+  uint8_t* sf;  // blocked (groups, rows, K)
+};
+
+// Column mode: input [groups][rows][cols] (optional row gather as above),
+// output the transposed MX tensor [groups][cols][rows] quantised along rows.
+struct QuantColsArgs {
+  const uint8_t* src;
+  int64_t ld;
+  const int32_t* row_map;
+  int32_t map_div;
+  int32_t groups;
+  int64_t rows, cols;
+  uint8_t* q;   // [groups][cols][rows]
+  uint8_t* sf;  // blocked (groups, cols, rows)
+};
+
+cudaError_t launch_quant_rows(const QuantRowsArgs& a, cudaStream_t st);
+cudaError_t launch_quant_cols(const QuantColsArgs& a, cudaStream_t st);
+
+}  // namespace moe

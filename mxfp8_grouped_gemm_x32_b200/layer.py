@@ -1,0 +1,140 @@
+"""Device buffers for one grouped MXFP8 MoE expert layer, driven through the
+C ABI.  PyTorch only allocates device memory and provides the stream; every
+step of the layer runs in the CUDA library (see lib.py).
+
+Steps (names of the C entry points):
+  quantize_weights  moe_mlp_quantize_mxfp8 x4: W_gate_up and W_down, along K
+                    for the forward and along the other axis for the backward
+  permute           moe_permute: counting sort by expert, gather + quantise x
+  forward           moe_grouped_mlp_fwd: gate_up GEMM + ScaledSwiGLU + requant,
+                    down GEMM, top-k combine
+  backward          moe_grouped_mlp_bwd: dgrad/wgrad of both projections,
+                    ScaledSwiGLU backward, d(prob)
+"""
+from __future__ import annotations
+
+import torch
+
+from . import lib
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def _u8(n: int, dev) -> torch.Tensor:
+    # 256-byte aligned by the caching allocator; sizes rounded to 16 bytes
+    return torch.empty(max(16, (n + 15) // 16 * 16), dtype=torch.uint8, device=dev)
+
+
+class GroupedMLP:
+    """One layer: T tokens, hidden H, intermediate I, E experts, top-k."""
+
+    def __init__(self, T: int, H: int, I: int, E: int, k: int, device="cuda", backward: bool = True):
+        self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
+        self.dev = torch.device(device)
+        dev = self.dev
+        self.rows_cap = lib.moe_padded_rows(T, k, E)
+        rc = self.rows_cap
+        sb = lib.moe_mx_scale_bytes
+        # quantised weights (forward: along H for gate_up, along I for down)
+        self.w1q = _u8(2 * E * I * H, dev)
+        self.w1sf = _u8(sb(2 * E, I, H), dev)
+        self.w2q = _u8(E * H * I, dev)
+        self.w2sf = _u8(sb(E, H, I), dev)
+        # routing
+        self.split_sizes = torch.empty(E, dtype=torch.int32, device=dev)
+        self.group_offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        self.row_to_slot = torch.empty(rc, dtype=torch.int32, device=dev)
+        self.slot_to_row = torch.empty(T * k, dtype=torch.int32, device=dev)
+        self.prob_perm = torch.empty(rc, dtype=torch.float32, device=dev)
+        self.xq = _u8(rc * H, dev)
+        self.xq_sf = _u8(sb(1, rc, H), dev)
+        self.hq = _u8(rc * I, dev)
+        self.hq_sf = _u8(sb(1, rc, I), dev)
+        self.out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        self.ws_perm_bytes = lib.moe_workspace_size(lib.MOE_OP_PERMUTE, T, k, E, H, I)
+        self.ws_fwd_bytes = lib.moe_workspace_size(lib.MOE_OP_FWD, T, k, E, H, I)
+        self.ws_perm = _u8(self.ws_perm_bytes, dev)
+        self.ws_fwd = _u8(self.ws_fwd_bytes, dev)
+        self.backward_enabled = backward
+        if backward:
+            self.w1tq = _u8(E * H * 2 * I, dev)
+            self.w1tsf = _u8(sb(E, H, 2 * I), dev)
+            self.w2tq = _u8(E * I * H, dev)
+            self.w2tsf = _u8(sb(E, I, H), dev)
+            self.xq_col = _u8(H * rc, dev)
+            self.xq_col_sf = _u8(sb(1, H, rc), dev)
+            self.saved_a = torch.empty(rc, 2 * I, dtype=torch.bfloat16, device=dev)
+            self.dX = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+            self.dW1 = torch.empty(E, 2 * I, H, dtype=torch.bfloat16, device=dev)
+            self.dW2 = torch.empty(E, H, I, dtype=torch.bfloat16, device=dev)
+            self.dprob = torch.empty(T, k, dtype=torch.float32, device=dev)
+            self.ws_bwd_bytes = lib.moe_workspace_size(lib.MOE_OP_BWD, T, k, E, H, I)
+            self.ws_bwd = _u8(self.ws_bwd_bytes, dev)
+        else:
+            self.saved_a = None
+
+    @staticmethod
+    def _stream() -> int:
+        return torch.cuda.current_stream().cuda_stream
+
+    def quantize_weights(self, w1: torch.Tensor, w2: torch.Tensor) -> None:
+        """w1 bf16 [E, 2I, H] (gate rows first), w2 bf16 [E, H, I]."""
+        E, H, I, s = self.E, self.H, self.I, self._stream()
+        assert w1.dtype == torch.bfloat16 and w1.is_contiguous() and w1.shape == (E, 2 * I, H)
+        assert w2.dtype == torch.bfloat16 and w2.is_contiguous() and w2.shape == (E, H, I)
+        lib.moe_mlp_quantize_mxfp8(w1.data_ptr(), 2 * E, I, H, lib.MOE_QUANT_ROW, _ptr(self.w1q), _ptr(self.w1sf), s)
+        lib.moe_mlp_quantize_mxfp8(w2.data_ptr(), E, H, I, lib.MOE_QUANT_ROW, _ptr(self.w2q), _ptr(self.w2sf), s)
+        if self.backward_enabled:
+            lib.moe_mlp_quantize_mxfp8(w1.data_ptr(), E, 2 * I, H, lib.MOE_QUANT_COL, _ptr(self.w1tq),
+                                       _ptr(self.w1tsf), s)
+            lib.moe_mlp_quantize_mxfp8(w2.data_ptr(), E, H, I, lib.MOE_QUANT_COL, _ptr(self.w2tq),
+                                       _ptr(self.w2tsf), s)
+
+    def permute(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_prob: torch.Tensor) -> None:
+        """x bf16 [T, H]; topk_idx int32 [T, k]; topk_prob float32 [T, k]."""
+        assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.shape == (self.T, self.H)
+        assert topk_idx.dtype == torch.int32 and topk_idx.is_contiguous()
+        assert topk_prob.dtype == torch.float32 and topk_prob.is_contiguous()
+        bw = self.backward_enabled
+        lib.moe_permute(x.data_ptr(), topk_idx.data_ptr(), topk_prob.data_ptr(), self.T, self.H, self.k,
+                        self.E, self.rows_cap, _ptr(self.split_sizes), _ptr(self.group_offsets),
+                        _ptr(self.row_to_slot), _ptr(self.slot_to_row), _ptr(self.prob_perm),
+                        _ptr(self.xq), _ptr(self.xq_sf), _ptr(self.xq_col) if bw else 0,
+                        _ptr(self.xq_col_sf) if bw else 0, _ptr(self.ws_perm), self.ws_perm_bytes,
+                        self._stream())
+
+    def forward(self) -> torch.Tensor:
+        lib.moe_grouped_mlp_fwd(_ptr(self.w1q), _ptr(self.w1sf), _ptr(self.w2q), _ptr(self.w2sf), self.T,
+                                self.H, self.I, self.E, self.k, self.rows_cap, _ptr(self.split_sizes),
+                                _ptr(self.group_offsets), _ptr(self.row_to_slot), _ptr(self.prob_perm),
+                                _ptr(self.xq), _ptr(self.xq_sf), _ptr(self.out), _ptr(self.saved_a),
+                                _ptr(self.hq), _ptr(self.hq_sf), _ptr(self.ws_fwd), self.ws_fwd_bytes,
+                                self._stream())
+        return self.out
+
+    def backward(self, dY: torch.Tensor):
+        assert self.backward_enabled
+        assert dY.dtype == torch.bfloat16 and dY.is_contiguous() and dY.shape == (self.T, self.H)
+        lib.moe_grouped_mlp_bwd(_ptr(self.w2tq), _ptr(self.w2tsf), _ptr(self.w1tq), _ptr(self.w1tsf),
+                                self.T, self.H, self.I, self.E, self.k, self.rows_cap,
+                                _ptr(self.split_sizes), _ptr(self.group_offsets), _ptr(self.row_to_slot),
+                                _ptr(self.slot_to_row), _ptr(self.prob_perm), dY.data_ptr(),
+                                _ptr(self.saved_a), _ptr(self.xq_col), _ptr(self.xq_col_sf),
+                                _ptr(self.dX), _ptr(self.dW1), _ptr(self.dW2), _ptr(self.dprob),
+                                _ptr(self.ws_bwd), self.ws_bwd_bytes, self._stream())
+        return self.dX, self.dW1, self.dW2, self.dprob
+
+    def step(self, x, topk_idx, topk_prob, w1, w2, dY=None):
+        """One pass of the whole layer: weight quantisation, permutation,
+        forward and (if dY is given) backward."""
+        self.quantize_weights(w1, w2)
+        self.permute(x, topk_idx, topk_prob)
+        out = self.forward()
+        if dY is None:
+            return out
+        return (out,) + tuple(self.backward(dY))
+
+    def device_status(self) -> int:
+        return lib.moe_get_device_status(self._stream())

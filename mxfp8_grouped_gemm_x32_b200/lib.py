@@ -1,0 +1,140 @@
+"""ctypes binding of the C ABI in include/moe_mxfp8.h.
+
+Argument marshalling only: every function here has the name and the
+arguments of its C counterpart (device pointers as Python ints, sizes as
+ints, streams as raw cudaStream_t handles) and raises MoeError on a non-zero
+status.  All computation happens in the CUDA library; if the library is
+missing this module raises at import time instead of falling back to any
+other implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_mxfp8.so")
+
+MOE_QUANT_ROW = 1
+MOE_QUANT_COL = 2
+MOE_OP_PERMUTE = 1
+MOE_OP_FWD = 2
+MOE_OP_BWD = 3
+MOE_MAX_EXPERTS = 256
+
+STATUS = {
+    0: "MOE_OK", 1: "MOE_ERR_INVALID", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+    4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_INDEX", 6: "MOE_ERR_TIMEOUT", 7: "MOE_ERR_NO_DEVICE",
+}
+
+EXPORTED = [
+    "moe_mx_scale_bytes", "moe_padded_rows", "moe_workspace_size", "moe_mlp_quantize_mxfp8",
+    "moe_permute", "moe_grouped_mlp_fwd", "moe_combine", "moe_grouped_mlp_bwd",
+    "moe_get_device_status", "moe_status_string", "moe_launch_count", "moe_selftest_wait_timeout",
+]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)} ({status_string(code)})")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"CUDA library not built: {LIB_PATH} (run python -m "
+                      "mxfp8_grouped_gemm_x32_b200.build_lib)")
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+
+def _decl(name, res, *args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = list(args)
+    return f
+
+
+_decl("moe_mx_scale_bytes", _I64, _I32, _I64, _I64)
+_decl("moe_padded_rows", _I64, _I32, _I32, _I32)
+_decl("moe_workspace_size", _I64, _I32, _I32, _I32, _I32, _I32, _I32)
+_decl("moe_mlp_quantize_mxfp8", _I32, _P, _I32, _I64, _I64, _I32, _P, _P, _P)
+_decl("moe_permute", _I32, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
+      _P, _P, _SZ, _P)
+_decl("moe_grouped_mlp_fwd", _I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P,
+      _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
+_decl("moe_combine", _I32, _P, _I32, _I32, _I32, _P, _P)
+_decl("moe_grouped_mlp_bwd", _I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P,
+      _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
+_decl("moe_get_device_status", _I32, _P)
+_decl("moe_status_string", ctypes.c_char_p, _I32)
+_decl("moe_launch_count", _I64, _I32)
+_decl("moe_selftest_wait_timeout", _I32, _I32, _P)
+
+
+def _check(fn: str, code: int) -> None:
+    if code != 0:
+        raise MoeError(fn, code)
+
+
+def status_string(code: int) -> str:
+    return _lib.moe_status_string(code).decode()
+
+
+def moe_mx_scale_bytes(groups: int, rows: int, k: int) -> int:
+    return _lib.moe_mx_scale_bytes(groups, rows, k)
+
+
+def moe_padded_rows(T: int, k: int, E: int) -> int:
+    return _lib.moe_padded_rows(T, k, E)
+
+
+def moe_workspace_size(op: int, T: int, k: int, E: int, H: int, I: int) -> int:
+    return _lib.moe_workspace_size(op, T, k, E, H, I)
+
+
+def moe_mlp_quantize_mxfp8(src, groups, rows, cols, mode, q, sf, stream=0):
+    _check("moe_mlp_quantize_mxfp8", _lib.moe_mlp_quantize_mxfp8(src, groups, rows, cols, mode, q, sf, stream))
+
+
+def moe_permute(x, topk_idx, topk_prob, T, H, k, E, rows_cap, split_sizes, group_offsets, row_to_slot,
+                slot_to_row, prob_perm, xq, xq_sf, xq_col, xq_col_sf, workspace, workspace_bytes, stream=0):
+    _check("moe_permute", _lib.moe_permute(x, topk_idx, topk_prob, T, H, k, E, rows_cap, split_sizes,
+                                           group_offsets, row_to_slot, slot_to_row, prob_perm, xq, xq_sf,
+                                           xq_col, xq_col_sf, workspace, workspace_bytes, stream))
+
+
+def moe_grouped_mlp_fwd(w1q, w1sf, w2q, w2sf, T, H, I, E, k, rows_cap, split_sizes, group_offsets,
+                        row_to_slot, prob_perm, xq, xq_sf, out, saved_a, hq, hq_sf, workspace,
+                        workspace_bytes, stream=0):
+    _check("moe_grouped_mlp_fwd", _lib.moe_grouped_mlp_fwd(
+        w1q, w1sf, w2q, w2sf, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot, prob_perm,
+        xq, xq_sf, out, saved_a, hq, hq_sf, workspace, workspace_bytes, stream))
+
+
+def moe_combine(y, T, k, H, out, stream=0):
+    _check("moe_combine", _lib.moe_combine(y, T, k, H, out, stream))
+
+
+def moe_grouped_mlp_bwd(w2tq, w2tsf, w1tq, w1tsf, T, H, I, E, k, rows_cap, split_sizes, group_offsets,
+                        row_to_slot, slot_to_row, prob_perm, dY, saved_a, xq_col, xq_col_sf, dX, dW1,
+                        dW2, dprob, workspace, workspace_bytes, stream=0):
+    _check("moe_grouped_mlp_bwd", _lib.moe_grouped_mlp_bwd(
+        w2tq, w2tsf, w1tq, w1tsf, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot,
+        slot_to_row, prob_perm, dY, saved_a, xq_col, xq_col_sf, dX, dW1, dW2, dprob, workspace,
+        workspace_bytes, stream))
+
+
+def moe_get_device_status(stream=0) -> int:
+    return _lib.moe_get_device_status(stream)
+
+
+def moe_launch_count(reset: bool = False) -> int:
+    return _lib.moe_launch_count(1 if reset else 0)
+
+
+def moe_selftest_wait_timeout(wait_ms: int, stream=0) -> int:
+    return _lib.moe_selftest_wait_timeout(wait_ms, stream)
