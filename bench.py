@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark of the grouped MXFP8 MoE expert MLP (forward + backward).
+
+One step = one pass of the whole hot path over one batch: weight
+quantisation (both directions), permutation + quantisation of x, the fused
+forward (gate_up GEMM + ScaledSwiGLU + requant, down GEMM, top-k combine)
+and the backward (dY quantisation, dgrad / wgrad of both projections,
+ScaledSwiGLU backward).  Metric: algorithmic TFLOP/s = 18 * R * H * I / step
+time (R = T * k routed rows), and its fraction of the dense MXFP8 peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs an independent
+replica of the layer on its own batch (data-parallel tokens, weak scaling,
+no collective on the data path); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mxfp8_grouped_gemm_x32_b200.workloads import get_config  # noqa: E402
+
+METRIC = "grouped MoE MLP fwd/bwd TFLOP/s on 1 B200 and % of dense MXFP8 peak"
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+MXFP8_OVER_BF16 = 2.0       # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemm_gate_up_swiglu.mixtral_8x7b.md")
+GEMM_SOURCES = ["mxfp8_grouped_gemm_x32_b200/csrc/gemm.cu", "mxfp8_grouped_gemm_x32_b200/csrc/gemm.cuh",
+                "mxfp8_grouped_gemm_x32_b200/csrc/common.cuh"]
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="mixtral_8x7b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# host helpers (no GPU needed; covered by tests/test_bench_host.py)
+# ---------------------------------------------------------------------------
+
+def step_flops(cfg) -> float:
+    """Algorithmic FLOPs of one forward + backward step (6RHI + 12RHI)."""
+    return cfg.fwd_flops() + cfg.bwd_flops()
+
+
+def gate_up_flops(cfg) -> float:
+    """Algorithmic FLOPs of one launch of the gate_up GEMM: 2 * R * H * 2I."""
+    return 4.0 * cfg.R * cfg.H * cfg.I
+
+
+def load_peaks(path=os.path.join(ROOT, "MEASURED_PEAKS.json")):
+    """Dense MXFP8 peak (TFLOP/s) and HBM (GB/s) with the source named."""
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        bf16 = float(p["bf16_tflops"])
+        bf16_s = float(p.get("bf16_tflops_sustained", bf16))
+        return {"mxfp8_burst": bf16 * MXFP8_OVER_BF16, "mxfp8_sustained": bf16_s * MXFP8_OVER_BF16,
+                "hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"mxfp8_burst": FALLBACK_BF16_TFLOPS * MXFP8_OVER_BF16,
+                "mxfp8_sustained": 1400.0 * MXFP8_OVER_BF16, "hbm_gbs": FALLBACK_HBM_GBS,
+                "source": "fallback"}
+
+
+def gemm_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(cfg_name: str):
+    """DRAM bytes per gate_up launch from the committed ncu summary, or None
+    when the summary is missing, for another workload, or the kernel source
+    changed since it was captured."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"traffic_bytes_per_launch_full:\s*([0-9.eE+]+)", text)
+    m_w = re.search(r"workload:\s*(\S+)", text)
+    if not (m_sha and m_b and m_w) or m_w.group(1) != cfg_name:
+        return None
+    if m_sha.group(1) != gemm_source_sha():
+        return None
+    return float(m_b.group(1))
+
+
+def parse_clocks(csv_text: str, t0: float, t1: float):
+    """nvidia-smi samples (timestamp, index, clocks.sm, clocks.max.sm,
+    power, reasons...) -> summary over the samples inside [t0, t1] (the
+    nearest ones if none fell inside)."""
+    rows = []
+    for line in csv_text.strip().splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9 or not parts[2].replace(" MHz", "").isdigit():
+            continue
+        try:
+            ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            continue
+        rows.append((ts, int(parts[2].split()[0]), int(parts[3].split()[0]), parts[5:9]))
+    if not rows:
+        return None
+    inside = [r for r in rows if t0 - 0.25 <= r[0] <= t1 + 0.25]
+    if not inside:
+        mid = 0.5 * (t0 + t1)
+        inside = sorted(rows, key=lambda r: abs(r[0] - mid))[:3]
+    mhz = sorted(r[1] for r in inside)
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v.lower() == "active"})
+    return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": max(r[2] for r in inside),
+            "reasons": reasons, "samples": len(inside)}
+
+
+class ClockSampler:
+    """Background nvidia-smi sampler (200 ms) for one GPU index."""
+
+    def __init__(self, index: int):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader",
+                                          "-i", str(index), "-lms", "200"], stdout=self.file,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> str:
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        text = self.file.read()
+        self.file.close()
+        os.unlink(self.file.name)
+        return text
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(cfg, rows: int, seed: int, i_div: int = 1):
+    """One bounded sample of the workload for the CPU oracle: `rows` routed
+    rows of one expert and a 1/i_div slice of that expert's intermediate
+    dimension (gate, up and down weights of those I/i_div channels; their
+    weight quantisation in both directions included), forward + backward.
+    Every element of the sample goes through the same arithmetic as in the
+    full layer; the work scales linearly in rows and I.  Returns (seconds,
+    algorithmic FLOPs of the sample, description)."""
+    import numpy as np
+    from oracle import moe as omoe
+    rng = np.random.default_rng(seed)
+    H, I = cfg.H, cfg.I // i_div
+    x = rng.standard_normal((rows, H)).astype(np.float32).astype(np.float64)
+    w1 = (rng.standard_normal((1, 2 * I, H)).astype(np.float32) / np.sqrt(H)).astype(np.float64)
+    w2 = (rng.standard_normal((1, H, I)).astype(np.float32) / np.sqrt(I)).astype(np.float64)
+    dy = rng.standard_normal((rows, H)).astype(np.float32).astype(np.float64)
+    idx = np.zeros((rows, 1), np.int32)
+    prob = rng.uniform(0.2, 0.8, (rows, 1)).astype(np.float32)
+    t = time.perf_counter()
+    f = omoe.forward(x, w1, w2, idx, prob)
+    omoe.backward(f, x, w1, w2, prob, dy)
+    dt = time.perf_counter() - t
+    flops = 18.0 * rows * H * I
+    desc = (f"{rows} routed rows of one expert of {cfg.name}, H={H}, a 1/{i_div} slice of I "
+            f"({I} of {cfg.I} channels) with those weights; their MXFP8 quantisation in both "
+            f"directions included; fwd+bwd; float64 numpy")
+    return dt, flops, desc
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle as it stands, timed on the host
+    cores on bounded samples of the same workload.  Under torchrun only
+    rank 0 runs it."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    cfg = get_config(args.config)
+    rows, i_div = 64, 16
+    for _ in range(args.warmup):
+        oracle_sample(cfg, rows, args.seed, i_div)
+    tot_t = tot_f = 0.0
+    desc = ""
+    for s in range(args.steps):
+        dt, fl, desc = oracle_sample(cfg, rows, args.seed + s, i_div)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
+                       "sample_rows_per_step": rows, "sample_i_fraction": f"1/{i_div}"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def make_device_inputs(torch, cfg, seed: int, dev):
+    """Seeded synthetic inputs drawn on the device with the recipe of
+    mxfp8_grouped_gemm_x32_b200.workloads (bf16 normals, N(0, 1/fan_in)
+    weights, softmax/top-k routing renormalised)."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
+    x = torch.randn(T, H, generator=g, device=dev).to(torch.bfloat16)
+    w1 = (torch.randn(E, 2 * I, H, generator=g, device=dev) / H ** 0.5).to(torch.bfloat16)
+    w2 = (torch.randn(E, H, I, generator=g, device=dev) / I ** 0.5).to(torch.bfloat16)
+    dy = torch.randn(T, H, generator=g, device=dev).to(torch.bfloat16)
+    logits = torch.randn(T, E, generator=g, device=dev, dtype=torch.float64)
+    if cfg.expert_bias_std:
+        logits = logits + cfg.expert_bias_std * torch.randn(E, generator=g, device=dev, dtype=torch.float64)
+    if cfg.router == "topk_softmax":
+        top, idx = torch.topk(logits, k, dim=1)
+        prob = torch.softmax(top, dim=1)
+    else:
+        p = torch.softmax(logits, dim=1)
+        prob, idx = torch.topk(p, k, dim=1)
+        prob = prob / prob.sum(dim=1, keepdim=True)
+    return x, idx.to(torch.int32).contiguous(), prob.to(torch.float32).contiguous(), w1, w2, dy
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    from mxfp8_grouped_gemm_x32_b200.layer import GroupedMLP
+
+    cfg = get_config(args.config)
+    x, idx, prob, w1, w2, dy = make_device_inputs(torch, cfg, args.seed + rank, dev)
+    layer = GroupedMLP(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def step():
+        layer.step(x, idx, prob, w1, w2, dy)
+
+    for _ in range(args.warmup):
+        step()
+    st = layer.device_status()
+    if st != 0:
+        raise SystemExit(f"device status after warm-up: {lib.status_string(st)}")
+
+    # ---- timed region: K steps, inputs resident in HBM --------------------
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    lib.moe_timing_enable(True)
+    lib.moe_timing_read()
+    barrier()
+    launches0 = lib.moe_launch_count()
+    t_wall0 = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    t_wall1 = time.time()
+    launches = lib.moe_launch_count() - launches0
+    per_kernel = lib.moe_timing_read()
+    lib.moe_timing_enable(False)
+    time.sleep(0.3)
+    clocks = parse_clocks(sampler.stop(), t_wall0, t_wall1)
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    flops = step_flops(cfg)
+    value = world * flops / (ms_max * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers --------------
+    hx = x.cpu().pin_memory()
+    hidx = idx.cpu().pin_memory()
+    hprob = prob.cpu().pin_memory()
+    hdy = dy.cpu().pin_memory()
+    hout = torch.empty_like(layer.out, device="cpu").pin_memory()
+    hdx = torch.empty_like(layer.dX, device="cpu").pin_memory()
+    hdp = torch.empty_like(layer.dprob, device="cpu").pin_memory()
+    dx_in, didx, dprob_in, ddy = (torch.empty_like(t) for t in (x, idx, prob, dy))
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hidx, hprob, hdy))
+    d2h = sum(t.numel() * t.element_size() for t in (hout, hdx, hdp))
+
+    def e2e_step():
+        dx_in.copy_(hx, non_blocking=True)
+        didx.copy_(hidx, non_blocking=True)
+        dprob_in.copy_(hprob, non_blocking=True)
+        ddy.copy_(hdy, non_blocking=True)
+        layer.step(dx_in, didx, dprob_in, w1, w2, ddy)
+        hout.copy_(layer.out, non_blocking=True)
+        hdx.copy_(layer.dX, non_blocking=True)
+        hdp.copy_(layer.dprob, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    ms_e2e = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    value_e2e = world * flops / (ms_e2e * 1e-3) / 1e12
+    st = layer.device_status()
+    if st != 0:
+        raise SystemExit(f"device status after timing: {lib.status_string(st)}")
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks = load_peaks()
+    kernels = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
+               for k, v in per_kernel.items()}
+    g1 = per_kernel.get("gemm_gate_up_swiglu")
+    roofline = None
+    if g1 and g1[1]:
+        t_launch = g1[0] / g1[1] * 1e-3
+        achieved = gate_up_flops(cfg) / t_launch / 1e12
+        peak = peaks["mxfp8_sustained"]
+        roofline = {"bound": "tensor", "kernel": "gemm_gate_up_swiglu", "achieved": achieved,
+                    "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                    "traffic": profiled_traffic(cfg.name),
+                    "peak_source": f"{peaks['source']} bf16 sustained x {MXFP8_OVER_BF16} (nominal MXFP8/BF16)",
+                    "frac_of_burst": achieved / peaks["mxfp8_burst"]}
+    fwd_ms = sum(kernels[k]["ms_per_step"] for k in ("gemm_gate_up_swiglu", "gemm_down", "combine")
+                 if k in kernels)
+    bwd_keys = ("dy_quant_rows", "dy_quant_cols", "gemm_dgrad_down", "swiglu_bwd", "gemm_wgrad_down",
+                "gemm_dgrad_gate_up", "combine_dx", "gemm_wgrad_gate_up")
+    bwd_ms = sum(kernels[k]["ms_per_step"] for k in bwd_keys if k in kernels)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "mxfp8 (e4m3 x e4m3, e8m0 block scales, fp32 accumulate)",
+        "data": "synthetic (seeded, drawn on device; bf16 N(0,1) tokens, N(0,1/fan_in) weights, "
+                "softmax top-k routing)",
+        "config": {"workload": f"{cfg.name} expert layer fwd+bwd", "T": cfg.T, "H": cfg.H, "I": cfg.I,
+                   "E": cfg.E, "k": cfg.k, "R": cfg.R, "parallelism": f"replicas x{world} (data-parallel tokens)",
+                   "l2": "inputs larger than L2 (bf16 weights 2.8 GB re-read each step)",
+                   "step": "weight quant (both directions) + permute + fwd + bwd",
+                   "flops_per_step": flops},
+        "frac_of_mxfp8_peak": value / world / peaks["mxfp8_sustained"],
+        "fwd_tflops": cfg.fwd_flops() / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,
+        "bwd_tflops": cfg.bwd_flops() / (bwd_ms * 1e-3) / 1e12 if bwd_ms else None,
+        "kernels": kernels,
+        "roofline": roofline,
+        "clocks": clocks,
+        "e2e": {"value": value_e2e, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": ms_e2e},
+        "gpu_launches": launches,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        dt, fl, desc = oracle_sample(cfg, 256, args.seed, 4)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
+                                "kind": "oracle", "sample": desc, "seconds": dt}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

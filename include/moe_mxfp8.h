@@ -225,6 +225,18 @@ const char* moe_status_string(moe_status_t status);
  * the last reset (host-side counter; for launch accounting in benchmarks). */
 int64_t moe_launch_count(int32_t reset);
 
+/* Per-kernel timing.  While enabled, every kernel launch of the library is
+ * bracketed by two CUDA events recorded on its stream (host-created events,
+ * no device memory).  moe_timing_enable returns the previous state.
+ * moe_timing_read synchronises on the recorded events, aggregates them by
+ * kernel tag in order of first launch, writes up to max_entries totals (ms)
+ * and launch counts, the tags as '\n'-separated text into `names` (host,
+ * NUL-terminated, truncated to names_len), clears the record and returns
+ * the number of tags. */
+int32_t moe_timing_enable(int32_t on);
+int32_t moe_timing_read(char* names, int64_t names_len, double* ms, int64_t* count,
+                        int32_t max_entries);
+
 /* Self-test of the bounded-wait machinery: launches one CTA that waits on a
  * pipeline barrier nobody arrives on, with a limit of about `wait_ms`
  * milliseconds; the kernel gives up, records MOE_ERR_TIMEOUT and exits

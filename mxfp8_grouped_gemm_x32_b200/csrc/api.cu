@@ -1,6 +1,10 @@
 // C ABI of the grouped MXFP8 MoE expert MLP (declared in include/moe_mxfp8.h):
 // argument checks, workspace carving and the launch sequence of each call.
 #include <atomic>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
 
 #include "gemm.cuh"
 #include "permute.cuh"
@@ -11,6 +15,41 @@ namespace moe {
 
 static std::atomic<int64_t> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+namespace {
+struct TimingRec {
+  const char* tag;
+  cudaEvent_t a, b;
+};
+std::mutex g_tmu;
+bool g_timing = false;
+std::vector<TimingRec> g_recs;
+std::vector<cudaEvent_t> g_pool;
+cudaEvent_t pool_take() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace
+
+void timing_begin(cudaStream_t st, const char* tag) {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  if (!g_timing) return;
+  TimingRec r{tag, pool_take(), pool_take()};
+  cudaEventRecord(r.a, st);
+  g_recs.push_back(r);
+}
+
+void timing_end(cudaStream_t st) {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  if (!g_timing || g_recs.empty()) return;
+  cudaEventRecord(g_recs.back().b, st);
+}
 
 namespace {
 
@@ -137,11 +176,13 @@ moe_status_t moe_mlp_quantize_mxfp8(const void* src, int32_t groups, int64_t row
   if (mode == MOE_QUANT_ROW) {
     if (cols % 32) return MOE_ERR_UNSUPPORTED;
     QuantRowsArgs a{static_cast<const uint8_t*>(src), cols, nullptr, 1, groups, rows, cols, q, sf};
+    TimeScope ts(st, "quant_rows");
     return cuda_status(launch_quant_rows(a, st));
   }
   if (mode == MOE_QUANT_COL) {
     if (rows % 32 || cols % 8) return MOE_ERR_UNSUPPORTED;
     QuantColsArgs a{static_cast<const uint8_t*>(src), cols, nullptr, 1, groups, rows, cols, q, sf};
+    TimeScope ts(st, "quant_cols");
     return cuda_status(launch_quant_cols(a, st));
   }
   return MOE_ERR_INVALID;
@@ -167,13 +208,21 @@ moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* to
   if (!device_ok()) return MOE_ERR_NO_DEVICE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t R = int64_t(T) * k;
-  cudaError_t e = launch_permute_index(topk_idx, topk_prob, R, E, rows_cap, split_sizes, group_offsets,
-                                       row_to_slot, slot_to_row, prob_perm, workspace, st);
+  cudaError_t e;
+  {
+    TimeScope ts(st, "permute_index");
+    e = launch_permute_index(topk_idx, topk_prob, R, E, rows_cap, split_sizes, group_offsets,
+                             row_to_slot, slot_to_row, prob_perm, workspace, st);
+  }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq, xq_sf};
-  if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    TimeScope ts(st, "permute_quant_rows");
+    if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
   if (xq_col) {
     QuantColsArgs qc{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq_col, xq_col_sf};
+    TimeScope ts(st, "permute_quant_cols");
     if ((e = launch_quant_cols(qc, st)) != cudaSuccess) return MOE_ERR_CUDA;
   }
   return MOE_OK;
@@ -183,7 +232,9 @@ moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* o
   if (!y || !out || T < 0 || k <= 0 || H <= 0 || H % 8) return MOE_ERR_INVALID;
   if (!al16(y) || !al16(out)) return MOE_ERR_INVALID;
   if (!device_ok()) return MOE_ERR_NO_DEVICE;
-  return cuda_status(launch_combine(y, false, T, k, H, out, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  TimeScope ts(st, "combine");
+  return cuda_status(launch_combine(y, false, T, k, H, out, st));
 }
 
 moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const uint8_t* w2q,
@@ -224,7 +275,10 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   g1.prob = prob_perm; g1.row_to_slot = row_to_slot;
   g1.out2 = static_cast<uint8_t*>(saved_a);
   g1.q_out = w.hq; g1.sf_out = w.hq_sf; g1.q_KT = int32_t(cdiv(I, 128));
-  if ((e = launch_grouped_gemm(EPI_SWIGLU, m1, g1, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    TimeScope ts(st, "gemm_gate_up_swiglu");
+    if ((e = launch_grouped_gemm(EPI_SWIGLU, m1, g1, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
 
   // down grouped GEMM, rows scattered to slot order
   GemmMaps m2;
@@ -236,9 +290,13 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   g2.sfa = w.hq_sf; g2.a_KT = int32_t(cdiv(I, 128));
   g2.sfb = w2sf; g2.b_RT = int32_t(cdiv(H, 128)); g2.b_KT = int32_t(cdiv(I, 128));
   g2.row_to_slot = row_to_slot; g2.out = w.y; g2.ld_out = H;
-  if ((e = launch_grouped_gemm(EPI_F32_SCATTER, m2, g2, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    TimeScope ts(st, "gemm_down");
+    if ((e = launch_grouped_gemm(EPI_F32_SCATTER, m2, g2, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
 
   // top-k combine back to token order
+  TimeScope ts(st, "combine");
   return cuda_status(launch_combine(w.y, true, T, k, H, out, st));
 }
 
@@ -269,9 +327,15 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
 
   // dy rows gathered to permuted order, quantised along H and along tokens
   QuantRowsArgs qr{static_cast<const uint8_t*>(dY), H, row_to_slot, k, 1, rows_cap, H, w.dyq, w.dyq_sf};
-  if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    TimeScope ts(st, "dy_quant_rows");
+    if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
   QuantColsArgs qc{static_cast<const uint8_t*>(dY), H, row_to_slot, k, 1, rows_cap, H, w.dyc, w.dyc_sf};
-  if ((e = launch_quant_cols(qc, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    TimeScope ts(st, "dy_quant_cols");
+    if ((e = launch_quant_cols(qc, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
 
   // dgrad2: dh = dy W_down (contraction over H)
   GemmMaps m;
@@ -283,13 +347,19 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   g.sfa = w.dyq_sf; g.a_KT = int32_t(cdiv(H, 128));
   g.sfb = w2tsf; g.b_RT = int32_t(cdiv(I, 128)); g.b_KT = int32_t(cdiv(H, 128));
   g.out = w.dh; g.ld_out = I;
-  if (launch_grouped_gemm(EPI_F32_ROWS, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    TimeScope ts(st, "gemm_dgrad_down");
+    if (launch_grouped_gemm(EPI_F32_ROWS, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
 
   // ScaledSwiGLU backward + quantisation of da (both ways) and h (along tokens)
   SwigluBwdArgs sb{I, E, rows_cap, group_offsets, row_to_slot, prob_perm, w.dh,
                    static_cast<const uint8_t*>(saved_a), w.daq, w.daq_sf, w.dac, w.dac_sf, w.hc, w.hc_sf,
                    dprob};
-  if (launch_swiglu_bwd(sb, st) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    TimeScope ts(st, "swiglu_bwd");
+    if (launch_swiglu_bwd(sb, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
 
   // wgrad2: dW_down_e = dy_e^T h_e (contraction over the group's tokens)
   if (make_map_2d(&m.a, w.dyc, rows_cap, H, 128) != cudaSuccess) return MOE_ERR_CUDA;
@@ -301,7 +371,10 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   g.sfa = w.dyc_sf; g.a_KT = int32_t(rows_cap / 128);
   g.sfb = w.hc_sf; g.b_RT = int32_t(cdiv(I, 128)); g.b_KT = int32_t(rows_cap / 128);
   g.out = static_cast<uint8_t*>(dW2); g.ld_out = I; g.out_group_stride = int64_t(H) * I;
-  if (launch_grouped_gemm(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    TimeScope ts(st, "gemm_wgrad_down");
+    if (launch_grouped_gemm(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
 
   // dgrad1: dx = da W_gate_up (contraction over 2I), rows scattered to slots
   if (make_map_2d(&m.a, w.daq, 2 * int64_t(I), rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
@@ -313,8 +386,14 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   g.sfa = w.daq_sf; g.a_KT = int32_t(cdiv(2 * int64_t(I), 128));
   g.sfb = w1tsf; g.b_RT = int32_t(cdiv(H, 128)); g.b_KT = int32_t(cdiv(2 * int64_t(I), 128));
   g.row_to_slot = row_to_slot; g.out = w.dx; g.ld_out = H;
-  if (launch_grouped_gemm(EPI_F32_SCATTER, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_combine(w.dx, true, T, k, H, dX, st) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    TimeScope ts(st, "gemm_dgrad_gate_up");
+    if (launch_grouped_gemm(EPI_F32_SCATTER, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  {
+    TimeScope ts(st, "combine_dx");
+    if (launch_combine(w.dx, true, T, k, H, dX, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
 
   // wgrad1: dW_gate_up_e = da_e^T x_e (contraction over the group's tokens)
   if (make_map_2d(&m.a, w.dac, rows_cap, 2 * int64_t(I), 128) != cudaSuccess) return MOE_ERR_CUDA;
@@ -326,7 +405,10 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   g.sfa = w.dac_sf; g.a_KT = int32_t(rows_cap / 128);
   g.sfb = xq_col_sf; g.b_RT = int32_t(cdiv(H, 128)); g.b_KT = int32_t(rows_cap / 128);
   g.out = static_cast<uint8_t*>(dW1); g.ld_out = H; g.out_group_stride = 2 * int64_t(I) * H;
-  if (launch_grouped_gemm(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    TimeScope ts(st, "gemm_wgrad_gate_up");
+    if (launch_grouped_gemm(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
   (void)slot_to_row;
   return MOE_OK;
 }
@@ -351,6 +433,53 @@ const char* moe_status_string(moe_status_t s) {
     case MOE_ERR_NO_DEVICE: return "no sm_100 CUDA device current";
   }
   return "unknown status";
+}
+
+int32_t moe_timing_enable(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  const int32_t prev = g_timing ? 1 : 0;
+  g_timing = on != 0;
+  return prev;
+}
+
+int32_t moe_timing_read(char* names, int64_t names_len, double* ms, int64_t* count, int32_t max_entries) {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  std::vector<std::string> tags;
+  std::vector<double> tot;
+  std::vector<int64_t> cnt;
+  for (const TimingRec& r : g_recs) {
+    float t = 0.0f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
+      t = -1.0f;
+      cudaGetLastError();
+    }
+    size_t i = 0;
+    while (i < tags.size() && tags[i] != r.tag) ++i;
+    if (i == tags.size()) {
+      tags.emplace_back(r.tag);
+      tot.push_back(0.0);
+      cnt.push_back(0);
+    }
+    tot[i] += t;
+    cnt[i] += 1;
+    g_pool.push_back(r.a);
+    g_pool.push_back(r.b);
+  }
+  g_recs.clear();
+  const int32_t n = int32_t(tags.size()) < max_entries ? int32_t(tags.size()) : max_entries;
+  std::string joined;
+  for (int32_t i = 0; i < n; ++i) {
+    if (ms) ms[i] = tot[i];
+    if (count) count[i] = cnt[i];
+    joined += tags[i];
+    joined += '\n';
+  }
+  if (names && names_len > 0) {
+    const size_t m = joined.size() < size_t(names_len - 1) ? joined.size() : size_t(names_len - 1);
+    std::memcpy(names, joined.data(), m);
+    names[m] = 0;
+  }
+  return n;
 }
 
 int64_t moe_launch_count(int32_t reset) {

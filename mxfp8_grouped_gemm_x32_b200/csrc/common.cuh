@@ -23,6 +23,16 @@ __device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, c
 
 void count_launch(int n = 1);
 
+// Optional per-kernel timing (moe_timing_enable): CUDA events recorded on
+// the launching stream around each tagged launch, aggregated by tag on read.
+void timing_begin(cudaStream_t st, const char* tag);
+void timing_end(cudaStream_t st);
+struct TimeScope {
+  cudaStream_t st;
+  TimeScope(cudaStream_t s, const char* tag) : st(s) { timing_begin(s, tag); }
+  ~TimeScope() { timing_end(st); }
+};
+
 // ----------------------------------------------------------------------------
 // MXFP8 encoding
 // ----------------------------------------------------------------------------

@@ -31,6 +31,7 @@ EXPORTED = [
     "moe_mx_scale_bytes", "moe_padded_rows", "moe_workspace_size", "moe_mlp_quantize_mxfp8",
     "moe_permute", "moe_grouped_mlp_fwd", "moe_combine", "moe_grouped_mlp_bwd",
     "moe_get_device_status", "moe_status_string", "moe_launch_count", "moe_selftest_wait_timeout",
+    "moe_timing_enable", "moe_timing_read",
 ]
 
 
@@ -73,6 +74,9 @@ _decl("moe_get_device_status", _I32, _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
 _decl("moe_launch_count", _I64, _I32)
 _decl("moe_selftest_wait_timeout", _I32, _I32, _P)
+_decl("moe_timing_enable", _I32, _I32)
+_decl("moe_timing_read", _I32, ctypes.c_char_p, _I64, ctypes.POINTER(ctypes.c_double),
+      ctypes.POINTER(_I64), _I32)
 
 
 def _check(fn: str, code: int) -> None:
@@ -138,3 +142,17 @@ def moe_launch_count(reset: bool = False) -> int:
 
 def moe_selftest_wait_timeout(wait_ms: int, stream=0) -> int:
     return _lib.moe_selftest_wait_timeout(wait_ms, stream)
+
+
+def moe_timing_enable(on: bool) -> bool:
+    return bool(_lib.moe_timing_enable(1 if on else 0))
+
+
+def moe_timing_read(max_entries: int = 64) -> dict:
+    """{kernel tag: (total ms, launches)} since the last read."""
+    buf = ctypes.create_string_buffer(8192)
+    ms = (ctypes.c_double * max_entries)()
+    cnt = (_I64 * max_entries)()
+    n = _lib.moe_timing_read(buf, len(buf), ms, cnt, max_entries)
+    names = buf.value.decode().split("\n")[:n]
+    return {names[i]: (ms[i], int(cnt[i])) for i in range(n)}
