@@ -66,7 +66,8 @@ typedef enum {
   MOE_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
   MOE_ERR_DEVICE_INDEX = 5, /* device: an expert id outside [0, E) */
   MOE_ERR_TIMEOUT = 6,      /* device: a bounded pipeline wait ran out */
-  MOE_ERR_NO_DEVICE = 7     /* no sm_100 device current */
+  MOE_ERR_NO_DEVICE = 7,    /* no sm_100 device current */
+  MOE_ERR_TOO_LARGE = 8     /* needs more scratch than moe_permute_noalloc's built-in array */
 } moe_status_t;
 
 /* Quantisation modes of moe_mlp_quantize_mxfp8. */
@@ -147,6 +148,30 @@ moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* to
                          int32_t* slot_to_row, float* prob_perm, uint8_t* xq, uint8_t* xq_sf,
                          uint8_t* xq_col, uint8_t* xq_col_sf, void* workspace, size_t workspace_bytes,
                          moe_stream_t stream);
+
+/* No-allocation variant of moe_permute.  The paper has no counterpart: this
+ * exists for callers that cannot provide device scratch memory -- their
+ * device memory is planned up front by another component (a runtime with a
+ * fixed memory plan, or host code with no device allocator of its own) -- so
+ * they cannot pass the workspace moe_permute needs.  Arguments, outputs and
+ * errors are those of moe_permute without `workspace`; the results are
+ * identical.  The scratch (per-block expert histograms,
+ * ceil(T*k/1024)*E*4 + 256 bytes) lives in a file-scope device array of
+ * MOE_PERMUTE_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
+ * library holds until the process exits; larger problems are rejected with
+ * MOE_ERR_TOO_LARGE before anything is launched.  Nothing is allocated: no
+ * cudaMalloc, no cudaFree, no allocating library routine.  The first call on
+ * a device looks up the array's device address (cudaGetSymbolAddress, once
+ * per device, with that device current); make that first call before any
+ * stream capture.  All calls share the one array: calls whose kernels
+ * overlap on the GPU (different streams or host threads) race and must be
+ * serialised by the caller. */
+#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (256 * 1024)
+moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_idx, const float* topk_prob,
+                                 int32_t T, int32_t H, int32_t k, int32_t E, int64_t rows_cap,
+                                 int32_t* split_sizes, int32_t* group_offsets, int32_t* row_to_slot,
+                                 int32_t* slot_to_row, float* prob_perm, uint8_t* xq, uint8_t* xq_sf,
+                                 uint8_t* xq_col, uint8_t* xq_col_sf, moe_stream_t stream);
 
 /* ------------------------------------------------------------ forward --- */
 

@@ -431,6 +431,7 @@ const char* moe_status_string(moe_status_t s) {
     case MOE_ERR_DEVICE_INDEX: return "device: expert id out of range";
     case MOE_ERR_TIMEOUT: return "device: bounded pipeline wait timed out";
     case MOE_ERR_NO_DEVICE: return "no sm_100 CUDA device current";
+    case MOE_ERR_TOO_LARGE: return "problem needs more scratch than the no-allocation entry point's built-in array";
   }
   return "unknown status";
 }

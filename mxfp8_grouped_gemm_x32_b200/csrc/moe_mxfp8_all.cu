@@ -5,3 +5,4 @@
 #include "permute.cu"
 #include "quant.cu"
 #include "swiglu_bwd.cu"
+#include "noalloc.cu"

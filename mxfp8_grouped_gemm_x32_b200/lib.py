@@ -25,13 +25,15 @@ MOE_MAX_EXPERTS = 256
 STATUS = {
     0: "MOE_OK", 1: "MOE_ERR_INVALID", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
     4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_INDEX", 6: "MOE_ERR_TIMEOUT", 7: "MOE_ERR_NO_DEVICE",
+    8: "MOE_ERR_TOO_LARGE",
 }
+MOE_PERMUTE_NOALLOC_SCRATCH_BYTES = 256 * 1024
 
 EXPORTED = [
     "moe_mx_scale_bytes", "moe_padded_rows", "moe_workspace_size", "moe_mlp_quantize_mxfp8",
     "moe_permute", "moe_grouped_mlp_fwd", "moe_combine", "moe_grouped_mlp_bwd",
     "moe_get_device_status", "moe_status_string", "moe_launch_count", "moe_selftest_wait_timeout",
-    "moe_timing_enable", "moe_timing_read",
+    "moe_timing_enable", "moe_timing_read", "moe_permute_noalloc",
 ]
 
 
@@ -74,6 +76,8 @@ _decl("moe_get_device_status", _I32, _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
 _decl("moe_launch_count", _I64, _I32)
 _decl("moe_selftest_wait_timeout", _I32, _I32, _P)
+_decl("moe_permute_noalloc", _I32, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P,
+      _P, _P, _P, _P)
 _decl("moe_timing_enable", _I32, _I32)
 _decl("moe_timing_read", _I32, ctypes.c_char_p, _I64, ctypes.POINTER(ctypes.c_double),
       ctypes.POINTER(_I64), _I32)
@@ -109,6 +113,15 @@ def moe_permute(x, topk_idx, topk_prob, T, H, k, E, rows_cap, split_sizes, group
     _check("moe_permute", _lib.moe_permute(x, topk_idx, topk_prob, T, H, k, E, rows_cap, split_sizes,
                                            group_offsets, row_to_slot, slot_to_row, prob_perm, xq, xq_sf,
                                            xq_col, xq_col_sf, workspace, workspace_bytes, stream))
+
+
+def moe_permute_noalloc(x, topk_idx, topk_prob, T, H, k, E, rows_cap, split_sizes, group_offsets,
+                        row_to_slot, slot_to_row, prob_perm, xq, xq_sf, xq_col, xq_col_sf, stream=0):
+    """moe_permute for callers that cannot provide a device workspace: the
+    scratch lives in the library's built-in device array (see the header)."""
+    _check("moe_permute_noalloc", _lib.moe_permute_noalloc(
+        x, topk_idx, topk_prob, T, H, k, E, rows_cap, split_sizes, group_offsets, row_to_slot,
+        slot_to_row, prob_perm, xq, xq_sf, xq_col, xq_col_sf, stream))
 
 
 def moe_grouped_mlp_fwd(w1q, w1sf, w2q, w2sf, T, H, I, E, k, rows_cap, split_sizes, group_offsets,
