@@ -69,6 +69,10 @@ CONFIGS = {
                         note="T512 H256 I512 E4 top2"),
     "mixtral_8x7b": LayerConfig("mixtral_8x7b", T=8192, H=4096, I=14336, E=8, k=2,
                                 note="Mixtral-8x7B expert layer, 2x4096 tokens"),
+    # Mixtral expert shapes with 2 of the 8 experts and the same 2048 rows per
+    # expert: a profiler-sized slice of the Mixtral layer
+    "mixtral_profile": LayerConfig("mixtral_profile", T=4096, H=4096, I=14336, E=2, k=1,
+                                   note="Mixtral-8x7B expert shapes, 2 experts x 2048 rows"),
     "qwen3_30b_ragged": LayerConfig("qwen3_30b_ragged", T=16384, H=2048, I=768, E=128, k=8,
                                     expert_bias_std=1.5,
                                     note="Qwen3-MoE-30B-shaped, skewed routing"),
