@@ -67,6 +67,18 @@ def gate_up_flops(cfg) -> float:
     return 4.0 * cfg.R * cfg.H * cfg.I
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over the process group (the step time of a
+    multi-GPU run is the slowest rank's)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks(path=os.path.join(ROOT, "MEASURED_PEAKS.json")):
     """Dense MXFP8 peak (TFLOP/s) and HBM (GB/s) with the source named."""
     try:
@@ -320,12 +332,7 @@ def run_ours(args):
     lib.moe_timing_enable(False)
     time.sleep(0.3)
     clocks = parse_clocks(sampler.stop(), t_wall0, t_wall1)
-    ms = e0.elapsed_time(e1) / args.steps
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     flops = step_flops(cfg)
     value = world * flops / (ms_max * 1e-3) / 1e12
 
@@ -359,11 +366,7 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     barrier()
-    ms_e2e = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     value_e2e = world * flops / (ms_e2e * 1e-3) / 1e12
     st = layer.device_status()
     if st != 0:

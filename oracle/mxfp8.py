@@ -47,25 +47,26 @@ def e4m3_decode(codes: np.ndarray) -> np.ndarray:
     return E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
 
 
+# Non-negative finite E4M3 values in code order (codes 0x00..0x7E are
+# increasing) and the midpoints between neighbours.
+_POS_VALUES = E4M3_TABLE[:0x7F]
+_MIDPOINTS = 0.5 * (_POS_VALUES[:-1] + _POS_VALUES[1:])
+
+
 def e4m3_encode(v: np.ndarray) -> np.ndarray:
-    """float64 -> E4M3 codes, round-to-nearest-even, saturating at 448.
-    NaN (and infinity, which the scale rule never produces here) -> 0x7F
-    with the sign bit of the input."""
+    """float64 -> E4M3 codes: the nearest finite E4M3 value, ties to the even
+    code (even mantissa), saturating at +-448 (values above 448 round to the
+    largest code).  NaN (and infinity, which the scale rule never produces
+    here) -> 0x7F with the sign bit of the input."""
     v = np.asarray(v, dtype=np.float64)
     a = np.abs(v)
     bad = ~np.isfinite(a)
     a = np.where(bad, 0.0, a)
-    _, ex = np.frexp(a)                      # a = f * 2^ex, f in [0.5, 1)
-    e = np.maximum(ex - 1, -6)               # binade exponent, subnormals share -6
-    step = np.ldexp(1.0, e - 3)              # spacing of 3-bit mantissas
-    q = np.round(a / step) * step            # numpy rounds half to even
-    q = np.minimum(q, E4M3_MAX)
-    _, qx = np.frexp(q)
-    qe = qx - 1
-    normal = q >= 2.0 ** -6
-    biased = np.where(normal, qe + 7, 0)
-    man = np.where(normal, q / np.ldexp(1.0, qe) * 8.0 - 8.0, q / 2.0 ** -9)
-    code = (biased.astype(np.int64) << 3) | np.rint(man).astype(np.int64)
+    # number of midpoints strictly below a = index of the nearest value,
+    # except at an exact midpoint, where it is the lower neighbour
+    code = np.searchsorted(_MIDPOINTS, a, side="left")
+    tie = (code < _MIDPOINTS.size) & (a == _MIDPOINTS[np.minimum(code, _MIDPOINTS.size - 1)])
+    code = code + (tie & (code % 2 == 1))
     code = np.where(bad, CODE_NAN, code)
     code = code | (np.signbit(v).astype(np.int64) << 7)
     return code.astype(np.uint8)

@@ -28,6 +28,16 @@ ACC = 2.0 ** -22
 ACT = 2.0 ** -19
 
 
+def wbound(w: np.ndarray) -> np.ndarray:
+    """Element-wise upper bound on |dequantised MXFP8 weight| without
+    quantising: normal codes are within half a step (2^-4 relative) of |w|;
+    subnormal codes within 2^-10 * 2^s, and 2^s < block amax / 224, so
+    within 2^-17 of the block maximum -- bounded here by 2^-12 of the row
+    maximum."""
+    a = np.abs(np.asarray(w, np.float64))
+    return a * (1.0 + 2.0 ** -4) + 2.0 ** -12 * a.max(axis=-1, keepdims=True)
+
+
 def acc_band(a_deq: np.ndarray, b_deq: np.ndarray) -> np.ndarray:
     """Accumulation error band of a_deq @ b_deq.T (a [M,K], b [N,K])."""
     K = a_deq.shape[1]
@@ -96,8 +106,7 @@ def forward_allowance(f, x, w1, w2, topk_idx):
         if sl.stop == sl.start:
             continue
         xd = omx.roundtrip_rows(x[f["tok"][sl]])
-        w1d = omx.roundtrip_rows(w1[e])
-        bA = acc_band(xd, w1d)
+        bA = acc_band(xd, wbound(w1[e]))
         A = f["A"][sl]
         g, u = A[:, :I], A[:, I:]
         p = f["p"][sl][:, None]
@@ -105,7 +114,7 @@ def forward_allowance(f, x, w1, w2, topk_idx):
         h = p * g * sg * u
         bh = np.abs(p * u * sg * (1 + g * (1 - sg))) * bA[:, :I] + np.abs(p * g * sg) * bA[:, I:] + ACT * np.abs(h)
         Dh = code_ambiguity(h, bh)
-        allow_rows[sl] = Dh @ np.abs(omx.roundtrip_rows(w2[e])).T
+        allow_rows[sl] = Dh @ wbound(w2[e]).T
     return allow_rows[f["slot_row"]].reshape(T, k, -1).sum(axis=1)
 
 
@@ -127,16 +136,14 @@ def backward_allowance(f, b, x, w1, w2, dy, topk_idx):
         p = f["p"][sl][:, None]
         # saved activation: bf16 of A, A known to within its accumulation band
         xd = omx.roundtrip_rows(x[tok])
-        w1d = omx.roundtrip_rows(w1[e])
-        bA = acc_band(xd, w1d)
+        bA = acc_band(xd, wbound(w1[e]))
         lo, hi = bf16_alternatives(f["A"][sl], bA)
         a = f["saved"][sl]
         g, u = a[:, :I], a[:, I:]
         # dh = dy W2 from exact operand codes
         dyd = omx.roundtrip_rows(dy[tok])
-        w2td = omx.roundtrip_rows(w2[e].T)
         dh = b["dh"][sl]
-        bdh = acc_band(dyd, w2td)
+        bdh = acc_band(dyd, wbound(w2[e].T))
 
         def parts(gg, uu, dd):
             sg = omoe.sigmoid(gg)
@@ -160,7 +167,7 @@ def backward_allowance(f, b, x, w1, w2, dy, topk_idx):
         bda = np.concatenate([band[0], band[1]], axis=1)
         # dgrad1: ambiguous row-wise da codes times |W1| (quantised along 2I)
         Dr = code_ambiguity(da, bda)
-        allow_dx[sl] = Dr @ np.abs(omx.roundtrip_rows(w1[e].T)).T
+        allow_dx[sl] = Dr @ wbound(w1[e].T).T
         # wgrad2: |dy| (exact codes) times ambiguous h codes along tokens
         Dh = code_ambiguity_cols(base[2], band[2], [m])[0]
         dyc = omx.roundtrip_cols_grouped(dy[tok], [m])[0]

@@ -1,0 +1,88 @@
+"""Host logic of bench.py (no GPU): FLOP accounting, peaks, provenance of
+the profiled traffic, nvidia-smi clock parsing, and the multi-process path
+-- the max-over-ranks step time under a 2-rank gloo process group on CPU,
+and the reference arm's rank handling."""
+import json
+import os
+import socket
+
+import pytest
+
+import bench
+from mxfp8_grouped_gemm_x32_b200.workloads import get_config
+
+
+def test_step_flops_mixtral():
+    cfg = get_config("mixtral_8x7b")
+    R, H, I = 16384, 4096, 14336
+    assert bench.step_flops(cfg) == 18.0 * R * H * I
+    assert bench.gate_up_flops(cfg) == 2.0 * R * H * 2 * I
+
+
+def test_load_peaks(tmp_path):
+    p = tmp_path / "peaks.json"
+    p.write_text(json.dumps({"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0}))
+    pk = bench.load_peaks(str(p))
+    assert pk["source"] == "measured" and pk["mxfp8_burst"] == 3200.0 and pk["mxfp8_sustained"] == 2800.0
+    fb = bench.load_peaks(str(tmp_path / "missing.json"))
+    assert fb["source"] == "fallback" and fb["mxfp8_burst"] == 2 * 1590.0
+
+
+def test_profiled_traffic_tracks_kernel_source(tmp_path, monkeypatch):
+    sha = bench.gemm_source_sha()
+    f = tmp_path / "summary.md"
+    f.write_text(f"workload: mixtral_8x7b\nsource_sha256_16: {sha}\ntraffic_bytes_per_launch_full: 2.0e9\n")
+    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(f))
+    assert bench.profiled_traffic("mixtral_8x7b") == 2.0e9
+    assert bench.profiled_traffic("gpt_oss_20b") is None
+    f.write_text("workload: mixtral_8x7b\nsource_sha256_16: 0000000000000000\ntraffic_bytes_per_launch_full: 2e9\n")
+    assert bench.profiled_traffic("mixtral_8x7b") is None
+
+
+def test_parse_clocks():
+    csv = ("2026/12/02 16:00:00.000, 0, 1900 MHz, 1965 MHz, 900.00 W, Not Active, Not Active, Not Active, Active\n"
+           "2026/12/02 16:00:00.200, 0, 1950 MHz, 1965 MHz, 950.00 W, Not Active, Not Active, Not Active, Not Active\n"
+           "2026/12/02 16:00:00.400, 0, 1800 MHz, 1965 MHz, 990.00 W, Not Active, Not Active, Not Active, Active\n"
+           "2026/12/02 16:00:05.000, 0, 300 MHz, 1965 MHz, 100.00 W, Not Active, Not Active, Not Active, Not Active\n")
+    import datetime
+    t0 = datetime.datetime(2026, 12, 2, 16, 0, 0).timestamp()
+    c = bench.parse_clocks(csv, t0, t0 + 0.4)
+    assert c["sm_mhz"] == 1900 and c["sm_max_mhz"] == 1965 and c["samples"] == 3
+    assert c["reasons"] == ["sw_power_cap"]
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        v = bench.max_over_ranks(10.0 + 5.0 * rank, world)
+        with open(os.path.join(out_dir, f"r{rank}"), "w") as fh:
+            fh.write(repr(v))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_two_processes(tmp_path):
+    import torch.multiprocessing as mp
+    port = _free_port()
+    mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True, start_method="spawn")
+    vals = [float(open(tmp_path / f"r{r}").read()) for r in range(2)]
+    assert vals == [15.0, 15.0]
+
+
+def test_reference_arm_non_zero_rank_exits_without_output(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_max_over_ranks_single_process():
+    assert bench.max_over_ranks(3.5, 1) == 3.5
