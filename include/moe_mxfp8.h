@@ -120,6 +120,21 @@ int64_t moe_workspace_size(int32_t op, int32_t T, int32_t k, int32_t E, int32_t 
 moe_status_t moe_mlp_quantize_mxfp8(const void* src, int32_t groups, int64_t rows, int64_t cols,
                                     int32_t mode, uint8_t* q, uint8_t* sf, moe_stream_t stream);
 
+/* Both MXFP8 forms of both expert weights from one read of each (the per-step
+ * weight quantisation of Challenge 3: BF16 master weights quantised before
+ * the low-precision GEMMs of the forward and of the backward).  Results are
+ * identical to the four moe_mlp_quantize_mxfp8 calls named in parentheses.
+ *   w_gate_up  bf16 [E][2I][H];  w_down bf16 [E][H][I].
+ *   w1q, w1sf    MX (2E, I, H)   (ROW of w_gate_up, groups=2E rows=I cols=H)
+ *   w2q, w2sf    MX (E, H, I)    (ROW of w_down,    groups=E rows=H cols=I)
+ *   w1tq, w1tsf  MX (E, H, 2I)   (COL of w_gate_up, groups=E rows=2I cols=H)
+ *   w2tq, w2tsf  MX (E, I, H)    (COL of w_down,    groups=E rows=H cols=I)
+ * Needs H % 32 == 0, I % 64 == 0; all pointers 16-byte aligned. */
+moe_status_t moe_mlp_quantize_weights(const void* w_gate_up, const void* w_down, int32_t E, int32_t H,
+                                      int32_t I, uint8_t* w1q, uint8_t* w1sf, uint8_t* w2q, uint8_t* w2sf,
+                                      uint8_t* w1tq, uint8_t* w1tsf, uint8_t* w2tq, uint8_t* w2tsf,
+                                      moe_stream_t stream);
+
 /* ------------------------------------------------------------ permute --- */
 
 /* Group routed tokens by expert and quantise them (Challenge 1:

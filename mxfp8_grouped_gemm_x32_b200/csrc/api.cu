@@ -188,6 +188,24 @@ moe_status_t moe_mlp_quantize_mxfp8(const void* src, int32_t groups, int64_t row
   return MOE_ERR_INVALID;
 }
 
+moe_status_t moe_mlp_quantize_weights(const void* w_gate_up, const void* w_down, int32_t E, int32_t H,
+                                      int32_t I, uint8_t* w1q, uint8_t* w1sf, uint8_t* w2q, uint8_t* w2sf,
+                                      uint8_t* w1tq, uint8_t* w1tsf, uint8_t* w2tq, uint8_t* w2tsf,
+                                      moe_stream_t stream) {
+  const void* ptrs[] = {w_gate_up, w_down, w1q, w1sf, w2q, w2sf, w1tq, w1tsf, w2tq, w2tsf};
+  for (const void* p : ptrs)
+    if (!p || !al16(p)) return MOE_ERR_INVALID;
+  if (E <= 0 || H <= 0 || I <= 0) return MOE_ERR_INVALID;
+  if (H % 32 || I % 64) return MOE_ERR_UNSUPPORTED;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  QuantBothArgs a1{static_cast<const uint8_t*>(w_gate_up), E, 2 * int64_t(I), H, I, w1q, w1sf, w1tq, w1tsf};
+  QuantBothArgs a2{static_cast<const uint8_t*>(w_down), E, H, I, H, w2q, w2sf, w2tq, w2tsf};
+  TimeScope ts(st, "quant_weights");
+  if (launch_quant_both(a1, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(launch_quant_both(a2, st));
+}
+
 moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* topk_prob, int32_t T,
                          int32_t H, int32_t k, int32_t E, int64_t rows_cap, int32_t* split_sizes,
                          int32_t* group_offsets, int32_t* row_to_slot, int32_t* slot_to_row,

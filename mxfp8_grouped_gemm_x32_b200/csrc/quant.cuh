@@ -34,3 +34,26 @@ cudaError_t launch_quant_rows(const QuantRowsArgs& a, cudaStream_t st);
 cudaError_t launch_quant_cols(const QuantColsArgs& a, cudaStream_t st);
 
 }  // namespace moe
+
+namespace moe {
+
+// Both modes from one read of the source: input [groups][rows][cols] bf16.
+//  row mode output: MX tensor whose groups split each input group into
+//    rows / row_split row-groups of row_split rows (W_gate_up: gate and up
+//    halves) -- q_row [groups*rows][cols], sf_row blocked
+//    (groups*rows/row_split, row_split, cols);
+//  column mode output: q_col [groups][cols][rows], sf_col blocked
+//    (groups, cols, rows).
+struct QuantBothArgs {
+  const uint8_t* src;
+  int32_t groups;
+  int64_t rows, cols, row_split;
+  uint8_t* q_row;
+  uint8_t* sf_row;
+  uint8_t* q_col;
+  uint8_t* sf_col;
+};
+
+cudaError_t launch_quant_both(const QuantBothArgs& a, cudaStream_t st);
+
+}  // namespace moe

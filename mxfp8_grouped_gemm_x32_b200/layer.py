@@ -3,8 +3,9 @@ C ABI.  PyTorch only allocates device memory and provides the stream; every
 step of the layer runs in the CUDA library (see lib.py).
 
 Steps (names of the C entry points):
-  quantize_weights  moe_mlp_quantize_mxfp8 x4: W_gate_up and W_down, along K
+  quantize_weights  moe_mlp_quantize_weights: W_gate_up and W_down, along K
                     for the forward and along the other axis for the backward
+                    (forward only: moe_mlp_quantize_mxfp8 x2)
   permute           moe_permute: counting sort by expert, gather + quantise x
   forward           moe_grouped_mlp_fwd: gate_up GEMM + ScaledSwiGLU + requant,
                     down GEMM, top-k combine
@@ -84,13 +85,14 @@ class GroupedMLP:
         E, H, I, s = self.E, self.H, self.I, self._stream()
         assert w1.dtype == torch.bfloat16 and w1.is_contiguous() and w1.shape == (E, 2 * I, H)
         assert w2.dtype == torch.bfloat16 and w2.is_contiguous() and w2.shape == (E, H, I)
+        if self.backward_enabled:
+            # both directions of both weights from one read of each
+            lib.moe_mlp_quantize_weights(w1.data_ptr(), w2.data_ptr(), E, H, I, _ptr(self.w1q), _ptr(self.w1sf),
+                                         _ptr(self.w2q), _ptr(self.w2sf), _ptr(self.w1tq), _ptr(self.w1tsf),
+                                         _ptr(self.w2tq), _ptr(self.w2tsf), s)
+            return
         lib.moe_mlp_quantize_mxfp8(w1.data_ptr(), 2 * E, I, H, lib.MOE_QUANT_ROW, _ptr(self.w1q), _ptr(self.w1sf), s)
         lib.moe_mlp_quantize_mxfp8(w2.data_ptr(), E, H, I, lib.MOE_QUANT_ROW, _ptr(self.w2q), _ptr(self.w2sf), s)
-        if self.backward_enabled:
-            lib.moe_mlp_quantize_mxfp8(w1.data_ptr(), E, 2 * I, H, lib.MOE_QUANT_COL, _ptr(self.w1tq),
-                                       _ptr(self.w1tsf), s)
-            lib.moe_mlp_quantize_mxfp8(w2.data_ptr(), E, H, I, lib.MOE_QUANT_COL, _ptr(self.w2tq),
-                                       _ptr(self.w2tsf), s)
 
     def permute(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_prob: torch.Tensor) -> None:
         """x bf16 [T, H]; topk_idx int32 [T, k]; topk_prob float32 [T, k]."""

@@ -33,7 +33,7 @@ EXPORTED = [
     "moe_mx_scale_bytes", "moe_padded_rows", "moe_workspace_size", "moe_mlp_quantize_mxfp8",
     "moe_permute", "moe_grouped_mlp_fwd", "moe_combine", "moe_grouped_mlp_bwd",
     "moe_get_device_status", "moe_status_string", "moe_launch_count", "moe_selftest_wait_timeout",
-    "moe_timing_enable", "moe_timing_read", "moe_permute_noalloc",
+    "moe_timing_enable", "moe_timing_read", "moe_permute_noalloc", "moe_mlp_quantize_weights",
 ]
 
 
@@ -65,6 +65,7 @@ _decl("moe_mx_scale_bytes", _I64, _I32, _I64, _I64)
 _decl("moe_padded_rows", _I64, _I32, _I32, _I32)
 _decl("moe_workspace_size", _I64, _I32, _I32, _I32, _I32, _I32, _I32)
 _decl("moe_mlp_quantize_mxfp8", _I32, _P, _I32, _I64, _I64, _I32, _P, _P, _P)
+_decl("moe_mlp_quantize_weights", _I32, _P, _P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P)
 _decl("moe_permute", _I32, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
       _P, _P, _SZ, _P)
 _decl("moe_grouped_mlp_fwd", _I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P,
@@ -106,6 +107,12 @@ def moe_workspace_size(op: int, T: int, k: int, E: int, H: int, I: int) -> int:
 
 def moe_mlp_quantize_mxfp8(src, groups, rows, cols, mode, q, sf, stream=0):
     _check("moe_mlp_quantize_mxfp8", _lib.moe_mlp_quantize_mxfp8(src, groups, rows, cols, mode, q, sf, stream))
+
+
+def moe_mlp_quantize_weights(w_gate_up, w_down, E, H, I, w1q, w1sf, w2q, w2sf, w1tq, w1tsf, w2tq, w2tsf,
+                             stream=0):
+    _check("moe_mlp_quantize_weights", _lib.moe_mlp_quantize_weights(
+        w_gate_up, w_down, E, H, I, w1q, w1sf, w2q, w2sf, w1tq, w1tsf, w2tq, w2tsf, stream))
 
 
 def moe_permute(x, topk_idx, topk_prob, T, H, k, E, rows_cap, split_sizes, group_offsets, row_to_slot,

@@ -317,3 +317,37 @@ def test_bad_expert_id_reported(torch_cuda):
     L.permute(_bf(torch, inp["x"]), torch.from_numpy(idx).cuda(), torch.from_numpy(inp["topk_prob"]).cuda())
     assert lib.moe_get_device_status(0) == 5       # MOE_ERR_DEVICE_INDEX
     assert L.slot_to_row.cpu().numpy()[3 * cfg.k + 1] == -1
+
+
+@pytest.mark.parametrize("E,H,I", [(3, 256, 192), (2, 2880, 2880), (2, 4096, 512)])
+def test_quantize_weights_fused_equals_separate(torch_cuda, E, H, I):
+    """moe_mlp_quantize_weights (one read of each weight) writes exactly what
+    the four single-mode calls write, including zero padding scale bytes."""
+    torch = torch_cuda
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    rng = np.random.default_rng(E * H + I)
+    from mxfp8_grouped_gemm_x32_b200.workloads import bf16_bits_from_f32
+    w1 = _bf(torch, bf16_bits_from_f32(rng.standard_normal((E, 2 * I, H)).astype(np.float32) * 0.05))
+    w2 = _bf(torch, bf16_bits_from_f32(rng.standard_normal((E, H, I)).astype(np.float32) * 0.05))
+    sb = lib.moe_mx_scale_bytes
+    sizes = [(2 * E * I * H, sb(2 * E, I, H)), (E * H * I, sb(E, H, I)), (E * H * 2 * I, sb(E, H, 2 * I)),
+             (E * I * H, sb(E, I, H))]
+
+    def bufs():
+        return [(torch.full((q,), 0x33, dtype=torch.uint8, device="cuda"),
+                 torch.full((s,), 0x33, dtype=torch.uint8, device="cuda")) for q, s in sizes]
+    a, b = bufs(), bufs()
+    p = lambda t: t.data_ptr()
+    lib.moe_mlp_quantize_mxfp8(p(w1), 2 * E, I, H, lib.MOE_QUANT_ROW, p(a[0][0]), p(a[0][1]), 0)
+    lib.moe_mlp_quantize_mxfp8(p(w2), E, H, I, lib.MOE_QUANT_ROW, p(a[1][0]), p(a[1][1]), 0)
+    lib.moe_mlp_quantize_mxfp8(p(w1), E, 2 * I, H, lib.MOE_QUANT_COL, p(a[2][0]), p(a[2][1]), 0)
+    lib.moe_mlp_quantize_mxfp8(p(w2), E, H, I, lib.MOE_QUANT_COL, p(a[3][0]), p(a[3][1]), 0)
+    lib.moe_mlp_quantize_weights(p(w1), p(w2), E, H, I, p(b[0][0]), p(b[0][1]), p(b[1][0]), p(b[1][1]),
+                                 p(b[2][0]), p(b[2][1]), p(b[3][0]), p(b[3][1]), 0)
+    torch.cuda.synchronize()
+    for (qa, sa), (qb, sb_) in zip(a, b):
+        assert torch.equal(qa, qb) and torch.equal(sa, sb_)
+    # and against the oracle for the forward operands
+    c, s = omx.quantize_rows(_f64(w1.cpu().view(torch.int16).numpy().view(np.uint16)).reshape(2 * E * I, H))
+    assert np.array_equal(b[0][0].cpu().numpy().reshape(2 * E * I, H), c)
+    assert np.array_equal(sf_unblock(b[0][1].cpu().numpy(), 2 * E, I, H).reshape(2 * E * I, -1), s)
