@@ -21,6 +21,8 @@
 //   warps 2-9   epilogue: drain the accumulator into registers
 //               (tcgen05.ld), release it to the MMA warp at once, then apply
 //               the epilogue and store -- so the next tile's MMAs overlap it.
+//               Rows go out through a per-warp shared staging buffer so that
+//               each store instruction writes 8 rows x 64 contiguous bytes.
 // Tiles (128 rows x 256 columns) walk a device-side schedule derived from
 // the group offsets; every CTA strides through them (persistent grid).
 // Every wait is bounded; on time-out the kernel records MOE_ERR_TIMEOUT,
@@ -50,7 +52,10 @@ constexpr int OFF_BAR = OFF_SFB + STAGES * SMEM_SFB;
 constexpr int NUM_BARS = 2 * STAGES + 2;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem address, abort flag
 constexpr int OFF_GO = OFF_MISC + 16;              // group offsets [E+1]
-constexpr int SMEM_TOTAL = OFF_GO + (MOE_MAX_EXPERTS + 1) * 4;
+constexpr int STAGE_PITCH_W = 20;                  // words per staged row (16 used): conflict-free v4
+constexpr int STAGE_WARP_BYTES = 32 * STAGE_PITCH_W * 4;
+constexpr int OFF_STAGE = (OFF_GO + (MOE_MAX_EXPERTS + 1) * 4 + 127) / 128 * 128;
+constexpr int SMEM_TOTAL = OFF_STAGE + NUM_EPI_WARPS * STAGE_WARP_BYTES;
 constexpr int SMEM_LAUNCH = SMEM_TOTAL + 1024;     // slack for 1 KB alignment
 
 struct Tile {
@@ -98,104 +103,117 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, in
   return ti;
 }
 
-__device__ __forceinline__ uint32_t block_amax_bits(const float* f) {
-  uint32_t am = 0;
+// Writes the warp's 32 rows (one per lane) of NW 32-bit words each to global
+// memory through the warp's shared staging buffer, 16 words (64 bytes) of
+// every row at a time, so that each global store instruction covers 8 rows x
+// 64 contiguous bytes instead of 32 rows x 16 bytes.  `row` is this lane's
+// destination (nullptr: row not stored); only the first `bytes` bytes of a
+// row are stored (a multiple of 16).
+template <int NW>
+__device__ __forceinline__ void warp_store_rows(uint32_t* stage, uint8_t* row, const uint32_t* w, int bytes,
+                                                int lane) {
+  static_assert(NW % 16 == 0, "rows are staged 16 words at a time");
+  const uint64_t rp = reinterpret_cast<uint64_t>(row);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) am = max(am, __float_as_uint(f[j]) & 0x7FFFFFFFu);
-  return am;
-}
-
-// Quantise 32 fp32 values to E4M3 codes with scale byte sb, store 32 bytes.
-__device__ __forceinline__ void store_block_e4m3(uint8_t* dst, const float* f, uint32_t sb) {
-  const float inv = inv_scale_from_e8m0(sb);
-  uint32_t w[8];
+  for (int c = 0; c < NW / 16; ++c) {
+    __syncwarp();
+    uint4* srow = reinterpret_cast<uint4*>(stage + lane * STAGE_PITCH_W);
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    w[j] = pack4_e4m3(f[4 * j] * inv, f[4 * j + 1] * inv, f[4 * j + 2] * inv, f[4 * j + 3] * inv);
-  uint4* d = reinterpret_cast<uint4*>(dst);
-  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  d[1] = make_uint4(w[4], w[5], w[6], w[7]);
-}
-
-// 128 fp32 (as bits) -> bf16, 16 x 16-byte stores, columns >= ncols skipped
-// in units of 8.
-__device__ __forceinline__ void store_row_bf16(uint8_t* dst, const uint32_t* v, int ncols) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
+    for (int q = 0; q < 4; ++q)
+      srow[q] = make_uint4(w[16 * c + 4 * q], w[16 * c + 4 * q + 1], w[16 * c + 4 * q + 2], w[16 * c + 4 * q + 3]);
+    __syncwarp();
+    const int piece = lane & 3;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    if (8 * i < ncols)
-      d[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1])),
-                        pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
-                        pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
-                        pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+    for (int it = 0; it < 4; ++it) {
+      const int rr = (lane >> 2) + 8 * it;
+      const uint64_t dst = __shfl_sync(0xFFFFFFFFu, rp, rr);
+      const int off = 64 * c + 16 * piece;
+      if (dst != 0 && off < bytes)
+        *reinterpret_cast<uint4*>(dst + off) =
+            *reinterpret_cast<const uint4*>(stage + rr * STAGE_PITCH_W + 4 * piece);
+    }
   }
 }
 
+// 2*NW fp32 values (as bits) -> NW bf16x2 words, in place at the front.
+template <int NW>
+__device__ __forceinline__ void pack_bf16_inplace(uint32_t* v) {
+#pragma unroll
+  for (int i = 0; i < NW; ++i) v[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+}
+
 template <int EPI>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti, const uint32_t* v,
-                                              int q, int half, int lane) {
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti, uint32_t* v, int q, int half,
+                                              int lane, uint32_t* stage) {
   const int r = ti.m0 + 32 * q + lane;
-  if (r >= ti.row_end) return;
+  const bool rv = r < ti.row_end;
   if constexpr (EPI == EPI_SWIGLU) {
     // v[0:64] gate columns nb..nb+63, v[64:128] the matching up columns
     const int nb = ti.n0 + 64 * half;
-    if (nb >= a.N) return;
+    if (nb >= a.N) return;  // uniform across the warp
     const int N = a.N;
     if (a.out2) {
-      uint4* dg = reinterpret_cast<uint4*>(a.out2 + (int64_t(r) * 2 * N + nb) * 2);
-      uint4* du = reinterpret_cast<uint4*>(a.out2 + (int64_t(r) * 2 * N + N + nb) * 2);
+      // saved A in bf16, 32 columns at a time (keeps the fp32 values for h)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t* g = v + 8 * i;
-        const uint32_t* u = v + 64 + 8 * i;
-        dg[i] = make_uint4(pack_bf16x2(__uint_as_float(g[0]), __uint_as_float(g[1])),
-                           pack_bf16x2(__uint_as_float(g[2]), __uint_as_float(g[3])),
-                           pack_bf16x2(__uint_as_float(g[4]), __uint_as_float(g[5])),
-                           pack_bf16x2(__uint_as_float(g[6]), __uint_as_float(g[7])));
-        du[i] = make_uint4(pack_bf16x2(__uint_as_float(u[0]), __uint_as_float(u[1])),
-                           pack_bf16x2(__uint_as_float(u[2]), __uint_as_float(u[3])),
-                           pack_bf16x2(__uint_as_float(u[4]), __uint_as_float(u[5])),
-                           pack_bf16x2(__uint_as_float(u[6]), __uint_as_float(u[7])));
+      for (int c = 0; c < 4; ++c) {
+        uint32_t t[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          t[j] = pack_bf16x2(__uint_as_float(v[32 * c + 2 * j]), __uint_as_float(v[32 * c + 2 * j + 1]));
+        const int64_t col = (c < 2 ? 0 : N) + nb + 32 * (c & 1);
+        warp_store_rows<16>(stage, rv ? a.out2 + (int64_t(r) * 2 * N + col) * 2 : nullptr, t, 64, lane);
       }
     }
-    const float p = a.prob[r];
+    float p = 0.0f;
+    if (rv) p = a.prob[r];
+    uint32_t hw[16];  // 64 E4M3 codes of h
     uint32_t sbs = 0;
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-      float h[32];
+      // h in place of the gate values of this block
+      uint32_t am = 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float g = __uint_as_float(v[32 * b + j]);
         const float u = __uint_as_float(v[64 + 32 * b + j]);
-        h[j] = p * __fdividef(g, 1.0f + __expf(-g)) * u;
+        const float h = p * __fdividef(g, 1.0f + __expf(-g)) * u;
+        v[32 * b + j] = __float_as_uint(h);
+        am = max(am, __float_as_uint(h) & 0x7FFFFFFFu);
       }
-      const uint32_t sb = e8m0_from_amax_bits(block_amax_bits(h));
-      store_block_e4m3(a.q_out + int64_t(r) * N + nb + 32 * b, h, sb);
+      const uint32_t sb = e8m0_from_amax_bits(am);
+      const float inv = inv_scale_from_e8m0(sb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        hw[8 * b + j] = pack4_e4m3(__uint_as_float(v[32 * b + 4 * j]) * inv, __uint_as_float(v[32 * b + 4 * j + 1]) * inv,
+                                   __uint_as_float(v[32 * b + 4 * j + 2]) * inv, __uint_as_float(v[32 * b + 4 * j + 3]) * inv);
       sbs |= sb << (8 * b);
     }
-    const int kb0 = nb >> 5;
-    uint8_t* sfp = a.sf_out + sf_offset(0, r, kb0, 0, a.q_KT);
-    if (nb + 64 == N && (kb0 & 3) == 0)
-      *reinterpret_cast<uint32_t*>(sfp) = sbs;  // also zero the two padding blocks of the K tile
-    else
-      *reinterpret_cast<uint16_t*>(sfp) = uint16_t(sbs);
+    warp_store_rows<16>(stage, rv ? a.q_out + int64_t(r) * N + nb : nullptr, hw, 64, lane);
+    if (rv) {
+      const int kb0 = nb >> 5;
+      uint8_t* sfp = a.sf_out + sf_offset(0, r, kb0, 0, a.q_KT);
+      if (nb + 64 == N && (kb0 & 3) == 0)
+        *reinterpret_cast<uint32_t*>(sfp) = sbs;  // also zero the two padding blocks of the K tile
+      else
+        *reinterpret_cast<uint16_t*>(sfp) = uint16_t(sbs);
+    }
   } else {
     const int nb = ti.n0 + 128 * half;
-    if (nb >= a.N) return;
+    if (nb >= a.N) return;  // uniform across the warp
+    const int ncols = min(128, a.N - nb);
     if constexpr (EPI == EPI_F32_SCATTER || EPI == EPI_F32_ROWS) {
-      int64_t orow = r;
-      if constexpr (EPI == EPI_F32_SCATTER) {
-        orow = a.row_to_slot[r];
-        if (orow < 0) return;
+      uint8_t* dst = nullptr;
+      if (rv) {
+        int64_t orow = r;
+        if constexpr (EPI == EPI_F32_SCATTER) orow = a.row_to_slot[r];
+        if (orow >= 0) dst = a.out + (orow * a.ld_out + nb) * 4;
       }
-      uint4* d = reinterpret_cast<uint4*>(a.out + (orow * a.ld_out + nb) * 4);
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (4 * i < a.N - nb) d[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      return;
+      warp_store_rows<128>(stage, dst, v, ncols * 4, lane);
+    } else {
+      pack_bf16_inplace<64>(v);
+      uint8_t* dst = rv ? a.out + (int64_t(ti.e) * a.out_group_stride + int64_t(r) * a.ld_out + nb) * 2 : nullptr;
+      warp_store_rows<64>(stage, dst, v, ncols * 2, lane);
     }
-    uint8_t* dst = a.out + (int64_t(ti.e) * a.out_group_stride + int64_t(r) * a.ld_out + nb) * 2;
-    store_row_bf16(dst, v, a.N - nb);
   }
 }
 
@@ -321,6 +339,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ---------------- epilogue warps ----------------
     const int q = warp & 3;            // TMEM sub-partition this warp may read
     const int half = (warp - 2) >> 2;  // which half of the tile's columns
+    uint32_t* stage = reinterpret_cast<uint32_t*>(smem + OFF_STAGE + (warp - 2) * STAGE_WARP_BYTES);
     uint32_t acc_it = 0;
     uint32_t v[128];
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -329,7 +348,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if constexpr (EPI == EPI_WGRAD) {
 #pragma unroll
           for (int i = 0; i < 128; ++i) v[i] = 0u;
-          epilogue_tile<EPI>(a, ti, v, q, half, lane);
+          epilogue_tile<EPI>(a, ti, v, q, half, lane, stage);
         }
         continue;
       }
@@ -352,7 +371,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
       ++acc_it;
-      epilogue_tile<EPI>(a, ti, v, q, half, lane);
+      epilogue_tile<EPI>(a, ti, v, q, half, lane, stage);
     }
   }
 
