@@ -154,8 +154,11 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(QuantColsArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Both modes from one read.  A CTA stages a 128-row x 128-column tile of one
-// group (bf16, shared memory); thread t then quantises
+// Both modes from one read.  Persistent CTAs walk 128-row x 128-column tiles
+// of the source; each tile is brought into shared memory with cp.async while
+// the previous one is quantised (two buffers), so the loads of the next tile
+// overlap the arithmetic and stores of this one.  For a staged tile, thread t
+// quantises
 //   row mode: row t%128, column blocks 2*(t/128), +1 -> 64 code bytes and
 //             two scale bytes of that row;
 //   column mode: column t%128, row blocks 2*(t/128), +1 -> 64 code bytes of
@@ -163,23 +166,54 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(QuantColsArgs a) {
 // Weights are read from HBM once for both the forward (row) and the
 // backward (column) operand.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256, 4) quant_both_kernel(QuantBothArgs a) {
-  __shared__ __align__(16) uint16_t tile[QC_TILE * QC_PITCH];
-  const int64_t g = blockIdx.z;
-  const int64_t r0 = int64_t(blockIdx.x) * QC_TILE;
-  const int64_t c0 = int64_t(blockIdx.y) * QC_TILE;
-  const int tid = threadIdx.x;
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+constexpr int QB_TILE_ELEMS = QC_TILE * QC_PITCH;
+constexpr int QB_OUT_PITCH = 144;  // bytes per staged output row (128 codes + 16: conflict-free 16-byte writes)
+constexpr int QB_OUT_BYTES = QC_TILE * QB_OUT_PITCH;
+
+struct QbTile {
+  int64_t g, r0, c0;
+};
+
+__device__ __forceinline__ QbTile qb_tile(const QuantBothArgs& a, int64_t t, int64_t rt, int64_t ct) {
+  QbTile q;
+  q.g = t / (rt * ct);
+  const int64_t rem = t - q.g * rt * ct;
+  q.r0 = (rem / ct) * QC_TILE;
+  q.c0 = (rem % ct) * QC_TILE;
+  return q;
+}
+
+__device__ __forceinline__ void qb_load(const QuantBothArgs& a, const QbTile& q, uint16_t* tile, int tid) {
   for (int i = tid; i < QC_TILE * (QC_TILE / 8); i += 256) {
     const int rr = i / (QC_TILE / 8);
     const int cc = (i % (QC_TILE / 8)) * 8;
-    const int64_t r = r0 + rr, c = c0 + cc;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < a.rows && c < a.cols)
-      v = __ldg(reinterpret_cast<const uint4*>(a.src + ((g * a.rows + r) * a.cols + c) * 2));
-    *reinterpret_cast<uint4*>(&tile[rr * QC_PITCH + cc]) = v;
+    const int64_t r = q.r0 + rr, c = q.c0 + cc;
+    const bool in = r < a.rows && c < a.cols;
+    const uint8_t* src = in ? a.src + ((q.g * a.rows + r) * a.cols + c) * 2 : a.src;
+    cp_async16(&tile[rr * QC_PITCH + cc], src, in ? 16u : 0u);  // zero fill outside the matrix
   }
-  __syncthreads();
+}
 
+// Quantise one staged tile.  The codes of both modes go to shared staging
+// tiles (out_row: 128 rows x 128 codes, out_col: 128 transposed rows x 128
+// codes) and the scale bytes to `atoms` (2 x 512 bytes: the row-mode and the
+// column-mode scale atom of this tile, zero where no row / block exists);
+// qb_store writes them to global memory as whole 128-byte lines.
+__device__ __forceinline__ void qb_compute(const QuantBothArgs& a, const QbTile& q, const uint16_t* tile,
+                                           uint8_t* out_row, uint8_t* out_col, uint8_t* atoms, bool row_atom,
+                                           int tid) {
+  const int64_t g = q.g, r0 = q.r0, c0 = q.c0;
   // ---- row mode: blocks of 32 along the columns --------------------------
   // thread -> (row tid % 128, column half tid / 128): a warp reads 32
   // consecutive staged rows with 16-byte loads, conflict-free for the
@@ -187,12 +221,8 @@ __global__ void __launch_bounds__(256, 4) quant_both_kernel(QuantBothArgs a) {
   {
     const int rl = tid & 127, hb = tid >> 7;
     const int64_t r = r0 + rl;
+    uint32_t sbs = 0;
     if (r < a.rows) {
-      const int64_t rg = g * (a.rows / a.row_split) + r / a.row_split;  // row-group
-      const int64_t rr = r % a.row_split;
-      const int64_t RT = cdiv(a.row_split, 128), KT = cdiv(a.cols, 128);
-      const int64_t kb0 = c0 / 32 + 2 * hb;
-      uint32_t sbs = 0;
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         const int64_t cb = c0 + 64 * hb + 32 * b;
@@ -216,50 +246,118 @@ __global__ void __launch_bounds__(256, 4) quant_both_kernel(QuantBothArgs a) {
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           w[j] = pack4_e4m3(f[4 * j] * inv, f[4 * j + 1] * inv, f[4 * j + 2] * inv, f[4 * j + 3] * inv);
-        uint4* d = reinterpret_cast<uint4*>(a.q_row + (g * a.rows + r) * a.cols + cb);
+        uint4* d = reinterpret_cast<uint4*>(out_row + rl * QB_OUT_PITCH + 64 * hb + 32 * b);
         d[0] = make_uint4(w[0], w[1], w[2], w[3]);
         d[1] = make_uint4(w[4], w[5], w[6], w[7]);
         sbs |= sb << (8 * b);
       }
-      *reinterpret_cast<uint16_t*>(a.sf_row + sf_offset(rg, rr, kb0, RT, KT)) = uint16_t(sbs);
+      if (!row_atom) {  // the tile spans two row-groups: scale bytes one by one
+        const int64_t rg = g * (a.rows / a.row_split) + r / a.row_split;
+        const int64_t rr = r % a.row_split;
+        *reinterpret_cast<uint16_t*>(a.sf_row + sf_offset(rg, rr, c0 / 32 + 2 * hb, cdiv(a.row_split, 128),
+                                                          cdiv(a.cols, 128))) = uint16_t(sbs);
+      }
     }
+    // position of (row rl, blocks 2hb, 2hb+1) inside the 512-byte atom
+    *reinterpret_cast<uint16_t*>(atoms + (rl & 31) * 16 + (rl >> 5) * 4 + 2 * hb) = uint16_t(sbs);
   }
-
   // ---- column mode: blocks of 32 along the rows, stored transposed --------
+  // thread -> (column pair tid % 64, row block tid / 64): 32 four-byte loads
+  // give both columns of the pair
   {
-    const int cl = tid & 127, half = tid >> 7;
-    const int64_t c = c0 + cl;
-    const int64_t RT = cdiv(a.cols, 128), KT = cdiv(a.rows, 128);
-    const int64_t kb0 = r0 / 32 + 2 * half;
-    uint8_t* sfp = a.sf_col + sf_offset(g, c, kb0, RT, KT);
-    if (c >= a.cols) {
-      *reinterpret_cast<uint16_t*>(sfp) = 0;
-      return;
-    }
-    uint32_t sbs = 0;
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      const int64_t rb = r0 + 64 * half + 32 * b;
-      if (rb >= a.rows) break;
-      float f[32];
+    const int cp = tid & 63, rb = tid >> 6;
+    const int64_t c = c0 + 2 * cp;
+    const int64_t rbeg = r0 + 32 * rb;
+    uint32_t sb2[2] = {0u, 0u};
+    if (c < a.cols && rbeg < a.rows) {
+      uint32_t wv[32];  // bf16 pairs: column c in the low half, c + 1 in the high half
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        f[j] = __uint_as_float(uint32_t(tile[(64 * half + 32 * b + j) * QC_PITCH + cl]) << 16);
-      uint32_t am = 0;
+        wv[j] = *reinterpret_cast<const uint32_t*>(&tile[(32 * rb + j) * QC_PITCH + 2 * cp]);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) am = max(am, __float_as_uint(f[j]) & 0x7FFFFFFFu);
-      const uint32_t sb = e8m0_from_amax_bits(am);
-      const float inv = inv_scale_from_e8m0(sb);
-      uint32_t w[8];
+      for (int h = 0; h < 2; ++h) {
+        uint32_t am = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        w[j] = pack4_e4m3(f[4 * j] * inv, f[4 * j + 1] * inv, f[4 * j + 2] * inv, f[4 * j + 3] * inv);
-      uint4* d = reinterpret_cast<uint4*>(a.q_col + (g * a.cols + c) * a.rows + rb);
-      d[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      d[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      sbs |= sb << (8 * b);
+        for (int j = 0; j < 32; ++j) am = max(am, (h ? (wv[j] & 0xFFFF0000u) : (wv[j] << 16)) & 0x7FFFFFFFu);
+        const uint32_t sb = e8m0_from_amax_bits(am);
+        const float inv = inv_scale_from_e8m0(sb);
+        uint32_t w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t* q4 = wv + 4 * j;
+          w[j] = h ? pack4_e4m3(bf16hi(q4[0]) * inv, bf16hi(q4[1]) * inv, bf16hi(q4[2]) * inv, bf16hi(q4[3]) * inv)
+                   : pack4_e4m3(bf16lo(q4[0]) * inv, bf16lo(q4[1]) * inv, bf16lo(q4[2]) * inv, bf16lo(q4[3]) * inv);
+        }
+        uint4* d = reinterpret_cast<uint4*>(out_col + (2 * cp + h) * QB_OUT_PITCH + 32 * rb);
+        d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        sb2[h] = sb;
+      }
     }
-    *reinterpret_cast<uint16_t*>(sfp) = uint16_t(sbs);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int cl = 2 * cp + h;  // output row inside the tile
+      atoms[512 + (cl & 31) * 16 + (cl >> 5) * 4 + rb] = uint8_t(sb2[h]);
+    }
+  }
+}
+
+// Staged codes and scale atoms of one tile -> global memory: every warp
+// store instruction covers 4 rows x 128 contiguous bytes.
+__device__ __forceinline__ void qb_store(const QuantBothArgs& a, const QbTile& q, const uint8_t* out_row,
+                                         const uint8_t* out_col, const uint8_t* atoms, bool row_atom,
+                                         int64_t rt, int64_t ct, int tid) {
+  const int chunk = tid & 7;
+  const int64_t vrow_bytes = a.cols - q.c0 < 128 ? a.cols - q.c0 : 128;  // valid codes of a row-mode row
+  const int64_t vcol_bytes = a.rows - q.r0 < 128 ? a.rows - q.r0 : 128;  // valid codes of a column-mode row
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = (tid >> 3) + 32 * i;
+    if (q.r0 + rr < a.rows && 16 * chunk < vrow_bytes)
+      *reinterpret_cast<uint4*>(a.q_row + (q.g * a.rows + q.r0 + rr) * a.cols + q.c0 + 16 * chunk) =
+          *reinterpret_cast<const uint4*>(out_row + rr * QB_OUT_PITCH + 16 * chunk);
+    if (q.c0 + rr < a.cols && 16 * chunk < vcol_bytes)
+      *reinterpret_cast<uint4*>(a.q_col + (q.g * a.cols + q.c0 + rr) * a.rows + q.r0 + 16 * chunk) =
+          *reinterpret_cast<const uint4*>(out_col + rr * QB_OUT_PITCH + 16 * chunk);
+  }
+  if (tid < 32) {
+    if (row_atom) {
+      const int64_t rg = q.g * (a.rows / a.row_split) + q.r0 / a.row_split;
+      const int64_t rr = q.r0 % a.row_split;
+      reinterpret_cast<uint4*>(a.sf_row + sf_offset(rg, rr, q.c0 / 32, cdiv(a.row_split, 128),
+                                                    cdiv(a.cols, 128)))[tid] = reinterpret_cast<const uint4*>(atoms)[tid];
+    }
+  } else if (tid < 64) {
+    reinterpret_cast<uint4*>(a.sf_col + sf_offset(q.g, q.c0, q.r0 / 32, ct, rt))[tid - 32] =
+        reinterpret_cast<const uint4*>(atoms + 512)[tid - 32];
+  }
+}
+
+__global__ void __launch_bounds__(256, 2) quant_both_kernel(QuantBothArgs a) {
+  extern __shared__ __align__(16) uint16_t qb_smem[];
+  uint8_t* out_row = reinterpret_cast<uint8_t*>(qb_smem + 2 * QB_TILE_ELEMS);
+  uint8_t* out_col = out_row + QB_OUT_BYTES;
+  uint8_t* atoms = out_col + QB_OUT_BYTES;  // 1 KB
+  const int tid = threadIdx.x;
+  const int64_t rt = cdiv(a.rows, QC_TILE), ct = cdiv(a.cols, QC_TILE);
+  const int64_t ntiles = int64_t(a.groups) * rt * ct;
+  // whole row-mode atoms need row-groups of a multiple of 128 rows
+  const bool row_atom = a.row_split % QC_TILE == 0;
+  int64_t t = blockIdx.x;
+  if (t >= ntiles) return;
+  qb_load(a, qb_tile(a, t, rt, ct), qb_smem, tid);
+  cp_async_commit();
+  for (int it = 0; t < ntiles; ++it, t += gridDim.x) {
+    const int64_t tn = t + gridDim.x;
+    if (tn < ntiles) qb_load(a, qb_tile(a, tn, rt, ct), qb_smem + ((it + 1) & 1) * QB_TILE_ELEMS, tid);
+    cp_async_commit();  // (possibly empty group: keeps the wait count uniform)
+    cp_async_wait<1>();
+    __syncthreads();
+    const QbTile q = qb_tile(a, t, rt, ct);
+    qb_compute(a, q, qb_smem + (it & 1) * QB_TILE_ELEMS, out_row, out_col, atoms, row_atom, tid);
+    __syncthreads();  // staging complete
+    qb_store(a, q, out_row, out_col, atoms, row_atom, rt, ct, tid);
+    __syncthreads();  // staging and this input buffer are reused
   }
 }
 
@@ -294,8 +392,17 @@ cudaError_t launch_quant_both(const QuantBothArgs& a, cudaStream_t st) {
     cudaError_t e = cudaMemsetAsync(a.sf_row, 0, size_t(n), st);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(unsigned(cdiv(a.rows, 128)), unsigned(cdiv(a.cols, 128)), unsigned(a.groups));
-  quant_both_kernel<<<grid, 256, 0, st>>>(a);
+  const size_t smem = 2 * QB_TILE_ELEMS * sizeof(uint16_t) + 2 * QB_OUT_BYTES + 1024;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(quant_both_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int64_t ntiles = int64_t(a.groups) * cdiv(a.rows, QC_TILE) * cdiv(a.cols, QC_TILE);
+  int64_t grid = int64_t(num_sms()) * 2;
+  if (grid > ntiles) grid = ntiles;
+  quant_both_kernel<<<unsigned(grid), 256, smem, st>>>(a);
   count_launch();
   return cudaGetLastError();
 }
