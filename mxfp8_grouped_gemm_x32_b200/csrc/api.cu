@@ -87,7 +87,7 @@ FwdWs carve_fwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t r
 }
 
 struct BwdWs {
-  uint8_t *dyq, *dyq_sf, *dyc, *dyc_sf, *dh, *daq, *daq_sf, *dac, *dac_sf, *hc, *hc_sf, *dx;
+  uint8_t *dyq, *dyq_sf, *dyc, *dyc_sf, *dh, *daq, *daq_sf, *dac, *dac_sf, *hc, *hc_sf, *dx, *dpp;
 };
 BwdWs carve_bwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t rows_cap) {
   BwdWs w{};
@@ -103,6 +103,7 @@ BwdWs carve_bwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t r
   w.hc = c.take(I * rows_cap);
   w.hc_sf = c.take(mx_scale_bytes(1, I, rows_cap));
   w.dx = c.take(T * k * H * 4);
+  w.dpp = c.take(swiglu_partial_bytes(rows_cap, int32_t(I)));
   return w;
 }
 
@@ -373,7 +374,7 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   // ScaledSwiGLU backward + quantisation of da (both ways) and h (along tokens)
   SwigluBwdArgs sb{I, E, rows_cap, group_offsets, row_to_slot, prob_perm, w.dh,
                    static_cast<const uint8_t*>(saved_a), w.daq, w.daq_sf, w.dac, w.dac_sf, w.hc, w.hc_sf,
-                   dprob};
+                   dprob, reinterpret_cast<float*>(w.dpp)};
   {
     TimeScope ts(st, "swiglu_bwd");
     if (launch_swiglu_bwd(sb, st) != cudaSuccess) return MOE_ERR_CUDA;

@@ -37,6 +37,28 @@ struct TimeScope {
 // MXFP8 encoding
 // ----------------------------------------------------------------------------
 
+// max(|a|, |b|), NaN if either is NaN, so that a block holding a NaN gets
+// the NaN scale.  One min/max instruction (the absolute values fold into it).
+__device__ __forceinline__ float abs_max(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(fabsf(a)), "f"(fabsf(b)));
+  return d;
+}
+
+// max |v[i]| over N values (N a power of two), as a balanced tree.
+template <int N>
+__device__ __forceinline__ float abs_max_n(const float* v) {
+  float m[N / 2];
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) m[i] = abs_max(v[2 * i], v[2 * i + 1]);
+#pragma unroll
+  for (int w = N / 4; w >= 1; w /= 2) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = abs_max(m[2 * i], m[2 * i + 1]);
+  }
+  return m[0];
+}
+
 // E8M0 scale byte from the bit pattern of a block's amax (|.| bits of an
 // fp32 value, so NaN/Inf compare above every finite value).  The scale is the
 // smallest power of two 2^s with amax / 2^s <= 448: amax = m * 2^e with

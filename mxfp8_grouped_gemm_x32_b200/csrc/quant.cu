@@ -66,10 +66,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantRowsArgs a) {
         f[8 * j + 4] = bf16lo(v[j].z); f[8 * j + 5] = bf16hi(v[j].z);
         f[8 * j + 6] = bf16lo(v[j].w); f[8 * j + 7] = bf16hi(v[j].w);
       }
-      uint32_t am = 0;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) am = max(am, __float_as_uint(f[j]) & 0x7FFFFFFFu);
-      const uint32_t sb = e8m0_from_amax_bits(am);
+      const uint32_t sb = e8m0_from_amax_bits(__float_as_uint(abs_max_n<32>(f)));
       const float inv = inv_scale_from_e8m0(sb);
       uint32_t c[8];
 #pragma unroll
@@ -136,10 +133,7 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(QuantColsArgs a) {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
       f[j] = __uint_as_float(uint32_t(tile[(64 * half + 32 * b + j) * QC_PITCH + cl]) << 16);
-    uint32_t am = 0;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) am = max(am, __float_as_uint(f[j]) & 0x7FFFFFFFu);
-    const uint32_t sb = e8m0_from_amax_bits(am);
+    const uint32_t sb = e8m0_from_amax_bits(__float_as_uint(abs_max_n<32>(f)));
     const float inv = inv_scale_from_e8m0(sb);
     uint32_t w[8];
 #pragma unroll
@@ -237,10 +231,7 @@ __device__ __forceinline__ void qb_compute(const QuantBothArgs& a, const QbTile&
           f[8 * j + 4] = bf16lo(v.z); f[8 * j + 5] = bf16hi(v.z);
           f[8 * j + 6] = bf16lo(v.w); f[8 * j + 7] = bf16hi(v.w);
         }
-        uint32_t am = 0;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) am = max(am, __float_as_uint(f[j]) & 0x7FFFFFFFu);
-        const uint32_t sb = e8m0_from_amax_bits(am);
+        const uint32_t sb = e8m0_from_amax_bits(__float_as_uint(abs_max_n<32>(f)));
         const float inv = inv_scale_from_e8m0(sb);
         uint32_t w[8];
 #pragma unroll
@@ -276,18 +267,15 @@ __device__ __forceinline__ void qb_compute(const QuantBothArgs& a, const QbTile&
         wv[j] = *reinterpret_cast<const uint32_t*>(&tile[(32 * rb + j) * QC_PITCH + 2 * cp]);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        uint32_t am = 0;
+        float f[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) am = max(am, (h ? (wv[j] & 0xFFFF0000u) : (wv[j] << 16)) & 0x7FFFFFFFu);
-        const uint32_t sb = e8m0_from_amax_bits(am);
+        for (int j = 0; j < 32; ++j) f[j] = h ? bf16hi(wv[j]) : bf16lo(wv[j]);
+        const uint32_t sb = e8m0_from_amax_bits(__float_as_uint(abs_max_n<32>(f)));
         const float inv = inv_scale_from_e8m0(sb);
         uint32_t w[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t* q4 = wv + 4 * j;
-          w[j] = h ? pack4_e4m3(bf16hi(q4[0]) * inv, bf16hi(q4[1]) * inv, bf16hi(q4[2]) * inv, bf16hi(q4[3]) * inv)
-                   : pack4_e4m3(bf16lo(q4[0]) * inv, bf16lo(q4[1]) * inv, bf16lo(q4[2]) * inv, bf16lo(q4[3]) * inv);
-        }
+        for (int j = 0; j < 8; ++j)
+          w[j] = pack4_e4m3(f[4 * j] * inv, f[4 * j + 1] * inv, f[4 * j + 2] * inv, f[4 * j + 3] * inv);
         uint4* d = reinterpret_cast<uint4*>(out_col + (2 * cp + h) * QB_OUT_PITCH + 32 * rb);
         d[0] = make_uint4(w[0], w[1], w[2], w[3]);
         d[1] = make_uint4(w[4], w[5], w[6], w[7]);

@@ -19,8 +19,12 @@ struct SwigluBwdArgs {
   uint8_t* hcol;                 // MX (1, I, rows_cap)
   uint8_t* hcol_sf;
   float* dprob;                  // [T*k] slot order
+  float* dprob_part;             // [ceil(I/128)][rows_cap] per-chunk partial sums (scratch)
 };
 
+// Bytes of the dprob_part scratch.
+int64_t swiglu_partial_bytes(int64_t rows_cap, int32_t I);
+// Two launches: the fused kernel, then the dprob reduction over chunks.
 cudaError_t launch_swiglu_bwd(const SwigluBwdArgs& a, cudaStream_t st);
 
 }  // namespace moe
