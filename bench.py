@@ -391,9 +391,12 @@ def run_ours(args):
                     "traffic": profiled_traffic(cfg.name),
                     "peak_source": f"{peaks['source']} bf16 sustained x {MXFP8_OVER_BF16} (nominal MXFP8/BF16)",
                     "frac_of_burst": achieved / peaks["mxfp8_burst"]}
-    fwd_ms = sum(kernels[k]["ms_per_step"] for k in ("gemm_gate_up_swiglu", "gemm_down", "combine")
-                 if k in kernels)
-    bwd_keys = ("dy_quant_rows", "dy_quant_cols", "gemm_dgrad_down", "swiglu_bwd", "gemm_wgrad_down",
+    # layer forward = permute + gate_up GEMM + down GEMM + combine; layer backward = dY
+    # quantisation + both dgrads + SwiGLU backward + both wgrads + dX combine (weight
+    # quantisation reported on its own)
+    fwd_keys = ("permute_index", "permute_quant", "gemm_gate_up_swiglu", "gemm_down", "combine")
+    fwd_ms = sum(kernels[k]["ms_per_step"] for k in fwd_keys if k in kernels)
+    bwd_keys = ("dy_quant", "gemm_dgrad_down", "swiglu_bwd", "gemm_wgrad_down",
                 "gemm_dgrad_gate_up", "combine_dx", "gemm_wgrad_gate_up")
     bwd_ms = sum(kernels[k]["ms_per_step"] for k in bwd_keys if k in kernels)
     line = {

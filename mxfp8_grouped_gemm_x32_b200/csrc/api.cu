@@ -234,15 +234,16 @@ moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* to
                              row_to_slot, slot_to_row, prob_perm, workspace, st);
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq, xq_sf};
-  {
-    TimeScope ts(st, "permute_quant_rows");
-    if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
-  }
   if (xq_col) {
-    QuantColsArgs qc{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq_col, xq_col_sf};
-    TimeScope ts(st, "permute_quant_cols");
-    if ((e = launch_quant_cols(qc, st)) != cudaSuccess) return MOE_ERR_CUDA;
+    // training: x rows gathered once, quantised along H and along tokens
+    QuantBothArgs qb{static_cast<const uint8_t*>(x), 1, rows_cap, H, rows_cap, xq, xq_sf, xq_col, xq_col_sf,
+                     row_to_slot, k};
+    TimeScope ts(st, "permute_quant");
+    if ((e = launch_quant_both(qb, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq, xq_sf};
+    TimeScope ts(st, "permute_quant");
+    if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
   }
   return MOE_OK;
 }
@@ -345,15 +346,11 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   cudaError_t e;
 
   // dy rows gathered to permuted order, quantised along H and along tokens
-  QuantRowsArgs qr{static_cast<const uint8_t*>(dY), H, row_to_slot, k, 1, rows_cap, H, w.dyq, w.dyq_sf};
+  QuantBothArgs qb{static_cast<const uint8_t*>(dY), 1, rows_cap, H, rows_cap, w.dyq, w.dyq_sf, w.dyc, w.dyc_sf,
+                   row_to_slot, k};
   {
-    TimeScope ts(st, "dy_quant_rows");
-    if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
-  }
-  QuantColsArgs qc{static_cast<const uint8_t*>(dY), H, row_to_slot, k, 1, rows_cap, H, w.dyc, w.dyc_sf};
-  {
-    TimeScope ts(st, "dy_quant_cols");
-    if ((e = launch_quant_cols(qc, st)) != cudaSuccess) return MOE_ERR_CUDA;
+    TimeScope ts(st, "dy_quant");
+    if ((e = launch_quant_both(qb, st)) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // dgrad2: dh = dy W_down (contraction over H)

@@ -104,6 +104,30 @@ __host__ __device__ __forceinline__ int64_t sf_offset(int64_t g, int64_t r, int6
 
 __host__ __device__ __forceinline__ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// floor(m / d) for 0 <= m < 2^31 and a divisor fixed at launch, by a
+// multiply-high (Granlund & Montgomery, "Division by invariant integers using
+// multiplication", 1994): with l = ceil(log2 d), p = 31 + l and
+// magic = ceil(2^p / d) < 2^32, floor(m * magic / 2^p) = floor(m / d) because
+// the rounding excess m * (magic - 2^p/d) / 2^p stays below 1/d.
+struct FastDiv {
+  uint32_t d = 1, magic = 0, shift = 0;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  if (d > 1) {
+    uint32_t l = 0;
+    while ((uint64_t(1) << l) < d) ++l;
+    const uint64_t p2 = uint64_t(1) << (31 + l);
+    f.magic = uint32_t((p2 + d - 1) / d);
+    f.shift = l - 1;
+  }
+  return f;
+}
+__device__ __forceinline__ uint32_t fastdiv(uint32_t m, const FastDiv& f) {
+  return f.d == 1 ? m : (__umulhi(m, f.magic) >> f.shift);
+}
+
 // ----------------------------------------------------------------------------
 // small vector helpers
 // ----------------------------------------------------------------------------

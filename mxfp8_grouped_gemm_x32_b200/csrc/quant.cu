@@ -188,14 +188,36 @@ __device__ __forceinline__ QbTile qb_tile(const QuantBothArgs& a, int64_t t, int
   return q;
 }
 
+// One 128 x 128 tile into shared memory: 16-byte cp.async chunks, thread t
+// takes column chunk t % 16 of rows t / 16 + 16 j.  With a gather map the
+// eight source rows are looked up first (independent loads), then the eight
+// copies are issued.
 __device__ __forceinline__ void qb_load(const QuantBothArgs& a, const QbTile& q, uint16_t* tile, int tid) {
-  for (int i = tid; i < QC_TILE * (QC_TILE / 8); i += 256) {
-    const int rr = i / (QC_TILE / 8);
-    const int cc = (i % (QC_TILE / 8)) * 8;
-    const int64_t r = q.r0 + rr, c = q.c0 + cc;
-    const bool in = r < a.rows && c < a.cols;
-    const uint8_t* src = in ? a.src + ((q.g * a.rows + r) * a.cols + c) * 2 : a.src;
-    cp_async16(&tile[rr * QC_PITCH + cc], src, in ? 16u : 0u);  // zero fill outside the matrix
+  const int cc = (tid & 15) * 8;
+  const int64_t c = q.c0 + cc;
+  int64_t src_row[QC_TILE / 16];
+  bool in[QC_TILE / 16];
+#pragma unroll
+  for (int j = 0; j < QC_TILE / 16; ++j) {
+    const int64_t r = q.r0 + (tid >> 4) + 16 * j;
+    in[j] = r < a.rows && c < a.cols;
+    src_row[j] = q.g * a.rows + r;
+  }
+  if (a.row_map) {
+    int32_t m[QC_TILE / 16];
+#pragma unroll
+    for (int j = 0; j < QC_TILE / 16; ++j) m[j] = in[j] ? __ldg(a.row_map + src_row[j]) : -1;
+#pragma unroll
+    for (int j = 0; j < QC_TILE / 16; ++j) {
+      in[j] = m[j] >= 0;
+      src_row[j] = m[j] >= 0 ? int64_t(fastdiv(uint32_t(m[j]), a.div)) : 0;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < QC_TILE / 16; ++j) {
+    const int rr = (tid >> 4) + 16 * j;
+    const uint8_t* src = in[j] ? a.src + (src_row[j] * a.cols + c) * 2 : a.src;
+    cp_async16(&tile[rr * QC_PITCH + cc], src, in[j] ? 16u : 0u);  // zero fill outside the matrix
   }
 }
 
@@ -370,8 +392,10 @@ cudaError_t launch_quant_rows(const QuantRowsArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_both(const QuantBothArgs& a, cudaStream_t st) {
-  if (a.rows == 0 || a.cols == 0 || a.groups == 0) return cudaSuccess;
+cudaError_t launch_quant_both(const QuantBothArgs& args, cudaStream_t st) {
+  if (args.rows == 0 || args.cols == 0 || args.groups == 0) return cudaSuccess;
+  QuantBothArgs a = args;
+  a.div = make_fastdiv(uint32_t(a.map_div > 0 ? a.map_div : 1));
   if (a.row_split % 128) {
     // row-groups whose last 128-row tile is partial own padding scale bytes
     // that no source row maps to: clear the row-mode scales first

@@ -37,7 +37,9 @@ cudaError_t launch_quant_cols(const QuantColsArgs& a, cudaStream_t st);
 
 namespace moe {
 
-// Both modes from one read of the source: input [groups][rows][cols] bf16.
+// Both modes from one read of the source: input [groups][rows][cols] bf16,
+// or, with row_map, input row (g*rows + r) = source row
+// row_map[g*rows + r] / map_div (a negative entry gives a zero row).
 //  row mode output: MX tensor whose groups split each input group into
 //    rows / row_split row-groups of row_split rows (W_gate_up: gate and up
 //    halves) -- q_row [groups*rows][cols], sf_row blocked
@@ -52,6 +54,9 @@ struct QuantBothArgs {
   uint8_t* sf_row;
   uint8_t* q_col;
   uint8_t* sf_col;
+  const int32_t* row_map = nullptr;  // optional gather map
+  int32_t map_div = 1;
+  FastDiv div;                        // map_div as a multiply-high (set by the launcher)
 };
 
 cudaError_t launch_quant_both(const QuantBothArgs& a, cudaStream_t st);
