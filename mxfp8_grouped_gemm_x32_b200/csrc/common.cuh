@@ -45,18 +45,21 @@ __device__ __forceinline__ float abs_max(float a, float b) {
   return d;
 }
 
-// max |v[i]| over N values (N a power of two), as a balanced tree.
+// max(|a|, |b|, |c|), NaN if any is NaN (three-input form: two new values
+// per instruction).
+__device__ __forceinline__ float abs_max3(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
+  return d;
+}
+
+// max |v[i]| over N values (N even, N >= 4).
 template <int N>
 __device__ __forceinline__ float abs_max_n(const float* v) {
-  float m[N / 2];
+  float m = abs_max3(v[0], v[1], v[2]);
 #pragma unroll
-  for (int i = 0; i < N / 2; ++i) m[i] = abs_max(v[2 * i], v[2 * i + 1]);
-#pragma unroll
-  for (int w = N / 4; w >= 1; w /= 2) {
-#pragma unroll
-    for (int i = 0; i < w; ++i) m[i] = abs_max(m[2 * i], m[2 * i + 1]);
-  }
-  return m[0];
+  for (int i = 3; i + 1 < N; i += 2) m = abs_max3(m, v[i], v[i + 1]);
+  return abs_max(m, v[N - 1]);
 }
 
 // E8M0 scale byte from the bit pattern of a block's amax (|.| bits of an
@@ -85,14 +88,15 @@ __device__ __forceinline__ float inv_scale_from_e8m0(uint32_t b) {
 
 // Two fp32 -> packed E4M3x2 (round to nearest even, saturating to +-448).
 // The low byte holds `lo`.
-__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
+// Four codes in one word (a in the low byte): the two 16-bit conversions are
+// assembled in place rather than widened, shifted and or-ed.
 __device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float d) {
-  return uint32_t(cvt_e4m3x2(a, b)) | (uint32_t(cvt_e4m3x2(c, d)) << 16);
+  uint32_t r;
+  asm("{\n .reg .b16 lo, hi;\n cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n"
+      " cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n mov.b32 %0, {lo, hi};\n}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
 }
 
 // Byte offset of the scale of (group g, row r, 32-block kb) in the blocked

@@ -171,16 +171,16 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
       // h in place of the gate values of this block
-      uint32_t am = 0;
+      float am = 0.0f;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float g = __uint_as_float(v[32 * b + j]);
         const float u = __uint_as_float(v[64 + 32 * b + j]);
         const float h = p * __fdividef(g, 1.0f + __expf(-g)) * u;
         v[32 * b + j] = __float_as_uint(h);
-        am = max(am, __float_as_uint(h) & 0x7FFFFFFFu);
+        am = abs_max(am, h);
       }
-      const uint32_t sb = e8m0_from_amax_bits(am);
+      const uint32_t sb = e8m0_from_amax_bits(__float_as_uint(am));
       const float inv = inv_scale_from_e8m0(sb);
 #pragma unroll
       for (int j = 0; j < 8; ++j)

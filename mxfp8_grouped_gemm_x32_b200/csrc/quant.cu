@@ -54,28 +54,29 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantRowsArgs a) {
     uint32_t word = 0;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      if (b >= nblk) break;
-      uint4 v[4];
+      if (b < nblk) {
+        uint4 v[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = __ldg(s + 4 * b + j);
-      float f[32];
+        for (int j = 0; j < 4; ++j) v[j] = __ldg(s + 4 * b + j);
+        float f[32];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        f[8 * j + 0] = bf16lo(v[j].x); f[8 * j + 1] = bf16hi(v[j].x);
-        f[8 * j + 2] = bf16lo(v[j].y); f[8 * j + 3] = bf16hi(v[j].y);
-        f[8 * j + 4] = bf16lo(v[j].z); f[8 * j + 5] = bf16hi(v[j].z);
-        f[8 * j + 6] = bf16lo(v[j].w); f[8 * j + 7] = bf16hi(v[j].w);
+        for (int j = 0; j < 4; ++j) {
+          f[8 * j + 0] = bf16lo(v[j].x); f[8 * j + 1] = bf16hi(v[j].x);
+          f[8 * j + 2] = bf16lo(v[j].y); f[8 * j + 3] = bf16hi(v[j].y);
+          f[8 * j + 4] = bf16lo(v[j].z); f[8 * j + 5] = bf16hi(v[j].z);
+          f[8 * j + 6] = bf16lo(v[j].w); f[8 * j + 7] = bf16hi(v[j].w);
+        }
+        const uint32_t sb = e8m0_from_amax_bits(__float_as_uint(abs_max_n<32>(f)));
+        const float inv = inv_scale_from_e8m0(sb);
+        uint32_t c[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          c[j] = pack4_e4m3(f[4 * j] * inv, f[4 * j + 1] * inv, f[4 * j + 2] * inv, f[4 * j + 3] * inv);
+        uint4* d = reinterpret_cast<uint4*>(qrow + 32 * b);
+        d[0] = make_uint4(c[0], c[1], c[2], c[3]);
+        d[1] = make_uint4(c[4], c[5], c[6], c[7]);
+        word |= sb << (8 * b);
       }
-      const uint32_t sb = e8m0_from_amax_bits(__float_as_uint(abs_max_n<32>(f)));
-      const float inv = inv_scale_from_e8m0(sb);
-      uint32_t c[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        c[j] = pack4_e4m3(f[4 * j] * inv, f[4 * j + 1] * inv, f[4 * j + 2] * inv, f[4 * j + 3] * inv);
-      uint4* d = reinterpret_cast<uint4*>(qrow + 32 * b);
-      d[0] = make_uint4(c[0], c[1], c[2], c[3]);
-      d[1] = make_uint4(c[4], c[5], c[6], c[7]);
-      word |= sb << (8 * b);
     }
     *sfw = word;
   }
@@ -179,12 +180,15 @@ struct QbTile {
   int64_t g, r0, c0;
 };
 
-__device__ __forceinline__ QbTile qb_tile(const QuantBothArgs& a, int64_t t, int64_t rt, int64_t ct) {
+// Tile t -> (group, first row, first column), 32-bit multiply-high divisions.
+__device__ __forceinline__ QbTile qb_tile(const QuantBothArgs& a, uint32_t t) {
   QbTile q;
-  q.g = t / (rt * ct);
-  const int64_t rem = t - q.g * rt * ct;
-  q.r0 = (rem / ct) * QC_TILE;
-  q.c0 = (rem % ct) * QC_TILE;
+  const uint32_t g = fastdiv(t, a.tpg_div);
+  const uint32_t rem = t - g * a.tiles_per_group;
+  const uint32_t rt = fastdiv(rem, a.ct_div);
+  q.g = g;
+  q.r0 = int64_t(rt) * QC_TILE;
+  q.c0 = int64_t(rem - rt * a.ct) * QC_TILE;
   return q;
 }
 
@@ -265,8 +269,9 @@ __device__ __forceinline__ void qb_compute(const QuantBothArgs& a, const QbTile&
         sbs |= sb << (8 * b);
       }
       if (!row_atom) {  // the tile spans two row-groups: scale bytes one by one
-        const int64_t rg = g * (a.rows / a.row_split) + r / a.row_split;
-        const int64_t rr = r % a.row_split;
+        const uint32_t rq = fastdiv(uint32_t(r), a.rs_div);
+        const int64_t rg = g * a.row_groups + rq;
+        const int64_t rr = r - int64_t(rq) * a.row_split;
         *reinterpret_cast<uint16_t*>(a.sf_row + sf_offset(rg, rr, c0 / 32 + 2 * hb, cdiv(a.row_split, 128),
                                                           cdiv(a.cols, 128))) = uint16_t(sbs);
       }
@@ -316,29 +321,32 @@ __device__ __forceinline__ void qb_compute(const QuantBothArgs& a, const QbTile&
 // store instruction covers 4 rows x 128 contiguous bytes.
 __device__ __forceinline__ void qb_store(const QuantBothArgs& a, const QbTile& q, const uint8_t* out_row,
                                          const uint8_t* out_col, const uint8_t* atoms, bool row_atom,
-                                         int64_t rt, int64_t ct, int tid) {
+                                         int tid) {
   const int chunk = tid & 7;
+  uint8_t* const qr = a.q_row + (q.g * a.rows + q.r0) * a.cols + q.c0 + 16 * chunk;
+  uint8_t* const qc = a.q_col + (q.g * a.cols + q.c0) * a.rows + q.r0 + 16 * chunk;
   const int64_t vrow_bytes = a.cols - q.c0 < 128 ? a.cols - q.c0 : 128;  // valid codes of a row-mode row
   const int64_t vcol_bytes = a.rows - q.r0 < 128 ? a.rows - q.r0 : 128;  // valid codes of a column-mode row
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int rr = (tid >> 3) + 32 * i;
     if (q.r0 + rr < a.rows && 16 * chunk < vrow_bytes)
-      *reinterpret_cast<uint4*>(a.q_row + (q.g * a.rows + q.r0 + rr) * a.cols + q.c0 + 16 * chunk) =
+      *reinterpret_cast<uint4*>(qr + int64_t(rr) * a.cols) =
           *reinterpret_cast<const uint4*>(out_row + rr * QB_OUT_PITCH + 16 * chunk);
     if (q.c0 + rr < a.cols && 16 * chunk < vcol_bytes)
-      *reinterpret_cast<uint4*>(a.q_col + (q.g * a.cols + q.c0 + rr) * a.rows + q.r0 + 16 * chunk) =
+      *reinterpret_cast<uint4*>(qc + int64_t(rr) * a.rows) =
           *reinterpret_cast<const uint4*>(out_col + rr * QB_OUT_PITCH + 16 * chunk);
   }
   if (tid < 32) {
     if (row_atom) {
-      const int64_t rg = q.g * (a.rows / a.row_split) + q.r0 / a.row_split;
-      const int64_t rr = q.r0 % a.row_split;
+      const uint32_t rq = fastdiv(uint32_t(q.r0), a.rs_div);
+      const int64_t rg = q.g * a.row_groups + rq;
+      const int64_t rr = q.r0 - int64_t(rq) * a.row_split;
       reinterpret_cast<uint4*>(a.sf_row + sf_offset(rg, rr, q.c0 / 32, cdiv(a.row_split, 128),
                                                     cdiv(a.cols, 128)))[tid] = reinterpret_cast<const uint4*>(atoms)[tid];
     }
   } else if (tid < 64) {
-    reinterpret_cast<uint4*>(a.sf_col + sf_offset(q.g, q.c0, q.r0 / 32, ct, rt))[tid - 32] =
+    reinterpret_cast<uint4*>(a.sf_col + sf_offset(q.g, q.c0, q.r0 / 32, cdiv(a.cols, QC_TILE), cdiv(a.rows, QC_TILE)))[tid - 32] =
         reinterpret_cast<const uint4*>(atoms + 512)[tid - 32];
   }
 }
@@ -349,24 +357,22 @@ __global__ void __launch_bounds__(256, 2) quant_both_kernel(QuantBothArgs a) {
   uint8_t* out_col = out_row + QB_OUT_BYTES;
   uint8_t* atoms = out_col + QB_OUT_BYTES;  // 1 KB
   const int tid = threadIdx.x;
-  const int64_t rt = cdiv(a.rows, QC_TILE), ct = cdiv(a.cols, QC_TILE);
-  const int64_t ntiles = int64_t(a.groups) * rt * ct;
   // whole row-mode atoms need row-groups of a multiple of 128 rows
   const bool row_atom = a.row_split % QC_TILE == 0;
-  int64_t t = blockIdx.x;
-  if (t >= ntiles) return;
-  qb_load(a, qb_tile(a, t, rt, ct), qb_smem, tid);
+  uint32_t t = blockIdx.x;
+  if (t >= a.ntiles) return;
+  qb_load(a, qb_tile(a, t), qb_smem, tid);
   cp_async_commit();
-  for (int it = 0; t < ntiles; ++it, t += gridDim.x) {
-    const int64_t tn = t + gridDim.x;
-    if (tn < ntiles) qb_load(a, qb_tile(a, tn, rt, ct), qb_smem + ((it + 1) & 1) * QB_TILE_ELEMS, tid);
+  for (int it = 0; t < a.ntiles; ++it, t += gridDim.x) {
+    const uint32_t tn = t + gridDim.x;
+    if (tn < a.ntiles) qb_load(a, qb_tile(a, tn), qb_smem + ((it + 1) & 1) * QB_TILE_ELEMS, tid);
     cp_async_commit();  // (possibly empty group: keeps the wait count uniform)
     cp_async_wait<1>();
     __syncthreads();
-    const QbTile q = qb_tile(a, t, rt, ct);
+    const QbTile q = qb_tile(a, t);
     qb_compute(a, q, qb_smem + (it & 1) * QB_TILE_ELEMS, out_row, out_col, atoms, row_atom, tid);
     __syncthreads();  // staging complete
-    qb_store(a, q, out_row, out_col, atoms, row_atom, rt, ct, tid);
+    qb_store(a, q, out_row, out_col, atoms, row_atom, tid);
     __syncthreads();  // staging and this input buffer are reused
   }
 }
@@ -396,6 +402,17 @@ cudaError_t launch_quant_both(const QuantBothArgs& args, cudaStream_t st) {
   if (args.rows == 0 || args.cols == 0 || args.groups == 0) return cudaSuccess;
   QuantBothArgs a = args;
   a.div = make_fastdiv(uint32_t(a.map_div > 0 ? a.map_div : 1));
+  const int64_t rt = cdiv(a.rows, QC_TILE), ct = cdiv(a.cols, QC_TILE);
+  const int64_t tiles = int64_t(a.groups) * rt * ct;
+  if (tiles >= (int64_t(1) << 31) - (int64_t(1) << 20)) return cudaErrorInvalidValue;  // 32-bit tile schedule
+  a.ct = uint32_t(ct);
+  a.tiles_per_group = uint32_t(rt * ct);
+  a.ntiles = uint32_t(tiles);
+  a.ct_div = make_fastdiv(a.ct);
+  a.tpg_div = make_fastdiv(a.tiles_per_group);
+  if (a.row_split <= 0 || a.row_split >= (int64_t(1) << 31) || a.rows >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  a.rs_div = make_fastdiv(uint32_t(a.row_split));
+  a.row_groups = uint32_t(a.rows / a.row_split);
   if (a.row_split % 128) {
     // row-groups whose last 128-row tile is partial own padding scale bytes
     // that no source row maps to: clear the row-mode scales first
@@ -411,9 +428,8 @@ cudaError_t launch_quant_both(const QuantBothArgs& args, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int64_t ntiles = int64_t(a.groups) * cdiv(a.rows, QC_TILE) * cdiv(a.cols, QC_TILE);
   int64_t grid = int64_t(num_sms()) * 2;
-  if (grid > ntiles) grid = ntiles;
+  if (grid > tiles) grid = tiles;
   quant_both_kernel<<<unsigned(grid), 256, smem, st>>>(a);
   count_launch();
   return cudaGetLastError();

@@ -57,6 +57,11 @@ struct QuantBothArgs {
   const int32_t* row_map = nullptr;  // optional gather map
   int32_t map_div = 1;
   FastDiv div;                        // map_div as a multiply-high (set by the launcher)
+  // tile schedule (set by the launcher): 128 x 128 tiles, columns fastest
+  uint32_t ct = 0, tiles_per_group = 0, ntiles = 0;
+  FastDiv ct_div, tpg_div;
+  FastDiv rs_div;                     // row_split
+  uint32_t row_groups = 0;            // rows / row_split
 };
 
 cudaError_t launch_quant_both(const QuantBothArgs& a, cudaStream_t st);

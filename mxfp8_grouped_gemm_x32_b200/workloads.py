@@ -76,6 +76,10 @@ CONFIGS = {
     "qwen3_30b_ragged": LayerConfig("qwen3_30b_ragged", T=16384, H=2048, I=768, E=128, k=8,
                                     expert_bias_std=1.5,
                                     note="Qwen3-MoE-30B-shaped, skewed routing"),
+    # Qwen3 shapes and routing with a quarter of the tokens: a profiler-sized
+    # slice of the ragged layer (about 32 rows per expert instead of 128)
+    "qwen3_profile": LayerConfig("qwen3_profile", T=4096, H=2048, I=768, E=128, k=8, expert_bias_std=1.5,
+                                 note="Qwen3-MoE-30B-shaped, skewed routing, T=4096"),
     "gpt_oss_20b": LayerConfig("gpt_oss_20b", T=8192, H=2880, I=2880, E=32, k=4,
                                router="topk_softmax",
                                note="GPT-OSS-20B-shaped, K=2880 not a multiple of 128"),
