@@ -104,35 +104,72 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, in
 }
 
 // Writes the warp's 32 rows (one per lane) of NW 32-bit words each to global
-// memory through the warp's shared staging buffer, 16 words (64 bytes) of
-// every row at a time, so that each global store instruction covers 8 rows x
-// 64 contiguous bytes instead of 32 rows x 16 bytes.  `row` is this lane's
+// memory through the warp's shared staging buffer.  `row` is this lane's
 // destination (nullptr: row not stored); only the first `bytes` bytes of a
 // row are stored (a multiple of 16).
+//  NW % 32 == 0: 32 words (128 bytes) of 16 rows at a time, so that each
+//    global store instruction writes 4 rows x 128 contiguous bytes (whole
+//    L2 lines wherever the row starts are 128-byte aligned, as they are for
+//    the layer shapes benchmarked here);
+//  NW == 16: 16 words of all 32 rows, 8 rows x 64 bytes per instruction.
+// The staged pitch (144 bytes, or 80 for 64-byte rows) keeps the 16-byte
+// shared stores and loads free of bank conflicts.
+constexpr int STAGE128_PITCH_W = 36;
+static_assert(16 * STAGE128_PITCH_W * 4 <= STAGE_WARP_BYTES, "staging buffer too small");
+
 template <int NW>
 __device__ __forceinline__ void warp_store_rows(uint32_t* stage, uint8_t* row, const uint32_t* w, int bytes,
                                                 int lane) {
   static_assert(NW % 16 == 0, "rows are staged 16 words at a time");
   const uint64_t rp = reinterpret_cast<uint64_t>(row);
+  if constexpr (NW % 32 == 0) {
+    const int piece = lane & 7;
 #pragma unroll
-  for (int c = 0; c < NW / 16; ++c) {
-    __syncwarp();
-    uint4* srow = reinterpret_cast<uint4*>(stage + lane * STAGE_PITCH_W);
+    for (int c = 0; c < NW / 32; ++c) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      srow[q] = make_uint4(w[16 * c + 4 * q], w[16 * c + 4 * q + 1], w[16 * c + 4 * q + 2], w[16 * c + 4 * q + 3]);
-    __syncwarp();
-    const int piece = lane & 3;
+      for (int hh = 0; hh < 2; ++hh) {
+        __syncwarp();
+        if ((lane >> 4) == hh) {
+          uint4* srow = reinterpret_cast<uint4*>(stage + (lane & 15) * STAGE128_PITCH_W);
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int rr = (lane >> 2) + 8 * it;
-      const uint64_t dst = __shfl_sync(0xFFFFFFFFu, rp, rr);
-      const int off = 64 * c + 16 * piece;
-      if (dst != 0 && off < bytes)
-        *reinterpret_cast<uint4*>(dst + off) =
-            *reinterpret_cast<const uint4*>(stage + rr * STAGE_PITCH_W + 4 * piece);
+          for (int q = 0; q < 8; ++q)
+            srow[q] = make_uint4(w[32 * c + 4 * q], w[32 * c + 4 * q + 1], w[32 * c + 4 * q + 2],
+                                 w[32 * c + 4 * q + 3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int rr = (lane >> 3) + 4 * it;  // staged row 0..15
+          const uint64_t dst = __shfl_sync(0xFFFFFFFFu, rp, 16 * hh + rr);
+          const int off = 128 * c + 16 * piece;
+          if (dst != 0 && off < bytes)
+            *reinterpret_cast<uint4*>(dst + off) =
+                *reinterpret_cast<const uint4*>(stage + rr * STAGE128_PITCH_W + 4 * piece);
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < NW / 16; ++c) {
+      __syncwarp();
+      uint4* srow = reinterpret_cast<uint4*>(stage + lane * STAGE_PITCH_W);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        srow[q] = make_uint4(w[16 * c + 4 * q], w[16 * c + 4 * q + 1], w[16 * c + 4 * q + 2], w[16 * c + 4 * q + 3]);
+      __syncwarp();
+      const int piece = lane & 3;
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int rr = (lane >> 2) + 8 * it;
+        const uint64_t dst = __shfl_sync(0xFFFFFFFFu, rp, rr);
+        const int off = 64 * c + 16 * piece;
+        if (dst != 0 && off < bytes)
+          *reinterpret_cast<uint4*>(dst + off) =
+              *reinterpret_cast<const uint4*>(stage + rr * STAGE_PITCH_W + 4 * piece);
+      }
     }
   }
+  __syncwarp();
 }
 
 // 2*NW fp32 values (as bits) -> NW bf16x2 words, in place at the front.
