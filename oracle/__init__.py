@@ -14,6 +14,10 @@ Sources (pages of "Efficient MoE Training for Biological Foundation Models"):
   weights, GroupedLinear(gate_up) -> ScaledSwiGLU -> GroupedLinear(down),
   with the routing probability applied inside ScaledSwiGLU.
 
+* The router (router.py): the pages show only where the routing weights
+  are consumed; softmax over the experts, the k largest kept (ties to the
+  lower id) and renormalised is the reading taken.
+
 Every reading the pages leave open (scale rounding, gate/up order, saved
 activations, backward quantisation directions, padding of ragged blocks) is
 stated at the function that takes it.
@@ -22,8 +26,9 @@ Pins (tests/test_oracle_*.py): the codec against brute force and library
 casts over every bf16 pattern; the forward against an independent
 restatement of the per-expert loop; an identity-weight expert against its
 closed form; the backward against central finite differences and the
-closed form of d(prob); invariants of the permutation and the codec.
+closed form of d(prob); invariants of the permutation and the codec; the
+router against brute force over expert subsets, its closed form and torch.
 Parity unpinned: bit-level agreement of the scale rule with NVIDIA
 Transformer Engine (not available here).
 """
-from . import mxfp8, moe  # noqa: F401
+from . import mxfp8, moe, router  # noqa: F401
