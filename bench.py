@@ -368,6 +368,19 @@ def run_ours(args):
     barrier()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     value_e2e = world * flops / (ms_e2e * 1e-3) / 1e12
+    # router (moe_router_topk): reported beside the step, which starts from
+    # top-k routing; fp32 logits of the workload's shape
+    glog = torch.Generator(device=dev)
+    glog.manual_seed(args.seed + 7)
+    logits = torch.randn(cfg.T, cfg.E, generator=glog, device=dev)
+    for _ in range(3):
+        layer.route(logits)
+    e0.record(stream)
+    for _ in range(20):
+        layer.route(logits)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    router_ms = e0.elapsed_time(e1) / 20
     st = layer.device_status()
     if st != 0:
         raise SystemExit(f"device status after timing: {lib.status_string(st)}")
@@ -414,6 +427,8 @@ def run_ours(args):
         "fwd_tflops": cfg.fwd_flops() / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,
         "bwd_tflops": cfg.bwd_flops() / (bwd_ms * 1e-3) / 1e12 if bwd_ms else None,
         "kernels": kernels,
+        "router": {"ms_per_call": router_ms, "in_step": False,
+                   "what": "moe_router_topk on fp32 logits [T, E] (softmax, top-k, renormalise)"},
         "roofline": roofline,
         "clocks": clocks,
         "e2e": {"value": value_e2e, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -74,6 +74,10 @@ typedef enum {
 #define MOE_QUANT_ROW 1 /* quantise along the last axis (cols) */
 #define MOE_QUANT_COL 2 /* quantise along rows, store transposed */
 
+/* Element types of moe_router_topk's logits. */
+#define MOE_DTYPE_F32 0
+#define MOE_DTYPE_BF16 1
+
 /* Workspace sizes for moe_workspace_size(op, ...). */
 #define MOE_OP_PERMUTE 1
 #define MOE_OP_FWD 2
@@ -219,6 +223,22 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
  *   summed in fp32, j ascending. */
 moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* out,
                          moe_stream_t stream);
+
+/* Router: the inputs of moe_permute from router logits.  The pages show the
+ * routing weights only where the per-expert loop scales each expert's output
+ * (Challenge 1); reading taken: softmax over the E experts, the k largest
+ * kept in descending order (ties to the lower expert id), renormalised --
+ * equal to a softmax over the k kept logits, so the selection compares
+ * logits exactly.
+ *   logits      device [T][E], fp32 (MOE_DTYPE_F32) or bf16 (MOE_DTYPE_BF16);
+ *               NaN ranks as -inf; rows whose kept logits include +inf or
+ *               are all -inf get NaN probabilities
+ *   topk_idx    device int32 [T][k] (written), expert ids, descending logit
+ *   topk_prob   device fp32 [T][k] (written), exp(l_j - l_0) / sum over kept
+ * Limits: 1 <= k <= E <= 256 and k <= 32 (MOE_ERR_UNSUPPORTED otherwise).
+ * No allocation, no workspace; asynchronous on `stream`. */
+moe_status_t moe_router_topk(const void* logits, int32_t logits_dtype, int32_t T, int32_t E, int32_t k,
+                             int32_t* topk_idx, float* topk_prob, moe_stream_t stream);
 
 /* ----------------------------------------------------------- backward --- */
 

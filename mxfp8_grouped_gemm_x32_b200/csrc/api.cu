@@ -10,6 +10,7 @@
 #include "permute.cuh"
 #include "quant.cuh"
 #include "swiglu_bwd.cuh"
+#include "router.cuh"
 
 namespace moe {
 
@@ -427,6 +428,18 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   }
   (void)slot_to_row;
   return MOE_OK;
+}
+
+moe_status_t moe_router_topk(const void* logits, int32_t logits_dtype, int32_t T, int32_t E, int32_t k,
+                             int32_t* topk_idx, float* topk_prob, moe_stream_t stream) {
+  if (!logits || !topk_idx || !topk_prob || T < 0) return MOE_ERR_INVALID;
+  if (logits_dtype != MOE_DTYPE_F32 && logits_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID;
+  if (E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID;
+  if (E > MOE_MAX_EXPERTS || k > 32) return MOE_ERR_UNSUPPORTED;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  TimeScope ts(st, "router");
+  return cuda_status(launch_router_topk(logits, logits_dtype == MOE_DTYPE_BF16, T, E, k, topk_idx, topk_prob, st));
 }
 
 moe_status_t moe_get_device_status(moe_stream_t stream) {

@@ -6,3 +6,4 @@
 #include "quant.cu"
 #include "swiglu_bwd.cu"
 #include "noalloc.cu"
+#include "router.cu"

@@ -6,6 +6,7 @@ Steps (names of the C entry points):
   quantize_weights  moe_mlp_quantize_weights: W_gate_up and W_down, along K
                     for the forward and along the other axis for the backward
                     (forward only: moe_mlp_quantize_mxfp8 x2)
+  route             moe_router_topk: router logits -> top-k experts + probabilities
   permute           moe_permute: counting sort by expert, gather + quantise x
   forward           moe_grouped_mlp_fwd: gate_up GEMM + ScaledSwiGLU + requant,
                     down GEMM, top-k combine
@@ -93,6 +94,18 @@ class GroupedMLP:
             return
         lib.moe_mlp_quantize_mxfp8(w1.data_ptr(), 2 * E, I, H, lib.MOE_QUANT_ROW, _ptr(self.w1q), _ptr(self.w1sf), s)
         lib.moe_mlp_quantize_mxfp8(w2.data_ptr(), E, H, I, lib.MOE_QUANT_ROW, _ptr(self.w2q), _ptr(self.w2sf), s)
+
+    def route(self, logits: torch.Tensor):
+        """Router logits fp32 or bf16 [T, E] -> (topk_idx int32 [T, k],
+        topk_prob float32 [T, k]) in this layer's routing buffers."""
+        assert logits.is_contiguous() and logits.shape == (self.T, self.E)
+        dt = {torch.float32: lib.MOE_DTYPE_F32, torch.bfloat16: lib.MOE_DTYPE_BF16}[logits.dtype]
+        if not hasattr(self, "topk_idx"):
+            self.topk_idx = torch.empty(self.T, self.k, dtype=torch.int32, device=self.dev)
+            self.topk_prob = torch.empty(self.T, self.k, dtype=torch.float32, device=self.dev)
+        lib.moe_router_topk(logits.data_ptr(), dt, self.T, self.E, self.k, _ptr(self.topk_idx),
+                            _ptr(self.topk_prob), self._stream())
+        return self.topk_idx, self.topk_prob
 
     def permute(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_prob: torch.Tensor) -> None:
         """x bf16 [T, H]; topk_idx int32 [T, k]; topk_prob float32 [T, k]."""

@@ -34,7 +34,9 @@ EXPORTED = [
     "moe_permute", "moe_grouped_mlp_fwd", "moe_combine", "moe_grouped_mlp_bwd",
     "moe_get_device_status", "moe_status_string", "moe_launch_count", "moe_selftest_wait_timeout",
     "moe_timing_enable", "moe_timing_read", "moe_permute_noalloc", "moe_mlp_quantize_weights",
+    "moe_router_topk",
 ]
+MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 
 
 class MoeError(RuntimeError):
@@ -71,6 +73,7 @@ _decl("moe_permute", _I32, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _P, _P, _P,
 _decl("moe_grouped_mlp_fwd", _I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P,
       _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
 _decl("moe_combine", _I32, _P, _I32, _I32, _I32, _P, _P)
+_decl("moe_router_topk", _I32, _P, _I32, _I32, _I32, _I32, _P, _P, _P)
 _decl("moe_grouped_mlp_bwd", _I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P,
       _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
 _decl("moe_get_device_status", _I32, _P)
@@ -141,6 +144,10 @@ def moe_grouped_mlp_fwd(w1q, w1sf, w2q, w2sf, T, H, I, E, k, rows_cap, split_siz
 
 def moe_combine(y, T, k, H, out, stream=0):
     _check("moe_combine", _lib.moe_combine(y, T, k, H, out, stream))
+
+
+def moe_router_topk(logits, logits_dtype, T, E, k, topk_idx, topk_prob, stream=0):
+    _check("moe_router_topk", _lib.moe_router_topk(logits, logits_dtype, T, E, k, topk_idx, topk_prob, stream))
 
 
 def moe_grouped_mlp_bwd(w2tq, w2tsf, w1tq, w1tsf, T, H, I, E, k, rows_cap, split_sizes, group_offsets,

@@ -3,9 +3,10 @@
 This module is shared by the CUDA path's tests and benchmark and by the CPU
 oracle's tests.  It holds only the input recipe: random draws, rounding of
 those draws to bf16 (the storage format of every input tensor), and the
-router that turns logits into per-token top-k expert ids and probabilities.
-It contains none of the layer's own arithmetic (no quantisation, no GEMM, no
-activation).
+routing used to synthesise the expert MLP's top-k inputs.  It contains none
+of the expert MLP's arithmetic (no quantisation, no GEMM, no activation).
+The router step itself (moe_router_topk) is checked against its own oracle
+(oracle/router.py) on the raw `router_logits`; neither side uses `route`.
 
 Recipe (the workloads of "Efficient MoE Training for Biological Foundation
 Models", Challenge 1-3, and the MoE table of the NeMo Automodel page, with the
@@ -181,6 +182,7 @@ def make_inputs(cfg: LayerConfig, seed: int = 0, *, weights: bool = True,
       w1     uint16 bf16 bits [E, 2I, H]   (gate rows 0..I-1, up rows I..2I-1)
       w2     uint16 bf16 bits [E, H, I]
       topk_idx int32 [T, k], topk_prob float32 [T, k]
+      router_logits float32 [T, E]           (the logits the routing was drawn from)
       dy     uint16 bf16 bits [T, H]        (when grad)
     ``topk_idx`` may be given to force a routing pattern (edge cases); the
     probabilities are then drawn from the same router over those experts.
@@ -193,6 +195,7 @@ def make_inputs(cfg: LayerConfig, seed: int = 0, *, weights: bool = True,
     logits = _normal_f32(seed, _S_LOGITS, T * E, 1.0).reshape(T, E).astype(np.float64)
     if cfg.expert_bias_std:
         logits = logits + _normal_f32(seed, _S_BIAS, E, cfg.expert_bias_std).astype(np.float64)[None, :]
+    out["router_logits"] = logits.astype(np.float32)
     if topk_idx is None:
         idx, prob = route(logits, k, cfg.router)
     else:

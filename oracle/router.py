@@ -14,8 +14,9 @@ the plainest one consistent with the Mixtral model the pages benchmark:
 Because the renormalisation divides out the softmax denominator, the kept
 probabilities equal a softmax over the k kept logits, and the selection only
 compares logits (softmax is strictly increasing).  A NaN logit ranks below
-every number.  This module follows the definition step by step (softmax
-first); the tests pin it against the reduced forms.
+every number (as -inf).  A row whose kept logits include +inf, or are all
+-inf, has no defined probabilities (NaN).  This module follows the definition
+step by step (softmax first); the tests pin it against the reduced forms.
 """
 from __future__ import annotations
 
@@ -29,14 +30,15 @@ def route_topk(logits: np.ndarray, k: int):
     if not 1 <= k <= E:
         raise ValueError("need 1 <= k <= E")
     key = np.where(np.isnan(lg), -np.inf, lg)
-    # softmax over all experts (finite rows; a row of -inf keeps equal weights)
-    m = key.max(axis=1, keepdims=True)
-    m = np.where(np.isfinite(m), m, 0.0)
-    p = np.exp(key - m)
-    p = p / p.sum(axis=1, keepdims=True)
+    # softmax over all experts, shifted by the row maximum
+    with np.errstate(invalid="ignore"):
+        m = key.max(axis=1, keepdims=True)
+        p = np.exp(key - m)
+        p = p / p.sum(axis=1, keepdims=True)
     # k largest, descending, ties to the lower id: a stable sort of -key
     # (ranking the logits ranks the probabilities, and keeps ties exact)
     order = np.argsort(-key, axis=1, kind="stable")[:, :k]
     top = np.take_along_axis(p, order, axis=1)
-    top = top / top.sum(axis=1, keepdims=True)
+    with np.errstate(invalid="ignore"):
+        top = top / top.sum(axis=1, keepdims=True)
     return order.astype(np.int32), top

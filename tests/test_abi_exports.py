@@ -53,3 +53,15 @@ def test_host_side_argument_errors():
     assert lib._lib.moe_mlp_quantize_mxfp8(None, 1, 32, 32, 1, None, None, None) == 1
     assert lib._lib.moe_combine(None, 1, 1, 8, None, None) == 1
     assert lib.status_string(6).startswith("device: bounded")
+
+
+def test_router_argument_errors():
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    f = lib._lib.moe_router_topk
+    p = 16  # a non-null dummy pointer: every case below is rejected before it is used
+    assert f(None, 0, 4, 8, 2, p, p, None) == 1            # null logits
+    assert f(p, 2, 4, 8, 2, p, p, None) == 1               # unknown dtype
+    assert f(p, 0, 4, 8, 9, p, p, None) == 1               # k > E
+    assert f(p, 0, 4, 8, 0, p, p, None) == 1               # k = 0
+    assert f(p, 0, 4, 300, 2, p, p, None) == 2             # E > 256
+    assert f(p, 0, 4, 64, 33, p, p, None) == 2             # k > 32
