@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-library-probe", action="store_true",
+                    help="skip the dense MXFP8 GEMM rate of the CUDA library (context for the roofline)")
     return ap.parse_args(argv)
 
 
@@ -92,6 +94,48 @@ def load_peaks(path=os.path.join(ROOT, "MEASURED_PEAKS.json")):
         return {"mxfp8_burst": FALLBACK_BF16_TFLOPS * MXFP8_OVER_BF16,
                 "mxfp8_sustained": 1400.0 * MXFP8_OVER_BF16, "hbm_gbs": FALLBACK_HBM_GBS,
                 "source": "fallback"}
+
+
+def mxfp8_library_probe(torch, dev, seconds: float = 3.0):
+    """Dense MXFP8 GEMM rate of the CUDA library on this GPU (torch scaled_mm,
+    1x32 block scales, 8192^3): best of 10 (burst) and a seconds-long loop
+    (sustained, under the power cap).  Context for the roofline only -- it is
+    not on the measured path.  None when the library does not offer it."""
+    try:
+        import torch.nn.functional as F
+        M = N = K = 8192
+        a = torch.randn(M, K, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(N, K, device=dev).to(torch.float8_e4m3fn)
+        sa = torch.full((M * K // 32,), 127, dtype=torch.uint8, device=dev).view(torch.float8_e8m0fnu)
+        sb = torch.full((N * K // 32,), 127, dtype=torch.uint8, device=dev).view(torch.float8_e8m0fnu)
+        bw, sw = F.ScalingType.BlockWise1x32, F.SwizzleType.SWIZZLE_32_4_4
+
+        def run():
+            return F.scaled_mm(a, b.t(), sa, bw, sb, bw, swizzle_a=sw, swizzle_b=sw, output_dtype=torch.bfloat16)
+        run()
+        torch.cuda.synchronize()
+        best = float("inf")
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(10):
+            e0.record()
+            run()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        n, t0 = 0, time.time()
+        e0.record()
+        while time.time() - t0 < seconds:
+            for _ in range(20):
+                run()
+            n += 20
+            torch.cuda.synchronize()
+        e1.record()
+        torch.cuda.synchronize()
+        fl = 2.0 * M * N * K
+        return {"what": "torch scaled_mm (cuBLAS) dense MXFP8 8192^3, 1x32 E8M0 scales",
+                "burst_tflops": fl / best / 1e9, "sustained_tflops": fl / (e0.elapsed_time(e1) / n) / 1e9}
+    except Exception as exc:  # library without MXFP8 scaled_mm
+        return {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
 
 
 def gemm_source_sha() -> str:
@@ -463,6 +507,11 @@ def run_ours(args):
                 "pipeline": "copy stream: inputs of step i+1 in, results of step i out, while step i+1 computes"},
         "gpu_launches": launches,
     }
+    if not args.no_library_probe:
+        probe = mxfp8_library_probe(torch, dev)
+        line["mxfp8_library_probe"] = probe
+        if "sustained_tflops" in probe and roofline:
+            roofline["frac_of_library_sustained"] = roofline["achieved"] / probe["sustained_tflops"]
     if world == 1 and not args.no_cpu_baseline:
         dt, fl, desc = oracle_sample(cfg, 256, args.seed, 4)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),

@@ -26,9 +26,11 @@
 // and leave as whole 512-byte atoms (16-bit pairs / 32-bit words on ragged
 // edges).  dprob is summed per 128-column chunk in a fixed order into a
 // partial buffer and reduced over the chunks by swiglu_dprob_kernel.
-// (Measured on B200: issuing the next slice's loads before the column pass,
-// a persistent grid and packed fp32x2 arithmetic each cost more issue slots
-// than they saved.)
+// Three CTAs per SM (80 registers, 54 KB of shared memory each): 24 warps
+// hide more latency than 16 at 128 registers; four CTAs (64 registers) lose
+// more to spilled work than they gain.  (Also measured on B200 and rejected:
+// issuing the next slice's loads before the column pass, a persistent grid
+// and packed fp32x2 arithmetic each cost more issue slots than they saved.)
 #include "swiglu_bwd.cuh"
 
 namespace moe {
@@ -105,7 +107,7 @@ __device__ __forceinline__ uint32_t word4(const uint4& v, int i) {
   return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
-__global__ void __launch_bounds__(SB_THREADS, 2) swiglu_bwd_kernel(SwigluBwdArgs a) {
+__global__ void __launch_bounds__(SB_THREADS, 3) swiglu_bwd_kernel(SwigluBwdArgs a) {
   extern __shared__ __align__(16) uint8_t sb_raw[];
   SwigluSmem& sm = *reinterpret_cast<SwigluSmem*>(sb_raw);
   const int64_t r0 = int64_t(blockIdx.x) * SB_TILE;
