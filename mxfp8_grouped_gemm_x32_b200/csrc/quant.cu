@@ -149,10 +149,11 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(QuantColsArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Both modes from one read.  Persistent CTAs walk 128-row x 128-column tiles
-// of the source; each tile is brought into shared memory with cp.async while
-// the previous one is quantised (two buffers), so the loads of the next tile
-// overlap the arithmetic and stores of this one.  For a staged tile, thread t
+// Both modes from one read.  Persistent CTAs (three per SM, 73 KB of shared
+// memory each) walk 128-row x 128-column tiles of the source; a tile comes
+// into shared memory with cp.async, and the next tile's copies are issued as
+// soon as this one has been read, so they overlap its stores and the other
+// CTAs' arithmetic.  For a staged tile, thread t
 // quantises
 //   row mode: row t%128, column blocks 2*(t/128), +1 -> 64 code bytes and
 //             two scale bytes of that row;
@@ -351,29 +352,27 @@ __device__ __forceinline__ void qb_store(const QuantBothArgs& a, const QbTile& q
   }
 }
 
-__global__ void __launch_bounds__(256, 2) quant_both_kernel(QuantBothArgs a) {
+__global__ void __launch_bounds__(256, 3) quant_both_kernel(QuantBothArgs a) {
   extern __shared__ __align__(16) uint16_t qb_smem[];
-  uint8_t* out_row = reinterpret_cast<uint8_t*>(qb_smem + 2 * QB_TILE_ELEMS);
+  uint8_t* out_row = reinterpret_cast<uint8_t*>(qb_smem + QB_TILE_ELEMS);
   uint8_t* out_col = out_row + QB_OUT_BYTES;
   uint8_t* atoms = out_col + QB_OUT_BYTES;  // 1 KB
   const int tid = threadIdx.x;
-  // whole row-mode atoms need row-groups of a multiple of 128 rows
   const bool row_atom = a.row_split % QC_TILE == 0;
   uint32_t t = blockIdx.x;
   if (t >= a.ntiles) return;
   qb_load(a, qb_tile(a, t), qb_smem, tid);
   cp_async_commit();
-  for (int it = 0; t < a.ntiles; ++it, t += gridDim.x) {
-    const uint32_t tn = t + gridDim.x;
-    if (tn < a.ntiles) qb_load(a, qb_tile(a, tn), qb_smem + ((it + 1) & 1) * QB_TILE_ELEMS, tid);
-    cp_async_commit();  // (possibly empty group: keeps the wait count uniform)
-    cp_async_wait<1>();
-    __syncthreads();
+  for (; t < a.ntiles; t += gridDim.x) {
+    cp_async_wait<0>();
+    __syncthreads();  // input landed; the previous tile's staging has been stored
     const QbTile q = qb_tile(a, t);
-    qb_compute(a, q, qb_smem + (it & 1) * QB_TILE_ELEMS, out_row, out_col, atoms, row_atom, tid);
-    __syncthreads();  // staging complete
+    qb_compute(a, q, qb_smem, out_row, out_col, atoms, row_atom, tid);
+    __syncthreads();  // staging complete, input buffer free
+    const uint32_t tn = t + gridDim.x;
+    if (tn < a.ntiles) qb_load(a, qb_tile(a, tn), qb_smem, tid);
+    cp_async_commit();
     qb_store(a, q, out_row, out_col, atoms, row_atom, tid);
-    __syncthreads();  // staging and this input buffer are reused
   }
 }
 
@@ -421,14 +420,14 @@ cudaError_t launch_quant_both(const QuantBothArgs& args, cudaStream_t st) {
     cudaError_t e = cudaMemsetAsync(a.sf_row, 0, size_t(n), st);
     if (e != cudaSuccess) return e;
   }
-  const size_t smem = 2 * QB_TILE_ELEMS * sizeof(uint16_t) + 2 * QB_OUT_BYTES + 1024;
+  const size_t smem = QB_TILE_ELEMS * sizeof(uint16_t) + 2 * QB_OUT_BYTES + 1024;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(quant_both_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  int64_t grid = int64_t(num_sms()) * 2;
+  int64_t grid = int64_t(num_sms()) * 3;
   if (grid > tiles) grid = tiles;
   quant_both_kernel<<<unsigned(grid), 256, smem, st>>>(a);
   count_launch();
