@@ -14,9 +14,7 @@
 // HBM-bound: 8 bytes read and 5 written per (row, intermediate channel), and
 // close to issue-bound, so the kernel keeps instructions per element low.  A
 // CTA owns a 128-row x 128-column tile (rows of one expert group: groups
-// start on multiples of 128); on entry it asks L2 to prefetch the tile's
-// inputs (bulk prefetch, one request per row segment), then walks the tile
-// in four 32-row slices.  In a slice, eight threads share a row, each with
+// start on multiples of 128) and walks it in four 32-row slices.  In a slice, eight threads share a row, each with
 // 16 contiguous columns: a 32-block of the row-wise quantisation spans two
 // threads (one shuffle), and the two write its codes as one 32-byte sector.
 // dg, du, h are staged in shared memory (fp32, 16-byte stores; rows 16..31
@@ -29,8 +27,9 @@
 // Three CTAs per SM (80 registers, 54 KB of shared memory each): 24 warps
 // hide more latency than 16 at 128 registers; four CTAs (64 registers) lose
 // more to spilled work than they gain.  (Also measured on B200 and rejected:
-// issuing the next slice's loads before the column pass, a persistent grid
-// and packed fp32x2 arithmetic each cost more issue slots than they saved.)
+// issuing the next slice's loads before the column pass, a persistent grid,
+// packed fp32x2 arithmetic, and at three CTAs per SM an L2 bulk prefetch of
+// the tile's inputs on entry: each cost more than it saved.)
 #include "swiglu_bwd.cuh"
 
 namespace moe {
@@ -49,10 +48,6 @@ struct SwigluSmem {
 
 __device__ __forceinline__ int vidx(int row, int col) {
   return row * SB_VPITCH + (row >= 16 ? 16 : 0) + col;
-}
-
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // 16 values -> 16 E4M3 codes scaled by inv (a power of two: the products are exact)
@@ -89,20 +84,6 @@ __device__ __forceinline__ void load_slice(SliceIn& in, const SwigluBwdArgs& a, 
   }
 }
 
-// L2 prefetch of a tile's inputs (routed rows only: padding rows are never read)
-__device__ __forceinline__ void prefetch_tile(const SwigluBwdArgs& a, int64_t r0, int c0, int tid, int I, int64_t I2) {
-  const int rr = tid & 127;
-  const int64_t r = r0 + rr;
-  if (a.row_to_slot[r] < 0) return;
-  const uint32_t width = uint32_t(min(SB_TILE, I - c0));
-  if (tid < SB_TILE) {
-    prefetch_l2(a.dh + (r * I + c0) * 4, width * 4);
-  } else {
-    prefetch_l2(a.saved + (r * I2 + c0) * 2, width * 2);
-    prefetch_l2(a.saved + (r * I2 + I + c0) * 2, width * 2);
-  }
-}
-
 __device__ __forceinline__ uint32_t word4(const uint4& v, int i) {
   return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
@@ -120,7 +101,6 @@ __global__ void __launch_bounds__(SB_THREADS, 3) swiglu_bwd_kernel(SwigluBwdArgs
   const int64_t KTt = a.rows_cap / 128;
   const int rl = warp * 4 + (lane & 3), t = lane >> 2;  // row in the slice, column group
   const int cs = 16 * t;
-  prefetch_tile(a, r0, c0, tid, I, I2);
   {
     if (tid < SB_TILE) {
       const bool ok = a.row_to_slot[r0 + tid] >= 0;
