@@ -10,7 +10,7 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
-    config.addinivalue_line("markers", "slow: full-size workload, minutes on a GPU box")
+    config.addinivalue_line("markers", "slow: full-size workload, minutes on a B200")
 
 
 @pytest.fixture(scope="session")
