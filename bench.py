@@ -497,6 +497,13 @@ def run_ours(args):
         "frac_of_mxfp8_peak": value / world / peaks["mxfp8_sustained"],
         "fwd_tflops": cfg.fwd_flops() / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,
         "bwd_tflops": cfg.bwd_flops() / (bwd_ms * 1e-3) / 1e12 if bwd_ms else None,
+        # the step without the weight quantisation (whose time is measured in
+        # the same run): a gradient-accumulation micro-step, where the MX
+        # weights of the optimizer step are reused
+        "excl_weight_quant": ({"value": world * flops / ((ms_max - kernels["quant_weights"]["ms_per_step"]) * 1e-3)
+                               / 1e12, "unit": "TFLOP/s",
+                               "ms_per_step": ms_max - kernels["quant_weights"]["ms_per_step"]}
+                              if "quant_weights" in kernels else None),
         "kernels": kernels,
         "router": {"ms_per_call": router_ms, "in_step": False,
                    "what": "moe_router_topk on fp32 logits [T, E] (softmax, top-k, renormalise)"},
@@ -510,8 +517,13 @@ def run_ours(args):
     if not args.no_library_probe:
         probe = mxfp8_library_probe(torch, dev)
         line["mxfp8_library_probe"] = probe
-        if "sustained_tflops" in probe and roofline:
-            roofline["frac_of_library_sustained"] = roofline["achieved"] / probe["sustained_tflops"]
+        if "sustained_tflops" in probe:
+            lib_s = probe["sustained_tflops"]
+            probe["frac"] = {"step": value / world / lib_s,
+                             "layer_fwd": (line["fwd_tflops"] or 0.0) / lib_s,
+                             "layer_bwd": (line["bwd_tflops"] or 0.0) / lib_s}
+            if roofline:
+                roofline["frac_of_library_sustained"] = roofline["achieved"] / lib_s
     if world == 1 and not args.no_cpu_baseline:
         dt, fl, desc = oracle_sample(cfg, 256, args.seed, 4)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
