@@ -16,16 +16,15 @@ namespace moe {
 // `rows` inside the last 128-row tile only get zero scale words.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quant_rows_kernel(QuantRowsArgs a) {
-  const int64_t units = cdiv(a.K, 128);
-  const int64_t rows_pad = cdiv(a.rows, 128) * 128;
-  const int64_t total = int64_t(a.groups) * rows_pad * units;
+  const uint32_t units = a.units_div.d;
+  const uint32_t rows_pad = a.rowpad_div.d;
+  const uint32_t total = uint32_t(a.groups) * rows_pad * units;  // < 2^31 (checked by the launcher)
   const int64_t RT = rows_pad / 128, KT = units;
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
-       i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t u = i % units;
-    const int64_t rr = i / units;
-    const int64_t g = rr / rows_pad;
-    const int64_t r = rr % rows_pad;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const uint32_t rr = fastdiv(i, a.units_div);
+    const int64_t u = i - rr * units;
+    const uint32_t g = fastdiv(rr, a.rowpad_div);
+    const int64_t r = rr - g * rows_pad;
     uint32_t* sfw = reinterpret_cast<uint32_t*>(a.sf + sf_offset(g, r, u * 4, RT, KT));
     if (r >= a.rows) {
       *sfw = 0u;
@@ -35,7 +34,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantRowsArgs a) {
     int64_t src_row = out_row;
     if (a.row_map) {
       const int32_t m = a.row_map[out_row];
-      src_row = m < 0 ? -1 : int64_t(m / a.map_div);
+      src_row = m < 0 ? -1 : int64_t(fastdiv(uint32_t(m), a.div));
     }
     const int64_t k0 = u * 128;
     const int64_t rem = (a.K - k0) / 32;
@@ -387,9 +386,14 @@ static int num_sms() {
   return n;
 }
 
-cudaError_t launch_quant_rows(const QuantRowsArgs& a, cudaStream_t st) {
-  const int64_t total = int64_t(a.groups) * cdiv(a.rows, 128) * 128 * cdiv(a.K, 128);
+cudaError_t launch_quant_rows(const QuantRowsArgs& args, cudaStream_t st) {
+  const int64_t total = int64_t(args.groups) * cdiv(args.rows, 128) * 128 * cdiv(args.K, 128);
   if (total == 0) return cudaSuccess;
+  if (total >= (int64_t(1) << 31) - (int64_t(1) << 24)) return cudaErrorInvalidValue;  // 32-bit unit schedule
+  QuantRowsArgs a = args;
+  a.units_div = make_fastdiv(uint32_t(cdiv(a.K, 128)));
+  a.rowpad_div = make_fastdiv(uint32_t(cdiv(a.rows, 128) * 128));
+  a.div = make_fastdiv(uint32_t(a.map_div > 0 ? a.map_div : 1));
   int64_t blocks = cdiv(total, 256);
   blocks = blocks > int64_t(num_sms()) * 16 ? int64_t(num_sms()) * 16 : blocks;
   quant_rows_kernel<<<unsigned(blocks), 256, 0, st>>>(a);

@@ -15,6 +15,8 @@ struct QuantRowsArgs {
   int64_t rows, K;
   uint8_t* q;   // [groups][rows][K]
   uint8_t* sf;  // blocked (groups, rows, K)
+  // unit schedule (set by the launcher): units of 128 values, 32-bit indices
+  FastDiv units_div, rowpad_div, div;
 };
 
 // Column mode: input [groups][rows][cols] (optional row gather as above),
