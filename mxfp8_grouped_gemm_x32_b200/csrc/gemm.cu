@@ -392,16 +392,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(acc_full, acc_it & 1u, abort_flag)) break;
       tc_fence_after();
       const uint32_t tl = tmem + (uint32_t(32 * q) << 16) + ACC_COL;
-      if constexpr (EPI == EPI_SWIGLU) {
-        tmem_ld32(tl + 64 * half, v);
-        tmem_ld32(tl + 64 * half + 32, v + 32);
-        tmem_ld32(tl + 128 + 64 * half, v + 64);
-        tmem_ld32(tl + 128 + 64 * half + 32, v + 96);
+      if constexpr (EPI == EPI_SWIGLU) {  // gate columns 64*half.., up columns 128 + 64*half..
+        tmem_ld64(tl + 64 * half, v);
+        tmem_ld64(tl + 128 + 64 * half, v + 64);
       } else {
-        tmem_ld32(tl + 128 * half, v);
-        tmem_ld32(tl + 128 * half + 32, v + 32);
-        tmem_ld32(tl + 128 * half + 64, v + 64);
-        tmem_ld32(tl + 128 * half + 96, v + 96);
+        tmem_ld128(tl + 128 * half, v);
       }
       tc_wait_ld();
       tc_fence_before();
