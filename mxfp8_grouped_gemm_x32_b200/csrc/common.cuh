@@ -3,6 +3,7 @@
 // consumed by tcgen05 block-scaled MMA, the device status word, and thin
 // inline-PTX wrappers for mbarrier / TMA / tcgen05 (sm_100a).
 #pragma once
+#include <atomic>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -107,6 +108,36 @@ __host__ __device__ __forceinline__ int64_t sf_offset(int64_t g, int64_t r, int6
 }
 
 __host__ __device__ __forceinline__ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---- per-device host-side setup --------------------------------------------
+// SM count of the current device (cached per device; 148 if unknown).
+inline int device_sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) dev = 0;
+  std::atomic<int>* slot = dev < 64 ? &cache[dev] : nullptr;
+  int n = slot ? slot->load(std::memory_order_relaxed) : 0;
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (slot) slot->store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` once per device
+// (the attribute belongs to the device's context); `done` holds one bit per
+// device id below 64 (higher ids set it on every call).
+template <typename Kernel>
+inline cudaError_t ensure_smem_limit(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // floor(m / d) for 0 <= m < 2^31 and a divisor fixed at launch, by a
 // multiply-high (Granlund & Montgomery, "Division by invariant integers using

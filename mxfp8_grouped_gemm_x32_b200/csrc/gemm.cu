@@ -432,27 +432,12 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 template <int EPI>
 cudaError_t launch_epi(const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_mxf8_gemm_kernel<EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LAUNCH);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  grouped_mxf8_gemm_kernel<EPI><<<sm_count(), NUM_THREADS, SMEM_LAUNCH, st>>>(maps.a, maps.b, a);
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = ensure_smem_limit(grouped_mxf8_gemm_kernel<EPI>, SMEM_LAUNCH, configured);
+  if (e != cudaSuccess) return e;
+  grouped_mxf8_gemm_kernel<EPI><<<device_sm_count(), NUM_THREADS, SMEM_LAUNCH, st>>>(maps.a, maps.b, a);
   count_launch();
   return cudaGetLastError();
 }

@@ -375,17 +375,6 @@ __global__ void __launch_bounds__(256, 3) quant_both_kernel(QuantBothArgs a) {
   }
 }
 
-static int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 cudaError_t launch_quant_rows(const QuantRowsArgs& args, cudaStream_t st) {
   const int64_t total = int64_t(args.groups) * cdiv(args.rows, 128) * 128 * cdiv(args.K, 128);
   if (total == 0) return cudaSuccess;
@@ -395,7 +384,7 @@ cudaError_t launch_quant_rows(const QuantRowsArgs& args, cudaStream_t st) {
   a.rowpad_div = make_fastdiv(uint32_t(cdiv(a.rows, 128) * 128));
   a.div = make_fastdiv(uint32_t(a.map_div > 0 ? a.map_div : 1));
   int64_t blocks = cdiv(total, 256);
-  blocks = blocks > int64_t(num_sms()) * 16 ? int64_t(num_sms()) * 16 : blocks;
+  blocks = blocks > int64_t(device_sm_count()) * 16 ? int64_t(device_sm_count()) * 16 : blocks;
   quant_rows_kernel<<<unsigned(blocks), 256, 0, st>>>(a);
   count_launch();
   return cudaGetLastError();
@@ -425,13 +414,10 @@ cudaError_t launch_quant_both(const QuantBothArgs& args, cudaStream_t st) {
     if (e != cudaSuccess) return e;
   }
   const size_t smem = QB_TILE_ELEMS * sizeof(uint16_t) + 2 * QB_OUT_BYTES + 1024;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(quant_both_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  int64_t grid = int64_t(num_sms()) * 3;
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = ensure_smem_limit(quant_both_kernel, int(smem), configured);
+  if (e != cudaSuccess) return e;
+  int64_t grid = int64_t(device_sm_count()) * 3;
   if (grid > tiles) grid = tiles;
   quant_both_kernel<<<unsigned(grid), 256, smem, st>>>(a);
   count_launch();

@@ -241,13 +241,9 @@ int64_t swiglu_partial_bytes(int64_t rows_cap, int32_t I) { return cdiv(I, SB_TI
 
 cudaError_t launch_swiglu_bwd(const SwigluBwdArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(SwigluSmem);
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(swiglu_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(smem));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = ensure_smem_limit(swiglu_bwd_kernel, int(smem), configured);
+  if (e != cudaSuccess) return e;
   if (a.rows_cap == 0) return cudaSuccess;
   const int32_t nchunks = int32_t(cdiv(a.I, SB_TILE));
   dim3 grid(unsigned(a.rows_cap / SB_TILE), unsigned(nchunks));
