@@ -18,6 +18,8 @@
  *           parameter says "host".  The library never allocates device
  *           memory; scratch comes from the caller's workspace
  *           (moe_workspace_size).  Calls are asynchronous on `stream`.
+ *           For an empty batch (T == 0) arrays with a token dimension (x,
+ *           dY, out, dX, routing, logits, slot maps, dprob) may be null.
  * Errors.   Argument errors (null pointer, bad size, misalignment, an
  *           unsupported shape) are detected on the host before any launch
  *           and return MOE_ERR_INVALID / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE

@@ -214,8 +214,9 @@ moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* to
                          float* prob_perm, uint8_t* xq, uint8_t* xq_sf, uint8_t* xq_col,
                          uint8_t* xq_col_sf, void* workspace, size_t workspace_bytes,
                          moe_stream_t stream) {
-  if (!x || !topk_idx || !topk_prob || !split_sizes || !group_offsets || !row_to_slot ||
-      !slot_to_row || !prob_perm || !xq || !xq_sf)
+  // arrays with a token dimension may be null for an empty batch (T == 0)
+  if ((T > 0 && (!x || !topk_idx || !topk_prob || !slot_to_row)) || !split_sizes || !group_offsets ||
+      !row_to_slot || !prob_perm || !xq || !xq_sf)
     return MOE_ERR_INVALID;
   if ((xq_col == nullptr) != (xq_col_sf == nullptr)) return MOE_ERR_INVALID;
   if (T < 0 || H <= 0 || k <= 0 || E <= 0 || k > E) return MOE_ERR_INVALID;
@@ -250,7 +251,7 @@ moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* to
 }
 
 moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* out, moe_stream_t stream) {
-  if (!y || !out || T < 0 || k <= 0 || H <= 0 || H % 8) return MOE_ERR_INVALID;
+  if ((T > 0 && (!y || !out)) || T < 0 || k <= 0 || H <= 0 || H % 8) return MOE_ERR_INVALID;
   if (!al16(y) || !al16(out)) return MOE_ERR_INVALID;
   if (!device_ok()) return MOE_ERR_NO_DEVICE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -266,7 +267,7 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
                                  void* out, void* saved_a, uint8_t* hq, uint8_t* hq_sf, void* workspace,
                                  size_t workspace_bytes, moe_stream_t stream) {
   if (!w1q || !w1sf || !w2q || !w2sf || !split_sizes || !group_offsets || !row_to_slot || !prob_perm ||
-      !xq || !xq_sf || !out)
+      !xq || !xq_sf || (T > 0 && !out))
     return MOE_ERR_INVALID;
   if ((hq == nullptr) != (hq_sf == nullptr)) return MOE_ERR_INVALID;
   if (!layer_dims_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
@@ -330,8 +331,8 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
                                  void* dX, void* dW1, void* dW2, float* dprob, void* workspace,
                                  size_t workspace_bytes, moe_stream_t stream) {
   if (!w2tq || !w2tsf || !w1tq || !w1tsf || !split_sizes || !group_offsets || !row_to_slot ||
-      !slot_to_row || !prob_perm || !dY || !saved_a || !xq_col || !xq_col_sf || !dX || !dW1 || !dW2 ||
-      !dprob)
+      (T > 0 && (!slot_to_row || !dY || !dX || !dprob)) || !prob_perm || !saved_a || !xq_col || !xq_col_sf ||
+      !dW1 || !dW2)
     return MOE_ERR_INVALID;
   if (!layer_dims_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
   if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
@@ -432,7 +433,7 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
 
 moe_status_t moe_router_topk(const void* logits, int32_t logits_dtype, int32_t T, int32_t E, int32_t k,
                              int32_t* topk_idx, float* topk_prob, moe_stream_t stream) {
-  if (!logits || !topk_idx || !topk_prob || T < 0) return MOE_ERR_INVALID;
+  if ((T > 0 && (!logits || !topk_idx || !topk_prob)) || T < 0) return MOE_ERR_INVALID;
   if (logits_dtype != MOE_DTYPE_F32 && logits_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID;
   if (E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID;
   if (E > MOE_MAX_EXPERTS || k > 32) return MOE_ERR_UNSUPPORTED;

@@ -64,8 +64,8 @@ extern "C" moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_i
                                             uint8_t* xq_sf, uint8_t* xq_col, uint8_t* xq_col_sf,
                                             moe_stream_t stream) {
   using namespace moe;
-  if (!x || !topk_idx || !topk_prob || !split_sizes || !group_offsets || !row_to_slot ||
-      !slot_to_row || !prob_perm || !xq || !xq_sf)
+  if ((T > 0 && (!x || !topk_idx || !topk_prob || !slot_to_row)) || !split_sizes || !group_offsets ||
+      !row_to_slot || !prob_perm || !xq || !xq_sf)
     return MOE_ERR_INVALID;
   if ((xq_col == nullptr) != (xq_col_sf == nullptr)) return MOE_ERR_INVALID;
   if (T < 0 || H <= 0 || k <= 0 || E <= 0 || k > E) return MOE_ERR_INVALID;

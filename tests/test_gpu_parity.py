@@ -351,3 +351,35 @@ def test_quantize_weights_fused_equals_separate(torch_cuda, E, H, I):
     c, s = omx.quantize_rows(_f64(w1.cpu().view(torch.int16).numpy().view(np.uint16)).reshape(2 * E * I, H))
     assert np.array_equal(b[0][0].cpu().numpy().reshape(2 * E * I, H), c)
     assert np.array_equal(sf_unblock(b[0][1].cpu().numpy(), 2 * E, I, H).reshape(2 * E * I, -1), s)
+
+
+@pytest.mark.parametrize("T", [0, 1])
+def test_zero_and_one_token(torch_cuda, T):
+    """A batch with no tokens runs every launch of the step and leaves nothing
+    to compute (zero weight gradients); a single token is one row in each of
+    its k experts' groups."""
+    import torch
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    from mxfp8_grouped_gemm_x32_b200.layer import GroupedMLP
+    cfg = get_config("tiny", T=T)
+    inp = make_inputs(cfg, seed=3)
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    L = GroupedMLP(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k)
+    res = L.step(bf(inp["x"]), torch.from_numpy(inp["topk_idx"]).cuda(), torch.from_numpy(inp["topk_prob"]).cuda(),
+                 bf(inp["w1"]), bf(inp["w2"]), bf(inp["dy"]))
+    torch.cuda.synchronize()
+    assert lib.moe_get_device_status(0) == 0
+    out, dX, dW1, dW2, dprob = res
+    assert out.shape == (T, cfg.H) and dprob.shape == (T, cfg.k)
+    if T == 0:
+        assert float(dW1.float().abs().max()) == 0.0 and float(dW2.float().abs().max()) == 0.0
+        return
+    f = omoe.forward(_f64(inp["x"]), _f64(inp["w1"]), _f64(inp["w2"]), inp["topk_idx"], inp["topk_prob"])
+    b = omoe.backward(f, _f64(inp["x"]), _f64(inp["w1"]), _f64(inp["w2"]), inp["topk_prob"], _f64(inp["dy"]))
+    x, w1, w2, dy = (_f64(inp[k]) for k in ("x", "w1", "w2", "dy"))
+    allow = ambiguity.backward_allowance(f, b, x, w1, w2, dy, inp["topk_idx"])
+    allow["out"] = ambiguity.forward_allowance(f, x, w1, w2, inp["topk_idx"])
+    assert ambiguity.within(bf16_to_f64(out), f["out"], OUT_TOL, allow["out"]) <= OUT_TOL
+    for key, gpu, ref, bfo in (("dX", dX, b["dX"], True), ("dprob", dprob, b["dprob_f64"], False)):
+        g = gpu.float().cpu().numpy().astype(np.float64)
+        assert ambiguity.within(g, ref, GRAD_TOL, allow[key], bf16_out=bfo) <= GRAD_TOL
