@@ -138,6 +138,29 @@ def mxfp8_library_probe(torch, dev, seconds: float = 3.0):
         return {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
 
 
+def attainable_fwd(cfg, split, p_tflops: float, bw_gbs: float, rows_cap: int) -> dict:
+    """Attainable layer-forward time: per expert e, max(FLOP_e / P, bytes_e / BW)
+    for each of the two GEMMs (tiny groups are bound by their weight bytes),
+    plus the permutation's and the combine's bytes at BW.  Bytes per GEMM:
+    MX weights (+1/32 scales) and the expert's activation rows in and out
+    (gate_up: x codes in, bf16 saved A and h codes out; down: h codes in,
+    fp32 per-slot rows out)."""
+    H, I, T, k = cfg.H, cfg.I, cfg.T, cfg.k
+    P, BW = p_tflops * 1e12, bw_gbs * 1e9
+    t = 0.0
+    for m in split:
+        m = float(m)
+        f1, f2 = 2 * m * H * 2 * I, 2 * m * I * H
+        b1 = 2 * I * H * (1 + 1 / 32) + m * H + m * 2 * I * 2 + m * I
+        b2 = H * I * (1 + 1 / 32) + m * I + m * H * 4
+        t += max(f1 / P, b1 / BW) + max(f2 / P, b2 / BW)
+    permute_bytes = T * H * 2 + 2 * rows_cap * H * (1 + 1 / 32)
+    combine_bytes = T * k * H * 4 + T * H * 2
+    t += (permute_bytes + combine_bytes) / BW
+    return {"ms": t * 1e3, "peak_tflops": p_tflops, "hbm_gbs": bw_gbs,
+            "what": "sum over experts of max(FLOP/P, bytes/BW) for both GEMMs + permutation and combine bytes / BW"}
+
+
 def gemm_source_sha() -> str:
     h = hashlib.sha256()
     for rel in GEMM_SOURCES:
@@ -455,6 +478,7 @@ def run_ours(args):
     st = layer.device_status()
     if st != 0:
         raise SystemExit(f"device status after timing: {lib.status_string(st)}")
+    split_host = layer.split_sizes.cpu().tolist()
 
     if world > 1:
         dist.destroy_process_group()
@@ -524,6 +548,14 @@ def run_ours(args):
                              "layer_bwd": (line["bwd_tflops"] or 0.0) / lib_s}
             if roofline:
                 roofline["frac_of_library_sustained"] = roofline["achieved"] / lib_s
+    # attainable layer forward for this routing (per-expert max of compute and
+    # bytes), with the library's sustained MXFP8 rate when measured
+    p_att = line.get("mxfp8_library_probe", {}).get("sustained_tflops", peaks["mxfp8_sustained"])
+    att = attainable_fwd(cfg, split_host, p_att, peaks["hbm_gbs"], layer.rows_cap)
+    if fwd_ms:
+        att["measured_ms"] = fwd_ms
+        att["frac"] = att["ms"] / fwd_ms
+    line["attainable_fwd"] = att
     if world == 1 and not args.no_cpu_baseline:
         dt, fl, desc = oracle_sample(cfg, 256, args.seed, 4)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
