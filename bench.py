@@ -305,7 +305,9 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k,
+            "config": {"workload": f"{cfg.name} expert layer fwd+bwd", "T": cfg.T, "H": cfg.H, "I": cfg.I,
+                       "E": cfg.E, "k": cfg.k, "R": cfg.R,
+                       "step": "weight quant (both directions) + permute + fwd + bwd",
                        "sample_rows_per_step": rows, "sample_i_fraction": f"1/{i_div}"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
                              "sample": desc},
