@@ -49,6 +49,8 @@ class GroupedMLP:
         self.group_offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
         self.row_to_slot = torch.empty(rc, dtype=torch.int32, device=dev)
         self.slot_to_row = torch.empty(T * k, dtype=torch.int32, device=dev)
+        self.topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev)     # router outputs
+        self.topk_prob = torch.empty(T, k, dtype=torch.float32, device=dev)
         self.prob_perm = torch.empty(rc, dtype=torch.float32, device=dev)
         self.xq = _u8(rc * H, dev)
         self.xq_sf = _u8(sb(1, rc, H), dev)
@@ -100,9 +102,6 @@ class GroupedMLP:
         topk_prob float32 [T, k]) in this layer's routing buffers."""
         assert logits.is_contiguous() and logits.shape == (self.T, self.E)
         dt = {torch.float32: lib.MOE_DTYPE_F32, torch.bfloat16: lib.MOE_DTYPE_BF16}[logits.dtype]
-        if not hasattr(self, "topk_idx"):
-            self.topk_idx = torch.empty(self.T, self.k, dtype=torch.int32, device=self.dev)
-            self.topk_prob = torch.empty(self.T, self.k, dtype=torch.float32, device=self.dev)
         lib.moe_router_topk(logits.data_ptr(), dt, self.T, self.E, self.k, _ptr(self.topk_idx),
                             _ptr(self.topk_prob), self._stream())
         return self.topk_idx, self.topk_prob
