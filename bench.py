@@ -174,7 +174,8 @@ def profiled_traffic(cfg_name: str):
     when the summary is missing, for another workload, or the kernel source
     changed since it was captured."""
     try:
-        text = open(PROFILE_SUMMARY).read()
+        with open(PROFILE_SUMMARY) as fh:
+            text = fh.read()
     except OSError:
         return None
     m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)

@@ -12,7 +12,8 @@ HEADER = os.path.join(ROOT, "include", "moe_mxfp8.h")
 
 
 def _declared():
-    text = open(HEADER).read()
+    with open(HEADER) as fh:
+        text = fh.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
 

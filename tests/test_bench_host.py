@@ -74,7 +74,7 @@ def test_max_over_ranks_gloo_two_processes(tmp_path):
     import torch.multiprocessing as mp
     port = _free_port()
     mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True, start_method="spawn")
-    vals = [float(open(tmp_path / f"r{r}").read()) for r in range(2)]
+    vals = [float((tmp_path / f"r{r}").read_text()) for r in range(2)]
     assert vals == [15.0, 15.0]
 
 
