@@ -383,3 +383,27 @@ def test_zero_and_one_token(torch_cuda, T):
     for key, gpu, ref, bfo in (("dX", dX, b["dX"], True), ("dprob", dprob, b["dprob_f64"], False)):
         g = gpu.float().cpu().numpy().astype(np.float64)
         assert ambiguity.within(g, ref, GRAD_TOL, allow[key], bf16_out=bfo) <= GRAD_TOL
+
+
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("gpt_oss_20b", dict(T=160, E=4, k=2))])
+def test_forward_only_equals_training_forward(torch_cuda, name, over):
+    """The inference path (permutation quantising x along H only, forward
+    without the saved activation) writes exactly the bytes of the training
+    path's permutation and forward."""
+    torch = torch_cuda
+    from mxfp8_grouped_gemm_x32_b200.layer import GroupedMLP
+    cfg = get_config(name, **over)
+    inp = make_inputs(cfg, seed=4, grad=False)
+    x, w1, w2 = (_bf(torch, inp[k]) for k in ("x", "w1", "w2"))
+    idx, prob = torch.from_numpy(inp["topk_idx"]).cuda(), torch.from_numpy(inp["topk_prob"]).cuda()
+    outs = []
+    for bwd in (False, True):
+        L = GroupedMLP(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, backward=bwd)
+        L.quantize_weights(w1, w2)
+        L.permute(x, idx, prob)
+        out = L.forward()
+        torch.cuda.synchronize()
+        outs.append([t.cpu().clone() for t in (L.xq, L.xq_sf, L.hq, L.hq_sf, out)])
+    for a, b in zip(*outs):
+        assert torch.equal(a.view(torch.uint8) if a.dtype != torch.uint8 else a,
+                           b.view(torch.uint8) if b.dtype != torch.uint8 else b)
