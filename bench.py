@@ -482,6 +482,21 @@ def run_ours(args):
     if st != 0:
         raise SystemExit(f"device status after timing: {lib.status_string(st)}")
     split_host = layer.split_sizes.cpu().tolist()
+    # forward-only layer (inference): weights quantised once, then permutation +
+    # forward per call, no saved activation and no quantisation along tokens
+    inf = GroupedMLP(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, device=dev, backward=False)
+    inf.quantize_weights(w1, w2)
+    for _ in range(3):
+        inf.permute(x, idx, prob)
+        inf.forward()
+    e0.record(stream)
+    for _ in range(10):
+        inf.permute(x, idx, prob)
+        inf.forward()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_inf = max_over_ranks(e0.elapsed_time(e1) / 10, world, dev)
+    del inf
 
     if world > 1:
         dist.destroy_process_group()
@@ -532,6 +547,9 @@ def run_ours(args):
                                "ms_per_step": ms_max - kernels["quant_weights"]["ms_per_step"]}
                               if "quant_weights" in kernels else None),
         "kernels": kernels,
+        "inference_fwd": {"value": world * cfg.fwd_flops() / (ms_inf * 1e-3) / 1e12, "unit": "TFLOP/s",
+                          "ms_per_call": ms_inf,
+                          "what": "forward-only layer: permutation + forward per call, MX weights reused"},
         "router": {"ms_per_call": router_ms, "in_step": False,
                    "what": "moe_router_topk on fp32 logits [T, E] (softmax, top-k, renormalise)"},
         "roofline": roofline,
