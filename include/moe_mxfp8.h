@@ -208,9 +208,10 @@ moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_idx, const f
  *   saved_a    bf16 [rows_cap][2I] or NULL: A rounded to bf16, kept for the
  *              backward (padding rows are not written).
  *   hq, hq_sf  optional outputs (both NULL or both set) of the requantised
- *              intermediate: MX tensor (1, rows_cap, I); rows at or past
- *              group_offsets[E] (and their scale atoms) are not written.  If
- *              NULL they live in the workspace.
+ *              intermediate: MX tensor (1, rows_cap, I); only routed rows
+ *              (row_to_slot >= 0) are written -- padding rows keep whatever
+ *              the buffer held and are never read as a result.  If NULL
+ *              they live in the workspace.
  *   workspace  >= moe_workspace_size(MOE_OP_FWD, T, k, E, H, I).
  * Needs H % 32 == 0, I % 64 == 0, E <= MOE_MAX_EXPERTS. */
 moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const uint8_t* w2q,

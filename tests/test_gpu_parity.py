@@ -403,9 +403,10 @@ def test_forward_only_equals_training_forward(torch_cuda, name, over):
         L.permute(x, idx, prob)
         out = L.forward()
         torch.cuda.synchronize()
-        used = int(L.group_offsets[cfg.E])          # h is written for the group rows only
-        hsf = used // 128 * (-(-cfg.I // 128)) * 512  # their scale atoms: a prefix of the blocked layout
-        outs.append([t.cpu().clone() for t in (L.xq, L.xq_sf, L.hq[: used * cfg.I], L.hq_sf[:hsf],
-                                               out.view(torch.uint8))])
+        routed = L.row_to_slot.cpu().numpy() >= 0    # h is written for routed rows only
+        rc = L.rows_cap
+        h = L.hq.cpu().numpy()[: rc * cfg.I].reshape(rc, cfg.I)[routed]
+        hs = sf_unblock(L.hq_sf.cpu().numpy(), 1, rc, cfg.I)[0][routed]
+        outs.append([L.xq.cpu().numpy(), L.xq_sf.cpu().numpy(), h, hs, out.view(torch.uint8).cpu().numpy()])
     for a, b in zip(*outs):
-        assert torch.equal(a, b)
+        assert np.array_equal(a, b)
