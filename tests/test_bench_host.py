@@ -86,3 +86,23 @@ def test_reference_arm_non_zero_rank_exits_without_output(monkeypatch, capsys):
 
 def test_max_over_ranks_single_process():
     assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def test_attainable_fwd_limits():
+    """The attainable forward is the sum over experts of the larger of the
+    compute and byte times: with no bandwidth limit it is FLOPs / P plus the
+    permutation and combine bytes; an expert with no rows still streams its
+    weights; more rows never make it smaller."""
+    cfg = get_config("tiny")                          # H256 I512 E4 k2, T512
+    H, I, T, k = cfg.H, cfg.I, cfg.T, cfg.k
+    split = [256, 256, 256, 256]
+    big_bw = bench.attainable_fwd(cfg, split, 1000.0, 1e12, 1536)["ms"]
+    flops = sum(6.0 * m * H * I for m in split)
+    pc_bytes = T * H * 2 + 2 * 1536 * H * (1 + 1 / 32) + T * k * H * 4 + T * H * 2
+    assert big_bw == pytest.approx((flops / 1e15 + pc_bytes / 1e21) * 1e3, rel=1e-12)  # GEMM bytes take no time
+    empty = bench.attainable_fwd(cfg, [0, 0, 0, 1024], 1e9, 1000.0, 1536)["ms"]
+    w_bytes = 3 * (1 + 1 / 32) * H * I                               # MX W_gate_up + W_down of one expert
+    assert empty >= 3 * w_bytes / 1e12 * 1e3                         # the three idle experts still read weights
+    a = bench.attainable_fwd(cfg, [100, 200, 300, 424], 2000.0, 6000.0, 1536)["ms"]
+    b = bench.attainable_fwd(cfg, [200, 200, 300, 424], 2000.0, 6000.0, 1536)["ms"]
+    assert b >= a
