@@ -145,7 +145,7 @@ moe_status_t moe_mlp_quantize_weights(const void* w_gate_up, const void* w_down,
 
 /* Group routed tokens by expert and quantise them (Challenge 1:
  * split_sizes; Challenge 3: quantise activations before the GEMM).
- *   x          bf16 [T][H], H % 128 == 0 or H % 32 == 0 (any multiple of 32).
+ *   x          bf16 [T][H], H any multiple of 32.
  *   topk_idx   int32 [T][k] expert ids; topk_prob float [T][k].
  *   rows_cap   = moe_padded_rows(T,k,E) (or larger, a multiple of 128).
  * Outputs (all device, caller-owned):
@@ -161,6 +161,9 @@ moe_status_t moe_mlp_quantize_weights(const void* w_gate_up, const void* w_down,
  *                  (32-token blocks inside each 128-aligned group; padding
  *                  tokens are zero) -- the weight-gradient operand.
  *   workspace  >= moe_workspace_size(MOE_OP_PERMUTE, T, k, E, H, 0) bytes.
+ * Limits: 1 <= k <= E, H % 32 == 0 (else MOE_ERR_INVALID / MOE_ERR_UNSUPPORTED
+ * as for the other calls); E <= MOE_MAX_EXPERTS and T*k < 2^30
+ * (MOE_ERR_UNSUPPORTED otherwise).
  * Expert ids outside [0,E) set MOE_ERR_DEVICE_INDEX in the device status and
  * are dropped. */
 moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* topk_prob,
@@ -213,7 +216,8 @@ moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_idx, const f
  *              the buffer held and are never read as a result.  If NULL
  *              they live in the workspace.
  *   workspace  >= moe_workspace_size(MOE_OP_FWD, T, k, E, H, I).
- * Needs H % 32 == 0, I % 64 == 0, E <= MOE_MAX_EXPERTS. */
+ * Needs H % 32 == 0, I % 64 == 0, 1 <= k <= E <= MOE_MAX_EXPERTS and
+ * T*k < 2^30 (MOE_ERR_UNSUPPORTED otherwise). */
 moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const uint8_t* w2q,
                                  const uint8_t* w2sf, int32_t T, int32_t H, int32_t I, int32_t E,
                                  int32_t k, int64_t rows_cap, const int32_t* split_sizes,
@@ -264,7 +268,8 @@ moe_status_t moe_router_topk(const void* logits, int32_t logits_dtype, int32_t T
  *   xq_col, xq_col_sf  MX tensor (1, H, rows_cap) from moe_permute.
  * Outputs: dX bf16 [T][H]; dW1 bf16 [E][2I][H]; dW2 bf16 [E][H][I];
  *   dprob float [T][k] (slot order).
- * Needs H % 128 == 0 or H % 32 == 0, I % 64 == 0. */
+ * Needs H % 32 == 0, I % 64 == 0, 1 <= k <= E <= MOE_MAX_EXPERTS and
+ * T*k < 2^30 (MOE_ERR_UNSUPPORTED otherwise). */
 moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, const uint8_t* w1tq,
                                  const uint8_t* w1tsf, int32_t T, int32_t H, int32_t I, int32_t E,
                                  int32_t k, int64_t rows_cap, const int32_t* split_sizes,

@@ -173,21 +173,18 @@ moe_status_t moe_mlp_quantize_mxfp8(const void* src, int32_t groups, int64_t row
                                     int32_t mode, uint8_t* q, uint8_t* sf, moe_stream_t stream) {
   if (!src || !q || !sf || groups < 0 || rows < 0 || cols < 0) return MOE_ERR_INVALID;
   if (!al16(src) || !al16(q) || !al16(sf)) return MOE_ERR_INVALID;
+  if (mode != MOE_QUANT_ROW && mode != MOE_QUANT_COL) return MOE_ERR_INVALID;
+  if (mode == MOE_QUANT_ROW ? cols % 32 != 0 : (rows % 32 != 0 || cols % 8 != 0)) return MOE_ERR_UNSUPPORTED;
   if (!device_ok()) return MOE_ERR_NO_DEVICE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (mode == MOE_QUANT_ROW) {
-    if (cols % 32) return MOE_ERR_UNSUPPORTED;
     QuantRowsArgs a{static_cast<const uint8_t*>(src), cols, nullptr, 1, groups, rows, cols, q, sf};
     TimeScope ts(st, "quant_rows");
     return cuda_status(launch_quant_rows(a, st));
   }
-  if (mode == MOE_QUANT_COL) {
-    if (rows % 32 || cols % 8) return MOE_ERR_UNSUPPORTED;
-    QuantColsArgs a{static_cast<const uint8_t*>(src), cols, nullptr, 1, groups, rows, cols, q, sf};
-    TimeScope ts(st, "quant_cols");
-    return cuda_status(launch_quant_cols(a, st));
-  }
-  return MOE_ERR_INVALID;
+  QuantColsArgs a{static_cast<const uint8_t*>(src), cols, nullptr, 1, groups, rows, cols, q, sf};
+  TimeScope ts(st, "quant_cols");
+  return cuda_status(launch_quant_cols(a, st));
 }
 
 moe_status_t moe_mlp_quantize_weights(const void* w_gate_up, const void* w_down, int32_t E, int32_t H,
@@ -220,7 +217,7 @@ moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* to
     return MOE_ERR_INVALID;
   if ((xq_col == nullptr) != (xq_col_sf == nullptr)) return MOE_ERR_INVALID;
   if (T < 0 || H <= 0 || k <= 0 || E <= 0 || k > E) return MOE_ERR_INVALID;
-  if (E > MOE_MAX_EXPERTS || H % 32) return MOE_ERR_UNSUPPORTED;
+  if (E > MOE_MAX_EXPERTS || H % 32 || int64_t(T) * k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
   if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
   if (!al16(x) || !al16(xq) || !al16(xq_sf) || (xq_col && (!al16(xq_col) || !al16(xq_col_sf))))
     return MOE_ERR_INVALID;

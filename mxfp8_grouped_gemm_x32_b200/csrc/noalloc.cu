@@ -69,7 +69,7 @@ extern "C" moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_i
     return MOE_ERR_INVALID;
   if ((xq_col == nullptr) != (xq_col_sf == nullptr)) return MOE_ERR_INVALID;
   if (T < 0 || H <= 0 || k <= 0 || E <= 0 || k > E) return MOE_ERR_INVALID;
-  if (E > MOE_MAX_EXPERTS || H % 32) return MOE_ERR_UNSUPPORTED;
+  if (E > MOE_MAX_EXPERTS || H % 32 || int64_t(T) * k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
   if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (!al16(x) || !al16(xq) || !al16(xq_sf) || (xq_col && (!al16(xq_col) || !al16(xq_col_sf))))

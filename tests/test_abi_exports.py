@@ -66,3 +66,99 @@ def test_router_argument_errors():
     assert f(p, 0, 4, 8, 0, p, p, None) == 1               # k = 0
     assert f(p, 0, 4, 300, 2, p, p, None) == 2             # E > 256
     assert f(p, 0, 4, 64, 33, p, p, None) == 2             # k > 32
+
+
+# Every case below is rejected by the host-side checks before the library
+# looks for a device, so it returns the same code with or without a GPU and no
+# pointer is ever dereferenced.  P is an aligned non-null dummy, M a
+# misaligned one.
+P, M = 1 << 20, (1 << 20) + 8
+INVALID, UNSUPPORTED, WORKSPACE, TOO_LARGE = 1, 2, 3, 8
+
+
+def _permute_args(T=64, H=256, k=2, E=4, rows_cap=None, x=P, xq=P, xq_col=P, xq_col_sf=P, ws=P,
+                  ws_bytes=1 << 30):
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    if rows_cap is None:
+        rows_cap = lib.moe_padded_rows(T, k, E)
+    return (x, P, P, T, H, k, E, rows_cap, P, P, P, P, P, xq, P, xq_col, xq_col_sf, ws, ws_bytes, None)
+
+
+def test_permute_argument_errors():
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    f = lib._lib.moe_permute
+    assert f(*_permute_args(x=None)) == INVALID                      # null x with T > 0
+    assert f(*_permute_args(xq_col_sf=None)) == INVALID              # column form half given
+    assert f(*_permute_args(k=5, E=4)) == INVALID                    # k > E
+    assert f(*_permute_args(E=300)) == UNSUPPORTED                   # E > MOE_MAX_EXPERTS
+    assert f(*_permute_args(H=48)) == UNSUPPORTED                    # H % 32 != 0
+    assert f(*_permute_args(T=1 << 29, k=2, rows_cap=1 << 31)) == UNSUPPORTED   # T*k >= 2^30
+    assert f(*_permute_args(rows_cap=128)) == INVALID                # below moe_padded_rows
+    assert f(*_permute_args(rows_cap=lib.moe_padded_rows(64, 2, 4) + 64)) == INVALID  # not a multiple of 128
+    assert f(*_permute_args(xq=M)) == INVALID                        # misaligned output
+    assert f(*_permute_args(ws=None)) == WORKSPACE
+    assert f(*_permute_args(ws_bytes=16)) == WORKSPACE
+    g = lib._lib.moe_permute_noalloc
+    assert g(*_permute_args(x=None)[:17], None) == INVALID
+    assert g(*_permute_args(T=1 << 29, k=2, rows_cap=1 << 31)[:17], None) == UNSUPPORTED
+    T, k, E = 131073, 2, 256                                           # 257 histogram blocks x 256 experts
+    assert g(*_permute_args(T=T, k=k, E=E)[:17], None) == TOO_LARGE
+
+
+def _fwd_args(T=64, H=256, I=512, E=4, k=2, rows_cap=None, w1q=P, out=P, hq=P, hq_sf=P, ws=P, ws_bytes=1 << 40):
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    if rows_cap is None:
+        rows_cap = lib.moe_padded_rows(T, k, E)
+    return (w1q, P, P, P, T, H, I, E, k, rows_cap, P, P, P, P, P, P, out, P, hq, hq_sf, ws, ws_bytes, None)
+
+
+def test_forward_argument_errors():
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    f = lib._lib.moe_grouped_mlp_fwd
+    assert f(*_fwd_args(w1q=None)) == INVALID
+    assert f(*_fwd_args(hq_sf=None)) == INVALID                      # hq given without its scales
+    assert f(*_fwd_args(I=96)) == UNSUPPORTED                        # I % 64 != 0
+    assert f(*_fwd_args(H=48)) == UNSUPPORTED
+    assert f(*_fwd_args(k=5, E=4)) == UNSUPPORTED
+    assert f(*_fwd_args(T=1 << 29, k=2, rows_cap=1 << 31)) == UNSUPPORTED
+    assert f(*_fwd_args(rows_cap=128)) == INVALID
+    assert f(*_fwd_args(out=M)) == INVALID
+    assert f(*_fwd_args(ws_bytes=16)) == WORKSPACE
+    need = lib.moe_workspace_size(lib.MOE_OP_FWD, 64, 2, 4, 256, 512)
+    assert f(*_fwd_args(hq=None, hq_sf=None, ws_bytes=need - 1)) == WORKSPACE   # h in the workspace
+
+
+def _bwd_args(T=64, H=256, I=512, E=4, k=2, saved=P, dW1=P, ws_bytes=1 << 40):
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    rows_cap = lib.moe_padded_rows(T, k, E)
+    return (P, P, P, P, T, H, I, E, k, rows_cap, P, P, P, P, P, P, saved, P, P, P, dW1, P, P, P, ws_bytes, None)
+
+
+def test_backward_argument_errors():
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    f = lib._lib.moe_grouped_mlp_bwd
+    assert f(*_bwd_args(saved=None)) == INVALID
+    assert f(*_bwd_args(H=48)) == UNSUPPORTED
+    assert f(*_bwd_args(E=300, k=2)) == UNSUPPORTED
+    assert f(*_bwd_args(dW1=M)) == INVALID
+    need = lib.moe_workspace_size(lib.MOE_OP_BWD, 64, 2, 4, 256, 512)
+    assert f(*_bwd_args(ws_bytes=need - 1)) == WORKSPACE
+
+
+def test_quantise_and_combine_argument_errors():
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    q = lib._lib.moe_mlp_quantize_mxfp8
+    assert q(P, 1, 64, 48, lib.MOE_QUANT_ROW, P, P, None) == UNSUPPORTED    # cols % 32
+    assert q(P, 1, 48, 64, lib.MOE_QUANT_COL, P, P, None) == UNSUPPORTED    # rows % 32
+    assert q(P, 1, 64, 12, lib.MOE_QUANT_COL, P, P, None) == UNSUPPORTED    # cols % 8
+    assert q(P, 1, 64, 64, 3, P, P, None) == INVALID                        # unknown mode
+    assert q(M, 1, 64, 64, lib.MOE_QUANT_ROW, P, P, None) == INVALID
+    w = lib._lib.moe_mlp_quantize_weights
+    assert w(P, P, 4, 256, 512, *([P] * 7), None, None) == INVALID          # a null output
+    assert w(P, M, 4, 256, 512, *([P] * 8), None) == INVALID                # misaligned input
+    assert w(P, P, 0, 256, 512, *([P] * 8), None) == INVALID                # E = 0
+    assert w(P, P, 4, 256, 96, *([P] * 8), None) == UNSUPPORTED             # I % 64
+    c = lib._lib.moe_combine
+    assert c(P, 4, 2, 12, P, None) == INVALID                                # H % 8
+    assert c(P, 4, 2, 64, M, None) == INVALID
+    assert c(P, -1, 2, 64, P, None) == INVALID
