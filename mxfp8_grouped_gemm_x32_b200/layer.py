@@ -24,6 +24,22 @@ def _ptr(t) -> int:
     return 0 if t is None else t.data_ptr()
 
 
+def check_tensor(t, name: str, dtype, shape, device) -> None:
+    """Raise unless `t` is a contiguous tensor of `dtype` and `shape` on
+    `device`.  The library receives raw pointers, so a host tensor or a
+    wrong shape must be caught here, before any kernel reads through it."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name}: expected a tensor on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
 def _u8(n: int, dev) -> torch.Tensor:
     # 256-byte aligned by the caching allocator; sizes rounded to 16 bytes
     return torch.empty(max(16, (n + 15) // 16 * 16), dtype=torch.uint8, device=dev)
@@ -57,6 +73,7 @@ class GroupedMLP:
         self.hq = _u8(rc * I, dev)
         self.hq_sf = _u8(sb(1, rc, I), dev)
         self.out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        self.dev = self.out.device      # concrete device (index resolved) for the input checks
         self.ws_perm_bytes = lib.moe_workspace_size(lib.MOE_OP_PERMUTE, T, k, E, H, I)
         self.ws_fwd_bytes = lib.moe_workspace_size(lib.MOE_OP_FWD, T, k, E, H, I)
         self.ws_perm = _u8(self.ws_perm_bytes, dev)
@@ -86,8 +103,8 @@ class GroupedMLP:
     def quantize_weights(self, w1: torch.Tensor, w2: torch.Tensor) -> None:
         """w1 bf16 [E, 2I, H] (gate rows first), w2 bf16 [E, H, I]."""
         E, H, I, s = self.E, self.H, self.I, self._stream()
-        assert w1.dtype == torch.bfloat16 and w1.is_contiguous() and w1.shape == (E, 2 * I, H)
-        assert w2.dtype == torch.bfloat16 and w2.is_contiguous() and w2.shape == (E, H, I)
+        check_tensor(w1, "w_gate_up", torch.bfloat16, (E, 2 * I, H), self.dev)
+        check_tensor(w2, "w_down", torch.bfloat16, (E, H, I), self.dev)
         if self.backward_enabled:
             # both directions of both weights from one read of each
             lib.moe_mlp_quantize_weights(w1.data_ptr(), w2.data_ptr(), E, H, I, _ptr(self.w1q), _ptr(self.w1sf),
@@ -100,17 +117,19 @@ class GroupedMLP:
     def route(self, logits: torch.Tensor):
         """Router logits fp32 or bf16 [T, E] -> (topk_idx int32 [T, k],
         topk_prob float32 [T, k]) in this layer's routing buffers."""
-        assert logits.is_contiguous() and logits.shape == (self.T, self.E)
-        dt = {torch.float32: lib.MOE_DTYPE_F32, torch.bfloat16: lib.MOE_DTYPE_BF16}[logits.dtype]
+        dt = {torch.float32: lib.MOE_DTYPE_F32, torch.bfloat16: lib.MOE_DTYPE_BF16}.get(logits.dtype)
+        if dt is None:
+            raise TypeError(f"logits: expected float32 or bfloat16, got {logits.dtype}")
+        check_tensor(logits, "logits", logits.dtype, (self.T, self.E), self.dev)
         lib.moe_router_topk(logits.data_ptr(), dt, self.T, self.E, self.k, _ptr(self.topk_idx),
                             _ptr(self.topk_prob), self._stream())
         return self.topk_idx, self.topk_prob
 
     def permute(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_prob: torch.Tensor) -> None:
         """x bf16 [T, H]; topk_idx int32 [T, k]; topk_prob float32 [T, k]."""
-        assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.shape == (self.T, self.H)
-        assert topk_idx.dtype == torch.int32 and topk_idx.is_contiguous()
-        assert topk_prob.dtype == torch.float32 and topk_prob.is_contiguous()
+        check_tensor(x, "x", torch.bfloat16, (self.T, self.H), self.dev)
+        check_tensor(topk_idx, "topk_idx", torch.int32, (self.T, self.k), self.dev)
+        check_tensor(topk_prob, "topk_prob", torch.float32, (self.T, self.k), self.dev)
         bw = self.backward_enabled
         lib.moe_permute(x.data_ptr(), topk_idx.data_ptr(), topk_prob.data_ptr(), self.T, self.H, self.k,
                         self.E, self.rows_cap, _ptr(self.split_sizes), _ptr(self.group_offsets),
@@ -129,8 +148,9 @@ class GroupedMLP:
         return self.out
 
     def backward(self, dY: torch.Tensor):
-        assert self.backward_enabled
-        assert dY.dtype == torch.bfloat16 and dY.is_contiguous() and dY.shape == (self.T, self.H)
+        if not self.backward_enabled:
+            raise RuntimeError("this layer was built with backward=False")
+        check_tensor(dY, "dY", torch.bfloat16, (self.T, self.H), self.dev)
         lib.moe_grouped_mlp_bwd(_ptr(self.w2tq), _ptr(self.w2tsf), _ptr(self.w1tq), _ptr(self.w1tsf),
                                 self.T, self.H, self.I, self.E, self.k, self.rows_cap,
                                 _ptr(self.split_sizes), _ptr(self.group_offsets), _ptr(self.row_to_slot),
