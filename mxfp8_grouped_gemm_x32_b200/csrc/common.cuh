@@ -347,9 +347,9 @@ __host__ __device__ constexpr uint32_t make_idesc_mxf8(int M, int N, uint32_t a_
 
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives
-// lane (base lane + i), columns [col, col+32).
-// One warp: 32 lanes x N consecutive 32-bit TMEM columns in one instruction.
+// TMEM -> registers, one warp, one instruction: 32 lanes x N consecutive
+// 32-bit columns (N = 64 or 128); thread i receives lane (base lane + i),
+// columns [col, col + N) of the address `taddr` = (lane << 16) | col.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"

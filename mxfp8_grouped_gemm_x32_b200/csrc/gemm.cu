@@ -22,7 +22,8 @@
 //               (tcgen05.ld), release it to the MMA warp at once, then apply
 //               the epilogue and store -- so the next tile's MMAs overlap it.
 //               Rows go out through a per-warp shared staging buffer so that
-//               each store instruction writes 8 rows x 64 contiguous bytes.
+//               each store instruction writes 4 rows x 128 contiguous bytes
+//               (8 rows x 64 bytes for the SwiGLU epilogue's 64-byte pieces).
 // Tiles (128 rows x 256 columns) walk a device-side schedule derived from
 // the group offsets; every CTA strides through them (persistent grid).
 // Every wait is bounded; on time-out the kernel records MOE_ERR_TIMEOUT,

@@ -35,7 +35,7 @@ struct GemmArgs {
   int32_t b_RT, b_KT;  // row tiles per group and K tiles in B's scale layout
   const float* prob;
   const int32_t* row_to_slot;
-  uint8_t* out;       // bf16 output
+  uint8_t* out;       // output: fp32 rows (EPI_F32_*), bf16 per-expert matrices (EPI_WGRAD)
   int64_t ld_out;     // elements between output rows
   int64_t out_group_stride;  // mode 1: elements between experts' matrices
   uint8_t* out2;      // EPI_SWIGLU: saved A, bf16 [rows][2N] (nullable)
