@@ -27,7 +27,9 @@ casts over every bf16 pattern; the forward against an independent
 restatement of the per-expert loop; an identity-weight expert against its
 closed form; the backward against central finite differences and the
 closed form of d(prob); invariants of the permutation and the codec; the
-router against brute force over expert subsets, its closed form and torch.
+quantisation axis of every GEMM operand by inputs scaled along one axis
+(with planted axis swaps that must fail); the router against brute force
+over expert subsets, its closed form and torch.
 Parity unpinned: bit-level agreement of the scale rule with NVIDIA
 Transformer Engine (not available here).
 """
