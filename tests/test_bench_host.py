@@ -106,3 +106,10 @@ def test_attainable_fwd_limits():
     a = bench.attainable_fwd(cfg, [100, 200, 300, 424], 2000.0, 6000.0, 1536)["ms"]
     b = bench.attainable_fwd(cfg, [200, 200, 300, 424], 2000.0, 6000.0, 1536)["ms"]
     assert b >= a
+
+
+def test_l2_note_states_the_weight_bytes():
+    assert bench.l2_note(get_config("mixtral_8x7b")).startswith("inputs larger than L2 (bf16 weights 2.82 GB")
+    assert "1.21 GB" in bench.l2_note(get_config("qwen3_30b_ragged"))
+    assert "1.59 GB" in bench.l2_note(get_config("gpt_oss_20b"))
+    assert bench.l2_note(get_config("tiny")).startswith("inputs smaller than L2")
