@@ -292,6 +292,16 @@ def oracle_sample(cfg, rows: int, seed: int, i_div: int = 1):
 
 
 def cpu_cores() -> int:
+    """Threads the oracle runs on: the BLAS pool numpy's matrix products use
+    (the bulk of its work; the rest is single-threaded numpy), else the
+    host cores this process may use."""
+    try:
+        from threadpoolctl import threadpool_info
+        blas = [p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"]
+        if blas and max(blas) > 0:
+            return int(max(blas))
+    except Exception:  # threadpoolctl missing or unable to inspect the BLAS
+        pass
     try:
         return len(os.sched_getaffinity(0))
     except AttributeError:

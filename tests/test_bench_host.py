@@ -113,3 +113,13 @@ def test_l2_note_states_the_weight_bytes():
     assert "1.21 GB" in bench.l2_note(get_config("qwen3_30b_ragged"))
     assert "1.59 GB" in bench.l2_note(get_config("gpt_oss_20b"))
     assert bench.l2_note(get_config("tiny")).startswith("inputs smaller than L2")
+
+
+def test_cpu_cores_reports_the_blas_threads():
+    import numpy  # noqa: F401  (loads the BLAS the oracle uses)
+    from threadpoolctl import threadpool_info, threadpool_limits
+    if not any(p.get("user_api") == "blas" for p in threadpool_info()):
+        pytest.skip("no BLAS pool visible")
+    with threadpool_limits(limits=1, user_api="blas"):
+        assert bench.cpu_cores() == 1
+    assert bench.cpu_cores() >= 1
