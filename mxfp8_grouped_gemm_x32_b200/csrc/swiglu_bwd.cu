@@ -14,9 +14,10 @@
 // HBM-bound: 8 bytes read and 5 written per (row, intermediate channel), and
 // close to issue-bound, so the kernel keeps instructions per element low.  A
 // CTA owns a 128-row x 128-column tile (rows of one expert group: groups
-// start on multiples of 128) and walks it in four 32-row slices.  In a slice, eight threads share a row, each with
-// 16 contiguous columns: a 32-block of the row-wise quantisation spans two
-// threads (one shuffle), and the two write its codes as one 32-byte sector.
+// start on multiples of 128) and walks it in four 32-row slices.  In a
+// slice, eight threads share a row, each with 16 contiguous columns: a
+// 32-block of the row-wise quantisation spans two threads (one shuffle),
+// and the two write its codes as one 32-byte sector.
 // dg, du, h are staged in shared memory (fp32, 16-byte stores; rows 16..31
 // shifted by 16 words so the column reads are conflict-free) and quantised
 // down the columns, two lanes per column of 32 rows; each column block
