@@ -45,8 +45,10 @@
  * Permuted rows.  Routed row (token t, choice j) is slot s = t*k + j.  Rows
  *           are ordered by (expert, slot) (stable counting sort) and every
  *           expert's group starts on a multiple of 128 rows in a padded row
- *           space of capacity moe_padded_rows(T,k,E); padding rows hold zero
- *           codes and zero scales.
+ *           space of capacity moe_padded_rows(T,k,E).  Padding rows of the
+ *           MX tensors moe_permute produces hold zero codes and zero
+ *           scales; the forward's requantised h is written for routed rows
+ *           only (see moe_grouped_mlp_fwd).
  */
 #ifndef MOE_MXFP8_H
 #define MOE_MXFP8_H
