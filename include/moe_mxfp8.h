@@ -230,7 +230,8 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
 
 /* Top-k combine (Challenge 1, index_add back to token order):
  *   y  bf16 [T*k][H] in slot order -> out bf16 [T][H], out[t] = sum_j y[t*k+j]
- *   summed in fp32, j ascending. */
+ *   summed in fp32, j ascending (deterministic).
+ * Needs H % 8 == 0 and 16-byte aligned y and out (MOE_ERR_INVALID otherwise). */
 moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* out,
                          moe_stream_t stream);
 
