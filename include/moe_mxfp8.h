@@ -246,7 +246,8 @@ moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* o
  *               are all -inf get NaN probabilities
  *   topk_idx    device int32 [T][k] (written), expert ids, descending logit
  *   topk_prob   device fp32 [T][k] (written), exp(l_j - l_0) / sum over kept
- * Limits: 1 <= k <= E <= 256 and k <= 32 (MOE_ERR_UNSUPPORTED otherwise).
+ * Limits: 1 <= k <= E (MOE_ERR_INVALID otherwise); E <= MOE_MAX_EXPERTS (256)
+ * and k <= 32 (MOE_ERR_UNSUPPORTED otherwise).
  * No allocation, no workspace; asynchronous on `stream`. */
 moe_status_t moe_router_topk(const void* logits, int32_t logits_dtype, int32_t T, int32_t E, int32_t k,
                              int32_t* topk_idx, float* topk_prob, moe_stream_t stream);
