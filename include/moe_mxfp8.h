@@ -186,12 +186,13 @@ moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* to
  * MOE_PERMUTE_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
  * library holds until the process exits; larger problems are rejected with
  * MOE_ERR_TOO_LARGE before anything is launched.  Nothing is allocated: no
- * cudaMalloc, no cudaFree, no allocating library routine.  The first call on
- * a device looks up the array's device address (cudaGetSymbolAddress, once
- * per device, with that device current); make that first call before any
- * stream capture.  All calls share the one array: calls whose kernels
- * overlap on the GPU (different streams or host threads) race and must be
- * serialised by the caller. */
+ * cudaMalloc, no cudaFree, no allocating library routine.  Every call looks
+ * up the array's device address on the current device (cudaGetSymbolAddress,
+ * a host-side query), so the address stays right after a device reset; the
+ * first call on a device is where the runtime loads the library's module
+ * there, so make that first call before any stream capture.  All calls
+ * share the one array: calls whose kernels overlap on the GPU (different
+ * streams or host threads) race and must be serialised by the caller. */
 #define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (256 * 1024)
 moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_idx, const float* topk_prob,
                                  int32_t T, int32_t H, int32_t k, int32_t E, int64_t rows_cap,

@@ -27,7 +27,8 @@
 // Tiles (128 rows x 256 columns) walk a device-side schedule derived from
 // the group offsets; every CTA strides through them (persistent grid).
 // Every wait is bounded; on time-out the kernel records MOE_ERR_TIMEOUT,
-// stops all roles and still frees its TMEM.
+// stops all roles, lets its copies and MMAs in flight finish (bounded
+// waits again) and still frees its TMEM.
 #include "gemm.cuh"
 
 namespace moe {
@@ -50,7 +51,7 @@ constexpr int OFF_B = OFF_A + STAGES * SMEM_A;
 constexpr int OFF_SFA = OFF_B + STAGES * SMEM_B;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SMEM_SFA;
 constexpr int OFF_BAR = OFF_SFB + STAGES * SMEM_SFB;
-constexpr int NUM_BARS = 2 * STAGES + 2;
+constexpr int NUM_BARS = 2 * STAGES + 3;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem address, abort flag
 constexpr int OFF_GO = OFF_MISC + 16;              // group offsets [E+1]
 constexpr int STAGE_PITCH_W = 20;                  // words per staged row (16 used): conflict-free v4
@@ -265,6 +266,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;  // MMA completion on the abort path
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
   int* go = reinterpret_cast<int*>(smem + OFF_GO);
@@ -278,6 +280,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, NUM_EPI_WARPS);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -299,11 +302,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       prefetch_tmap(&tmB);
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t issued = 0;  // stages armed so far
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const Tile ti = decode_tile<EPI>(a, go, t);
         for (int kt = 0; kt < ti.nkt; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          ++issued;
           uint64_t* bar = &full[stage];
           mbar_arrive_expect_tx(bar, STAGE_TX);
           const int kg = ti.kt0 + kt;
@@ -334,6 +339,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+      }
+      if (*abort_flag) {
+        // shutting down early: let the copies of the last armed stages land
+        // before the shared memory they write is released
+        const uint32_t first = issued > uint32_t(STAGES) ? issued - STAGES : 0u;
+        for (uint32_t i = first; i < issued; ++i)
+          mbar_wait_drain(&full[i % STAGES], (i / STAGES) & 1u);
       }
     }
   } else if (warp == 1) {
@@ -371,6 +383,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!ok) break;
         tc_commit(acc_full);
         ++acc_it;
+      }
+      if (*abort_flag) {
+        // shutting down early: wait until every MMA issued so far has
+        // finished writing TMEM before it is freed
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0);
       }
     }
   } else {

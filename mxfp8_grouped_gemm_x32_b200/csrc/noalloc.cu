@@ -11,15 +11,16 @@
 // The array is part of the library image, so every GPU that loads the
 // library holds it until the process exits.  Host code cannot use the
 // array's name as a device address (in host code it names a host-side
-// stand-in), so the device address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, the first time the entry
-// point runs on it; that first call should therefore come before any stream
-// capture.  Every call shares the array and it keeps the last call's
-// contents; every byte a call reads from it is written earlier in the same
-// call, so nothing needs clearing.  Calls whose kernels overlap on the GPU
-// (two streams, or two host threads) race on the array.
-#include <mutex>
-
+// stand-in), so every call looks the device address up with
+// cudaGetSymbolAddress on the current device (a host-side query, no
+// allocation) and passes it to the kernels.  Looking it up on every call
+// rather than caching it keeps the address right after a device reset,
+// which reloads the module.  The first call on a device is where the
+// runtime loads the library's module there, so that first call should come
+// before any stream capture.  Every call shares the array and it keeps the
+// last call's contents; every byte a call reads from it is written earlier
+// in the same call, so nothing needs clearing.  Calls whose kernels overlap
+// on the GPU (two streams, or two host threads) race on the array.
 #include "permute.cuh"
 #include "quant.cuh"
 
@@ -31,25 +32,12 @@ static __device__ __align__(256) uint8_t g_permute_scratch[kPermuteScratchBytes]
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_permute_scratch on the current device (looked up once
-// per device).
+// Device address of g_permute_scratch on the current device.
 cudaError_t permute_scratch(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_permute_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 
