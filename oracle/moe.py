@@ -114,12 +114,15 @@ def _ident(v):
 
 
 def forward(x, w1, w2, topk_idx, topk_prob, *, quantize=True, round_saved=True,
-            experts=None):
+            experts=None, h_bf16=False):
     """Forward pass of the layer.
 
     x [T, H], w1 [E, 2I, H], w2 [E, H, I] as float64 values (bf16 inputs
     already converted), topk_idx int [T, k], topk_prob [T, k].
     ``quantize=False`` replaces every MXFP8 round trip by the identity;
+    ``h_bf16=True`` (with ``quantize=False``: the BF16 recipe, Challenge 2's
+    "BF16 uses 16 bits to represent each activation") rounds h to bf16
+    between the two GEMMs;
     ``round_saved=False`` keeps the saved activation in float64.
     ``experts`` restricts the work to those experts (rows of other experts
     are left zero) -- used for sampled checks at full size.
@@ -169,7 +172,7 @@ def forward(x, w1, w2, topk_idx, topk_prob, *, quantize=True, round_saved=True,
             hd = mxfp8.dequantize_rows(c, s)
             w2d = mxfp8.roundtrip_rows(w2[e])
         else:
-            hd, w2d = h, _ident(w2[e])
+            hd, w2d = (bf16_round(h) if h_bf16 else h), _ident(w2[e])
         Y[r0:r1] = hd @ w2d.T                             # down GEMM
     out = np.zeros((T, w2.shape[1]))
     slot_row = np.empty(R, np.int64)

@@ -112,6 +112,34 @@ def test_identity_expert_closed_form():
     assert np.array_equal(out, want)
 
 
+def test_identity_expert_bf16_path():
+    """BF16 recipe (no MXFP8, h kept in bf16): with the identity expert the
+    output is h = silu(x1) x2 rounded to bf16, checked against the
+    definition of round-to-nearest-even by brute force over the neighbouring
+    bf16 values, not against the oracle's own rounding."""
+    I, H, T = 64, 128, 16
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((T, H))
+    w1 = np.eye(2 * I)[None]
+    w2 = np.concatenate([np.eye(I), np.zeros((H - I, I))], axis=0)[None]
+    idx = np.zeros((T, 1), np.int32)
+    prob = np.ones((T, 1), np.float32)
+    out = moe.forward(x, w1, w2, idx, prob, quantize=False, h_bf16=True)["out"]
+    h = x[:, :I] / (1 + np.exp(-x[:, :I])) * x[:, I:]
+    assert np.all(out[:, I:] == 0)
+    v = out[:, :I]
+    bits = v.astype(np.float32).view(np.uint32)
+    assert np.all(v.astype(np.float32).astype(np.float64) == v) and np.all(bits & 0xFFFF == 0)   # bf16 values
+    nb = bits >> 16
+    for step in (-1, 1):                        # neighbours one bf16 step down and up
+        w = ((nb.astype(np.int64) + step).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        dv, dw = np.abs(v - h), np.abs(w - h)
+        assert np.all((dv < dw) | ((dv == dw) & (nb % 2 == 0)))
+    # without the bf16 step h passes through unrounded
+    out2 = moe.forward(x, w1, w2, idx, prob, quantize=False)["out"]
+    assert np.allclose(out2[:, :I], h, rtol=1e-15, atol=0)
+
+
 def test_permutation_invariants(tiny):
     cfg, inp = tiny
     perm, split = moe.permute(inp["topk_idx"], cfg.E)
