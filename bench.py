@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 from mxfp8_grouped_gemm_x32_b200.workloads import get_config  # noqa: E402
 
 METRIC = "grouped MoE MLP fwd/bwd TFLOP/s on 1 B200 and % of dense MXFP8 peak"
+SIDE_WORKLOADS_DEFAULT = ("qwen3_30b_ragged", "gpt_oss_20b")
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 MXFP8_OVER_BF16 = 2.0       # nominal dense ratio (4.5 / 2.25 PFLOP/s)
@@ -50,6 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default=",".join(SIDE_WORKLOADS_DEFAULT),
+                    help="further layer shapes measured in the same run (comma list, '' for none)")
     ap.add_argument("--no-library-probe", action="store_true",
                     help="skip the dense MXFP8 GEMM rate of the CUDA library (context for the roofline)")
     return ap.parse_args(argv)
@@ -102,11 +105,11 @@ def load_peaks(path=os.path.join(ROOT, "MEASURED_PEAKS.json")):
         bf16 = float(p["bf16_tflops"])
         bf16_s = float(p.get("bf16_tflops_sustained", bf16))
         return {"mxfp8_burst": bf16 * MXFP8_OVER_BF16, "mxfp8_sustained": bf16_s * MXFP8_OVER_BF16,
-                "hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
+                "bf16_sustained": bf16_s, "hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
     except (OSError, KeyError, ValueError):
         return {"mxfp8_burst": FALLBACK_BF16_TFLOPS * MXFP8_OVER_BF16,
-                "mxfp8_sustained": 1400.0 * MXFP8_OVER_BF16, "hbm_gbs": FALLBACK_HBM_GBS,
-                "source": "fallback"}
+                "mxfp8_sustained": 1400.0 * MXFP8_OVER_BF16, "bf16_sustained": 1400.0,
+                "hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
 
 
 def mxfp8_library_probe(torch, dev, seconds: float = 3.0):
@@ -172,6 +175,37 @@ def attainable_fwd(cfg, split, p_tflops: float, bw_gbs: float, rows_cap: int) ->
     t += (permute_bytes + combine_bytes) / BW
     return {"ms": t * 1e3, "peak_tflops": p_tflops, "hbm_gbs": bw_gbs,
             "what": "sum over experts of max(FLOP/P, bytes/BW) for both GEMMs + permutation and combine bytes / BW"}
+
+
+def split_histogram(split) -> dict:
+    """Rows per expert (M_e) of one routing: min, median, max, and the number
+    of experts that received no token."""
+    m = sorted(int(v) for v in split)
+    n = len(m)
+    med = m[n // 2] if n % 2 else 0.5 * (m[n // 2 - 1] + m[n // 2])
+    return {"min": m[0], "median": med, "max": m[-1], "empty": sum(1 for v in m if v == 0), "experts": n}
+
+
+MXFP8_OPS_PER_CLK_SM = 16384  # dense MXFP8 tensor-core FLOPs per clock per SM (sm_100)
+
+
+def clock_peak_tflops(sm_mhz: float, n_sm: int = 148) -> float:
+    """Dense MXFP8 tensor-core peak at a given SM clock: 16384 FLOP per clock
+    per SM x SMs x clock."""
+    return MXFP8_OPS_PER_CLK_SM * n_sm * sm_mhz * 1e6 / 1e12
+
+
+def phase_rates(cfg, fwd_ms: float, bwd_ms: float, peak: float, clk_peak) -> dict:
+    """Layer forward / backward TFLOP/s and their fractions of the dense MXFP8
+    peak (`peak`, the roofline denominator) and of the clock-based peak."""
+    out = {}
+    for name, fl, ms in (("fwd", cfg.fwd_flops(), fwd_ms), ("bwd", cfg.bwd_flops(), bwd_ms)):
+        if not ms:
+            continue
+        tf = fl / (ms * 1e-3) / 1e12
+        out[name] = {"ms": ms, "tflops": tf, "frac_of_peak": tf / peak,
+                     "frac_of_clock_peak": (tf / clk_peak) if clk_peak else None}
+    return out
 
 
 def gemm_source_sha() -> str:
@@ -368,6 +402,110 @@ def make_device_inputs(torch, cfg, seed: int, dev):
     return x, idx.to(torch.int32).contiguous(), prob.to(torch.float32).contiguous(), w1, w2, dy
 
 
+class PhaseTimer:
+    """CUDA events recorded on the launching stream between the phases of
+    each step: weight quantisation | permutation + forward | backward."""
+
+    def __init__(self, torch, n_steps: int):
+        self.ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_steps)]
+        self.i = 0
+
+    def take(self):
+        if self.i >= len(self.ev):
+            return None
+        e = self.ev[self.i]
+        self.i += 1
+        return e
+
+    def phases(self):
+        """Per-step (weight quant, fwd, bwd) in ms for the steps recorded."""
+        return [(a.elapsed_time(b), b.elapsed_time(c), c.elapsed_time(d)) for a, b, c, d in self.ev[:self.i]]
+
+
+def median(v):
+    v = sorted(v)
+    n = len(v)
+    return v[n // 2] if n % 2 else 0.5 * (v[n // 2 - 1] + v[n // 2])
+
+
+def make_step(layer, stream, x, idx, prob, w1, w2, dy):
+    """One step of the layer; `rec` (four CUDA events) brackets its phases."""
+    def step(rec=None):
+        if rec:
+            rec[0].record(stream)
+        layer.quantize_weights(w1, w2)
+        if rec:
+            rec[1].record(stream)
+        layer.permute(x, idx, prob)
+        layer.forward()
+        if rec:
+            rec[2].record(stream)
+        layer.backward(dy)
+        if rec:
+            rec[3].record(stream)
+    return step
+
+
+def measure_workload(torch, lib, name: str, seed: int, dev, steps: int, warmup: int, local: int, peaks) -> dict:
+    """A further layer shape measured in the same run (1 GPU): `warmup`
+    untimed steps, then `steps` steps, each preceded by a 256 MB write that
+    flushes L2 (outside the timed phases).  Reports per-step medians of the
+    layer forward, backward and weight quantisation, their TFLOP/s and
+    fractions of the dense MXFP8 peak and of the clock-based peak, the
+    per-kernel times and the rows-per-expert histogram."""
+    from mxfp8_grouped_gemm_x32_b200.layer import GroupedMLP
+    cfg = get_config(name)
+    x, idx, prob, w1, w2, dy = make_device_inputs(torch, cfg, seed, dev)
+    layer = GroupedMLP(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, device=dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    step = make_step(layer, stream, x, idx, prob, w1, w2, dy)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    st = layer.device_status()
+    if st != 0:
+        raise SystemExit(f"{name}: device status after warm-up: {lib.status_string(st)}")
+    pt = PhaseTimer(torch, steps)
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    lib.moe_timing_enable(True)
+    lib.moe_timing_read()
+    t0 = time.time()
+    for _ in range(steps):
+        flush.fill_(1)
+        step(pt.take())
+    torch.cuda.synchronize()
+    t1 = time.time()
+    per_kernel = lib.moe_timing_read()
+    lib.moe_timing_enable(False)
+    time.sleep(0.3)
+    clocks = parse_clocks(sampler.stop(), t0, t1)
+    st = layer.device_status()
+    if st != 0:
+        raise SystemExit(f"{name}: device status after timing: {lib.status_string(st)}")
+    ph = pt.phases()
+    wq, fwd, bwd = (median([p[i] for p in ph]) for i in range(3))
+    step_ms = median([sum(p) for p in ph])
+    clk_peak = clock_peak_tflops(clocks["sm_mhz"]) if clocks else None
+    flops = step_flops(cfg)
+    out = {"config": {"T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "k": cfg.k, "R": cfg.R,
+                      "router": cfg.router, "expert_bias_std": cfg.expert_bias_std},
+           "steps": steps, "warmup": warmup, "timing": "median over steps; L2 flushed (256 MB write) before each step",
+           "ms_per_step": step_ms, "tflops": flops / (step_ms * 1e-3) / 1e12,
+           "frac_of_peak": flops / (step_ms * 1e-3) / 1e12 / peaks["mxfp8_sustained"],
+           "weight_quant_ms": wq,
+           "layer": phase_rates(cfg, fwd, bwd, peaks["mxfp8_sustained"], clk_peak),
+           "peak_tflops": peaks["mxfp8_sustained"], "clock_peak_tflops": clk_peak,
+           "rows_per_expert": split_histogram(layer.split_sizes.cpu().tolist()),
+           "kernels": {k: {"ms_per_step": v[0] / steps, "launches_per_step": v[1] / steps}
+                       for k, v in per_kernel.items()},
+           "clocks": clocks}
+    del layer, flush
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -396,9 +534,7 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def step():
-        layer.step(x, idx, prob, w1, w2, dy)
-
+    step = make_step(layer, stream, x, idx, prob, w1, w2, dy)
     for _ in range(args.warmup):
         step()
     st = layer.device_status()
@@ -406,6 +542,7 @@ def run_ours(args):
         raise SystemExit(f"device status after warm-up: {lib.status_string(st)}")
 
     # ---- timed region: K steps, inputs resident in HBM --------------------
+    pt = PhaseTimer(torch, args.steps)
     sampler = ClockSampler(local)
     time.sleep(0.3)
     lib.moe_timing_enable(True)
@@ -416,7 +553,7 @@ def run_ours(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        step()
+        step(pt.take())
     e1.record(stream)
     barrier()
     t_wall1 = time.time()
@@ -428,6 +565,8 @@ def run_ours(args):
     ms_max = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     flops = step_flops(cfg)
     value = world * flops / (ms_max * 1e-3) / 1e12
+    ph = pt.phases()
+    wq_ms, fwd_ms, bwd_ms = (sum(p[i] for p in ph) / len(ph) for i in range(3))
 
     # ---- end to end through the public API with host buffers --------------
     # Every step copies its own inputs (x, routing, dY) from pinned host memory
@@ -520,6 +659,20 @@ def run_ours(args):
     torch.cuda.synchronize()
     ms_inf = max_over_ranks(e0.elapsed_time(e1) / 10, world, dev)
     del inf
+    # the BF16 recipe's forward (bf16 operands, no MXFP8): routing + forward
+    for _ in range(3):
+        layer.permute_index(idx, prob)
+        layer.forward_bf16(x, w1, w2)
+    e0.record(stream)
+    for _ in range(10):
+        layer.permute_index(idx, prob)
+        layer.forward_bf16(x, w1, w2)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_bf16 = max_over_ranks(e0.elapsed_time(e1) / 10, world, dev)
+    st = layer.device_status()
+    if st != 0:
+        raise SystemExit(f"device status after the BF16 forward: {lib.status_string(st)}")
 
     if world > 1:
         dist.destroy_process_group()
@@ -527,6 +680,8 @@ def run_ours(args):
         return 0
 
     peaks = load_peaks()
+    peak = peaks["mxfp8_sustained"]
+    clk_peak = clock_peak_tflops(clocks["sm_mhz"]) if clocks else None
     kernels = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
                for k, v in per_kernel.items()}
     g1 = per_kernel.get("gemm_gate_up_swiglu")
@@ -534,20 +689,13 @@ def run_ours(args):
     if g1 and g1[1]:
         t_launch = g1[0] / g1[1] * 1e-3
         achieved = gate_up_flops(cfg) / t_launch / 1e12
-        peak = peaks["mxfp8_sustained"]
         roofline = {"bound": "tensor", "kernel": "gemm_gate_up_swiglu", "achieved": achieved,
                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                     "traffic": profiled_traffic(cfg.name),
                     "peak_source": f"{peaks['source']} bf16 sustained x {MXFP8_OVER_BF16} (nominal MXFP8/BF16)",
-                    "frac_of_burst": achieved / peaks["mxfp8_burst"]}
-    # layer forward = permute + gate_up GEMM + down GEMM + combine; layer backward = dY
-    # quantisation + both dgrads + SwiGLU backward + both wgrads + dX combine (weight
-    # quantisation reported on its own)
-    fwd_keys = ("permute_index", "permute_quant", "gemm_gate_up_swiglu", "gemm_down", "combine")
-    fwd_ms = sum(kernels[k]["ms_per_step"] for k in fwd_keys if k in kernels)
-    bwd_keys = ("dy_quant", "gemm_dgrad_down", "swiglu_bwd", "gemm_wgrad_down",
-                "gemm_dgrad_gate_up", "combine_dx", "gemm_wgrad_gate_up")
-    bwd_ms = sum(kernels[k]["ms_per_step"] for k in bwd_keys if k in kernels)
+                    "frac_of_burst": achieved / peaks["mxfp8_burst"],
+                    "frac_of_clock_peak": achieved / clk_peak if clk_peak else None}
+    layer_rates = phase_rates(cfg, fwd_ms, bwd_ms, peak, clk_peak)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
@@ -559,20 +707,29 @@ def run_ours(args):
                    "l2": l2_note(cfg),
                    "step": "weight quant (both directions) + permute + fwd + bwd",
                    "flops_per_step": flops},
-        "frac_of_mxfp8_peak": value / world / peaks["mxfp8_sustained"],
-        "fwd_tflops": cfg.fwd_flops() / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,
-        "bwd_tflops": cfg.bwd_flops() / (bwd_ms * 1e-3) / 1e12 if bwd_ms else None,
-        # the step without the weight quantisation (whose time is measured in
-        # the same run): a gradient-accumulation micro-step, where the MX
-        # weights of the optimizer step are reused
-        "excl_weight_quant": ({"value": world * flops / ((ms_max - kernels["quant_weights"]["ms_per_step"]) * 1e-3)
-                               / 1e12, "unit": "TFLOP/s",
-                               "ms_per_step": ms_max - kernels["quant_weights"]["ms_per_step"]}
-                              if "quant_weights" in kernels else None),
+        "frac_of_mxfp8_peak": value / world / peak,
+        "clock_peak_tflops": clk_peak,
+        "frac_of_clock_peak": value / world / clk_peak if clk_peak else None,
+        # layer forward = permutation + forward; layer backward = the backward
+        # call; CUDA events between the phases of every timed step (means)
+        "layer": layer_rates,
+        "fwd_tflops": layer_rates.get("fwd", {}).get("tflops"),
+        "bwd_tflops": layer_rates.get("bwd", {}).get("tflops"),
+        "weight_quant_ms": wq_ms,
+        # the step without the weight quantisation: a gradient-accumulation
+        # micro-step, where the MX weights of the optimizer step are reused
+        "excl_weight_quant": {"value": world * flops / ((fwd_ms + bwd_ms) * 1e-3) / 1e12, "unit": "TFLOP/s",
+                              "ms_per_step": fwd_ms + bwd_ms},
         "kernels": kernels,
+        "rows_per_expert": split_histogram(split_host),
         "inference_fwd": {"value": world * cfg.fwd_flops() / (ms_inf * 1e-3) / 1e12, "unit": "TFLOP/s",
                           "ms_per_call": ms_inf,
                           "what": "forward-only layer: permutation + forward per call, MX weights reused"},
+        "bf16_fwd": {"value": world * cfg.fwd_flops() / (ms_bf16 * 1e-3) / 1e12, "unit": "TFLOP/s",
+                     "ms_per_call": ms_bf16, "peak_bf16_tflops": peaks["bf16_sustained"],
+                     "frac_of_bf16_peak": cfg.fwd_flops() / (ms_bf16 * 1e-3) / 1e12 / peaks["bf16_sustained"],
+                     "what": "BF16 recipe layer forward (moe_permute without x + moe_grouped_mlp_fwd_bf16): "
+                             "bf16 operands, no MXFP8"},
         "router": {"ms_per_call": router_ms, "in_step": False,
                    "what": "moe_router_topk on fp32 logits [T, E] (softmax, top-k, renormalise)"},
         "roofline": roofline,
@@ -582,6 +739,21 @@ def run_ours(args):
                 "pipeline": "copy stream: inputs of step i+1 in, results of step i out, while step i+1 computes"},
         "gpu_launches": launches,
     }
+    # attainable layer forward for this routing (per-expert max of compute and
+    # bytes) at the roofline peak
+    att = attainable_fwd(cfg, split_host, peak, peaks["hbm_gbs"], layer.rows_cap)
+    att["measured_ms"] = fwd_ms
+    att["frac"] = att["ms"] / fwd_ms
+    line["attainable_fwd"] = att
+    del layer, x, idx, prob, w1, w2, dy, din, dsnap
+    torch.cuda.empty_cache()
+    if world == 1 and args.workloads:
+        # the other layer shapes, measured in the same run on the same GPU
+        line["workloads"] = {}
+        for name in args.workloads.split(","):
+            if name and name != cfg.name:
+                line["workloads"][name] = measure_workload(torch, lib, name, args.seed, dev, max(args.steps, 50),
+                                                           max(args.warmup, 10), local, peaks)
     if not args.no_library_probe:
         probe = mxfp8_library_probe(torch, dev)
         line["mxfp8_library_probe"] = probe
@@ -590,16 +762,7 @@ def run_ours(args):
             probe["frac"] = {"step": value / world / lib_s,
                              "layer_fwd": (line["fwd_tflops"] or 0.0) / lib_s,
                              "layer_bwd": (line["bwd_tflops"] or 0.0) / lib_s}
-            if roofline:
-                roofline["frac_of_library_sustained"] = roofline["achieved"] / lib_s
-    # attainable layer forward for this routing (per-expert max of compute and
-    # bytes), with the library's sustained MXFP8 rate when measured
-    p_att = line.get("mxfp8_library_probe", {}).get("sustained_tflops", peaks["mxfp8_sustained"])
-    att = attainable_fwd(cfg, split_host, p_att, peaks["hbm_gbs"], layer.rows_cap)
-    if fwd_ms:
-        att["measured_ms"] = fwd_ms
-        att["frac"] = att["ms"] / fwd_ms
-    line["attainable_fwd"] = att
+            probe["note"] = "context only: a library's achieved rate, not the peak the targets use"
     if world == 1 and not args.no_cpu_baseline:
         dt, fl, desc = oracle_sample(cfg, 256, args.seed, 4)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),

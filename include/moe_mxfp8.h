@@ -45,10 +45,13 @@
  * Permuted rows.  Routed row (token t, choice j) is slot s = t*k + j.  Rows
  *           are ordered by (expert, slot) (stable counting sort) and every
  *           expert's group starts on a multiple of 128 rows in a padded row
- *           space of capacity moe_padded_rows(T,k,E).  Padding rows of the
- *           MX tensors moe_permute produces hold zero codes and zero
- *           scales; the forward's requantised h is written for routed rows
- *           only (see moe_grouped_mlp_fwd).
+ *           space of capacity moe_padded_rows(T,k,E).  The groups fill
+ *           rows [0, group_offsets[E]); the rows from group_offsets[E] to the
+ *           capacity belong to no group, and no kernel writes or reads them.
+ *           Padding rows inside a group (after its last token, up to the
+ *           next multiple of 128) of the MX tensors moe_permute produces
+ *           hold zero codes and zero scales; the forward's requantised h is
+ *           written for routed rows only (see moe_grouped_mlp_fwd).
  */
 #ifndef MOE_MXFP8_H
 #define MOE_MXFP8_H
@@ -86,6 +89,7 @@ typedef enum {
 #define MOE_OP_PERMUTE 1
 #define MOE_OP_FWD 2
 #define MOE_OP_BWD 3
+#define MOE_OP_FWD_BF16 4
 
 /* Limits checked on the host. */
 #define MOE_MAX_EXPERTS 256
@@ -104,6 +108,25 @@ int64_t moe_padded_rows(int32_t T, int32_t k, int32_t E);
 /* Workspace bytes for op MOE_OP_PERMUTE / MOE_OP_FWD / MOE_OP_BWD of a layer
  * (T tokens, top-k, E experts, hidden H, intermediate I).  -1 if invalid. */
 int64_t moe_workspace_size(int32_t op, int32_t T, int32_t k, int32_t E, int32_t H, int32_t I);
+
+/* Plain <-> blocked scale order (Challenge 2: one E8M0 scale byte per 32
+ * consecutive values along K).  The plain order is the ordinary one,
+ * row-major [groups][rows][k/32] with `ld` bytes between rows (ld >= k/32);
+ * the blocked order is the layout above, which every MX operand of this
+ * library uses.  Callers holding MX scales from another quantiser convert
+ * them with moe_mx_scales_to_blocked (padding bytes of the layout are
+ * written as 0); moe_mx_scales_from_blocked reads the library's scales back
+ * in plain order.
+ *   plain    device, groups*rows rows of ld bytes (only the first k/32 of a
+ *            row are read or written).
+ *   blocked  device, moe_mx_scale_bytes(groups, rows, k) bytes, 4-byte
+ *            aligned for moe_mx_scales_to_blocked.
+ * Needs k % 32 == 0 and ld >= k/32 (MOE_ERR_INVALID otherwise).  No
+ * allocation; asynchronous on `stream`. */
+moe_status_t moe_mx_scales_to_blocked(const uint8_t* plain, int32_t groups, int64_t rows, int64_t k,
+                                      int64_t ld, uint8_t* blocked, moe_stream_t stream);
+moe_status_t moe_mx_scales_from_blocked(const uint8_t* blocked, int32_t groups, int64_t rows, int64_t k,
+                                        uint8_t* plain, int64_t ld, moe_stream_t stream);
 
 /* ----------------------------------------------------------- quantise --- */
 
@@ -157,7 +180,10 @@ moe_status_t moe_mlp_quantize_weights(const void* w_gate_up, const void* w_down,
  *   row_to_slot    int32 [rows_cap]  slot of each padded row, -1 = padding.
  *   slot_to_row    int32 [T*k]       padded row of each slot.
  *   prob_perm      float [rows_cap]  routing probability per padded row (0 pad).
- *   xq, xq_sf      MX tensor (1, rows_cap, H): gathered x, quantised along H.
+ *   xq, xq_sf      MX tensor (1, rows_cap, H): gathered x, quantised along H
+ *                  (rows from group_offsets[E] on are left unwritten).  Both
+ *                  NULL (then xq_col too): only the routing outputs above
+ *                  are produced, as the BF16 forward needs.
  *   xq_col, xq_col_sf  optional (both NULL or both set): MX tensor
  *                  (1, H, rows_cap) = gathered x^T quantised along tokens
  *                  (32-token blocks inside each 128-aligned group; padding
@@ -219,6 +245,11 @@ moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_idx, const f
  *              the buffer held and are never read as a result.  If NULL
  *              they live in the workspace.
  *   workspace  >= moe_workspace_size(MOE_OP_FWD, T, k, E, H, I).
+ * The combine is always applied (there is no flag for per-slot output): the
+ * down projection's rows are summed in fp32, in ascending j, from an fp32
+ * per-slot buffer in the workspace, so `out` is rounded to bf16 once.  A
+ * caller that wants per-slot rows instead uses moe_combine's input format
+ * (bf16 [T*k][H]) with its own down projection.
  * Needs H % 32 == 0, I % 64 == 0, 1 <= k <= E <= MOE_MAX_EXPERTS and
  * T*k < 2^30 (MOE_ERR_UNSUPPORTED otherwise). */
 moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const uint8_t* w2q,
@@ -228,6 +259,25 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
                                  const float* prob_perm, const uint8_t* xq, const uint8_t* xq_sf,
                                  void* out, void* saved_a, uint8_t* hq, uint8_t* hq_sf,
                                  void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* BF16 grouped MLP forward: the same layer with BF16 operands and no
+ * quantisation (the pages' "select BF16 or MXFP8": both recipes run the
+ * GroupedLinear -> ScaledSwiGLU -> GroupedLinear sequence).  x rows are
+ * gathered into permuted order, A = x W_gate_up^T and y = h W_down^T run on
+ * the bf16 tensor cores (fp32 accumulation), h = prob * silu(gate) * up is
+ * kept in bf16 between them, and out[t] = sum_j y[t*k+j] (fp32, ascending
+ * j, one bf16 rounding).
+ *   w_gate_up  bf16 [E][2I][H] (gate rows first); w_down bf16 [E][H][I].
+ *   routing    split_sizes, group_offsets, row_to_slot, prob_perm from
+ *              moe_permute (xq may be NULL there).
+ *   x          bf16 [T][H];  out bf16 [T][H].
+ *   workspace  >= moe_workspace_size(MOE_OP_FWD_BF16, T, k, E, H, I).
+ * Limits as moe_grouped_mlp_fwd. */
+moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down, int32_t T, int32_t H, int32_t I,
+                                      int32_t E, int32_t k, int64_t rows_cap, const int32_t* split_sizes,
+                                      const int32_t* group_offsets, const int32_t* row_to_slot,
+                                      const float* prob_perm, const void* x, void* out, void* workspace,
+                                      size_t workspace_bytes, moe_stream_t stream);
 
 /* Top-k combine (Challenge 1, index_add back to token order):
  *   y  bf16 [T*k][H] in slot order -> out bf16 [T][H], out[t] = sum_j y[t*k+j]
@@ -253,6 +303,23 @@ moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* o
 moe_status_t moe_router_topk(const void* logits, int32_t logits_dtype, int32_t T, int32_t E, int32_t k,
                              int32_t* topk_idx, float* topk_prob, moe_stream_t stream);
 
+/* Router fused with the permutation: moe_router_topk and moe_permute in one
+ * call (Challenge 1: the routing weights and the per-expert token groups
+ * the grouped GEMMs consume).  The router pass also counts each kept
+ * (token, choice) in the expert histogram of the permutation's counting
+ * sort, so the routing is read once and the histogram pass is not launched.
+ * Results are identical to moe_router_topk followed by moe_permute.
+ *   logits, logits_dtype   as moe_router_topk.
+ *   topk_idx, topk_prob    written, as moe_router_topk (also read back by
+ *                          the permutation).
+ *   every other argument   as moe_permute.
+ * Limits: those of both calls (k <= 32 included). */
+moe_status_t moe_route_permute(const void* logits, int32_t logits_dtype, const void* x, int32_t T, int32_t H,
+                               int32_t k, int32_t E, int64_t rows_cap, int32_t* topk_idx, float* topk_prob,
+                               int32_t* split_sizes, int32_t* group_offsets, int32_t* row_to_slot,
+                               int32_t* slot_to_row, float* prob_perm, uint8_t* xq, uint8_t* xq_sf, uint8_t* xq_col,
+                               uint8_t* xq_col_sf, void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
 /* ----------------------------------------------------------- backward --- */
 
 /* Matching fused backward (Challenge 3).  With dy_r = dY[token(r)]:
@@ -268,7 +335,8 @@ moe_status_t moe_router_topk(const void* logits, int32_t logits_dtype, int32_t T
  *                (moe_mlp_quantize_mxfp8 COL of W_down, groups=E rows=H cols=I).
  *   w1tq, w1tsf  MX tensor (E, H, 2I): W_gate_up^T quantised along 2I
  *                (COL of W_gate_up, groups=E rows=2I cols=H).
- *   routing      as in the forward, plus slot_to_row.
+ *   routing      as in the forward, plus slot_to_row (the dX combine
+ *                gathers each token's k dgrad rows through it).
  *   dY           bf16 [T][H].  saved_a bf16 [rows_cap][2I] from the forward.
  *   xq_col, xq_col_sf  MX tensor (1, H, rows_cap) from moe_permute.
  * Outputs: dX bf16 [T][H]; dW1 bf16 [E][2I][H]; dW2 bf16 [E][H][I];

@@ -87,8 +87,32 @@ FwdWs carve_fwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t r
   return w;
 }
 
+struct FwdBf16Ws {
+  uint8_t *xp, *h, *y;
+};
+FwdBf16Ws carve_fwd_bf16(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t rows_cap) {
+  FwdBf16Ws w{};
+  w.xp = c.take(rows_cap * H * 2);  // gathered x, bf16, permuted order
+  w.h = c.take(rows_cap * I * 2);   // h, bf16
+  w.y = c.take(T * k * H * 4);      // fp32 down-projection rows in slot order
+  return w;
+}
+
+// xp[r] = x[row_to_slot[r] / k] (bf16 rows, 16 bytes per thread) for the
+// rows of the groups; padding rows inside a group are zero.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ row_to_slot,
+                                                         const int32_t* __restrict__ rows_used, int32_t k, int64_t H16,
+                                                         uint4* __restrict__ xp) {
+  const int64_t n = int64_t(*rows_used) * H16;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / H16, c = i - r * H16;
+    const int32_t s = __ldg(row_to_slot + r);
+    xp[i] = s >= 0 ? __ldg(x + int64_t(s / k) * H16 + c) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 struct BwdWs {
-  uint8_t *dyq, *dyq_sf, *dyc, *dyc_sf, *dh, *daq, *daq_sf, *dac, *dac_sf, *hc, *hc_sf, *dx, *dpp;
+  uint8_t *dyq, *dyq_sf, *dyc, *dyc_sf, *daq, *daq_sf, *dac, *dac_sf, *hc, *hc_sf, *dx, *dpp;
 };
 BwdWs carve_bwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t rows_cap) {
   BwdWs w{};
@@ -96,15 +120,14 @@ BwdWs carve_bwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t r
   w.dyq_sf = c.take(mx_scale_bytes(1, rows_cap, H));
   w.dyc = c.take(H * rows_cap);
   w.dyc_sf = c.take(mx_scale_bytes(1, H, rows_cap));
-  w.dh = c.take(rows_cap * I * 4);
   w.daq = c.take(rows_cap * 2 * I);
   w.daq_sf = c.take(mx_scale_bytes(1, rows_cap, 2 * I));
   w.dac = c.take(2 * I * rows_cap);
   w.dac_sf = c.take(mx_scale_bytes(1, 2 * I, rows_cap));
   w.hc = c.take(I * rows_cap);
   w.hc_sf = c.take(mx_scale_bytes(1, I, rows_cap));
-  w.dx = c.take(T * k * H * 4);
-  w.dpp = c.take(swiglu_partial_bytes(rows_cap, int32_t(I)));
+  w.dx = c.take(rows_cap * H * 4);  // fp32 dgrad rows in permuted order
+  w.dpp = c.take(I / 64 * rows_cap * 4);  // dprob partial sums per 64-column chunk
   return w;
 }
 
@@ -165,6 +188,10 @@ int64_t moe_workspace_size(int32_t op, int32_t T, int32_t k, int32_t E, int32_t 
       if (H <= 0 || I <= 0) return -1;
       carve_bwd(c, T, k, H, I, rows_cap);
       return c.off;
+    case MOE_OP_FWD_BF16:
+      if (H <= 0 || I <= 0) return -1;
+      carve_fwd_bf16(c, T, k, H, I, rows_cap);
+      return c.off;
   }
   return -1;
 }
@@ -211,11 +238,13 @@ moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* to
                          float* prob_perm, uint8_t* xq, uint8_t* xq_sf, uint8_t* xq_col,
                          uint8_t* xq_col_sf, void* workspace, size_t workspace_bytes,
                          moe_stream_t stream) {
-  // arrays with a token dimension may be null for an empty batch (T == 0)
-  if ((T > 0 && (!x || !topk_idx || !topk_prob || !slot_to_row)) || !split_sizes || !group_offsets ||
-      !row_to_slot || !prob_perm || !xq || !xq_sf)
+  // arrays with a token dimension may be null for an empty batch (T == 0);
+  // without xq (and xq_sf) only the index maps are produced
+  if ((T > 0 && (!topk_idx || !topk_prob || !slot_to_row || (xq && !x))) || !split_sizes || !group_offsets ||
+      !row_to_slot || !prob_perm)
     return MOE_ERR_INVALID;
-  if ((xq_col == nullptr) != (xq_col_sf == nullptr)) return MOE_ERR_INVALID;
+  if ((xq == nullptr) != (xq_sf == nullptr) || (xq_col == nullptr) != (xq_col_sf == nullptr)) return MOE_ERR_INVALID;
+  if (!xq && xq_col) return MOE_ERR_INVALID;
   if (T < 0 || H <= 0 || k <= 0 || E <= 0 || k > E) return MOE_ERR_INVALID;
   if (E > MOE_MAX_EXPERTS || H % 32 || int64_t(T) * k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
   if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
@@ -233,14 +262,15 @@ moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* to
                              row_to_slot, slot_to_row, prob_perm, workspace, st);
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (!xq) return MOE_OK;
   if (xq_col) {
     // training: x rows gathered once, quantised along H and along tokens
     QuantBothArgs qb{static_cast<const uint8_t*>(x), 1, rows_cap, H, rows_cap, xq, xq_sf, xq_col, xq_col_sf,
-                     row_to_slot, k};
+                     row_to_slot, k, group_offsets + E};
     TimeScope ts(st, "permute_quant");
     if ((e = launch_quant_both(qb, st)) != cudaSuccess) return MOE_ERR_CUDA;
   } else {
-    QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq, xq_sf};
+    QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq, xq_sf, group_offsets + E};
     TimeScope ts(st, "permute_quant");
     if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
   }
@@ -253,7 +283,7 @@ moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* o
   if (!device_ok()) return MOE_ERR_NO_DEVICE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   TimeScope ts(st, "combine");
-  return cuda_status(launch_combine(y, false, T, k, H, out, st));
+  return cuda_status(launch_combine(y, false, nullptr, T, k, H, out, st));
 }
 
 moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const uint8_t* w2q,
@@ -296,7 +326,7 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   g1.q_out = w.hq; g1.sf_out = w.hq_sf; g1.q_KT = int32_t(cdiv(I, 128));
   {
     TimeScope ts(st, "gemm_gate_up_swiglu");
-    if ((e = launch_grouped_gemm(EPI_SWIGLU, m1, g1, st)) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((e = launch_grouped_gemm(EPI_SWIGLU, 256, m1, g1, st)) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // down grouped GEMM, rows scattered to slot order
@@ -311,12 +341,69 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   g2.row_to_slot = row_to_slot; g2.out = w.y; g2.ld_out = H;
   {
     TimeScope ts(st, "gemm_down");
-    if ((e = launch_grouped_gemm(EPI_F32_SCATTER, m2, g2, st)) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((e = launch_grouped_gemm(EPI_F32_SCATTER, 256, m2, g2, st)) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // top-k combine back to token order
   TimeScope ts(st, "combine");
-  return cuda_status(launch_combine(w.y, true, T, k, H, out, st));
+  return cuda_status(launch_combine(w.y, true, nullptr, T, k, H, out, st));
+}
+
+moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down, int32_t T, int32_t H, int32_t I,
+                                      int32_t E, int32_t k, int64_t rows_cap, const int32_t* split_sizes,
+                                      const int32_t* group_offsets, const int32_t* row_to_slot,
+                                      const float* prob_perm, const void* x, void* out, void* workspace,
+                                      size_t workspace_bytes, moe_stream_t stream) {
+  if (!w_gate_up || !w_down || !split_sizes || !group_offsets || !row_to_slot || !prob_perm ||
+      (T > 0 && (!x || !out)))
+    return MOE_ERR_INVALID;
+  if (!layer_dims_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
+  for (const void* p : {w_gate_up, w_down, x, (const void*)out})
+    if (!al16(p)) return MOE_ERR_INVALID;
+  Carver c{static_cast<uint8_t*>(workspace)};
+  FwdBf16Ws w = carve_fwd_bf16(c, T, k, H, I, rows_cap);
+  if (!workspace || int64_t(workspace_bytes) < c.off) return MOE_ERR_WORKSPACE;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) return MOE_OK;
+  {
+    TimeScope ts(st, "gather_x_bf16");
+    const int64_t H16 = int64_t(H) / 8;
+    int64_t blocks = cdiv(rows_cap * H16, 256);
+    const int64_t cap = int64_t(device_sm_count()) * 16;
+    gather_rows_kernel<<<unsigned(blocks < cap ? blocks : cap), 256, 0, st>>>(
+        static_cast<const uint4*>(x), row_to_slot, group_offsets + E, k, H16, reinterpret_cast<uint4*>(w.xp));
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  // gate_up grouped GEMM (bf16) + ScaledSwiGLU, h in bf16; bf16 matrices
+  // are described to TMA as bytes (128-byte K tiles of 64 values)
+  GemmMaps m1;
+  if (make_map_2d(&m1.a, w.xp, 2 * int64_t(H), rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m1.b, w_gate_up, 2 * int64_t(H), I, 2 * int64_t(E), 128) != cudaSuccess) return MOE_ERR_CUDA;
+  GemmArgs g1{};
+  g1.mode = 0; g1.E = E; g1.N = I; g1.num_kt = int32_t(cdiv(2 * int64_t(H), 128)); g1.n_tiles = int32_t(cdiv(I, 128));
+  g1.group_offsets = group_offsets; g1.split_sizes = split_sizes;
+  g1.prob = prob_perm; g1.row_to_slot = row_to_slot; g1.q_out = w.h;
+  {
+    TimeScope ts(st, "gemm_gate_up_swiglu_bf16");
+    if (launch_grouped_gemm_bf16(EPI_SWIGLU_BF16, m1, g1, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  // down grouped GEMM (bf16), fp32 rows scattered to slot order
+  GemmMaps m2;
+  if (make_map_2d(&m2.a, w.h, 2 * int64_t(I), rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m2.b, w_down, 2 * int64_t(I), H, E, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  GemmArgs g2{};
+  g2.mode = 0; g2.E = E; g2.N = H; g2.num_kt = int32_t(cdiv(2 * int64_t(I), 128)); g2.n_tiles = int32_t(cdiv(H, 256));
+  g2.group_offsets = group_offsets; g2.split_sizes = split_sizes;
+  g2.row_to_slot = row_to_slot; g2.out = w.y; g2.ld_out = H;
+  {
+    TimeScope ts(st, "gemm_down_bf16");
+    if (launch_grouped_gemm_bf16(EPI_F32_SCATTER, m2, g2, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  TimeScope ts(st, "combine");
+  return cuda_status(launch_combine(w.y, true, nullptr, T, k, H, out, st));
 }
 
 moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, const uint8_t* w1tq,
@@ -346,34 +433,35 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
 
   // dy rows gathered to permuted order, quantised along H and along tokens
   QuantBothArgs qb{static_cast<const uint8_t*>(dY), 1, rows_cap, H, rows_cap, w.dyq, w.dyq_sf, w.dyc, w.dyc_sf,
-                   row_to_slot, k};
+                   row_to_slot, k, group_offsets + E};
   {
     TimeScope ts(st, "dy_quant");
     if ((e = launch_quant_both(qb, st)) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
-  // dgrad2: dh = dy W_down (contraction over H)
+  // dgrad2 + ScaledSwiGLU backward: dh = dy W_down (contraction over H) in
+  // TMEM; the epilogue quantises da = [dg | du] along 2I and along tokens and
+  // h along tokens, and sums dprob per 64-column chunk
   GemmMaps m;
   if (make_map_2d(&m.a, w.dyq, H, rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
-  if (make_map_3d(&m.b, w2tq, H, I, E, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m.b, w2tq, H, I, E, 128) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs g{};
-  g.mode = 0; g.E = E; g.N = I; g.num_kt = int32_t(cdiv(H, 128)); g.n_tiles = int32_t(cdiv(I, 256));
+  g.mode = 0; g.E = E; g.N = I; g.num_kt = int32_t(cdiv(H, 128)); g.n_tiles = int32_t(cdiv(I, 128));
   g.group_offsets = group_offsets; g.split_sizes = split_sizes;
   g.sfa = w.dyq_sf; g.a_KT = int32_t(cdiv(H, 128));
   g.sfb = w2tsf; g.b_RT = int32_t(cdiv(I, 128)); g.b_KT = int32_t(cdiv(H, 128));
-  g.out = w.dh; g.ld_out = I;
+  g.prob = prob_perm; g.saved = static_cast<const uint8_t*>(saved_a); g.rows_cap = rows_cap;
+  g.daq = w.daq; g.daq_sf = w.daq_sf; g.dacol = w.dac; g.dacol_sf = w.dac_sf; g.hcol = w.hc; g.hcol_sf = w.hc_sf;
+  g.dprob_part = reinterpret_cast<float*>(w.dpp);
   {
-    TimeScope ts(st, "gemm_dgrad_down");
-    if (launch_grouped_gemm(EPI_F32_ROWS, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+    TimeScope ts(st, "gemm_dgrad_down_swiglu");
+    if (launch_grouped_gemm(EPI_SWIGLU_BWD, 128, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
-
-  // ScaledSwiGLU backward + quantisation of da (both ways) and h (along tokens)
-  SwigluBwdArgs sb{I, E, rows_cap, group_offsets, row_to_slot, prob_perm, w.dh,
-                   static_cast<const uint8_t*>(saved_a), w.daq, w.daq_sf, w.dac, w.dac_sf, w.hc, w.hc_sf,
-                   dprob, reinterpret_cast<float*>(w.dpp)};
   {
-    TimeScope ts(st, "swiglu_bwd");
-    if (launch_swiglu_bwd(sb, st) != cudaSuccess) return MOE_ERR_CUDA;
+    TimeScope ts(st, "dprob_reduce");
+    if (launch_dprob_reduce(group_offsets, E, row_to_slot, rows_cap, reinterpret_cast<const float*>(w.dpp),
+                            I / 64, dprob, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
 
   // wgrad2: dW_down_e = dy_e^T h_e (contraction over the group's tokens)
@@ -388,10 +476,11 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   g.out = static_cast<uint8_t*>(dW2); g.ld_out = I; g.out_group_stride = int64_t(H) * I;
   {
     TimeScope ts(st, "gemm_wgrad_down");
-    if (launch_grouped_gemm(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_grouped_gemm(EPI_WGRAD, 256, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
-  // dgrad1: dx = da W_gate_up (contraction over 2I), rows scattered to slots
+  // dgrad1: dx = da W_gate_up (contraction over 2I), fp32 rows in permuted
+  // order; the combine gathers a token's k rows through slot_to_row
   if (make_map_2d(&m.a, w.daq, 2 * int64_t(I), rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
   if (make_map_3d(&m.b, w1tq, 2 * int64_t(I), H, E, 256) != cudaSuccess) return MOE_ERR_CUDA;
   g = GemmArgs{};
@@ -400,14 +489,14 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   g.group_offsets = group_offsets; g.split_sizes = split_sizes;
   g.sfa = w.daq_sf; g.a_KT = int32_t(cdiv(2 * int64_t(I), 128));
   g.sfb = w1tsf; g.b_RT = int32_t(cdiv(H, 128)); g.b_KT = int32_t(cdiv(2 * int64_t(I), 128));
-  g.row_to_slot = row_to_slot; g.out = w.dx; g.ld_out = H;
+  g.out = w.dx; g.ld_out = H;
   {
     TimeScope ts(st, "gemm_dgrad_gate_up");
-    if (launch_grouped_gemm(EPI_F32_SCATTER, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_grouped_gemm(EPI_F32_ROWS, 256, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
   {
     TimeScope ts(st, "combine_dx");
-    if (launch_combine(w.dx, true, T, k, H, dX, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_combine(w.dx, true, slot_to_row, T, k, H, dX, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // wgrad1: dW_gate_up_e = da_e^T x_e (contraction over the group's tokens)
@@ -422,9 +511,8 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   g.out = static_cast<uint8_t*>(dW1); g.ld_out = H; g.out_group_stride = 2 * int64_t(I) * H;
   {
     TimeScope ts(st, "gemm_wgrad_gate_up");
-    if (launch_grouped_gemm(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_grouped_gemm(EPI_WGRAD, 256, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
-  (void)slot_to_row;
   return MOE_OK;
 }
 
@@ -437,7 +525,54 @@ moe_status_t moe_router_topk(const void* logits, int32_t logits_dtype, int32_t T
   if (!device_ok()) return MOE_ERR_NO_DEVICE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   TimeScope ts(st, "router");
-  return cuda_status(launch_router_topk(logits, logits_dtype == MOE_DTYPE_BF16, T, E, k, topk_idx, topk_prob, st));
+  return cuda_status(launch_router_topk(logits, logits_dtype == MOE_DTYPE_BF16, T, E, k, topk_idx, topk_prob,
+                                       nullptr, st));
+}
+
+moe_status_t moe_route_permute(const void* logits, int32_t logits_dtype, const void* x, int32_t T, int32_t H,
+                               int32_t k, int32_t E, int64_t rows_cap, int32_t* topk_idx, float* topk_prob,
+                               int32_t* split_sizes, int32_t* group_offsets, int32_t* row_to_slot,
+                               int32_t* slot_to_row, float* prob_perm, uint8_t* xq, uint8_t* xq_sf, uint8_t* xq_col,
+                               uint8_t* xq_col_sf, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  if ((T > 0 && (!logits || !x || !topk_idx || !topk_prob || !slot_to_row)) || !split_sizes || !group_offsets ||
+      !row_to_slot || !prob_perm || !xq || !xq_sf)
+    return MOE_ERR_INVALID;
+  if (logits_dtype != MOE_DTYPE_F32 && logits_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID;
+  if ((xq_col == nullptr) != (xq_col_sf == nullptr)) return MOE_ERR_INVALID;
+  if (T < 0 || H <= 0 || k <= 0 || E <= 0 || k > E) return MOE_ERR_INVALID;
+  if (E > MOE_MAX_EXPERTS || k > 32 || H % 32 || int64_t(T) * k >= (int64_t(1) << 30)) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
+  if (!al16(x) || !al16(xq) || !al16(xq_sf) || (xq_col && (!al16(xq_col) || !al16(xq_col_sf))))
+    return MOE_ERR_INVALID;
+  const int64_t need = moe_workspace_size(MOE_OP_PERMUTE, T, k, E, H, 0);
+  if (!workspace || int64_t(workspace_bytes) < need) return MOE_ERR_WORKSPACE;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t R = int64_t(T) * k;
+  {
+    TimeScope ts(st, "route_permute_index");
+    if (cudaMemsetAsync(row_to_slot, 0xFF, size_t(rows_cap) * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(prob_perm, 0, size_t(rows_cap) * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(workspace, 0, size_t(cdiv(R, PERM_BLOCK) * E * 4), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (launch_router_topk(logits, logits_dtype == MOE_DTYPE_BF16, T, E, k, topk_idx, topk_prob,
+                           static_cast<int32_t*>(workspace), st) != cudaSuccess ||
+        launch_permute_scan_scatter(topk_idx, topk_prob, R, E, split_sizes, group_offsets, row_to_slot, slot_to_row,
+                                    prob_perm, workspace, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  cudaError_t e;
+  if (xq_col) {
+    QuantBothArgs qb{static_cast<const uint8_t*>(x), 1, rows_cap, H, rows_cap, xq, xq_sf, xq_col, xq_col_sf,
+                     row_to_slot, k, group_offsets + E};
+    TimeScope ts(st, "permute_quant");
+    if ((e = launch_quant_both(qb, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq, xq_sf, group_offsets + E};
+    TimeScope ts(st, "permute_quant");
+    if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
 }
 
 moe_status_t moe_get_device_status(moe_stream_t stream) {

@@ -341,6 +341,29 @@ __device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// D[tmem] (+)= A x B^T, bf16 operands from shared memory, fp32 accumulators
+// in TMEM (kind::f16).
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor of kind::f16 MMA: bf16 x bf16 -> fp32, both
+// K-major, M x N.
+__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N) {
+  return 1u << 4                  // D format F32
+         | 1u << 7                // A format BF16
+         | 1u << 10               // B format BF16
+         | 0u << 15 | 0u << 16    // both K-major
+         | uint32_t(N >> 3) << 17 // N / 8
+         | uint32_t(M >> 4) << 24;// M / 16
+}
+
 // Instruction descriptor of kind::mxf8f6f4 block-scaled MMA: E4M3 x E4M3,
 // both K-major, E8M0 scales, M x N, scale-factor byte ids for A and B.
 __host__ __device__ constexpr uint32_t make_idesc_mxf8(int M, int N, uint32_t a_sf_id,
@@ -358,8 +381,22 @@ __host__ __device__ constexpr uint32_t make_idesc_mxf8(int M, int N, uint32_t a_
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // TMEM -> registers, one warp, one instruction: 32 lanes x N consecutive
-// 32-bit columns (N = 64 or 128); thread i receives lane (base lane + i),
+// 32-bit columns (N = 32, 64 or 128); thread i receives lane (base lane + i),
 // columns [col, col + N) of the address `taddr` = (lane << 16) | col.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+      "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,"
+      "%24,%25,%26,%27,%28,%29,%30,%31"
+      "}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"

@@ -8,24 +8,32 @@
 //   Challenge 3 / Figure 4 -- gate_up GEMM, SwiGLU, routing-probability
 //                   scaling and requantisation fused into one kernel before
 //                   the down projection, so the BF16 intermediate is never
-//                   written.
+//                   written; the matching fused backward folds the
+//                   ScaledSwiGLU backward into the epilogue of the GEMM that
+//                   produces dh, so dh is never written either.
 //
-// Design (one CTA per SM, 320 threads):
-//   warp 0      TMA producer: A tile 128x128 B, B tile 256x128 B (2-D or
-//               3-D tensor maps, 128-byte swizzle), both scale atoms by bulk
-//               copy, into a 4-stage shared-memory ring (mbarrier pipeline).
+// Design (one CTA per SM, 320 threads), two tile widths BN:
+//   BN = 256: 128 x 256 tiles, one fp32 accumulator of 256 TMEM columns,
+//             4-stage shared-memory ring;
+//   BN = 128: 128 x 128 tiles, two accumulators of 128 columns (the MMAs of
+//             the next tile run while the epilogue drains the previous one,
+//             so the epilogue may read TMEM lazily and hold it longer),
+//             5-stage ring.
+//   warp 0      TMA producer: A tile 128x128 B, B tile BNx128 B (2-D or
+//               3-D tensor maps, 128-byte swizzle), the scale atoms by bulk
+//               copy, into the shared-memory ring (mbarrier pipeline).
 //   warp 1      TMEM owner and MMA issuer: per 128-wide K tile, copies the
 //               scale atoms to TMEM (tcgen05.cp 32x128b.warpx4) and issues
-//               four tcgen05.mma.kind::mxf8f6f4.block_scale (M128 N256 K32)
-//               into an fp32 accumulator of 256 TMEM columns.
+//               four tcgen05.mma.kind::mxf8f6f4.block_scale (M128 NBN K32)
+//               into the current accumulator.
 //   warps 2-9   epilogue: drain the accumulator into registers
-//               (tcgen05.ld), release it to the MMA warp at once, then apply
-//               the epilogue and store -- so the next tile's MMAs overlap it.
+//               (tcgen05.ld), release it to the MMA warp, then apply the
+//               epilogue and store -- so the next tile's MMAs overlap it.
 //               Rows go out through a per-warp shared staging buffer so that
 //               each store instruction writes 4 rows x 128 contiguous bytes
 //               (8 rows x 64 bytes for the SwiGLU epilogue's 64-byte pieces).
-// Tiles (128 rows x 256 columns) walk a device-side schedule derived from
-// the group offsets; every CTA strides through them (persistent grid).
+// Tiles walk a device-side schedule derived from the group offsets; every
+// CTA strides through them (persistent grid).
 // Every wait is bounded; on time-out the kernel records MOE_ERR_TIMEOUT,
 // stops all roles, lets its copies and MMAs in flight finish (bounded
 // waits again) and still frees its TMEM.
@@ -35,42 +43,50 @@ namespace moe {
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128, STAGES = 4;
-constexpr int SMEM_A = BM * BK;  // 16 KB
-constexpr int SMEM_B = BN * BK;  // 32 KB
-constexpr int SMEM_SFA = 512;
-constexpr int SMEM_SFB = 1024;
-constexpr uint32_t STAGE_TX = SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB;
+constexpr int BM = 128, BK = 128;
 constexpr int NUM_THREADS = 320;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 260;
+constexpr uint32_t SFA_COL = 256, SFB_COL = 260;  // accumulators use columns 0..255
+constexpr int STAGE_PITCH_W = 20;                  // words per staged 64-byte row (16 used): conflict-free v4
 
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * SMEM_A;
-constexpr int OFF_SFA = OFF_B + STAGES * SMEM_B;
-constexpr int OFF_SFB = OFF_SFA + STAGES * SMEM_SFA;
-constexpr int OFF_BAR = OFF_SFB + STAGES * SMEM_SFB;
-constexpr int NUM_BARS = 2 * STAGES + 3;
-constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem address, abort flag
-constexpr int OFF_GO = OFF_MISC + 16;              // group offsets [E+1]
-constexpr int STAGE_PITCH_W = 20;                  // words per staged row (16 used): conflict-free v4
-constexpr int STAGE_WARP_BYTES = 32 * STAGE_PITCH_W * 4;
-constexpr int OFF_STAGE = (OFF_GO + (MOE_MAX_EXPERTS + 1) * 4 + 127) / 128 * 128;
-constexpr int SMEM_TOTAL = OFF_STAGE + NUM_EPI_WARPS * STAGE_WARP_BYTES;
-constexpr int SMEM_LAUNCH = SMEM_TOTAL + 1024;     // slack for 1 KB alignment
+// Shared-memory plan and pipeline depth of the two tile widths.
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = BN == 256 ? 4 : 5;
+  static constexpr int ACC = BN == 256 ? 1 : 2;   // TMEM accumulators
+  static constexpr int SMEM_A = BM * BK;
+  static constexpr int SMEM_B = BN * BK;
+  static constexpr int SMEM_SFA = 512;
+  static constexpr int SMEM_SFB = BN * 4;          // one 512-byte atom per 128 rows of B
+  static constexpr uint32_t STAGE_TX = SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * SMEM_A;
+  static constexpr int OFF_SFA = OFF_B + STAGES * SMEM_B;
+  static constexpr int OFF_SFB = OFF_SFA + STAGES * SMEM_SFA;
+  static constexpr int OFF_BAR = OFF_SFB + STAGES * SMEM_SFB;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem address, abort flag
+  static constexpr int OFF_GO = OFF_MISC + 16;              // group offsets [E+1]
+  // per-warp staging: 32 rows x 20 words (64-byte rows) or 16 rows x 36 words
+  // (128-byte rows); BN = 128 also transposes 32 x 32 fp32 values (pitch 36)
+  static constexpr int STAGE_WARP_BYTES = BN == 256 ? 2560 : 32 * 36 * 4;
+  static constexpr int OFF_STAGE = (OFF_GO + (MOE_MAX_EXPERTS + 1) * 4 + 127) / 128 * 128;
+  static constexpr int SMEM_TOTAL = OFF_STAGE + NUM_EPI_WARPS * STAGE_WARP_BYTES;
+  static constexpr int SMEM_LAUNCH = SMEM_TOTAL + 1024;     // slack for 1 KB alignment
+  static_assert(SMEM_LAUNCH <= 232448, "shared memory plan exceeds 227 KB");
+};
 
 struct Tile {
   int e, m0, n0, kt0, nkt, row_end;
 };
 
-template <int EPI>
 __device__ __forceinline__ int total_tiles(const GemmArgs& a, const int* go) {
   if (a.mode == 0) return (go[a.E] >> 7) * a.n_tiles;
   return a.E * a.m_tiles * a.n_tiles;
 }
 
-template <int EPI>
+template <int EPI, int BN>
 __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, int t) {
   Tile ti;
   if (a.mode == 0) {
@@ -86,7 +102,7 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, in
     const int n_idx = local / mt, m_idx = local - n_idx * mt;  // rows fastest: B panel reuse
     ti.e = e;
     ti.m0 = go[e] + (m_idx << 7);
-    ti.n0 = n_idx * (EPI == EPI_SWIGLU ? 128 : 256);
+    ti.n0 = n_idx * ((EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16) ? BN / 2 : BN);
     ti.kt0 = 0;
     ti.nkt = a.num_kt;
     ti.row_end = go[e] + a.split_sizes[e];
@@ -97,7 +113,7 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, in
     const int n_idx = local / a.m_tiles, m_idx = local - n_idx * a.m_tiles;
     ti.e = e;
     ti.m0 = m_idx << 7;
-    ti.n0 = n_idx << 8;
+    ti.n0 = n_idx * BN;
     ti.kt0 = go[e] >> 7;
     ti.nkt = (go[e + 1] - go[e]) >> 7;
     ti.row_end = a.M_out;
@@ -117,7 +133,8 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, in
 // The staged pitch (144 bytes, or 80 for 64-byte rows) keeps the 16-byte
 // shared stores and loads free of bank conflicts.
 constexpr int STAGE128_PITCH_W = 36;
-static_assert(16 * STAGE128_PITCH_W * 4 <= STAGE_WARP_BYTES, "staging buffer too small");
+static_assert(16 * STAGE128_PITCH_W * 4 <= Cfg<256>::STAGE_WARP_BYTES, "staging buffer too small");
+static_assert(32 * STAGE_PITCH_W * 4 <= Cfg<256>::STAGE_WARP_BYTES, "staging buffer too small");
 
 template <int NW>
 __device__ __forceinline__ void warp_store_rows(uint32_t* stage, uint8_t* row, const uint32_t* w, int bytes,
@@ -181,12 +198,38 @@ __device__ __forceinline__ void pack_bf16_inplace(uint32_t* v) {
   for (int i = 0; i < NW; ++i) v[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
 }
 
-template <int EPI>
+// Epilogue of one tile for the warp that owns TMEM sub-partition q (rows
+// 32q..32q+31 of the tile) and column half `half` (BN/2 columns).  v holds the
+// warp's accumulator values: EPI_SWIGLU (BN = 256) 64 gate + 64 up columns,
+// the others BN/2 columns.
+template <int EPI, int BN>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti, uint32_t* v, int q, int half,
                                               int lane, uint32_t* stage) {
+  constexpr int NC = BN / 2;  // accumulator columns per warp
   const int r = ti.m0 + 32 * q + lane;
   const bool rv = r < ti.row_end;
-  if constexpr (EPI == EPI_SWIGLU) {
+  if constexpr (EPI == EPI_SWIGLU_BF16) {
+    static_assert(BN == 256, "the gate_up epilogue pairs 128 gate with 128 up columns");
+    // v[0:64] gate columns nb..nb+63, v[64:128] the matching up columns;
+    // h = p * silu(g) * u leaves in bf16 (the BF16 path keeps h in 16 bits)
+    const int nb = ti.n0 + 64 * half;
+    if (nb >= a.N) return;  // uniform across the warp
+    const float p = rv ? a.prob[r] : 0.0f;
+    uint32_t hw[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float h2[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float g = __uint_as_float(v[2 * j + i]);
+        const float u = __uint_as_float(v[64 + 2 * j + i]);
+        h2[i] = p * __fdividef(g, 1.0f + __expf(-g)) * u;
+      }
+      hw[j] = pack_bf16x2(h2[0], h2[1]);
+    }
+    warp_store_rows<32>(stage, rv ? a.q_out + (int64_t(r) * a.N + nb) * 2 : nullptr, hw, 128, lane);
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    static_assert(BN == 256, "the gate_up epilogue pairs 128 gate with 128 up columns");
     // v[0:64] gate columns nb..nb+63, v[64:128] the matching up columns
     const int nb = ti.n0 + 64 * half;
     if (nb >= a.N) return;  // uniform across the warp
@@ -237,9 +280,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
         *reinterpret_cast<uint16_t*>(sfp) = uint16_t(sbs);
     }
   } else {
-    const int nb = ti.n0 + 128 * half;
+    const int nb = ti.n0 + NC * half;
     if (nb >= a.N) return;  // uniform across the warp
-    const int ncols = min(128, a.N - nb);
+    const int ncols = min(NC, a.N - nb);
     if constexpr (EPI == EPI_F32_SCATTER || EPI == EPI_F32_ROWS) {
       uint8_t* dst = nullptr;
       if (rv) {
@@ -247,29 +290,161 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
         if constexpr (EPI == EPI_F32_SCATTER) orow = a.row_to_slot[r];
         if (orow >= 0) dst = a.out + (orow * a.ld_out + nb) * 4;
       }
-      warp_store_rows<128>(stage, dst, v, ncols * 4, lane);
+      warp_store_rows<NC>(stage, dst, v, ncols * 4, lane);
     } else {
-      pack_bf16_inplace<64>(v);
+      pack_bf16_inplace<NC / 2>(v);
       uint8_t* dst = rv ? a.out + (int64_t(ti.e) * a.out_group_stride + int64_t(r) * a.ld_out + nb) * 2 : nullptr;
-      warp_store_rows<64>(stage, dst, v, ncols * 2, lane);
+      warp_store_rows<NC / 2>(stage, dst, v, ncols * 2, lane);
     }
   }
 }
 
-template <int EPI>
+// ---------------------------------------------------------------------------
+// EPI_SWIGLU_BWD (BN = 128): the ScaledSwiGLU backward on the dh tile.
+// The warp owns rows rb..rb+31 (one 32-row block along tokens: groups start
+// on multiples of 128) and dh columns cb..cb+63, read from TMEM in two
+// chunks of 32.  Per element, with g, u from the saved bf16 A and p the row's
+// routing probability:
+//   sig = 1/(1+exp(-g)), s = g*sig
+//   dg = dh*p*u*sig*(1+g*(1-sig)),  du = dh*p*s,  h = p*s*u,  dprob += dh*s*u
+// dg and du are quantised along 2I (one 32-block per chunk, in the thread)
+// and, like h, along tokens: the chunk is transposed through the warp's
+// staging buffer and lane c quantises column c over the warp's 32 rows.
+// Rows past the group's last token hold zeros in every output.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_elem(const uint4* v, int e) {
+  const uint4 w4 = v[e >> 3];
+  const int i = (e >> 1) & 3;
+  const uint32_t w = i == 0 ? w4.x : (i == 1 ? w4.y : (i == 2 ? w4.z : w4.w));
+  return (e & 1) ? bf16hi(w) : bf16lo(w);
+}
+
+// 32 values -> E4M3 codes + E8M0 scale byte; codes stored at dst (32 bytes).
+__device__ __forceinline__ uint32_t encode32_store(const float* o, uint8_t* dst) {
+  const uint32_t sb = e8m0_from_amax_bits(__float_as_uint(abs_max_n<32>(o)));
+  const float inv = inv_scale_from_e8m0(sb);
+  uint32_t w[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) w[j] = pack4_e4m3(o[4 * j] * inv, o[4 * j + 1] * inv, o[4 * j + 2] * inv, o[4 * j + 3] * inv);
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  return sb;
+}
+
+constexpr int TP_W = 36;  // words per transposed row (conflict-free 16-byte stores and column reads)
+
+// Column-wise quantisation of a 32 x 32 chunk held one row per lane: lane c
+// writes the codes of column `col0 + c` over the warp's 32 rows to
+// q + (col0 + c) * ld + rb and its scale byte to the blocked layout.
+__device__ __forceinline__ void quant_cols32(const float* o, uint32_t* stage, int lane, uint8_t* q, uint8_t* sf,
+                                             int64_t col0, int64_t ld, int64_t rb, int64_t KT) {
+  __syncwarp();
+  float4* srow = reinterpret_cast<float4*>(stage + lane * TP_W);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) srow[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+  __syncwarp();
+  float f[32];
+#pragma unroll
+  for (int rr = 0; rr < 32; ++rr) f[rr] = __uint_as_float(stage[rr * TP_W + lane]);
+  const int64_t col = col0 + lane;
+  const uint32_t sb = encode32_store(f, q + col * ld + rb);
+  sf[sf_offset(0, col, rb >> 5, 0, KT)] = uint8_t(sb);
+}
+
+// dh columns [col, col + 32) of the warp's 32 rows from TMEM (zero for rows
+// past the group's last token).
+__device__ __forceinline__ void load_dh32(uint32_t taddr, bool rv, uint32_t* d) {
+  tmem_ld32(taddr, d);
+  tc_wait_ld();
+  if (!rv) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) d[e] = 0u;
+  }
+}
+
+__device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Tile& ti, uint32_t tl, int q, int half,
+                                                    int lane, uint32_t* stage) {
+  const int I = a.N;
+  const int cb = ti.n0 + 64 * half;
+  if (cb >= I) return;  // uniform across the warp
+  const int64_t rb = ti.m0 + 32 * q;
+  const int64_t r = rb + lane;
+  const bool rv = r < ti.row_end;
+  const int64_t I2 = 2 * int64_t(I);
+  const int64_t KT2 = I2 / 128, KTt = a.rows_cap / 128;
+  const float p = rv ? a.prob[r] : 0.0f;
+  const uint8_t* grow = a.saved + (r * I2 + cb) * 2;
+  float dps = 0.0f;
+  uint32_t sb_dg = 0, sb_du = 0;
+  // dh is read from TMEM once per output quantity rather than held in
+  // registers across all three (the accumulator stays ours until released)
+#pragma unroll 1
+  for (int j = 0; j < 2; ++j) {
+    const int cc = cb + 32 * j;
+    const uint32_t tc = tl + 64 * half + 32 * j;
+    uint4 gv[4], uv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      gv[i] = rv ? __ldg(reinterpret_cast<const uint4*>(grow + 64 * j) + i) : make_uint4(0u, 0u, 0u, 0u);
+      uv[i] = rv ? __ldg(reinterpret_cast<const uint4*>(grow + int64_t(I) * 2 + 64 * j) + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float sg[32], o[32];
+    uint32_t d[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) sg[e] = __fdividef(1.0f, 1.0f + __expf(-bf16_elem(gv, e)));
+    // dg, quantised along 2I (columns cc..cc+31) and along tokens
+    load_dh32(tc, rv, d);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float g = bf16_elem(gv, e), u = bf16_elem(uv, e);
+      o[e] = (__uint_as_float(d[e]) * p) * (u * sg[e]) * fmaf(g, 1.0f - sg[e], 1.0f);
+    }
+    sb_dg |= encode32_store(o, a.daq + r * I2 + cc) << (8 * j);
+    quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, cc, a.rows_cap, rb, KTt);
+    // du, quantised along 2I (columns I+cc..) and along tokens
+    load_dh32(tc, rv, d);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) o[e] = (__uint_as_float(d[e]) * p) * (bf16_elem(gv, e) * sg[e]);
+    sb_du |= encode32_store(o, a.daq + r * I2 + I + cc) << (8 * j);
+    quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, int64_t(I) + cc, a.rows_cap, rb, KTt);
+    // h = p*s*u along tokens (operand of the down projection's weight
+    // gradient); dprob partial sum
+    load_dh32(tc, rv, d);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float su = (bf16_elem(gv, e) * sg[e]) * bf16_elem(uv, e);
+      o[e] = p * su;
+      dps = fmaf(__uint_as_float(d[e]), su, dps);
+    }
+    quant_cols32(o, stage, lane, a.hcol, a.hcol_sf, cc, a.rows_cap, rb, KTt);
+  }
+  // scale bytes of dg and du along 2I: blocks cb/32, cb/32+1 (cb % 64 == 0,
+  // so the pair shares a 4-byte group of the atom)
+  *reinterpret_cast<uint16_t*>(a.daq_sf + sf_offset(0, r, cb >> 5, 0, KT2)) = uint16_t(sb_dg);
+  *reinterpret_cast<uint16_t*>(a.daq_sf + sf_offset(0, r, (int64_t(I) + cb) >> 5, 0, KT2)) = uint16_t(sb_du);
+  a.dprob_part[int64_t(cb >> 6) * a.rows_cap + r] = dps;
+}
+
+template <int EPI, int BN, int KIND>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_mxf8_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB, const GemmArgs a) {
+  using C = Cfg<BN>;
+  constexpr int STAGES = C::STAGES, ACC = C::ACC;
+  constexpr bool MX = KIND == KIND_MXF8;
+  constexpr bool GATE_UP = EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16;  // B tile = gate rows + up rows
+  constexpr uint32_t TX = MX ? C::STAGE_TX : uint32_t(C::SMEM_A + C::SMEM_B);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;  // MMA completion on the abort path
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
-  int* go = reinterpret_cast<int*>(smem + OFF_GO);
+  uint64_t* acc_full = empty + STAGES;   // [ACC]
+  uint64_t* acc_empty = acc_full + ACC;  // [ACC]
+  uint64_t* drain = acc_empty + ACC;     // MMA completion on the abort path
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  int* go = reinterpret_cast<int*>(smem + C::OFF_GO);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -278,8 +453,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, NUM_EPI_WARPS);
+    for (int b = 0; b < ACC; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], NUM_EPI_WARPS);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -293,7 +470,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int ntiles = total_tiles<EPI>(a, go);
+  const int ntiles = total_tiles(a, go);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -305,36 +482,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t issued = 0;  // stages armed so far
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile ti = decode_tile<EPI>(a, go, t);
+        const Tile ti = decode_tile<EPI, BN>(a, go, t);
         for (int kt = 0; kt < ti.nkt; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           ++issued;
           uint64_t* bar = &full[stage];
-          mbar_arrive_expect_tx(bar, STAGE_TX);
+          mbar_arrive_expect_tx(bar, TX);
           const int kg = ti.kt0 + kt;
-          uint8_t* sa = smem + OFF_A + stage * SMEM_A;
-          uint8_t* sb = smem + OFF_B + stage * SMEM_B;
-          uint8_t* ssfa = smem + OFF_SFA + stage * SMEM_SFA;
-          uint8_t* ssfb = smem + OFF_SFB + stage * SMEM_SFB;
+          uint8_t* sa = smem + C::OFF_A + stage * C::SMEM_A;
+          uint8_t* sb = smem + C::OFF_B + stage * C::SMEM_B;
+          uint8_t* ssfa = smem + C::OFF_SFA + stage * C::SMEM_SFA;
+          uint8_t* ssfb = smem + C::OFF_SFB + stage * C::SMEM_SFB;
           tma_load_2d(sa, &tmA, bar, kg * BK, ti.m0);
-          bulk_load(ssfa, a.sfa + (int64_t(ti.m0 >> 7) * a.a_KT + kg) * 512, 512, bar);
-          if constexpr (EPI == EPI_SWIGLU) {
+          if constexpr (MX) bulk_load(ssfa, a.sfa + (int64_t(ti.m0 >> 7) * a.a_KT + kg) * 512, 512, bar);
+          if constexpr (GATE_UP) {
             tma_load_3d(sb, &tmB, bar, kg * BK, ti.n0, 2 * ti.e);
-            tma_load_3d(sb + SMEM_B / 2, &tmB, bar, kg * BK, ti.n0, 2 * ti.e + 1);
-            const int rb = ti.n0 >> 7;
-            bulk_load(ssfb, a.sfb + ((int64_t(2 * ti.e) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
-            bulk_load(ssfb + 512, a.sfb + ((int64_t(2 * ti.e + 1) * a.b_RT + rb) * a.b_KT + kg) * 512,
-                      512, bar);
+            tma_load_3d(sb + C::SMEM_B / 2, &tmB, bar, kg * BK, ti.n0, 2 * ti.e + 1);
+            if constexpr (MX) {
+              const int rb = ti.n0 >> 7;
+              bulk_load(ssfb, a.sfb + ((int64_t(2 * ti.e) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
+              bulk_load(ssfb + 512, a.sfb + ((int64_t(2 * ti.e + 1) * a.b_RT + rb) * a.b_KT + kg) * 512,
+                        512, bar);
+            }
           } else {
             if (a.mode == 0)
               tma_load_3d(sb, &tmB, bar, kg * BK, ti.n0, ti.e);
             else
               tma_load_2d(sb, &tmB, bar, kg * BK, ti.n0);
-            const int64_t gb = a.mode == 0 ? int64_t(ti.e) * a.b_RT : 0;
+            if constexpr (MX) {
+              const int64_t gb = a.mode == 0 ? int64_t(ti.e) * a.b_RT : 0;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int rb = min((ti.n0 >> 7) + h, a.b_RT - 1);  // rows past N: any finite atom
-              bulk_load(ssfb + 512 * h, a.sfb + ((gb + rb) * a.b_KT + kg) * 512, 512, bar);
+              for (int h = 0; h < BN / 128; ++h) {
+                const int rb = min((ti.n0 >> 7) + h, a.b_RT - 1);  // rows past N: any finite atom
+                bulk_load(ssfb + 512 * h, a.sfb + ((gb + rb) * a.b_KT + kg) * 512, 512, bar);
+              }
             }
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -356,32 +537,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       const uint32_t sfa_t = tmem + SFA_COL, sfb_t = tmem + SFB_COL;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile ti = decode_tile<EPI>(a, go, t);
+        const Tile ti = decode_tile<EPI, BN>(a, go, t);
         if (ti.nkt == 0) continue;
-        if (!mbar_wait(acc_empty, (acc_it & 1u) ^ 1u, abort_flag)) break;
+        const uint32_t buf = acc_it % ACC, use = acc_it / ACC;
+        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, abort_flag)) break;
         tc_fence_after();
+        const uint32_t acc = tmem + buf * BN;
         for (int kt = 0; kt < ti.nkt; ++kt) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + OFF_A + stage * SMEM_A);
-          const uint32_t sb = smem_u32(smem + OFF_B + stage * SMEM_B);
-          const uint32_t ssfa = smem_u32(smem + OFF_SFA + stage * SMEM_SFA);
-          const uint32_t ssfb = smem_u32(smem + OFF_SFB + stage * SMEM_SFB);
-          tc_cp_32x128b_warpx4(sfa_t, make_smem_desc(ssfa, 0, 128, 0));
-          tc_cp_32x128b_warpx4(sfb_t, make_smem_desc(ssfb, 0, 128, 0));
-          tc_cp_32x128b_warpx4(sfb_t + 4, make_smem_desc(ssfb + 512, 0, 128, 0));
+          const uint32_t sa = smem_u32(smem + C::OFF_A + stage * C::SMEM_A);
+          const uint32_t sb = smem_u32(smem + C::OFF_B + stage * C::SMEM_B);
+          const uint32_t ssfa = smem_u32(smem + C::OFF_SFA + stage * C::SMEM_SFA);
+          const uint32_t ssfb = smem_u32(smem + C::OFF_SFB + stage * C::SMEM_SFB);
+          if constexpr (MX) {
+            tc_cp_32x128b_warpx4(sfa_t, make_smem_desc(ssfa, 0, 128, 0));
+#pragma unroll
+            for (int h = 0; h < BN / 128; ++h)
+              tc_cp_32x128b_warpx4(sfb_t + 4 * h, make_smem_desc(ssfb + 512 * h, 0, 128, 0));
+          }
+          // four MMAs of 32 bytes of K each (32 E4M3 values, or 16 bf16)
 #pragma unroll
           for (uint32_t kk = 0; kk < 4; ++kk) {
             const uint64_t ad = make_smem_desc(sa + 32 * kk, 16, 1024, 2);
             const uint64_t bd = make_smem_desc(sb + 32 * kk, 16, 1024, 2);
-            tc_mma_mxf8(tmem + ACC_COL, ad, bd, make_idesc_mxf8(BM, BN, kk, kk), sfa_t | (kk << 30),
-                        sfb_t | (kk << 30), (kt | kk) != 0 ? 1u : 0u);
+            if constexpr (MX)
+              tc_mma_mxf8(acc, ad, bd, make_idesc_mxf8(BM, BN, kk, kk), sfa_t | (kk << 30),
+                          sfb_t | (kk << 30), (kt | kk) != 0 ? 1u : 0u);
+            else
+              tc_mma_bf16(acc, ad, bd, make_idesc_bf16(BM, BN), (kt | kk) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        tc_commit(&acc_full[buf]);
         ++acc_it;
       }
       if (*abort_flag) {
@@ -395,34 +585,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ---------------- epilogue warps ----------------
     const int q = warp & 3;            // TMEM sub-partition this warp may read
     const int half = (warp - 2) >> 2;  // which half of the tile's columns
-    uint32_t* stage = reinterpret_cast<uint32_t*>(smem + OFF_STAGE + (warp - 2) * STAGE_WARP_BYTES);
+    uint32_t* stage = reinterpret_cast<uint32_t*>(smem + C::OFF_STAGE + (warp - 2) * C::STAGE_WARP_BYTES);
     uint32_t acc_it = 0;
-    uint32_t v[128];
+    uint32_t v[BN / 2];
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      const Tile ti = decode_tile<EPI>(a, go, t);
+      const Tile ti = decode_tile<EPI, BN>(a, go, t);
       if (ti.nkt == 0) {
         if constexpr (EPI == EPI_WGRAD) {
 #pragma unroll
-          for (int i = 0; i < 128; ++i) v[i] = 0u;
-          epilogue_tile<EPI>(a, ti, v, q, half, lane, stage);
+          for (int i = 0; i < BN / 2; ++i) v[i] = 0u;
+          epilogue_tile<EPI, BN>(a, ti, v, q, half, lane, stage);
         }
         continue;
       }
-      if (!mbar_wait(acc_full, acc_it & 1u, abort_flag)) break;
+      const uint32_t buf = acc_it % ACC, use = acc_it / ACC;
+      if (!mbar_wait(&acc_full[buf], use & 1u, abort_flag)) break;
       tc_fence_after();
-      const uint32_t tl = tmem + (uint32_t(32 * q) << 16) + ACC_COL;
-      if constexpr (EPI == EPI_SWIGLU) {  // gate columns 64*half.., up columns 128 + 64*half..
-        tmem_ld64(tl + 64 * half, v);
-        tmem_ld64(tl + 128 + 64 * half, v + 64);
+      const uint32_t tl = tmem + (uint32_t(32 * q) << 16) + buf * BN;
+      if constexpr (EPI == EPI_SWIGLU_BWD) {
+        // reads TMEM chunk by chunk; the other accumulator keeps the MMAs busy
+        epilogue_swiglu_bwd(a, ti, tl, q, half, lane, stage);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
       } else {
-        tmem_ld128(tl + 128 * half, v);
+        if constexpr (GATE_UP) {  // gate columns 64*half.., up columns 128 + 64*half..
+          tmem_ld64(tl + 64 * half, v);
+          tmem_ld64(tl + 128 + 64 * half, v + 64);
+        } else if constexpr (BN == 256) {
+          tmem_ld128(tl + 128 * half, v);
+        } else {
+          tmem_ld64(tl + 64 * half, v);
+        }
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        epilogue_tile<EPI, BN>(a, ti, v, q, half, lane, stage);
       }
-      tc_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
       ++acc_it;
-      epilogue_tile<EPI>(a, ti, v, q, half, lane, stage);
     }
   }
 
@@ -451,12 +652,13 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <int EPI>
+template <int EPI, int BN, int KIND = KIND_MXF8>
 cudaError_t launch_epi(const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
   static std::atomic<uint64_t> configured{0};
-  cudaError_t e = ensure_smem_limit(grouped_mxf8_gemm_kernel<EPI>, SMEM_LAUNCH, configured);
+  constexpr int smem = Cfg<BN>::SMEM_LAUNCH;
+  cudaError_t e = ensure_smem_limit(grouped_mxf8_gemm_kernel<EPI, BN, KIND>, smem, configured);
   if (e != cudaSuccess) return e;
-  grouped_mxf8_gemm_kernel<EPI><<<device_sm_count(), NUM_THREADS, SMEM_LAUNCH, st>>>(maps.a, maps.b, a);
+  grouped_mxf8_gemm_kernel<EPI, BN, KIND><<<device_sm_count(), NUM_THREADS, smem, st>>>(maps.a, maps.b, a);
   count_launch();
   return cudaGetLastError();
 }
@@ -490,12 +692,29 @@ cudaError_t make_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t launch_grouped_gemm(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
+cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
+  if (bn == 256) {
+    switch (epi) {
+      case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, 256>(maps, a, st);
+      case EPI_F32_SCATTER: return launch_epi<EPI_F32_SCATTER, 256>(maps, a, st);
+      case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256>(maps, a, st);
+      case EPI_WGRAD: return launch_epi<EPI_WGRAD, 256>(maps, a, st);
+    }
+  } else if (bn == 128) {
+    switch (epi) {
+      case EPI_F32_SCATTER: return launch_epi<EPI_F32_SCATTER, 128>(maps, a, st);
+      case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 128>(maps, a, st);
+      case EPI_WGRAD: return launch_epi<EPI_WGRAD, 128>(maps, a, st);
+      case EPI_SWIGLU_BWD: return launch_epi<EPI_SWIGLU_BWD, 128>(maps, a, st);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_grouped_gemm_bf16(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
   switch (epi) {
-    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(maps, a, st);
-    case EPI_F32_SCATTER: return launch_epi<EPI_F32_SCATTER>(maps, a, st);
-    case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS>(maps, a, st);
-    case EPI_WGRAD: return launch_epi<EPI_WGRAD>(maps, a, st);
+    case EPI_SWIGLU_BF16: return launch_epi<EPI_SWIGLU_BF16, 256, KIND_BF16>(maps, a, st);
+    case EPI_F32_SCATTER: return launch_epi<EPI_F32_SCATTER, 256, KIND_BF16>(maps, a, st);
   }
   return cudaErrorInvalidValue;
 }

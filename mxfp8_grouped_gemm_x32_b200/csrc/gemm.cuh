@@ -9,7 +9,15 @@ enum EpiKind : int {
   EPI_SWIGLU = 0,        // gate_up: h = p * silu(gate) * up, requantised to MXFP8 (+ saved A in bf16)
   EPI_F32_SCATTER = 1,   // down / dgrad1: fp32 rows written to their slot (row_to_slot)
   EPI_F32_ROWS = 2,      // dgrad2: fp32 rows in permuted order (feeds the requantising SwiGLU backward)
-  EPI_WGRAD = 3          // weight gradients: one bf16 matrix per expert
+  EPI_WGRAD = 3,         // weight gradients: one bf16 matrix per expert
+  EPI_SWIGLU_BWD = 4,    // dgrad2 + ScaledSwiGLU backward: da (along 2I and tokens), h (tokens), dprob partials
+  EPI_SWIGLU_BF16 = 5    // BF16 path gate_up: h = p * silu(gate) * up written in bf16 (q_out)
+};
+
+// Operand kind of the tensor-core MMA.
+enum MmaKind : int {
+  KIND_MXF8 = 0,  // E4M3 x E4M3 with E8M0 block scales (kind::mxf8f6f4.block_scale)
+  KIND_BF16 = 1   // bf16 x bf16, no scales (kind::f16); operands are addressed as bytes, 64 values per K tile
 };
 
 // One grouped GEMM  D = (A * SFA) (B * SFB)^T  over ragged expert groups.
@@ -39,14 +47,26 @@ struct GemmArgs {
   int64_t ld_out;     // elements between output rows
   int64_t out_group_stride;  // mode 1: elements between experts' matrices
   uint8_t* out2;      // EPI_SWIGLU: saved A, bf16 [rows][2N] (nullable)
-  uint8_t* q_out;     // EPI_SWIGLU: h codes [rows][N]
+  uint8_t* q_out;     // EPI_SWIGLU: h codes [rows][N]; EPI_SWIGLU_BF16: h bf16 [rows][N]
   uint8_t* sf_out;    // EPI_SWIGLU: h scales, blocked (1, rows, N)
   int32_t q_KT;
+  // EPI_SWIGLU_BWD (N = I): saved A bf16 [rows_cap][2I] (gate | up); outputs
+  // da = [dg | du] MX (1, rows_cap, 2I) and MX along tokens (1, 2I, rows_cap),
+  // h MX along tokens (1, I, rows_cap), dprob partial sums [I/64][rows_cap]
+  const uint8_t* saved;
+  int64_t rows_cap;
+  uint8_t* daq;
+  uint8_t* daq_sf;
+  uint8_t* dacol;
+  uint8_t* dacol_sf;
+  uint8_t* hcol;
+  uint8_t* hcol_sf;
+  float* dprob_part;
 };
 
 // Tensor maps: A 2-D {K, rows} with a 128 x 128 box; B either 3-D
-// {K, rows, groups} or 2-D {K, rows} with a 128 x (128|256) box; all uint8
-// with 128-byte swizzle.
+// {K, rows, groups} or 2-D {K, rows} with a 128 x bn box (EPI_SWIGLU: two
+// boxes of bn/2 rows); all uint8 with 128-byte swizzle.
 struct GemmMaps {
   CUtensorMap a, b;
 };
@@ -56,6 +76,13 @@ cudaError_t make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64
 cudaError_t make_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                         uint64_t groups, uint32_t box_rows);
 
-cudaError_t launch_grouped_gemm(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);
+// bn: tile width, 256 (one accumulator) or 128 (two accumulators; required
+// by EPI_SWIGLU_BWD, not offered for EPI_SWIGLU).
+cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);
+
+// BF16 operands (kind::f16), bn = 256: EPI_SWIGLU_BF16 and EPI_F32_SCATTER.
+// The tensor maps describe the bf16 matrices as bytes (inner extent 2K), and
+// num_kt / a_KT count 128-byte K tiles.
+cudaError_t launch_grouped_gemm_bf16(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);
 
 }  // namespace moe

@@ -7,3 +7,4 @@
 #include "swiglu_bwd.cu"
 #include "noalloc.cu"
 #include "router.cu"
+#include "scales.cu"

@@ -11,7 +11,7 @@
 
 namespace moe {
 
-constexpr int PB = 1024;  // slots per block of the counting sort
+constexpr int PB = PERM_BLOCK;
 
 __device__ __forceinline__ bool id_ok(int32_t e, int32_t E) { return e >= 0 && e < E; }
 
@@ -106,24 +106,28 @@ __global__ void __launch_bounds__(PB) perm_scatter_kernel(const int32_t* __restr
   }
 }
 
-// out[t] = sum_j y[t*k + j], fp32 sum in ascending j, 8 columns per thread.
-// F32_IN: y holds fp32 rows (the grouped GEMM's scatter output), else bf16.
+// out[t] = sum_j y[row(t, j)], fp32 sum in ascending j, 8 columns per thread;
+// row(t, j) = t*k + j (rows in slot order) or slot_to_row[t*k + j] (rows in
+// permuted order).  F32_IN: y holds fp32 rows (a grouped GEMM's output),
+// else bf16.
 template <bool F32_IN>
-__global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ yv, int64_t T, int32_t k,
-                                                      int64_t H8, uint4* __restrict__ out) {
+__global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ yv, const int32_t* __restrict__ slot_to_row,
+                                                      int64_t T, int32_t k, int64_t H8, uint4* __restrict__ out) {
   const int64_t n = T * H8;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
        i += int64_t(gridDim.x) * blockDim.x) {
     const int64_t t = i / H8, c = i % H8;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     for (int j = 0; j < k; ++j) {
+      const int64_t row = slot_to_row ? int64_t(__ldg(slot_to_row + t * k + j)) : t * k + j;
+      if (row < 0) continue;  // a slot whose expert id was rejected
       if constexpr (F32_IN) {
-        const float4* y = static_cast<const float4*>(yv) + ((t * k + j) * H8 + c) * 2;
+        const float4* y = static_cast<const float4*>(yv) + (row * H8 + c) * 2;
         const float4 v0 = __ldg(y), v1 = __ldg(y + 1);
         acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
         acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
       } else {
-        const uint4 v = __ldg(static_cast<const uint4*>(yv) + (t * k + j) * H8 + c);
+        const uint4 v = __ldg(static_cast<const uint4*>(yv) + row * H8 + c);
         acc[0] += bf16lo(v.x); acc[1] += bf16hi(v.x);
         acc[2] += bf16lo(v.y); acc[3] += bf16hi(v.y);
         acc[4] += bf16lo(v.z); acc[5] += bf16hi(v.z);
@@ -137,6 +141,21 @@ __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y
 
 int64_t permute_workspace_bytes(int64_t R, int32_t E) {
   return cdiv(R, PB) * int64_t(E) * 4 + 256;
+}
+
+cudaError_t launch_permute_scan_scatter(const int32_t* idx, const float* prob, int64_t R, int32_t E,
+                                        int32_t* split, int32_t* offs, int32_t* row_to_slot, int32_t* slot_to_row,
+                                        float* prob_perm, void* ws, cudaStream_t st) {
+  const int32_t nb = int32_t(cdiv(R, PB));
+  int32_t* hist = static_cast<int32_t*>(ws);
+  perm_scan_kernel<<<1, MOE_MAX_EXPERTS, 0, st>>>(hist, nb, E, split, offs);
+  count_launch();
+  if (nb > 0) {
+    perm_scatter_kernel<<<nb, PB, 32 * E * sizeof(int), st>>>(idx, prob, R, E, hist, slot_to_row,
+                                                               row_to_slot, prob_perm);
+    count_launch();
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_permute_index(const int32_t* idx, const float* prob, int64_t R, int32_t E,
@@ -153,26 +172,19 @@ cudaError_t launch_permute_index(const int32_t* idx, const float* prob, int64_t 
     perm_hist_kernel<<<nb, PB, E * sizeof(int), st>>>(idx, R, E, hist);
     count_launch();
   }
-  perm_scan_kernel<<<1, MOE_MAX_EXPERTS, 0, st>>>(hist, nb, E, split, offs);
-  count_launch();
-  if (nb > 0) {
-    perm_scatter_kernel<<<nb, PB, 32 * E * sizeof(int), st>>>(idx, prob, R, E, hist, slot_to_row,
-                                                               row_to_slot, prob_perm);
-    count_launch();
-  }
-  return cudaGetLastError();
+  return launch_permute_scan_scatter(idx, prob, R, E, split, offs, row_to_slot, slot_to_row, prob_perm, ws, st);
 }
 
-cudaError_t launch_combine(const void* y, bool f32_in, int64_t T, int32_t k, int64_t H, void* out,
-                           cudaStream_t st) {
+cudaError_t launch_combine(const void* y, bool f32_in, const int32_t* slot_to_row, int64_t T, int32_t k, int64_t H,
+                           void* out, cudaStream_t st) {
   const int64_t n = T * (H / 8);
   if (n == 0) return cudaSuccess;
   int64_t blocks = cdiv(n, 256);
   if (blocks > 148 * 32) blocks = 148 * 32;
   if (f32_in)
-    combine_kernel<true><<<unsigned(blocks), 256, 0, st>>>(y, T, k, H / 8, static_cast<uint4*>(out));
+    combine_kernel<true><<<unsigned(blocks), 256, 0, st>>>(y, slot_to_row, T, k, H / 8, static_cast<uint4*>(out));
   else
-    combine_kernel<false><<<unsigned(blocks), 256, 0, st>>>(y, T, k, H / 8, static_cast<uint4*>(out));
+    combine_kernel<false><<<unsigned(blocks), 256, 0, st>>>(y, slot_to_row, T, k, H / 8, static_cast<uint4*>(out));
   count_launch();
   return cudaGetLastError();
 }

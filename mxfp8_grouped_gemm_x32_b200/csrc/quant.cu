@@ -18,7 +18,8 @@ namespace moe {
 __global__ void __launch_bounds__(256) quant_rows_kernel(QuantRowsArgs a) {
   const uint32_t units = a.units_div.d;
   const uint32_t rows_pad = a.rowpad_div.d;
-  const uint32_t total = uint32_t(a.groups) * rows_pad * units;  // < 2^31 (checked by the launcher)
+  uint32_t total = uint32_t(a.groups) * rows_pad * units;  // < 2^31 (checked by the launcher)
+  if (a.rows_used) total = min(total, uint32_t(max(*a.rows_used, 0)) * units);
   const int64_t RT = rows_pad / 128, KT = units;
   for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
     const uint32_t rr = fastdiv(i, a.units_div);
@@ -358,18 +359,21 @@ __global__ void __launch_bounds__(256, 3) quant_both_kernel(QuantBothArgs a) {
   uint8_t* atoms = out_col + QB_OUT_BYTES;  // 1 KB
   const int tid = threadIdx.x;
   const bool row_atom = a.row_split % QC_TILE == 0;
+  uint32_t ntiles = a.ntiles;
+  if (a.rows_used)  // one group: tiles run columns fastest, so the rows in use come first
+    ntiles = min(ntiles, uint32_t(cdiv(max(*a.rows_used, 0), QC_TILE)) * a.ct);
   uint32_t t = blockIdx.x;
-  if (t >= a.ntiles) return;
+  if (t >= ntiles) return;
   qb_load(a, qb_tile(a, t), qb_smem, tid);
   cp_async_commit();
-  for (; t < a.ntiles; t += gridDim.x) {
+  for (; t < ntiles; t += gridDim.x) {
     cp_async_wait<0>();
     __syncthreads();  // input landed; the previous tile's staging has been stored
     const QbTile q = qb_tile(a, t);
     qb_compute(a, q, qb_smem, out_row, out_col, atoms, row_atom, tid);
     __syncthreads();  // staging complete, input buffer free
     const uint32_t tn = t + gridDim.x;
-    if (tn < a.ntiles) qb_load(a, qb_tile(a, tn), qb_smem, tid);
+    if (tn < ntiles) qb_load(a, qb_tile(a, tn), qb_smem, tid);
     cp_async_commit();
     qb_store(a, q, out_row, out_col, atoms, row_atom, tid);
   }

@@ -15,6 +15,9 @@ struct QuantRowsArgs {
   int64_t rows, K;
   uint8_t* q;   // [groups][rows][K]
   uint8_t* sf;  // blocked (groups, rows, K)
+  // optional (groups == 1): device count of the leading rows in use, a
+  // multiple of 128; rows from there on are not written
+  const int32_t* rows_used = nullptr;
   // unit schedule (set by the launcher): units of 128 values, 32-bit indices
   FastDiv units_div, rowpad_div, div;
 };
@@ -58,6 +61,9 @@ struct QuantBothArgs {
   uint8_t* sf_col;
   const int32_t* row_map = nullptr;  // optional gather map
   int32_t map_div = 1;
+  // optional (groups == 1): device count of the leading rows in use, a
+  // multiple of 128; tiles from there on are skipped (nothing written)
+  const int32_t* rows_used = nullptr;
   FastDiv div;                        // map_div as a multiply-high (set by the launcher)
   // tile schedule (set by the launcher): 128 x 128 tiles, columns fastest
   uint32_t ct = 0, tiles_per_group = 0, ntiles = 0;

@@ -13,6 +13,13 @@
 // shuffles) and lane r keeps the r-th winner.  NaN logits rank as -inf.
 // Probabilities: exp(l_r - l_0) in fp32, summed over the kept lanes by a
 // fixed shuffle tree, divided.
+//
+// Fused with the permutation (the routing step that feeds the grouped
+// layer): with a histogram given, each kept (token, choice) also counts its
+// expert in the expert histogram of its block of PERM_BLOCK slots -- the
+// first pass of the permutation's counting sort -- so the permutation reads
+// the routing once instead of twice and needs no histogram launch.
+#include "permute.cuh"
 #include "router.cuh"
 
 namespace moe {
@@ -21,7 +28,8 @@ constexpr int RT_WARPS = 8;
 
 template <bool BF16>
 __global__ void __launch_bounds__(RT_WARPS * 32) router_topk_kernel(const void* logits, int32_t T, int32_t E,
-                                                                   int32_t k, int32_t* topk_idx, float* topk_prob) {
+                                                                   int32_t k, int32_t* topk_idx, float* topk_prob,
+                                                                   int32_t* hist) {
   const int64_t t = int64_t(blockIdx.x) * RT_WARPS + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;  // uniform across the warp
@@ -79,17 +87,20 @@ __global__ void __launch_bounds__(RT_WARPS * 32) router_topk_kernel(const void* 
   if (lane < k) {
     topk_idx[t * k + lane] = kept_e;
     topk_prob[t * k + lane] = ex / s;
+    // kept_e is a real expert unless every remaining logit is -inf; then the
+    // winner is still an expert id in [0, E) (ties go to the lowest id)
+    if (hist) atomicAdd(&hist[((t * k + lane) / PERM_BLOCK) * E + kept_e], 1);
   }
 }
 
 cudaError_t launch_router_topk(const void* logits, bool bf16, int32_t T, int32_t E, int32_t k,
-                               int32_t* topk_idx, float* topk_prob, cudaStream_t st) {
+                               int32_t* topk_idx, float* topk_prob, int32_t* hist, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const unsigned blocks = unsigned((int64_t(T) + RT_WARPS - 1) / RT_WARPS);
   if (bf16)
-    router_topk_kernel<true><<<blocks, RT_WARPS * 32, 0, st>>>(logits, T, E, k, topk_idx, topk_prob);
+    router_topk_kernel<true><<<blocks, RT_WARPS * 32, 0, st>>>(logits, T, E, k, topk_idx, topk_prob, hist);
   else
-    router_topk_kernel<false><<<blocks, RT_WARPS * 32, 0, st>>>(logits, T, E, k, topk_idx, topk_prob);
+    router_topk_kernel<false><<<blocks, RT_WARPS * 32, 0, st>>>(logits, T, E, k, topk_idx, topk_prob, hist);
   count_launch();
   return cudaGetLastError();
 }

@@ -10,6 +10,8 @@ Steps (names of the C entry points):
   permute           moe_permute: counting sort by expert, gather + quantise x
   forward           moe_grouped_mlp_fwd: gate_up GEMM + ScaledSwiGLU + requant,
                     down GEMM, top-k combine
+  forward_bf16      moe_grouped_mlp_fwd_bf16: the same layer with bf16 operands
+                    (routing from permute_index, moe_permute without x)
   backward          moe_grouped_mlp_bwd: dgrad/wgrad of both projections,
                     ScaledSwiGLU backward, d(prob)
 """
@@ -40,61 +42,125 @@ def check_tensor(t, name: str, dtype, shape, device) -> None:
         raise ValueError(f"{name}: must be contiguous")
 
 
-def _u8(n: int, dev) -> torch.Tensor:
-    # 256-byte aligned by the caching allocator; sizes rounded to 16 bytes
-    return torch.empty(max(16, (n + 15) // 16 * 16), dtype=torch.uint8, device=dev)
+GUARD_BYTE = 0xA5
+
+
+class _Alloc:
+    """Device buffers of one layer.  With guard > 0 every buffer is followed
+    by `guard` bytes of a fixed pattern (a debug aid: check() names every
+    buffer whose tail was written, i.e. a write past its end)."""
+
+    def __init__(self, dev, guard: int = 0):
+        self.dev, self.guard = dev, (guard + 255) // 256 * 256
+        self.tails = []
+
+    def raw(self, nbytes: int, name: str) -> torch.Tensor:
+        # 256-byte aligned by the caching allocator; sizes rounded to 16 bytes
+        n = max(16, (nbytes + 15) // 16 * 16)
+        if not self.guard:
+            return torch.empty(n, dtype=torch.uint8, device=self.dev)
+        n256 = (n + 255) // 256 * 256
+        buf = torch.empty(n256 + self.guard, dtype=torch.uint8, device=self.dev)
+        buf[n:].fill_(GUARD_BYTE)
+        self.tails.append((name, buf[n:]))
+        return buf[:n]
+
+    def typed(self, shape, dtype, name: str) -> torch.Tensor:
+        numel = 1
+        for d in shape:
+            numel *= d
+        esz = torch.empty(0, dtype=dtype).element_size()
+        return self.raw(numel * esz, name)[: numel * esz].view(dtype).view(*shape)
+
+    def check(self):
+        """Names of the buffers whose guard bytes changed."""
+        return [name for name, t in self.tails if not bool((t == GUARD_BYTE).all())]
 
 
 class GroupedMLP:
     """One layer: T tokens, hidden H, intermediate I, E experts, top-k."""
 
-    def __init__(self, T: int, H: int, I: int, E: int, k: int, device="cuda", backward: bool = True):
+    def __init__(self, T: int, H: int, I: int, E: int, k: int, device="cuda", backward: bool = True,
+                 guard: int = 0):
         self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
         self.dev = torch.device(device)
-        dev = self.dev
+        al = self._alloc = _Alloc(self.dev, guard)
+        u8 = al.raw
         self.rows_cap = lib.moe_padded_rows(T, k, E)
         rc = self.rows_cap
         sb = lib.moe_mx_scale_bytes
         # quantised weights (forward: along H for gate_up, along I for down)
-        self.w1q = _u8(2 * E * I * H, dev)
-        self.w1sf = _u8(sb(2 * E, I, H), dev)
-        self.w2q = _u8(E * H * I, dev)
-        self.w2sf = _u8(sb(E, H, I), dev)
+        self.w1q = u8(2 * E * I * H, "w1q")
+        self.w1sf = u8(sb(2 * E, I, H), "w1sf")
+        self.w2q = u8(E * H * I, "w2q")
+        self.w2sf = u8(sb(E, H, I), "w2sf")
         # routing
-        self.split_sizes = torch.empty(E, dtype=torch.int32, device=dev)
-        self.group_offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
-        self.row_to_slot = torch.empty(rc, dtype=torch.int32, device=dev)
-        self.slot_to_row = torch.empty(T * k, dtype=torch.int32, device=dev)
-        self.topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev)     # router outputs
-        self.topk_prob = torch.empty(T, k, dtype=torch.float32, device=dev)
-        self.prob_perm = torch.empty(rc, dtype=torch.float32, device=dev)
-        self.xq = _u8(rc * H, dev)
-        self.xq_sf = _u8(sb(1, rc, H), dev)
-        self.hq = _u8(rc * I, dev)
-        self.hq_sf = _u8(sb(1, rc, I), dev)
-        self.out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        self.split_sizes = al.typed((E,), torch.int32, "split_sizes")
+        self.group_offsets = al.typed((E + 1,), torch.int32, "group_offsets")
+        self.row_to_slot = al.typed((rc,), torch.int32, "row_to_slot")
+        self.slot_to_row = al.typed((T * k,), torch.int32, "slot_to_row")
+        self.topk_idx = al.typed((T, k), torch.int32, "topk_idx")        # router outputs
+        self.topk_prob = al.typed((T, k), torch.float32, "topk_prob")
+        self.prob_perm = al.typed((rc,), torch.float32, "prob_perm")
+        self.xq = u8(rc * H, "xq")
+        self.xq_sf = u8(sb(1, rc, H), "xq_sf")
+        self.hq = u8(rc * I, "hq")
+        self.hq_sf = u8(sb(1, rc, I), "hq_sf")
+        self.out = al.typed((T, H), torch.bfloat16, "out")
         self.dev = self.out.device      # concrete device (index resolved) for the input checks
         self.ws_perm_bytes = lib.moe_workspace_size(lib.MOE_OP_PERMUTE, T, k, E, H, I)
         self.ws_fwd_bytes = lib.moe_workspace_size(lib.MOE_OP_FWD, T, k, E, H, I)
-        self.ws_perm = _u8(self.ws_perm_bytes, dev)
-        self.ws_fwd = _u8(self.ws_fwd_bytes, dev)
+        self.ws_perm = u8(self.ws_perm_bytes, "ws_perm")
+        self.ws_fwd = u8(self.ws_fwd_bytes, "ws_fwd")
         self.backward_enabled = backward
         if backward:
-            self.w1tq = _u8(E * H * 2 * I, dev)
-            self.w1tsf = _u8(sb(E, H, 2 * I), dev)
-            self.w2tq = _u8(E * I * H, dev)
-            self.w2tsf = _u8(sb(E, I, H), dev)
-            self.xq_col = _u8(H * rc, dev)
-            self.xq_col_sf = _u8(sb(1, H, rc), dev)
-            self.saved_a = torch.empty(rc, 2 * I, dtype=torch.bfloat16, device=dev)
-            self.dX = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
-            self.dW1 = torch.empty(E, 2 * I, H, dtype=torch.bfloat16, device=dev)
-            self.dW2 = torch.empty(E, H, I, dtype=torch.bfloat16, device=dev)
-            self.dprob = torch.empty(T, k, dtype=torch.float32, device=dev)
+            self.w1tq = u8(E * H * 2 * I, "w1tq")
+            self.w1tsf = u8(sb(E, H, 2 * I), "w1tsf")
+            self.w2tq = u8(E * I * H, "w2tq")
+            self.w2tsf = u8(sb(E, I, H), "w2tsf")
+            self.xq_col = u8(H * rc, "xq_col")
+            self.xq_col_sf = u8(sb(1, H, rc), "xq_col_sf")
+            self.saved_a = al.typed((rc, 2 * I), torch.bfloat16, "saved_a")
+            self.dX = al.typed((T, H), torch.bfloat16, "dX")
+            self.dW1 = al.typed((E, 2 * I, H), torch.bfloat16, "dW1")
+            self.dW2 = al.typed((E, H, I), torch.bfloat16, "dW2")
+            self.dprob = al.typed((T, k), torch.float32, "dprob")
             self.ws_bwd_bytes = lib.moe_workspace_size(lib.MOE_OP_BWD, T, k, E, H, I)
-            self.ws_bwd = _u8(self.ws_bwd_bytes, dev)
+            self.ws_bwd = u8(self.ws_bwd_bytes, "ws_bwd")
         else:
             self.saved_a = None
+
+    def permute_index(self, topk_idx: torch.Tensor, topk_prob: torch.Tensor) -> None:
+        """Routing outputs of the permutation only (no quantisation of x):
+        what the BF16 forward needs."""
+        check_tensor(topk_idx, "topk_idx", torch.int32, (self.T, self.k), self.dev)
+        check_tensor(topk_prob, "topk_prob", torch.float32, (self.T, self.k), self.dev)
+        lib.moe_permute(0, topk_idx.data_ptr(), topk_prob.data_ptr(), self.T, self.H, self.k, self.E, self.rows_cap,
+                        _ptr(self.split_sizes), _ptr(self.group_offsets), _ptr(self.row_to_slot),
+                        _ptr(self.slot_to_row), _ptr(self.prob_perm), 0, 0, 0, 0, _ptr(self.ws_perm),
+                        self.ws_perm_bytes, self._stream())
+
+    def forward_bf16(self, x: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor) -> torch.Tensor:
+        """BF16 recipe forward (moe_grouped_mlp_fwd_bf16) on the routing of
+        the last permute / permute_index: x bf16 [T, H], w1 bf16 [E, 2I, H],
+        w2 bf16 [E, H, I] -> out."""
+        E, H, I = self.E, self.H, self.I
+        check_tensor(x, "x", torch.bfloat16, (self.T, H), self.dev)
+        check_tensor(w1, "w_gate_up", torch.bfloat16, (E, 2 * I, H), self.dev)
+        check_tensor(w2, "w_down", torch.bfloat16, (E, H, I), self.dev)
+        if getattr(self, "ws_bf16", None) is None:
+            self.ws_bf16_bytes = lib.moe_workspace_size(lib.MOE_OP_FWD_BF16, self.T, self.k, E, H, I)
+            self.ws_bf16 = self._alloc.raw(self.ws_bf16_bytes, "ws_bf16")
+        lib.moe_grouped_mlp_fwd_bf16(w1.data_ptr(), w2.data_ptr(), self.T, H, I, E, self.k, self.rows_cap,
+                                     _ptr(self.split_sizes), _ptr(self.group_offsets), _ptr(self.row_to_slot),
+                                     _ptr(self.prob_perm), x.data_ptr(), _ptr(self.out), _ptr(self.ws_bf16),
+                                     self.ws_bf16_bytes, self._stream())
+        return self.out
+
+    def check_guards(self):
+        """Names of the buffers written past their end (layers built with
+        guard > 0; always empty otherwise)."""
+        return self._alloc.check()
 
     @staticmethod
     def _stream() -> int:
@@ -123,6 +189,24 @@ class GroupedMLP:
         check_tensor(logits, "logits", logits.dtype, (self.T, self.E), self.dev)
         lib.moe_router_topk(logits.data_ptr(), dt, self.T, self.E, self.k, _ptr(self.topk_idx),
                             _ptr(self.topk_prob), self._stream())
+        return self.topk_idx, self.topk_prob
+
+    def route_permute(self, logits: torch.Tensor, x: torch.Tensor):
+        """Router and permutation in one call (moe_route_permute): logits fp32
+        or bf16 [T, E], x bf16 [T, H]; the routing lands in topk_idx /
+        topk_prob, the permuted and quantised x in this layer's buffers."""
+        dt = {torch.float32: lib.MOE_DTYPE_F32, torch.bfloat16: lib.MOE_DTYPE_BF16}.get(logits.dtype)
+        if dt is None:
+            raise TypeError(f"logits: expected float32 or bfloat16, got {logits.dtype}")
+        check_tensor(logits, "logits", logits.dtype, (self.T, self.E), self.dev)
+        check_tensor(x, "x", torch.bfloat16, (self.T, self.H), self.dev)
+        bw = self.backward_enabled
+        lib.moe_route_permute(logits.data_ptr(), dt, x.data_ptr(), self.T, self.H, self.k, self.E, self.rows_cap,
+                              _ptr(self.topk_idx), _ptr(self.topk_prob), _ptr(self.split_sizes),
+                              _ptr(self.group_offsets), _ptr(self.row_to_slot), _ptr(self.slot_to_row),
+                              _ptr(self.prob_perm), _ptr(self.xq), _ptr(self.xq_sf), _ptr(self.xq_col) if bw else 0,
+                              _ptr(self.xq_col_sf) if bw else 0, _ptr(self.ws_perm), self.ws_perm_bytes,
+                              self._stream())
         return self.topk_idx, self.topk_prob
 
     def permute(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_prob: torch.Tensor) -> None:

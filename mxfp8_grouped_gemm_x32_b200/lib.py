@@ -20,6 +20,7 @@ MOE_QUANT_COL = 2
 MOE_OP_PERMUTE = 1
 MOE_OP_FWD = 2
 MOE_OP_BWD = 3
+MOE_OP_FWD_BF16 = 4
 MOE_MAX_EXPERTS = 256
 
 STATUS = {
@@ -34,7 +35,8 @@ EXPORTED = [
     "moe_permute", "moe_grouped_mlp_fwd", "moe_combine", "moe_grouped_mlp_bwd",
     "moe_get_device_status", "moe_status_string", "moe_launch_count", "moe_selftest_wait_timeout",
     "moe_timing_enable", "moe_timing_read", "moe_permute_noalloc", "moe_mlp_quantize_weights",
-    "moe_router_topk",
+    "moe_router_topk", "moe_mx_scales_to_blocked", "moe_mx_scales_from_blocked", "moe_route_permute",
+    "moe_grouped_mlp_fwd_bf16",
 ]
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 
@@ -76,6 +78,12 @@ _decl("moe_combine", _I32, _P, _I32, _I32, _I32, _P, _P)
 _decl("moe_router_topk", _I32, _P, _I32, _I32, _I32, _I32, _P, _P, _P)
 _decl("moe_grouped_mlp_bwd", _I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P,
       _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
+_decl("moe_mx_scales_to_blocked", _I32, _P, _I32, _I64, _I64, _I64, _P, _P)
+_decl("moe_mx_scales_from_blocked", _I32, _P, _I32, _I64, _I64, _P, _I64, _P)
+_decl("moe_route_permute", _I32, _P, _I32, _P, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
+      _P, _P, _P, _P, _SZ, _P)
+_decl("moe_grouped_mlp_fwd_bf16", _I32, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P, _P,
+      _SZ, _P)
 _decl("moe_get_device_status", _I32, _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
 _decl("moe_launch_count", _I64, _I32)
@@ -142,12 +150,35 @@ def moe_grouped_mlp_fwd(w1q, w1sf, w2q, w2sf, T, H, I, E, k, rows_cap, split_siz
         xq, xq_sf, out, saved_a, hq, hq_sf, workspace, workspace_bytes, stream))
 
 
+def moe_mx_scales_to_blocked(plain, groups, rows, k, ld, blocked, stream=0):
+    _check("moe_mx_scales_to_blocked", _lib.moe_mx_scales_to_blocked(plain, groups, rows, k, ld, blocked, stream))
+
+
+def moe_mx_scales_from_blocked(blocked, groups, rows, k, plain, ld, stream=0):
+    _check("moe_mx_scales_from_blocked", _lib.moe_mx_scales_from_blocked(blocked, groups, rows, k, plain, ld, stream))
+
+
+def moe_grouped_mlp_fwd_bf16(w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot,
+                             prob_perm, x, out, workspace, workspace_bytes, stream=0):
+    _check("moe_grouped_mlp_fwd_bf16", _lib.moe_grouped_mlp_fwd_bf16(
+        w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot, prob_perm, x, out,
+        workspace, workspace_bytes, stream))
+
+
 def moe_combine(y, T, k, H, out, stream=0):
     _check("moe_combine", _lib.moe_combine(y, T, k, H, out, stream))
 
 
 def moe_router_topk(logits, logits_dtype, T, E, k, topk_idx, topk_prob, stream=0):
     _check("moe_router_topk", _lib.moe_router_topk(logits, logits_dtype, T, E, k, topk_idx, topk_prob, stream))
+
+
+def moe_route_permute(logits, logits_dtype, x, T, H, k, E, rows_cap, topk_idx, topk_prob, split_sizes,
+                      group_offsets, row_to_slot, slot_to_row, prob_perm, xq, xq_sf, xq_col, xq_col_sf, workspace,
+                      workspace_bytes, stream=0):
+    _check("moe_route_permute", _lib.moe_route_permute(
+        logits, logits_dtype, x, T, H, k, E, rows_cap, topk_idx, topk_prob, split_sizes, group_offsets,
+        row_to_slot, slot_to_row, prob_perm, xq, xq_sf, xq_col, xq_col_sf, workspace, workspace_bytes, stream))
 
 
 def moe_grouped_mlp_bwd(w2tq, w2tsf, w1tq, w1tsf, T, H, I, E, k, rows_cap, split_sizes, group_offsets,

@@ -162,3 +162,35 @@ def test_quantise_and_combine_argument_errors():
     assert c(P, 4, 2, 12, P, None) == INVALID                                # H % 8
     assert c(P, 4, 2, 64, M, None) == INVALID
     assert c(P, -1, 2, 64, P, None) == INVALID
+
+
+def test_scale_conversion_argument_errors():
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    t = lib._lib.moe_mx_scales_to_blocked
+    f = lib._lib.moe_mx_scales_from_blocked
+    assert t(P, 1, 64, 48, 2, P, None) == INVALID           # k % 32
+    assert t(P, 1, 64, 128, 3, P, None) == INVALID          # ld < k/32
+    assert t(None, 1, 64, 128, 4, P, None) == INVALID       # null plain
+    assert t(P, 1, 64, 128, 4, P + 2, None) == INVALID      # blocked not 4-byte aligned
+    assert t(P, -1, 64, 128, 4, P, None) == INVALID
+    assert t(None, 0, 64, 128, 4, None, None) == 0          # nothing to convert
+    assert f(P, 1, 64, 48, P, 2, None) == INVALID
+    assert f(P, 1, 64, 128, P, 3, None) == INVALID
+    assert f(None, 1, 64, 128, P, 4, None) == INVALID
+    assert f(P, 1, 0, 128, None, 4, None) == 0
+
+
+def test_route_permute_argument_errors():
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    f = lib._lib.moe_route_permute
+
+    def args(T=64, H=256, k=2, E=4, dtype=0, logits=P, x=P, ws_bytes=1 << 30):
+        rows_cap = lib.moe_padded_rows(T, k, E) if T < (1 << 28) else 1 << 31
+        return (logits, dtype, x, T, H, k, E, rows_cap, P, P, P, P, P, P, P, P, P, P, P, P, ws_bytes, None)
+    assert f(*args(logits=None)) == INVALID
+    assert f(*args(dtype=5)) == INVALID
+    assert f(*args(k=5, E=4)) == INVALID
+    assert f(*args(k=33, E=64)) == UNSUPPORTED                    # router keeps at most 32
+    assert f(*args(H=48)) == UNSUPPORTED
+    assert f(*args(x=M)) == INVALID
+    assert f(*args(ws_bytes=16)) == WORKSPACE

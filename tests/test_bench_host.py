@@ -123,3 +123,17 @@ def test_cpu_cores_reports_the_blas_threads():
     with threadpool_limits(limits=1, user_api="blas"):
         assert bench.cpu_cores() == 1
     assert bench.cpu_cores() >= 1
+
+
+def test_split_histogram_and_peaks():
+    h = bench.split_histogram([0, 5, 3, 0, 100, 7])
+    assert h == {"min": 0, "median": 4.0, "max": 100, "empty": 2, "experts": 6}
+    assert bench.split_histogram([4, 1, 9])["median"] == 4
+    # 16384 FLOP per clock per SM x 148 SMs at 1.965 GHz
+    assert abs(bench.clock_peak_tflops(1965) - 16384 * 148 * 1.965e9 / 1e12) < 1e-9
+    cfg = get_config("qwen3_30b_ragged")
+    r = bench.phase_rates(cfg, 1.0, 2.0, 2800.0, 4000.0)
+    assert abs(r["fwd"]["tflops"] - cfg.fwd_flops() / 1e-3 / 1e12) < 1e-6
+    assert abs(r["bwd"]["frac_of_peak"] - cfg.bwd_flops() / 2e-3 / 1e12 / 2800.0) < 1e-12
+    assert abs(r["fwd"]["frac_of_clock_peak"] - r["fwd"]["tflops"] / 4000.0) < 1e-12
+    assert bench.phase_rates(cfg, 1.0, 0.0, 2800.0, None)["fwd"]["frac_of_clock_peak"] is None

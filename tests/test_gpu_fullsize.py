@@ -9,11 +9,12 @@ the sampled outputs exactly (every row's forward and backward depend only on
 that row and its expert's weights; every intermediate channel's weight
 gradients depend only on that channel over the expert's rows, with the same
 32-row blocks along tokens):
-* per-slot outputs of a few routed rows of one expert: the down-projection
-  row y (fp32, before the combine), the dgrad row dx (fp32, before the
-  combine) and dprob;
-* two 32-channel blocks of that expert's weight gradients: dW_gate_up rows
-  (gate and up) and dW_down columns, over every routed row of the expert;
+* for three experts -- the median, the largest (many 128-row tiles) and the
+  smallest non-empty group: per-slot outputs of a few routed rows including
+  the group's first and last (the down-projection row y and the dgrad row dx,
+  fp32 before the combine, and dprob), and two 32-channel blocks of the
+  expert's weight gradients, one of them the last (dW_gate_up rows, gate and
+  up, and dW_down columns) over every routed row of the expert;
 * at every token: out = bf16(sum_j y) and dX = bf16(sum_j dx), bit-exact (the
   combine, a property that holds at any size).
 Bars as in test_gpu_parity.py (with the allowance of tests/ambiguity.py).
@@ -42,19 +43,20 @@ def _rel_rms(g, r):
 
 def _slot_buffers(L, cfg):
     """fp32 per-slot rows kept by the library in the caller's workspaces:
-    the forward's y (first piece when hq is caller-provided) and the
-    backward's dx (last piece), each [T*k][H]."""
+    the forward's y (first piece when hq is caller-provided, [T*k][H] in slot
+    order) and the backward's dx (the piece after the MX operands, [rows_cap][H]
+    in permuted order), both returned in slot order."""
     import torch
     from mxfp8_grouped_gemm_x32_b200 import lib
     rc, H, I, n = L.rows_cap, cfg.H, cfg.I, cfg.T * cfg.k * cfg.H
     a256 = lambda v: (v + 255) // 256 * 256
     sb = lib.moe_mx_scale_bytes
-    pieces = [rc * H, sb(1, rc, H), H * rc, sb(1, H, rc), rc * I * 4, rc * 2 * I, sb(1, rc, 2 * I),
+    pieces = [rc * H, sb(1, rc, H), H * rc, sb(1, H, rc), rc * 2 * I, sb(1, rc, 2 * I),
               2 * I * rc, sb(1, 2 * I, rc), I * rc, sb(1, I, rc)]
     off = sum(a256(p) for p in pieces)
     y = L.ws_fwd[: n * 4].view(torch.float32)
-    dx = L.ws_bwd[off: off + n * 4].view(torch.float32)
-    return y.view(cfg.T * cfg.k, H), dx.view(cfg.T * cfg.k, H)
+    dx = L.ws_bwd[off: off + rc * H * 4].view(torch.float32).view(rc, H)
+    return y.view(cfg.T * cfg.k, H), dx[L.slot_to_row.long()]
 
 
 @pytest.mark.parametrize("name", ["mixtral_8x7b", "qwen3_30b_ragged", "gpt_oss_20b"])
@@ -89,20 +91,35 @@ def test_full_size_sampled(name):
         got = gpu_sum.cpu().view(torch.int16).numpy().view(np.uint16)
         assert np.array_equal(got, want)
 
-    # --- the expert: the one holding the median number of rows (non-empty)
+    # --- three experts: the median, the largest and the smallest non-empty
+    # group (the largest spans many 128-row tiles; every group has a ragged
+    # last tile, and on the GPT-OSS shape both contractions end in a K tail)
     nz = np.flatnonzero(split)
-    e = int(nz[np.argsort(split[nz])[len(nz) // 2]])
-    slots = np.flatnonzero(idx.reshape(-1) == e)          # its rows, in permuted (slot) order
-    tk = slots // cfg.k
+    order = nz[np.argsort(split[nz], kind="stable")]
+    experts = []
+    for e in (int(order[len(order) // 2]), int(order[-1]), int(order[0])):
+        if e not in experts:
+            experts.append(e)
     x = _f64(inp["x"])
     dy = _f64(inp["dy"])
+    for n, e in enumerate(experts):
+        _check_expert(cfg, inp, L, e, x, dy, y_slot, dx_slot, dW1, dW2, dprob, seed=1 + n)
+
+
+def _check_expert(cfg, inp, L, e, x, dy, y_slot, dx_slot, dW1, dW2, dprob, seed):
+    import torch
+    idx, prob = inp["topk_idx"], inp["topk_prob"]
+    slots = np.flatnonzero(idx.reshape(-1) == e)          # its rows, in permuted (slot) order
+    tk = slots // cfg.k
     pe = prob.reshape(-1)[slots][:, None].astype(np.float32)
     w1e = _f64(inp["w1"][e:e + 1])
     w2e = _f64(inp["w2"][e:e + 1])
-    rng = np.random.default_rng(1)
+    rng = np.random.default_rng(seed)
 
-    # sampled rows: y, dx, dprob (k = 1 sub-problem over those rows)
-    s = np.sort(rng.choice(slots.size, min(8, slots.size), replace=False))
+    # sampled rows: y, dx, dprob (k = 1 sub-problem over those rows); the
+    # group's first and last rows are always among them
+    pick = rng.choice(slots.size, min(8, slots.size), replace=False)
+    s = np.unique(np.concatenate([pick, [0, slots.size - 1]]))
     xs, dys = x[tk[s]], dy[tk[s]]
     i1 = np.zeros((s.size, 1), np.int32)
     f = omoe.forward(xs, w1e, w2e, i1, pe[s])
@@ -112,17 +129,19 @@ def test_full_size_sampled(name):
     g_y = y_slot[torch.from_numpy(slots[s]).cuda()].cpu().numpy().astype(np.float64)
     g_dx = dx_slot[torch.from_numpy(slots[s]).cuda()].cpu().numpy().astype(np.float64)
     g_dp = dprob.reshape(-1)[torch.from_numpy(slots[s]).cuda()].cpu().numpy().astype(np.float64)
-    assert ambiguity.within(g_y, f["Y"], OUT_TOL, a_y, bf16_out=False) <= OUT_TOL
-    assert ambiguity.within(g_dx, b["dx_rows"], GRAD_TOL, a_b["dX"], bf16_out=False) <= GRAD_TOL
-    assert ambiguity.within(g_dp, b["dprob_f64"][:, 0], GRAD_TOL, a_b["dprob"][:, 0], bf16_out=False) <= GRAD_TOL
-    assert _rel_rms(g_y, f["Y"]) <= RMS_TOL and _rel_rms(g_dx, b["dx_rows"]) <= RMS_TOL
+    tag = f"expert {e} ({slots.size} rows)"
+    assert ambiguity.within(g_y, f["Y"], OUT_TOL, a_y, bf16_out=False) <= OUT_TOL, tag
+    assert ambiguity.within(g_dx, b["dx_rows"], GRAD_TOL, a_b["dX"], bf16_out=False) <= GRAD_TOL, tag
+    assert ambiguity.within(g_dp, b["dprob_f64"][:, 0], GRAD_TOL, a_b["dprob"][:, 0], bf16_out=False) <= GRAD_TOL, tag
+    assert _rel_rms(g_y, f["Y"]) <= RMS_TOL and _rel_rms(g_dx, b["dx_rows"]) <= RMS_TOL, tag
 
-    # two 32-channel blocks of the intermediate dimension, over all rows of e
+    # two 32-channel blocks of the intermediate dimension (one of them the
+    # last block), over all rows of e
     I = cfg.I
-    blocks = rng.choice(I // 32, 2, replace=False)
-    ch = np.concatenate([np.arange(32 * c, 32 * c + 32) for c in sorted(blocks)])
-    w1c = np.concatenate([w1e[:, ch], w1e[:, I + ch]], axis=1)      # [1, 2*64, H]
-    w2c = w2e[:, :, ch]                                              # [1, H, 64]
+    blocks = np.unique([rng.integers(0, I // 32 - 1), I // 32 - 1])
+    ch = np.concatenate([np.arange(32 * c, 32 * c + 32) for c in blocks])
+    w1c = np.concatenate([w1e[:, ch], w1e[:, I + ch]], axis=1)      # [1, 2*nch, H]
+    w2c = w2e[:, :, ch]                                              # [1, H, nch]
     ie = np.zeros((slots.size, 1), np.int32)
     fe = omoe.forward(x[tk], w1c, w2c, ie, pe)
     be = omoe.backward(fe, x[tk], w1c, w2c, pe, dy[tk])
@@ -130,6 +149,6 @@ def test_full_size_sampled(name):
     rows1 = torch.from_numpy(np.concatenate([ch, I + ch])).cuda()
     g_w1 = dW1[e][rows1].float().cpu().numpy().astype(np.float64)
     g_w2 = dW2[e][:, torch.from_numpy(ch).cuda()].float().cpu().numpy().astype(np.float64)
-    assert ambiguity.within(g_w1, be["dW1"][0], GRAD_TOL, ae["dW1"][0]) <= GRAD_TOL
-    assert ambiguity.within(g_w2, be["dW2"][0], GRAD_TOL, ae["dW2"][0]) <= GRAD_TOL
-    assert _rel_rms(g_w1, be["dW1"][0]) <= RMS_TOL and _rel_rms(g_w2, be["dW2"][0]) <= RMS_TOL
+    assert ambiguity.within(g_w1, be["dW1"][0], GRAD_TOL, ae["dW1"][0]) <= GRAD_TOL, tag
+    assert ambiguity.within(g_w2, be["dW2"][0], GRAD_TOL, ae["dW2"][0]) <= GRAD_TOL, tag
+    assert _rel_rms(g_w1, be["dW1"][0]) <= RMS_TOL and _rel_rms(g_w2, be["dW2"][0]) <= RMS_TOL, tag

@@ -113,7 +113,8 @@ class Layer:
     def __init__(self, torch, cfg, inp):
         from mxfp8_grouped_gemm_x32_b200.layer import GroupedMLP
         self.cfg, self.inp = cfg, inp
-        self.L = GroupedMLP(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, backward=True)
+        # every buffer is followed by 4 KB of guard bytes (checked below)
+        self.L = GroupedMLP(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, backward=True, guard=4096)
         self.args = (_bf(torch, inp["x"]), torch.from_numpy(inp["topk_idx"]).cuda(),
                      torch.from_numpy(inp["topk_prob"]).cuda(), _bf(torch, inp["w1"]),
                      _bf(torch, inp["w2"]), _bf(torch, inp["dy"]))
@@ -178,6 +179,13 @@ def test_device_status_clean(run):
     assert layer.status == 0
 
 
+def test_no_write_past_any_buffer(run):
+    """The guard bytes after every output and workspace buffer of the step
+    (weights, routing, activations, gradients, workspaces) are intact."""
+    cfg, inp, layer, f, b = run
+    assert layer.L.check_guards() == []
+
+
 def test_permute_bitexact(run):
     cfg, inp, layer, f, b = run
     L = layer.L
@@ -210,7 +218,8 @@ def test_permute_bitexact(run):
         assert np.array_equal(xcsf[:, g0 // 32:(g0 + mp) // 32], s)
         assert np.all(xcol[:, g0 + mp:go[e + 1]] == 0)
     assert np.all(r2s[~used] == -1)
-    assert np.all(xq[~used] == 0) and np.all(xsf[~used] == 0)
+    pad = ~used[: go[cfg.E]]        # padding rows inside the groups (rows past the last group are not written)
+    assert np.all(xq[: go[cfg.E]][pad] == 0) and np.all(xsf[: go[cfg.E]][pad] == 0)
     assert np.array_equal(s2r[r2s[used]], np.flatnonzero(used))
     assert np.all(pp[~used] == 0)
 
@@ -276,13 +285,13 @@ def test_backward_requant_da(run):
     to the oracle's da (read from the backward workspace)."""
     cfg, inp, layer, f, b = run
     # the row-quantised da lives in the backward workspace: see carve_bwd
-    # (dyq, dyq_sf, dyc, dyc_sf, dh, daq, ...), 256-byte aligned pieces
+    # (dyq, dyq_sf, dyc, dyc_sf, daq, ...), 256-byte aligned pieces
     L = layer.L
     rc, H, I = L.rows_cap, cfg.H, cfg.I
     from mxfp8_grouped_gemm_x32_b200 import lib
     a256 = lambda n: (n + 255) // 256 * 256
     off = (a256(rc * H) + a256(lib.moe_mx_scale_bytes(1, rc, H)) + a256(H * rc)
-           + a256(lib.moe_mx_scale_bytes(1, H, rc)) + a256(rc * I * 4))
+           + a256(lib.moe_mx_scale_bytes(1, H, rc)))
     ws = L.ws_bwd.cpu().numpy()
     daq = ws[off:off + rc * 2 * I].reshape(rc, 2 * I)
     off2 = off + a256(rc * 2 * I)
@@ -405,8 +414,11 @@ def test_forward_only_equals_training_forward(torch_cuda, name, over):
         torch.cuda.synchronize()
         routed = L.row_to_slot.cpu().numpy() >= 0    # h is written for routed rows only
         rc = L.rows_cap
+        used = int(L.group_offsets[cfg.E])           # rows past the last group are not written
         h = L.hq.cpu().numpy()[: rc * cfg.I].reshape(rc, cfg.I)[routed]
         hs = sf_unblock(L.hq_sf.cpu().numpy(), 1, rc, cfg.I)[0][routed]
-        outs.append([L.xq.cpu().numpy(), L.xq_sf.cpu().numpy(), h, hs, out.view(torch.uint8).cpu().numpy()])
+        xq = L.xq.cpu().numpy()[: used * cfg.H]
+        xs = sf_unblock(L.xq_sf.cpu().numpy(), 1, rc, cfg.H)[0][:used]
+        outs.append([xq, xs, h, hs, out.view(torch.uint8).cpu().numpy()])
     for a, b in zip(*outs):
         assert np.array_equal(a, b)

@@ -83,3 +83,38 @@ def test_router_empty(cuda):
     lib.moe_router_topk(z.data_ptr(), lib.MOE_DTYPE_F32, 0, 8, 2, z.data_ptr(), z.data_ptr(), 0)
     torch.cuda.synchronize()
     assert float(z[0]) == 0.0
+
+
+@pytest.mark.parametrize("name,T,training", [("qwen3_30b_ragged", 3000, True), ("tiny", 1000, False),
+                                             ("gpt_oss_20b", 517, True)])
+def test_route_permute_equals_router_then_permute(cuda, name, T, training):
+    """moe_route_permute (the router fused into the permutation's histogram
+    pass) writes exactly what moe_router_topk followed by moe_permute writes,
+    and its expert ids match the oracle's router."""
+    import torch
+    from mxfp8_grouped_gemm_x32_b200.layer import GroupedMLP
+    cfg = get_config(name, T=T)
+    inp = make_inputs(cfg, seed=3, weights=False, grad=False)
+    lg = torch.from_numpy(inp["router_logits"].astype(np.float32)).cuda()
+    x = torch.from_numpy(inp["x"].view(np.int16)).view(torch.bfloat16).cuda()
+    a = GroupedMLP(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, backward=training)
+    b = GroupedMLP(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, backward=training)
+    idx, prob = a.route(lg)
+    a.permute(x, idx, prob)
+    b.route_permute(lg, x)
+    torch.cuda.synchronize()
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    assert lib.moe_get_device_status(0) == 0
+    ri, _ = orouter.route_topk(inp["router_logits"].astype(np.float32), cfg.k)
+    assert np.array_equal(b.topk_idx.cpu().numpy(), ri)
+    go = int(a.group_offsets[cfg.E])
+    names = ["topk_idx", "topk_prob", "split_sizes", "group_offsets", "row_to_slot", "slot_to_row", "prob_perm"]
+    for n in names:
+        assert torch.equal(getattr(a, n), getattr(b, n)), n
+    assert torch.equal(a.xq[: go * cfg.H], b.xq[: go * cfg.H])
+    nsf = go // 128 * ((cfg.H + 127) // 128) * 512
+    assert torch.equal(a.xq_sf[:nsf], b.xq_sf[:nsf])
+    if training:
+        xa = a.xq_col[: cfg.H * a.rows_cap].view(cfg.H, a.rows_cap)[:, :go]
+        xb = b.xq_col[: cfg.H * b.rows_cap].view(cfg.H, b.rows_cap)[:, :go]
+        assert torch.equal(xa, xb)
