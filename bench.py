@@ -52,7 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workloads", default=",".join(SIDE_WORKLOADS_DEFAULT),
-                    help="further layer shapes measured in the same run (comma list, '' for none)")
+                    help="further layer shapes measured in the same run (comma list; 'none' for none)")
     ap.add_argument("--no-library-probe", action="store_true",
                     help="skip the dense MXFP8 GEMM rate of the CUDA library (context for the roofline)")
     return ap.parse_args(argv)
@@ -747,13 +747,13 @@ def run_ours(args):
     line["attainable_fwd"] = att
     del layer, x, idx, prob, w1, w2, dy, din, dsnap
     torch.cuda.empty_cache()
-    if world == 1 and args.workloads:
+    side = [n for n in args.workloads.split(",") if n and n not in ("none", cfg.name)]
+    if world == 1 and side:
         # the other layer shapes, measured in the same run on the same GPU
         line["workloads"] = {}
-        for name in args.workloads.split(","):
-            if name and name != cfg.name:
-                line["workloads"][name] = measure_workload(torch, lib, name, args.seed, dev, max(args.steps, 50),
-                                                           max(args.warmup, 10), local, peaks)
+        for name in side:
+            line["workloads"][name] = measure_workload(torch, lib, name, args.seed, dev, max(args.steps, 50),
+                                                       max(args.warmup, 10), local, peaks)
     if not args.no_library_probe:
         probe = mxfp8_library_probe(torch, dev)
         line["mxfp8_library_probe"] = probe

@@ -180,14 +180,16 @@ moe_status_t moe_mlp_quantize_weights(const void* w_gate_up, const void* w_down,
  *   row_to_slot    int32 [rows_cap]  slot of each padded row, -1 = padding.
  *   slot_to_row    int32 [T*k]       padded row of each slot.
  *   prob_perm      float [rows_cap]  routing probability per padded row (0 pad).
- *   xq, xq_sf      MX tensor (1, rows_cap, H): gathered x, quantised along H
- *                  (rows from group_offsets[E] on are left unwritten).  Both
- *                  NULL (then xq_col too): only the routing outputs above
- *                  are produced, as the BF16 forward needs.
+ *   xq, xq_sf      MX tensor (1, T, H): x quantised along H, in token order
+ *                  (each token once; the forward's gate_up GEMM gathers the
+ *                  rows of every group itself).  Both NULL (then xq_col
+ *                  too): only the routing outputs above are produced, as the
+ *                  BF16 forward needs.
  *   xq_col, xq_col_sf  optional (both NULL or both set): MX tensor
  *                  (1, H, rows_cap) = gathered x^T quantised along tokens
  *                  (32-token blocks inside each 128-aligned group; padding
- *                  tokens are zero) -- the weight-gradient operand.
+ *                  tokens are zero; columns from group_offsets[E] on are
+ *                  left unwritten) -- the weight-gradient operand.
  *   workspace  >= moe_workspace_size(MOE_OP_PERMUTE, T, k, E, H, 0) bytes.
  * Limits: 1 <= k <= E, H % 32 == 0 (else MOE_ERR_INVALID / MOE_ERR_UNSUPPORTED
  * as for the other calls); E <= MOE_MAX_EXPERTS and T*k < 2^30
@@ -232,8 +234,11 @@ moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_idx, const f
  * GroupedLinear; Figure 4: one fused kernel before the down projection).
  *   w1q, w1sf  MX tensor (2E, I, H): W_gate_up quantised along H.
  *   w2q, w2sf  MX tensor (E, H, I):  W_down quantised along I.
- *   routing    split_sizes, group_offsets, row_to_slot, prob_perm from moe_permute.
- *   xq, xq_sf  MX tensor (1, rows_cap, H) from moe_permute.
+ *   routing    split_sizes, group_offsets, row_to_slot, slot_to_row, prob_perm
+ *              from moe_permute (the combine gathers each token's k rows
+ *              through slot_to_row).
+ *   xq, xq_sf  MX tensor (1, T, H) from moe_permute (x in token order; the
+ *              gate_up GEMM gathers row r's token, row_to_slot[r] / k).
  *   out        bf16 [T][H]: out[t] = sum_j y[t*k+j], y = down(h),
  *              h = prob * silu(gate) * up, gate = A[:, :I], up = A[:, I:],
  *              A = x W_gate_up^T (fp32 accumulation).
@@ -247,7 +252,7 @@ moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_idx, const f
  *   workspace  >= moe_workspace_size(MOE_OP_FWD, T, k, E, H, I).
  * The combine is always applied (there is no flag for per-slot output): the
  * down projection's rows are summed in fp32, in ascending j, from an fp32
- * per-slot buffer in the workspace, so `out` is rounded to bf16 once.  A
+ * buffer of rows in the workspace, so `out` is rounded to bf16 once.  A
  * caller that wants per-slot rows instead uses moe_combine's input format
  * (bf16 [T*k][H]) with its own down projection.
  * Needs H % 32 == 0, I % 64 == 0, 1 <= k <= E <= MOE_MAX_EXPERTS and
@@ -256,7 +261,8 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
                                  const uint8_t* w2sf, int32_t T, int32_t H, int32_t I, int32_t E,
                                  int32_t k, int64_t rows_cap, const int32_t* split_sizes,
                                  const int32_t* group_offsets, const int32_t* row_to_slot,
-                                 const float* prob_perm, const uint8_t* xq, const uint8_t* xq_sf,
+                                 const int32_t* slot_to_row, const float* prob_perm,
+                                 const uint8_t* xq, const uint8_t* xq_sf,
                                  void* out, void* saved_a, uint8_t* hq, uint8_t* hq_sf,
                                  void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
@@ -268,16 +274,16 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
  * kept in bf16 between them, and out[t] = sum_j y[t*k+j] (fp32, ascending
  * j, one bf16 rounding).
  *   w_gate_up  bf16 [E][2I][H] (gate rows first); w_down bf16 [E][H][I].
- *   routing    split_sizes, group_offsets, row_to_slot, prob_perm from
- *              moe_permute (xq may be NULL there).
+ *   routing    split_sizes, group_offsets, row_to_slot, slot_to_row,
+ *              prob_perm from moe_permute (xq may be NULL there).
  *   x          bf16 [T][H];  out bf16 [T][H].
  *   workspace  >= moe_workspace_size(MOE_OP_FWD_BF16, T, k, E, H, I).
  * Limits as moe_grouped_mlp_fwd. */
 moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down, int32_t T, int32_t H, int32_t I,
                                       int32_t E, int32_t k, int64_t rows_cap, const int32_t* split_sizes,
                                       const int32_t* group_offsets, const int32_t* row_to_slot,
-                                      const float* prob_perm, const void* x, void* out, void* workspace,
-                                      size_t workspace_bytes, moe_stream_t stream);
+                                      const int32_t* slot_to_row, const float* prob_perm, const void* x,
+                                      void* out, void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* Top-k combine (Challenge 1, index_add back to token order):
  *   y  bf16 [T*k][H] in slot order -> out bf16 [T][H], out[t] = sum_j y[t*k+j]
@@ -338,7 +344,10 @@ moe_status_t moe_route_permute(const void* logits, int32_t logits_dtype, const v
  *   routing      as in the forward, plus slot_to_row (the dX combine
  *                gathers each token's k dgrad rows through it).
  *   dY           bf16 [T][H].  saved_a bf16 [rows_cap][2I] from the forward.
- *   xq_col, xq_col_sf  MX tensor (1, H, rows_cap) from moe_permute.
+ *   x            bf16 [T][H], the forward's input: quantised along tokens (in
+ *                permuted order, 32-token blocks per group) right before the
+ *                weight gradient of gate_up, so no column form of x has to
+ *                be kept between the forward and the backward.
  * Outputs: dX bf16 [T][H]; dW1 bf16 [E][2I][H]; dW2 bf16 [E][H][I];
  *   dprob float [T][k] (slot order).
  * Needs H % 32 == 0, I % 64 == 0, 1 <= k <= E <= MOE_MAX_EXPERTS and
@@ -348,8 +357,8 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
                                  int32_t k, int64_t rows_cap, const int32_t* split_sizes,
                                  const int32_t* group_offsets, const int32_t* row_to_slot,
                                  const int32_t* slot_to_row, const float* prob_perm,
-                                 const void* dY, const void* saved_a, const uint8_t* xq_col,
-                                 const uint8_t* xq_col_sf, void* dX, void* dW1, void* dW2,
+                                 const void* dY, const void* saved_a, const void* x, void* dX, void* dW1,
+                                 void* dW2,
                                  float* dprob, void* workspace, size_t workspace_bytes,
                                  moe_stream_t stream);
 

@@ -83,7 +83,7 @@ FwdWs carve_fwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t r
     w.hq = c.take(rows_cap * I);
     w.hq_sf = c.take(mx_scale_bytes(1, rows_cap, I));
   }
-  w.y = c.take(T * k * H * 4);
+  w.y = c.take(rows_cap * H * 4);  // fp32 down-projection rows in permuted order
   return w;
 }
 
@@ -94,7 +94,7 @@ FwdBf16Ws carve_fwd_bf16(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, 
   FwdBf16Ws w{};
   w.xp = c.take(rows_cap * H * 2);  // gathered x, bf16, permuted order
   w.h = c.take(rows_cap * I * 2);   // h, bf16
-  w.y = c.take(T * k * H * 4);      // fp32 down-projection rows in slot order
+  w.y = c.take(rows_cap * H * 4);   // fp32 down-projection rows in permuted order
   return w;
 }
 
@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 }
 
 struct BwdWs {
-  uint8_t *dyq, *dyq_sf, *dyc, *dyc_sf, *daq, *daq_sf, *dac, *dac_sf, *hc, *hc_sf, *dx, *dpp;
+  uint8_t *dyq, *dyq_sf, *dyc, *dyc_sf, *daq, *daq_sf, *dac, *dac_sf, *hc, *hc_sf, *dx, *dpp, *xc, *xc_sf;
 };
 BwdWs carve_bwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t rows_cap) {
   BwdWs w{};
@@ -128,6 +128,8 @@ BwdWs carve_bwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t r
   w.hc_sf = c.take(mx_scale_bytes(1, I, rows_cap));
   w.dx = c.take(rows_cap * H * 4);  // fp32 dgrad rows in permuted order
   w.dpp = c.take(I / 64 * rows_cap * 4);  // dprob partial sums per 64-column chunk
+  w.xc = c.take(H * rows_cap);             // gathered x quantised along tokens (wgrad1 operand)
+  w.xc_sf = c.take(mx_scale_bytes(1, H, rows_cap));
   return w;
 }
 
@@ -142,6 +144,26 @@ bool device_ok() {
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
   return major == 10;
 }
+
+}  // namespace
+
+// x quantised along H once per token (token order, the gate_up GEMM gathers
+// the rows it needs) and, for training, the gathered rows quantised along
+// tokens in permuted order (the weight-gradient operand).
+moe_status_t quantize_x(const void* x, int32_t T, int32_t H, int32_t k, int32_t E, int64_t rows_cap,
+                        const int32_t* row_to_slot, const int32_t* group_offsets, uint8_t* xq, uint8_t* xq_sf,
+                        uint8_t* xq_col, uint8_t* xq_col_sf, cudaStream_t st) {
+  QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, nullptr, 1, 1, T, H, xq, xq_sf};
+  if (launch_quant_rows(qr, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (xq_col) {
+    QuantBothArgs qb{static_cast<const uint8_t*>(x), 1, rows_cap, H, rows_cap, nullptr, nullptr, xq_col, xq_col_sf,
+                     row_to_slot, k, group_offsets + E};
+    if (launch_quant_both(qb, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+namespace {
 
 // Bounded-wait self test: one thread waits on a barrier nobody arrives on.
 __global__ void wait_timeout_kernel(long long limit_cycles) {
@@ -263,18 +285,8 @@ moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* to
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (!xq) return MOE_OK;
-  if (xq_col) {
-    // training: x rows gathered once, quantised along H and along tokens
-    QuantBothArgs qb{static_cast<const uint8_t*>(x), 1, rows_cap, H, rows_cap, xq, xq_sf, xq_col, xq_col_sf,
-                     row_to_slot, k, group_offsets + E};
-    TimeScope ts(st, "permute_quant");
-    if ((e = launch_quant_both(qb, st)) != cudaSuccess) return MOE_ERR_CUDA;
-  } else {
-    QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq, xq_sf, group_offsets + E};
-    TimeScope ts(st, "permute_quant");
-    if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
-  }
-  return MOE_OK;
+  TimeScope ts(st, "permute_quant");
+  return quantize_x(x, T, H, k, E, rows_cap, row_to_slot, group_offsets, xq, xq_sf, xq_col, xq_col_sf, st);
 }
 
 moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* out, moe_stream_t stream) {
@@ -290,11 +302,11 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
                                  const uint8_t* w2sf, int32_t T, int32_t H, int32_t I, int32_t E,
                                  int32_t k, int64_t rows_cap, const int32_t* split_sizes,
                                  const int32_t* group_offsets, const int32_t* row_to_slot,
-                                 const float* prob_perm, const uint8_t* xq, const uint8_t* xq_sf,
-                                 void* out, void* saved_a, uint8_t* hq, uint8_t* hq_sf, void* workspace,
-                                 size_t workspace_bytes, moe_stream_t stream) {
+                                 const int32_t* slot_to_row, const float* prob_perm, const uint8_t* xq,
+                                 const uint8_t* xq_sf, void* out, void* saved_a, uint8_t* hq, uint8_t* hq_sf,
+                                 void* workspace, size_t workspace_bytes, moe_stream_t stream) {
   if (!w1q || !w1sf || !w2q || !w2sf || !split_sizes || !group_offsets || !row_to_slot || !prob_perm ||
-      !xq || !xq_sf || (T > 0 && !out))
+      !xq || !xq_sf || (T > 0 && (!out || !slot_to_row)))
     return MOE_ERR_INVALID;
   if ((hq == nullptr) != (hq_sf == nullptr)) return MOE_ERR_INVALID;
   if (!layer_dims_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
@@ -311,10 +323,11 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (T == 0) return MOE_OK;
 
-  // gate_up grouped GEMM + ScaledSwiGLU + requantisation of h
-  GemmMaps m1;
+  // gate_up grouped GEMM + ScaledSwiGLU + requantisation of h; the A rows
+  // are gathered from x's codes in token order inside the GEMM
+  GemmMaps m1{};
   cudaError_t e;
-  if ((e = make_map_2d(&m1.a, xq, H, rows_cap, 128)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((e = make_map_2d(&m1.a, xq, H, T, 1)) != cudaSuccess) return MOE_ERR_CUDA;  // one-row box: gathers
   if ((e = make_map_3d(&m1.b, w1q, H, I, 2 * int64_t(E), 128)) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs g1{};
   g1.mode = 0; g1.E = E; g1.N = I; g1.num_kt = int32_t(cdiv(H, 128)); g1.n_tiles = int32_t(cdiv(I, 128));
@@ -324,12 +337,13 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   g1.prob = prob_perm; g1.row_to_slot = row_to_slot;
   g1.out2 = static_cast<uint8_t*>(saved_a);
   g1.q_out = w.hq; g1.sf_out = w.hq_sf; g1.q_KT = int32_t(cdiv(I, 128));
+  g1.gather_sf = xq_sf; g1.gather_k = k; g1.gather_rows = T;
   {
     TimeScope ts(st, "gemm_gate_up_swiglu");
     if ((e = launch_grouped_gemm(EPI_SWIGLU, 256, m1, g1, st)) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
-  // down grouped GEMM, rows scattered to slot order
+  // down grouped GEMM, fp32 rows in permuted order
   GemmMaps m2;
   if ((e = make_map_2d(&m2.a, w.hq, I, rows_cap, 128)) != cudaSuccess) return MOE_ERR_CUDA;
   if ((e = make_map_3d(&m2.b, w2q, I, H, E, 256)) != cudaSuccess) return MOE_ERR_CUDA;
@@ -338,24 +352,25 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   g2.group_offsets = group_offsets; g2.split_sizes = split_sizes;
   g2.sfa = w.hq_sf; g2.a_KT = int32_t(cdiv(I, 128));
   g2.sfb = w2sf; g2.b_RT = int32_t(cdiv(H, 128)); g2.b_KT = int32_t(cdiv(I, 128));
-  g2.row_to_slot = row_to_slot; g2.out = w.y; g2.ld_out = H;
+  g2.out = w.y; g2.ld_out = H;
   {
     TimeScope ts(st, "gemm_down");
-    if ((e = launch_grouped_gemm(EPI_F32_SCATTER, 256, m2, g2, st)) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((e = launch_grouped_gemm(EPI_F32_ROWS, 256, m2, g2, st)) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
-  // top-k combine back to token order
+  // top-k combine back to token order: a token's k rows gathered through
+  // slot_to_row and summed in ascending j
   TimeScope ts(st, "combine");
-  return cuda_status(launch_combine(w.y, true, nullptr, T, k, H, out, st));
+  return cuda_status(launch_combine(w.y, true, slot_to_row, T, k, H, out, st));
 }
 
 moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down, int32_t T, int32_t H, int32_t I,
                                       int32_t E, int32_t k, int64_t rows_cap, const int32_t* split_sizes,
                                       const int32_t* group_offsets, const int32_t* row_to_slot,
-                                      const float* prob_perm, const void* x, void* out, void* workspace,
-                                      size_t workspace_bytes, moe_stream_t stream) {
+                                      const int32_t* slot_to_row, const float* prob_perm, const void* x,
+                                      void* out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
   if (!w_gate_up || !w_down || !split_sizes || !group_offsets || !row_to_slot || !prob_perm ||
-      (T > 0 && (!x || !out)))
+      (T > 0 && (!x || !out || !slot_to_row)))
     return MOE_ERR_INVALID;
   if (!layer_dims_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
   if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
@@ -390,20 +405,20 @@ moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down,
     TimeScope ts(st, "gemm_gate_up_swiglu_bf16");
     if (launch_grouped_gemm_bf16(EPI_SWIGLU_BF16, m1, g1, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
-  // down grouped GEMM (bf16), fp32 rows scattered to slot order
+  // down grouped GEMM (bf16), fp32 rows in permuted order
   GemmMaps m2;
   if (make_map_2d(&m2.a, w.h, 2 * int64_t(I), rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
   if (make_map_3d(&m2.b, w_down, 2 * int64_t(I), H, E, 256) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs g2{};
   g2.mode = 0; g2.E = E; g2.N = H; g2.num_kt = int32_t(cdiv(2 * int64_t(I), 128)); g2.n_tiles = int32_t(cdiv(H, 256));
   g2.group_offsets = group_offsets; g2.split_sizes = split_sizes;
-  g2.row_to_slot = row_to_slot; g2.out = w.y; g2.ld_out = H;
+  g2.out = w.y; g2.ld_out = H;
   {
     TimeScope ts(st, "gemm_down_bf16");
-    if (launch_grouped_gemm_bf16(EPI_F32_SCATTER, m2, g2, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_grouped_gemm_bf16(EPI_F32_ROWS, m2, g2, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
   TimeScope ts(st, "combine");
-  return cuda_status(launch_combine(w.y, true, nullptr, T, k, H, out, st));
+  return cuda_status(launch_combine(w.y, true, slot_to_row, T, k, H, out, st));
 }
 
 moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, const uint8_t* w1tq,
@@ -411,17 +426,17 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
                                  int32_t k, int64_t rows_cap, const int32_t* split_sizes,
                                  const int32_t* group_offsets, const int32_t* row_to_slot,
                                  const int32_t* slot_to_row, const float* prob_perm, const void* dY,
-                                 const void* saved_a, const uint8_t* xq_col, const uint8_t* xq_col_sf,
+                                 const void* saved_a, const void* x,
                                  void* dX, void* dW1, void* dW2, float* dprob, void* workspace,
                                  size_t workspace_bytes, moe_stream_t stream) {
   if (!w2tq || !w2tsf || !w1tq || !w1tsf || !split_sizes || !group_offsets || !row_to_slot ||
-      (T > 0 && (!slot_to_row || !dY || !dX || !dprob)) || !prob_perm || !saved_a || !xq_col || !xq_col_sf ||
+      (T > 0 && (!slot_to_row || !dY || !dX || !dprob || !x)) || !prob_perm || !saved_a ||
       !dW1 || !dW2)
     return MOE_ERR_INVALID;
   if (!layer_dims_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
   if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
   for (const void* p : {(const void*)w2tq, (const void*)w2tsf, (const void*)w1tq, (const void*)w1tsf,
-                        dY, saved_a, (const void*)xq_col, (const void*)xq_col_sf, (const void*)dX,
+                        dY, saved_a, x, (const void*)dX,
                         (const void*)dW1, (const void*)dW2})
     if (!al16(p)) return MOE_ERR_INVALID;
   Carver c{static_cast<uint8_t*>(workspace)};
@@ -444,9 +459,9 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   // h along tokens, and sums dprob per 64-column chunk
   GemmMaps m;
   if (make_map_2d(&m.a, w.dyq, H, rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
-  if (make_map_3d(&m.b, w2tq, H, I, E, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m.b, w2tq, H, I, E, 192) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs g{};
-  g.mode = 0; g.E = E; g.N = I; g.num_kt = int32_t(cdiv(H, 128)); g.n_tiles = int32_t(cdiv(I, 128));
+  g.mode = 0; g.E = E; g.N = I; g.num_kt = int32_t(cdiv(H, 128)); g.n_tiles = int32_t(cdiv(I, 192));
   g.group_offsets = group_offsets; g.split_sizes = split_sizes;
   g.sfa = w.dyq_sf; g.a_KT = int32_t(cdiv(H, 128));
   g.sfb = w2tsf; g.b_RT = int32_t(cdiv(I, 128)); g.b_KT = int32_t(cdiv(H, 128));
@@ -455,7 +470,7 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   g.dprob_part = reinterpret_cast<float*>(w.dpp);
   {
     TimeScope ts(st, "gemm_dgrad_down_swiglu");
-    if (launch_grouped_gemm(EPI_SWIGLU_BWD, 128, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_grouped_gemm(EPI_SWIGLU_BWD, 192, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
   {
     TimeScope ts(st, "dprob_reduce");
@@ -499,15 +514,24 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
     if (launch_combine(w.dx, true, slot_to_row, T, k, H, dX, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
+  // x gathered and quantised along tokens (the operand of wgrad1), right
+  // before the GEMM that consumes it
+  {
+    QuantBothArgs qx{static_cast<const uint8_t*>(x), 1, rows_cap, H, rows_cap, nullptr, nullptr, w.xc, w.xc_sf,
+                     row_to_slot, k, group_offsets + E};
+    TimeScope ts(st, "x_quant_cols");
+    if (launch_quant_both(qx, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
   // wgrad1: dW_gate_up_e = da_e^T x_e (contraction over the group's tokens)
   if (make_map_2d(&m.a, w.dac, rows_cap, 2 * int64_t(I), 128) != cudaSuccess) return MOE_ERR_CUDA;
-  if (make_map_2d(&m.b, xq_col, rows_cap, H, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_2d(&m.b, w.xc, rows_cap, H, 256) != cudaSuccess) return MOE_ERR_CUDA;
   g = GemmArgs{};
   g.mode = 1; g.E = E; g.N = H; g.n_tiles = int32_t(cdiv(H, 256));
   g.m_tiles = int32_t(cdiv(2 * int64_t(I), 128)); g.M_out = 2 * I;
   g.group_offsets = group_offsets; g.split_sizes = split_sizes;
   g.sfa = w.dac_sf; g.a_KT = int32_t(rows_cap / 128);
-  g.sfb = xq_col_sf; g.b_RT = int32_t(cdiv(H, 128)); g.b_KT = int32_t(rows_cap / 128);
+  g.sfb = w.xc_sf; g.b_RT = int32_t(cdiv(H, 128)); g.b_KT = int32_t(rows_cap / 128);
   g.out = static_cast<uint8_t*>(dW1); g.ld_out = H; g.out_group_stride = 2 * int64_t(I) * H;
   {
     TimeScope ts(st, "gemm_wgrad_gate_up");
@@ -561,18 +585,8 @@ moe_status_t moe_route_permute(const void* logits, int32_t logits_dtype, const v
                                     prob_perm, workspace, st) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
-  cudaError_t e;
-  if (xq_col) {
-    QuantBothArgs qb{static_cast<const uint8_t*>(x), 1, rows_cap, H, rows_cap, xq, xq_sf, xq_col, xq_col_sf,
-                     row_to_slot, k, group_offsets + E};
-    TimeScope ts(st, "permute_quant");
-    if ((e = launch_quant_both(qb, st)) != cudaSuccess) return MOE_ERR_CUDA;
-  } else {
-    QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq, xq_sf, group_offsets + E};
-    TimeScope ts(st, "permute_quant");
-    if ((e = launch_quant_rows(qr, st)) != cudaSuccess) return MOE_ERR_CUDA;
-  }
-  return MOE_OK;
+  TimeScope ts(st, "permute_quant");
+  return quantize_x(x, T, H, k, E, rows_cap, row_to_slot, group_offsets, xq, xq_sf, xq_col, xq_col_sf, st);
 }
 
 moe_status_t moe_get_device_status(moe_stream_t stream) {

@@ -12,13 +12,15 @@
 //                   ScaledSwiGLU backward into the epilogue of the GEMM that
 //                   produces dh, so dh is never written either.
 //
-// Design (one CTA per SM, 320 threads), two tile widths BN:
+// Design (one CTA per SM), two tile widths BN:
 //   BN = 256: 128 x 256 tiles, one fp32 accumulator of 256 TMEM columns,
-//             4-stage shared-memory ring;
-//   BN = 128: 128 x 128 tiles, two accumulators of 128 columns (the MMAs of
+//             8 epilogue warps (320 threads);
+//   BN = 192: 128 x 192 tiles, two accumulators of 192 columns (the MMAs of
 //             the next tile run while the epilogue drains the previous one,
 //             so the epilogue may read TMEM lazily and hold it longer),
-//             5-stage ring.
+//             12 epilogue warps of 64 columns (448 threads) -- the fused
+//             ScaledSwiGLU backward, whose epilogue does the most work;
+//   both with a 4-stage shared-memory ring.
 //   warp 0      TMA producer: A tile 128x128 B, B tile BNx128 B (2-D or
 //               3-D tensor maps, 128-byte swizzle), the scale atoms by bulk
 //               copy, into the shared-memory ring (mbarrier pipeline).
@@ -26,7 +28,7 @@
 //               scale atoms to TMEM (tcgen05.cp 32x128b.warpx4) and issues
 //               four tcgen05.mma.kind::mxf8f6f4.block_scale (M128 NBN K32)
 //               into the current accumulator.
-//   warps 2-9   epilogue: drain the accumulator into registers
+//   warps 2..   epilogue: drain the accumulator into registers
 //               (tcgen05.ld), release it to the MMA warp, then apply the
 //               epilogue and store -- so the next tile's MMAs overlap it.
 //               Rows go out through a per-warp shared staging buffer so that
@@ -44,21 +46,25 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128, BK = 128;
-constexpr int NUM_THREADS = 320;
-constexpr int NUM_EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SFA_COL = 256, SFB_COL = 260;  // accumulators use columns 0..255
 constexpr int STAGE_PITCH_W = 20;                  // words per staged 64-byte row (16 used): conflict-free v4
 
-// Shared-memory plan and pipeline depth of the two tile widths.
+// Shared-memory plan, pipeline depth, TMEM plan and warp count of the two
+// tile widths: BN = 256 (one accumulator, 8 epilogue warps) and BN = 192
+// (two accumulators, 12 epilogue warps of 64 columns each).
 template <int BN>
 struct Cfg {
-  static constexpr int STAGES = BN == 256 ? 4 : 5;
+  static constexpr int STAGES = 4;
   static constexpr int ACC = BN == 256 ? 1 : 2;   // TMEM accumulators
+  static constexpr int EPI_WARPS = BN == 256 ? 8 : 12;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int NC = BN / (EPI_WARPS / 4);  // accumulator columns per epilogue warp
+  static constexpr uint32_t SFA_COL = ACC * BN, SFB_COL = ACC * BN + 4;  // scale factors after the accumulators
   static constexpr int SMEM_A = BM * BK;
   static constexpr int SMEM_B = BN * BK;
   static constexpr int SMEM_SFA = 512;
-  static constexpr int SMEM_SFB = BN * 4;          // one 512-byte atom per 128 rows of B
+  static constexpr int SFB_ATOMS = (BN + 127) / 128;
+  static constexpr int SMEM_SFB = SFB_ATOMS * 512;  // one 512-byte atom per 128 rows of B
   static constexpr uint32_t STAGE_TX = SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * SMEM_A;
@@ -69,12 +75,13 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem address, abort flag
   static constexpr int OFF_GO = OFF_MISC + 16;              // group offsets [E+1]
   // per-warp staging: 32 rows x 20 words (64-byte rows) or 16 rows x 36 words
-  // (128-byte rows); BN = 128 also transposes 32 x 32 fp32 values (pitch 36)
+  // (128-byte rows); BN = 192 transposes 32 x 32 fp32 values (pitch 36)
   static constexpr int STAGE_WARP_BYTES = BN == 256 ? 2560 : 32 * 36 * 4;
   static constexpr int OFF_STAGE = (OFF_GO + (MOE_MAX_EXPERTS + 1) * 4 + 127) / 128 * 128;
-  static constexpr int SMEM_TOTAL = OFF_STAGE + NUM_EPI_WARPS * STAGE_WARP_BYTES;
+  static constexpr int SMEM_TOTAL = OFF_STAGE + EPI_WARPS * STAGE_WARP_BYTES;
   static constexpr int SMEM_LAUNCH = SMEM_TOTAL + 1024;     // slack for 1 KB alignment
   static_assert(SMEM_LAUNCH <= 232448, "shared memory plan exceeds 227 KB");
+  static_assert(SFB_COL + 4 * SFB_ATOMS <= TMEM_COLS, "TMEM plan exceeds 512 columns");
 };
 
 struct Tile {
@@ -205,7 +212,7 @@ __device__ __forceinline__ void pack_bf16_inplace(uint32_t* v) {
 template <int EPI, int BN>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti, uint32_t* v, int q, int half,
                                               int lane, uint32_t* stage) {
-  constexpr int NC = BN / 2;  // accumulator columns per warp
+  constexpr int NC = Cfg<BN>::NC;  // accumulator columns per warp
   const int r = ti.m0 + 32 * q + lane;
   const bool rv = r < ti.row_end;
   if constexpr (EPI == EPI_SWIGLU_BF16) {
@@ -300,7 +307,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
 }
 
 // ---------------------------------------------------------------------------
-// EPI_SWIGLU_BWD (BN = 128): the ScaledSwiGLU backward on the dh tile.
+// EPI_SWIGLU_BWD (BN = 192): the ScaledSwiGLU backward on the dh tile.
 // The warp owns rows rb..rb+31 (one 32-row block along tokens: groups start
 // on multiples of 128) and dh columns cb..cb+63, read from TMEM in two
 // chunks of 32.  Per element, with g, u from the saved bf16 A and p the row's
@@ -363,6 +370,18 @@ __device__ __forceinline__ void load_dh32(uint32_t taddr, bool rv, uint32_t* d) 
   }
 }
 
+// Brings the saved-A lines a warp's EPI_SWIGLU_BWD epilogue will read for
+// tile ti into L2 (one 128-byte line of gate and one of up values per row),
+// so that the loads of the next tile do not wait on DRAM.
+__device__ __forceinline__ void prefetch_saved(const GemmArgs& a, const Tile& ti, int q, int half, int lane) {
+  const int cb = ti.n0 + 64 * half;
+  const int64_t r = ti.m0 + 32 * q + lane;
+  if (cb >= a.N || r >= ti.row_end) return;
+  const uint8_t* g = a.saved + (r * 2 * a.N + cb) * 2;
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(g));
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(g + int64_t(a.N) * 2));
+}
+
 __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Tile& ti, uint32_t tl, int q, int half,
                                                     int lane, uint32_t* stage) {
   const int I = a.N;
@@ -389,23 +408,24 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
       gv[i] = rv ? __ldg(reinterpret_cast<const uint4*>(grow + 64 * j) + i) : make_uint4(0u, 0u, 0u, 0u);
       uv[i] = rv ? __ldg(reinterpret_cast<const uint4*>(grow + int64_t(I) * 2 + 64 * j) + i) : make_uint4(0u, 0u, 0u, 0u);
     }
-    float sg[32], o[32];
+    float sv[32], o[32];  // sv: s = g * sigmoid(g), kept across the three passes
     uint32_t d[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) sg[e] = __fdividef(1.0f, 1.0f + __expf(-bf16_elem(gv, e)));
-    // dg, quantised along 2I (columns cc..cc+31) and along tokens
+    // dg = dh*p*u*sig*(1+g*(1-sig)), quantised along 2I (columns cc..cc+31)
+    // and along tokens
     load_dh32(tc, rv, d);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const float g = bf16_elem(gv, e), u = bf16_elem(uv, e);
-      o[e] = (__uint_as_float(d[e]) * p) * (u * sg[e]) * fmaf(g, 1.0f - sg[e], 1.0f);
+      const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
+      o[e] = (__uint_as_float(d[e]) * p) * (u * sg) * fmaf(g, 1.0f - sg, 1.0f);
+      sv[e] = g * sg;
     }
     sb_dg |= encode32_store(o, a.daq + r * I2 + cc) << (8 * j);
     quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, cc, a.rows_cap, rb, KTt);
-    // du, quantised along 2I (columns I+cc..) and along tokens
+    // du = dh*p*s, quantised along 2I (columns I+cc..) and along tokens
     load_dh32(tc, rv, d);
 #pragma unroll
-    for (int e = 0; e < 32; ++e) o[e] = (__uint_as_float(d[e]) * p) * (bf16_elem(gv, e) * sg[e]);
+    for (int e = 0; e < 32; ++e) o[e] = (__uint_as_float(d[e]) * p) * sv[e];
     sb_du |= encode32_store(o, a.daq + r * I2 + I + cc) << (8 * j);
     quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, int64_t(I) + cc, a.rows_cap, rb, KTt);
     // h = p*s*u along tokens (operand of the down projection's weight
@@ -413,7 +433,7 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
     load_dh32(tc, rv, d);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-      const float su = (bf16_elem(gv, e) * sg[e]) * bf16_elem(uv, e);
+      const float su = sv[e] * bf16_elem(uv, e);
       o[e] = p * su;
       dps = fmaf(__uint_as_float(d[e]), su, dps);
     }
@@ -427,14 +447,17 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
 }
 
 template <int EPI, int BN, int KIND>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
     grouped_mxf8_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB, const GemmArgs a) {
   using C = Cfg<BN>;
-  constexpr int STAGES = C::STAGES, ACC = C::ACC;
+  constexpr int STAGES = C::STAGES, ACC = C::ACC, NUM_THREADS = C::THREADS;
   constexpr bool MX = KIND == KIND_MXF8;
   constexpr bool GATE_UP = EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16;  // B tile = gate rows + up rows
   constexpr uint32_t TX = MX ? C::STAGE_TX : uint32_t(C::SMEM_A + C::SMEM_B);
+  // EPI_SWIGLU gathers the A rows (x in token order) with four-row TMA
+  // gathers issued by all of warp 0; the other launches load A with TMA
+  constexpr bool GATHER = EPI == EPI_SWIGLU;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -450,12 +473,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], GATHER ? 33 : 1);  // gather: + one arrival per producer lane
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < ACC; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], NUM_EPI_WARPS);
+      mbar_init(&acc_empty[b], C::EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -473,7 +496,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int ntiles = total_tiles(a, go);
 
   if (warp == 0) {
-    if (lane == 0) {
+    if constexpr (GATHER) {
+      // ---------------- gathering producer (whole warp) ----------------
+      // lane 0 arms the stage and loads B and its scales with TMA / bulk
+      // copies; lane l gathers the A rows 4l..4l+3 with one four-row TMA
+      // gather from x's codes in token order (padding rows read past the
+      // tensor: zeros) and copies their four scale bytes of the K tile
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const Tile ti = decode_tile<EPI, BN>(a, go, t);
+        int tok[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = ti.m0 + 4 * lane + i;
+          const int sl = r < ti.row_end ? __ldg(a.row_to_slot + r) : -1;
+          tok[i] = sl >= 0 ? sl / a.gather_k : a.gather_rows;  // a row past the tensor: zero fill
+        }
+        for (int kt = 0; kt < ti.nkt; ++kt) {
+          // every lane waits for the MMAs that read the stage, then all agree
+          const bool okl = mbar_wait(&empty[stage], phase ^ 1u, abort_flag);
+          if (!__all_sync(0xFFFFFFFFu, okl)) { ok = false; break; }
+          uint64_t* bar = &full[stage];
+          const int kg = ti.kt0 + kt;
+          uint8_t* sa = smem + C::OFF_A + stage * C::SMEM_A;
+          uint8_t* sb = smem + C::OFF_B + stage * C::SMEM_B;
+          uint8_t* ssfa = smem + C::OFF_SFA + stage * C::SMEM_SFA;
+          uint8_t* ssfb = smem + C::OFF_SFB + stage * C::SMEM_SFB;
+          if (lane == 0) {
+            ++issued;
+            mbar_arrive_expect_tx(bar, C::SMEM_A + C::SMEM_B + C::SMEM_SFB);
+            tma_load_3d(sb, &tmB, bar, kg * BK, ti.n0, 2 * ti.e);
+            tma_load_3d(sb + C::SMEM_B / 2, &tmB, bar, kg * BK, ti.n0, 2 * ti.e + 1);
+            const int rb = ti.n0 >> 7;
+            bulk_load(ssfb, a.sfb + ((int64_t(2 * ti.e) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
+            bulk_load(ssfb + 512, a.sfb + ((int64_t(2 * ti.e + 1) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
+          }
+          __syncwarp();  // the stage's byte count is armed before any gather lands
+          tma_gather4(sa + 512 * lane, &tmA, bar, kg * BK, tok[0], tok[1], tok[2], tok[3]);
+          const uint32_t sfa_u = smem_u32(ssfa);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int row = 4 * lane + i;
+            const bool val = tok[i] < a.gather_rows;
+            cp_async_4_zfill(sfa_u + (row & 31) * 16 + (row >> 5) * 4,
+                             val ? a.gather_sf + sf_offset(0, tok[i], 4 * kg, 0, a.a_KT) : a.gather_sf,
+                             val ? 4u : 0u);
+          }
+          cp_async_mbar_arrive_noinc(bar);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (lane == 0 && *abort_flag) {
+        const uint32_t first = issued > uint32_t(STAGES) ? issued - STAGES : 0u;
+        for (uint32_t i = first; i < issued; ++i)
+          mbar_wait_drain(&full[i % STAGES], (i / STAGES) & 1u);
+      }
+    } else if (lane == 0) {
       // ---------------- TMA producer ----------------
       prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
@@ -512,7 +595,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if constexpr (MX) {
               const int64_t gb = a.mode == 0 ? int64_t(ti.e) * a.b_RT : 0;
 #pragma unroll
-              for (int h = 0; h < BN / 128; ++h) {
+              for (int h = 0; h < C::SFB_ATOMS; ++h) {
                 const int rb = min((ti.n0 >> 7) + h, a.b_RT - 1);  // rows past N: any finite atom
                 bulk_load(ssfb + 512 * h, a.sfb + ((gb + rb) * a.b_KT + kg) * 512, 512, bar);
               }
@@ -535,7 +618,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, acc_it = 0;
       bool ok = true;
-      const uint32_t sfa_t = tmem + SFA_COL, sfb_t = tmem + SFB_COL;
+      const uint32_t sfa_t = tmem + C::SFA_COL, sfb_t = tmem + C::SFB_COL;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const Tile ti = decode_tile<EPI, BN>(a, go, t);
         if (ti.nkt == 0) continue;
@@ -546,6 +629,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kt = 0; kt < ti.nkt; ++kt) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
+          if constexpr (GATHER) fence_proxy_async_smem();  // A arrived through cp.async (generic proxy)
           const uint32_t sa = smem_u32(smem + C::OFF_A + stage * C::SMEM_A);
           const uint32_t sb = smem_u32(smem + C::OFF_B + stage * C::SMEM_B);
           const uint32_t ssfa = smem_u32(smem + C::OFF_SFA + stage * C::SMEM_SFA);
@@ -553,7 +637,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if constexpr (MX) {
             tc_cp_32x128b_warpx4(sfa_t, make_smem_desc(ssfa, 0, 128, 0));
 #pragma unroll
-            for (int h = 0; h < BN / 128; ++h)
+            for (int h = 0; h < C::SFB_ATOMS; ++h)
               tc_cp_32x128b_warpx4(sfb_t + 4 * h, make_smem_desc(ssfb + 512 * h, 0, 128, 0));
           }
           // four MMAs of 32 bytes of K each (32 E4M3 values, or 16 bf16)
@@ -584,16 +668,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------- epilogue warps ----------------
     const int q = warp & 3;            // TMEM sub-partition this warp may read
-    const int half = (warp - 2) >> 2;  // which half of the tile's columns
+    const int half = (warp - 2) >> 2;  // which NC-column part of the tile's columns
     uint32_t* stage = reinterpret_cast<uint32_t*>(smem + C::OFF_STAGE + (warp - 2) * C::STAGE_WARP_BYTES);
     uint32_t acc_it = 0;
-    uint32_t v[BN / 2];
+    uint32_t v[C::NC];
+    if constexpr (EPI == EPI_SWIGLU_BWD)
+      if (int(blockIdx.x) < ntiles) prefetch_saved(a, decode_tile<EPI, BN>(a, go, blockIdx.x), q, half, lane);
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       const Tile ti = decode_tile<EPI, BN>(a, go, t);
+      if constexpr (EPI == EPI_SWIGLU_BWD)  // one tile ahead
+        if (t + int(gridDim.x) < ntiles) prefetch_saved(a, decode_tile<EPI, BN>(a, go, t + gridDim.x), q, half, lane);
       if (ti.nkt == 0) {
         if constexpr (EPI == EPI_WGRAD) {
 #pragma unroll
-          for (int i = 0; i < BN / 2; ++i) v[i] = 0u;
+          for (int i = 0; i < C::NC; ++i) v[i] = 0u;
           epilogue_tile<EPI, BN>(a, ti, v, q, half, lane, stage);
         }
         continue;
@@ -612,7 +700,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if constexpr (GATE_UP) {  // gate columns 64*half.., up columns 128 + 64*half..
           tmem_ld64(tl + 64 * half, v);
           tmem_ld64(tl + 128 + 64 * half, v + 64);
-        } else if constexpr (BN == 256) {
+        } else if constexpr (C::NC == 128) {
           tmem_ld128(tl + 128 * half, v);
         } else {
           tmem_ld64(tl + 64 * half, v);
@@ -658,7 +746,7 @@ cudaError_t launch_epi(const GemmMaps& maps, const GemmArgs& a, cudaStream_t st)
   constexpr int smem = Cfg<BN>::SMEM_LAUNCH;
   cudaError_t e = ensure_smem_limit(grouped_mxf8_gemm_kernel<EPI, BN, KIND>, smem, configured);
   if (e != cudaSuccess) return e;
-  grouped_mxf8_gemm_kernel<EPI, BN, KIND><<<device_sm_count(), NUM_THREADS, smem, st>>>(maps.a, maps.b, a);
+  grouped_mxf8_gemm_kernel<EPI, BN, KIND><<<device_sm_count(), Cfg<BN>::THREADS, smem, st>>>(maps.a, maps.b, a);
   count_launch();
   return cudaGetLastError();
 }
@@ -700,13 +788,8 @@ cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const Gem
       case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256>(maps, a, st);
       case EPI_WGRAD: return launch_epi<EPI_WGRAD, 256>(maps, a, st);
     }
-  } else if (bn == 128) {
-    switch (epi) {
-      case EPI_F32_SCATTER: return launch_epi<EPI_F32_SCATTER, 128>(maps, a, st);
-      case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 128>(maps, a, st);
-      case EPI_WGRAD: return launch_epi<EPI_WGRAD, 128>(maps, a, st);
-      case EPI_SWIGLU_BWD: return launch_epi<EPI_SWIGLU_BWD, 128>(maps, a, st);
-    }
+  } else if (bn == 192) {
+    if (epi == EPI_SWIGLU_BWD) return launch_epi<EPI_SWIGLU_BWD, 192>(maps, a, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -714,7 +797,7 @@ cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const Gem
 cudaError_t launch_grouped_gemm_bf16(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
   switch (epi) {
     case EPI_SWIGLU_BF16: return launch_epi<EPI_SWIGLU_BF16, 256, KIND_BF16>(maps, a, st);
-    case EPI_F32_SCATTER: return launch_epi<EPI_F32_SCATTER, 256, KIND_BF16>(maps, a, st);
+    case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256, KIND_BF16>(maps, a, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -62,9 +62,17 @@ struct GemmArgs {
   uint8_t* hcol;
   uint8_t* hcol_sf;
   float* dprob_part;
+  // EPI_SWIGLU: A is gathered row by row from the MX tensor of x in token
+  // order (codes [T][K] through tensor map A with a one-row box, blocked
+  // scales (1, T, K)): row r of the permuted space reads token
+  // row_to_slot[r] / gather_k
+  const uint8_t* gather_sf;  // blocked scales (1, T, K) of x in token order (codes: tensor map A)
+  int32_t gather_k;
+  int32_t gather_rows;       // T
 };
 
-// Tensor maps: A 2-D {K, rows} with a 128 x 128 box; B either 3-D
+// Tensor maps: A 2-D {K, rows} with a 128 x 128 box (EPI_SWIGLU: x's codes
+// {K, T} with a 128 x 1 box, for four-row gathers); B either 3-D
 // {K, rows, groups} or 2-D {K, rows} with a 128 x bn box (EPI_SWIGLU: two
 // boxes of bn/2 rows); all uint8 with 128-byte swizzle.
 struct GemmMaps {
@@ -76,11 +84,11 @@ cudaError_t make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64
 cudaError_t make_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                         uint64_t groups, uint32_t box_rows);
 
-// bn: tile width, 256 (one accumulator) or 128 (two accumulators; required
-// by EPI_SWIGLU_BWD, not offered for EPI_SWIGLU).
+// bn: tile width, 256 (one accumulator; every epilogue but EPI_SWIGLU_BWD)
+// or 192 (two accumulators, 12 epilogue warps; EPI_SWIGLU_BWD).
 cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);
 
-// BF16 operands (kind::f16), bn = 256: EPI_SWIGLU_BF16 and EPI_F32_SCATTER.
+// BF16 operands (kind::f16), bn = 256: EPI_SWIGLU_BF16 and EPI_F32_ROWS.
 // The tensor maps describe the bf16 matrices as bytes (inner extent 2K), and
 // num_kt / a_KT count 128-byte K tiles.
 cudaError_t launch_grouped_gemm_bf16(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);

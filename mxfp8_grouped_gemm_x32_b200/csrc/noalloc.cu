@@ -74,13 +74,5 @@ extern "C" moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_i
   if (launch_permute_index(topk_idx, topk_prob, R, E, rows_cap, split_sizes, group_offsets, row_to_slot,
                            slot_to_row, prob_perm, scratch, st) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (xq_col) {
-    QuantBothArgs qb{static_cast<const uint8_t*>(x), 1, rows_cap, H, rows_cap, xq, xq_sf, xq_col, xq_col_sf,
-                     row_to_slot, k, group_offsets + E};
-    if (launch_quant_both(qb, st) != cudaSuccess) return MOE_ERR_CUDA;
-  } else {
-    QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, row_to_slot, k, 1, rows_cap, H, xq, xq_sf, group_offsets + E};
-    if (launch_quant_rows(qr, st) != cudaSuccess) return MOE_ERR_CUDA;
-  }
-  return MOE_OK;
+  return quantize_x(x, T, H, k, E, rows_cap, row_to_slot, group_offsets, xq, xq_sf, xq_col, xq_col_sf, st);
 }

@@ -34,7 +34,9 @@ __global__ void __launch_bounds__(PB) perm_hist_kernel(const int32_t* __restrict
 }
 
 // Pass 2 (one CTA): split_sizes, 128-aligned group offsets, and the first
-// output row of every (block, expert) pair, in place in `hist`.
+// row of every (block, expert) pair relative to its group's start, in place
+// in `hist` (the scatter adds the group offset).  Each expert's column of
+// block counts is read eight blocks at a time so that the loads overlap.
 __global__ void __launch_bounds__(MOE_MAX_EXPERTS) perm_scan_kernel(int32_t* __restrict__ hist,
                                                                     int32_t nblocks, int32_t E,
                                                                     int32_t* __restrict__ split,
@@ -43,10 +45,15 @@ __global__ void __launch_bounds__(MOE_MAX_EXPERTS) perm_scan_kernel(int32_t* __r
   const int e = threadIdx.x;
   int32_t total = 0;
   if (e < E) {
-    for (int b = 0; b < nblocks; ++b) {
-      const int32_t c = hist[int64_t(b) * E + e];
-      hist[int64_t(b) * E + e] = total;
-      total += c;
+    for (int b0 = 0; b0 < nblocks; b0 += 8) {
+      int32_t c[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[i] = b0 + i < nblocks ? hist[int64_t(b0 + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (b0 + i < nblocks) hist[int64_t(b0 + i) * E + e] = total;
+        total += c[i];
+      }
     }
     split[e] = total;
   }
@@ -59,14 +66,10 @@ __global__ void __launch_bounds__(MOE_MAX_EXPERTS) perm_scan_kernel(int32_t* __r
       padded[i] = run;
       run += p;
     }
-    padded[E] = run;
     offs[E] = run;
   }
   __syncthreads();
-  if (e < E) {
-    offs[e] = padded[e];
-    for (int b = 0; b < nblocks; ++b) hist[int64_t(b) * E + e] += padded[e];
-  }
+  if (e < E) offs[e] = padded[e];
 }
 
 // Pass 3: stable rank of every slot inside its block (warp match + per-warp
@@ -75,6 +78,7 @@ __global__ void __launch_bounds__(MOE_MAX_EXPERTS) perm_scan_kernel(int32_t* __r
 __global__ void __launch_bounds__(PB) perm_scatter_kernel(const int32_t* __restrict__ idx,
                                                           const float* __restrict__ prob, int64_t R,
                                                           int32_t E, const int32_t* __restrict__ base,
+                                                          const int32_t* __restrict__ offs,
                                                           int32_t* __restrict__ slot_to_row,
                                                           int32_t* __restrict__ row_to_slot,
                                                           float* __restrict__ prob_perm) {
@@ -99,7 +103,7 @@ __global__ void __launch_bounds__(PB) perm_scatter_kernel(const int32_t* __restr
     }
     int32_t pre = 0;
     for (int w = 0; w < warp; ++w) pre += wcnt[w * E + e];
-    const int32_t row = base[int64_t(blockIdx.x) * E + e] + pre + int32_t(lrank);
+    const int32_t row = offs[e] + base[int64_t(blockIdx.x) * E + e] + pre + int32_t(lrank);
     slot_to_row[s] = row;
     row_to_slot[row] = int32_t(s);
     prob_perm[row] = prob[s];
@@ -151,7 +155,7 @@ cudaError_t launch_permute_scan_scatter(const int32_t* idx, const float* prob, i
   perm_scan_kernel<<<1, MOE_MAX_EXPERTS, 0, st>>>(hist, nb, E, split, offs);
   count_launch();
   if (nb > 0) {
-    perm_scatter_kernel<<<nb, PB, 32 * E * sizeof(int), st>>>(idx, prob, R, E, hist, slot_to_row,
+    perm_scatter_kernel<<<nb, PB, 32 * E * sizeof(int), st>>>(idx, prob, R, E, hist, offs, slot_to_row,
                                                                row_to_slot, prob_perm);
     count_launch();
   }

@@ -239,7 +239,7 @@ __device__ __forceinline__ void qb_compute(const QuantBothArgs& a, const QbTile&
   // thread -> (row tid % 128, column half tid / 128): a warp reads 32
   // consecutive staged rows with 16-byte loads, conflict-free for the
   // 272-byte row pitch
-  {
+  if (a.q_row) {
     const int rl = tid & 127, hb = tid >> 7;
     const int64_t r = r0 + rl;
     uint32_t sbs = 0;
@@ -331,7 +331,7 @@ __device__ __forceinline__ void qb_store(const QuantBothArgs& a, const QbTile& q
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int rr = (tid >> 3) + 32 * i;
-    if (q.r0 + rr < a.rows && 16 * chunk < vrow_bytes)
+    if (a.q_row && q.r0 + rr < a.rows && 16 * chunk < vrow_bytes)
       *reinterpret_cast<uint4*>(qr + int64_t(rr) * a.cols) =
           *reinterpret_cast<const uint4*>(out_row + rr * QB_OUT_PITCH + 16 * chunk);
     if (q.c0 + rr < a.cols && 16 * chunk < vcol_bytes)
@@ -339,7 +339,7 @@ __device__ __forceinline__ void qb_store(const QuantBothArgs& a, const QbTile& q
           *reinterpret_cast<const uint4*>(out_col + rr * QB_OUT_PITCH + 16 * chunk);
   }
   if (tid < 32) {
-    if (row_atom) {
+    if (row_atom && a.q_row) {
       const uint32_t rq = fastdiv(uint32_t(q.r0), a.rs_div);
       const int64_t rg = q.g * a.row_groups + rq;
       const int64_t rr = q.r0 - int64_t(rq) * a.row_split;
@@ -409,7 +409,7 @@ cudaError_t launch_quant_both(const QuantBothArgs& args, cudaStream_t st) {
   if (a.row_split <= 0 || a.row_split >= (int64_t(1) << 31) || a.rows >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
   a.rs_div = make_fastdiv(uint32_t(a.row_split));
   a.row_groups = uint32_t(a.rows / a.row_split);
-  if (a.row_split % 128) {
+  if (a.q_row && a.row_split % 128) {
     // row-groups whose last 128-row tile is partial own padding scale bytes
     // that no source row maps to: clear the row-mode scales first
     const int64_t n = int64_t(a.groups) * (a.rows / a.row_split) * cdiv(a.row_split, 128) *

@@ -45,7 +45,7 @@ namespace moe {
 // Both modes from one read of the source: input [groups][rows][cols] bf16,
 // or, with row_map, input row (g*rows + r) = source row
 // row_map[g*rows + r] / map_div (a negative entry gives a zero row).
-//  row mode output: MX tensor whose groups split each input group into
+//  row mode output (skipped when q_row is null): MX tensor whose groups split each input group into
 //    rows / row_split row-groups of row_split rows (W_gate_up: gate and up
 //    halves) -- q_row [groups*rows][cols], sf_row blocked
 //    (groups*rows/row_split, row_split, cols);
@@ -73,5 +73,16 @@ struct QuantBothArgs {
 };
 
 cudaError_t launch_quant_both(const QuantBothArgs& a, cudaStream_t st);
+
+}  // namespace moe
+
+namespace moe {
+
+// The permutation's quantisation of x (defined with the C entry points):
+// xq, xq_sf = MX tensor (1, T, H) of x in token order; with xq_col, the
+// gathered rows quantised along tokens, MX tensor (1, H, rows_cap).
+moe_status_t quantize_x(const void* x, int32_t T, int32_t H, int32_t k, int32_t E, int64_t rows_cap,
+                        const int32_t* row_to_slot, const int32_t* group_offsets, uint8_t* xq, uint8_t* xq_sf,
+                        uint8_t* xq_col, uint8_t* xq_col_sf, cudaStream_t st);
 
 }  // namespace moe

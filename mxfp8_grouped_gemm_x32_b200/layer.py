@@ -102,8 +102,8 @@ class GroupedMLP:
         self.topk_idx = al.typed((T, k), torch.int32, "topk_idx")        # router outputs
         self.topk_prob = al.typed((T, k), torch.float32, "topk_prob")
         self.prob_perm = al.typed((rc,), torch.float32, "prob_perm")
-        self.xq = u8(rc * H, "xq")
-        self.xq_sf = u8(sb(1, rc, H), "xq_sf")
+        self.xq = u8(T * H, "xq")                # x quantised along H, token order
+        self.xq_sf = u8(sb(1, T, H), "xq_sf")
         self.hq = u8(rc * I, "hq")
         self.hq_sf = u8(sb(1, rc, I), "hq_sf")
         self.out = al.typed((T, H), torch.bfloat16, "out")
@@ -118,8 +118,6 @@ class GroupedMLP:
             self.w1tsf = u8(sb(E, H, 2 * I), "w1tsf")
             self.w2tq = u8(E * I * H, "w2tq")
             self.w2tsf = u8(sb(E, I, H), "w2tsf")
-            self.xq_col = u8(H * rc, "xq_col")
-            self.xq_col_sf = u8(sb(1, H, rc), "xq_col_sf")
             self.saved_a = al.typed((rc, 2 * I), torch.bfloat16, "saved_a")
             self.dX = al.typed((T, H), torch.bfloat16, "dX")
             self.dW1 = al.typed((E, 2 * I, H), torch.bfloat16, "dW1")
@@ -129,6 +127,18 @@ class GroupedMLP:
             self.ws_bwd = u8(self.ws_bwd_bytes, "ws_bwd")
         else:
             self.saved_a = None
+        self.xq_col = self.xq_col_sf = None   # x along tokens: only when permute(..., with_cols=True)
+        self._x = None                         # the input of the last permutation (the backward's x)
+
+    def _cols(self, with_cols: bool):
+        """Buffers of the optional column form of x (x^T quantised along
+        tokens in permuted order); the backward does not need them."""
+        if not with_cols:
+            return 0, 0
+        if self.xq_col is None:
+            self.xq_col = self._alloc.raw(self.H * self.rows_cap, "xq_col")
+            self.xq_col_sf = self._alloc.raw(lib.moe_mx_scale_bytes(1, self.H, self.rows_cap), "xq_col_sf")
+        return _ptr(self.xq_col), _ptr(self.xq_col_sf)
 
     def permute_index(self, topk_idx: torch.Tensor, topk_prob: torch.Tensor) -> None:
         """Routing outputs of the permutation only (no quantisation of x):
@@ -153,7 +163,8 @@ class GroupedMLP:
             self.ws_bf16 = self._alloc.raw(self.ws_bf16_bytes, "ws_bf16")
         lib.moe_grouped_mlp_fwd_bf16(w1.data_ptr(), w2.data_ptr(), self.T, H, I, E, self.k, self.rows_cap,
                                      _ptr(self.split_sizes), _ptr(self.group_offsets), _ptr(self.row_to_slot),
-                                     _ptr(self.prob_perm), x.data_ptr(), _ptr(self.out), _ptr(self.ws_bf16),
+                                     _ptr(self.slot_to_row), _ptr(self.prob_perm), x.data_ptr(), _ptr(self.out),
+                                     _ptr(self.ws_bf16),
                                      self.ws_bf16_bytes, self._stream())
         return self.out
 
@@ -191,55 +202,64 @@ class GroupedMLP:
                             _ptr(self.topk_prob), self._stream())
         return self.topk_idx, self.topk_prob
 
-    def route_permute(self, logits: torch.Tensor, x: torch.Tensor):
+    def route_permute(self, logits: torch.Tensor, x: torch.Tensor, with_cols: bool = False):
         """Router and permutation in one call (moe_route_permute): logits fp32
         or bf16 [T, E], x bf16 [T, H]; the routing lands in topk_idx /
-        topk_prob, the permuted and quantised x in this layer's buffers."""
+        topk_prob, the quantised x in this layer's buffers."""
         dt = {torch.float32: lib.MOE_DTYPE_F32, torch.bfloat16: lib.MOE_DTYPE_BF16}.get(logits.dtype)
         if dt is None:
             raise TypeError(f"logits: expected float32 or bfloat16, got {logits.dtype}")
         check_tensor(logits, "logits", logits.dtype, (self.T, self.E), self.dev)
         check_tensor(x, "x", torch.bfloat16, (self.T, self.H), self.dev)
-        bw = self.backward_enabled
+        xc, xcs = self._cols(with_cols)
         lib.moe_route_permute(logits.data_ptr(), dt, x.data_ptr(), self.T, self.H, self.k, self.E, self.rows_cap,
                               _ptr(self.topk_idx), _ptr(self.topk_prob), _ptr(self.split_sizes),
                               _ptr(self.group_offsets), _ptr(self.row_to_slot), _ptr(self.slot_to_row),
-                              _ptr(self.prob_perm), _ptr(self.xq), _ptr(self.xq_sf), _ptr(self.xq_col) if bw else 0,
-                              _ptr(self.xq_col_sf) if bw else 0, _ptr(self.ws_perm), self.ws_perm_bytes,
-                              self._stream())
+                              _ptr(self.prob_perm), _ptr(self.xq), _ptr(self.xq_sf), xc, xcs, _ptr(self.ws_perm),
+                              self.ws_perm_bytes, self._stream())
+        self._x = x
         return self.topk_idx, self.topk_prob
 
-    def permute(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_prob: torch.Tensor) -> None:
-        """x bf16 [T, H]; topk_idx int32 [T, k]; topk_prob float32 [T, k]."""
+    def permute(self, x: torch.Tensor, topk_idx: torch.Tensor, topk_prob: torch.Tensor,
+                with_cols: bool = False) -> None:
+        """x bf16 [T, H]; topk_idx int32 [T, k]; topk_prob float32 [T, k].
+        with_cols also writes x^T quantised along tokens (xq_col), which the
+        backward makes for itself from x."""
         check_tensor(x, "x", torch.bfloat16, (self.T, self.H), self.dev)
         check_tensor(topk_idx, "topk_idx", torch.int32, (self.T, self.k), self.dev)
         check_tensor(topk_prob, "topk_prob", torch.float32, (self.T, self.k), self.dev)
-        bw = self.backward_enabled
+        xc, xcs = self._cols(with_cols)
         lib.moe_permute(x.data_ptr(), topk_idx.data_ptr(), topk_prob.data_ptr(), self.T, self.H, self.k,
                         self.E, self.rows_cap, _ptr(self.split_sizes), _ptr(self.group_offsets),
                         _ptr(self.row_to_slot), _ptr(self.slot_to_row), _ptr(self.prob_perm),
-                        _ptr(self.xq), _ptr(self.xq_sf), _ptr(self.xq_col) if bw else 0,
-                        _ptr(self.xq_col_sf) if bw else 0, _ptr(self.ws_perm), self.ws_perm_bytes,
+                        _ptr(self.xq), _ptr(self.xq_sf), xc, xcs, _ptr(self.ws_perm), self.ws_perm_bytes,
                         self._stream())
+        self._x = x
 
     def forward(self) -> torch.Tensor:
         lib.moe_grouped_mlp_fwd(_ptr(self.w1q), _ptr(self.w1sf), _ptr(self.w2q), _ptr(self.w2sf), self.T,
                                 self.H, self.I, self.E, self.k, self.rows_cap, _ptr(self.split_sizes),
-                                _ptr(self.group_offsets), _ptr(self.row_to_slot), _ptr(self.prob_perm),
-                                _ptr(self.xq), _ptr(self.xq_sf), _ptr(self.out), _ptr(self.saved_a),
+                                _ptr(self.group_offsets), _ptr(self.row_to_slot), _ptr(self.slot_to_row),
+                                _ptr(self.prob_perm), _ptr(self.xq), _ptr(self.xq_sf), _ptr(self.out),
+                                _ptr(self.saved_a),
                                 _ptr(self.hq), _ptr(self.hq_sf), _ptr(self.ws_fwd), self.ws_fwd_bytes,
                                 self._stream())
         return self.out
 
-    def backward(self, dY: torch.Tensor):
+    def backward(self, dY: torch.Tensor, x: torch.Tensor = None):
+        """dY bf16 [T, H]; x defaults to the input of the last permutation."""
         if not self.backward_enabled:
             raise RuntimeError("this layer was built with backward=False")
+        x = self._x if x is None else x
+        if x is None:
+            raise RuntimeError("backward needs x: call permute first or pass x")
         check_tensor(dY, "dY", torch.bfloat16, (self.T, self.H), self.dev)
+        check_tensor(x, "x", torch.bfloat16, (self.T, self.H), self.dev)
         lib.moe_grouped_mlp_bwd(_ptr(self.w2tq), _ptr(self.w2tsf), _ptr(self.w1tq), _ptr(self.w1tsf),
                                 self.T, self.H, self.I, self.E, self.k, self.rows_cap,
                                 _ptr(self.split_sizes), _ptr(self.group_offsets), _ptr(self.row_to_slot),
                                 _ptr(self.slot_to_row), _ptr(self.prob_perm), dY.data_ptr(),
-                                _ptr(self.saved_a), _ptr(self.xq_col), _ptr(self.xq_col_sf),
+                                _ptr(self.saved_a), x.data_ptr(),
                                 _ptr(self.dX), _ptr(self.dW1), _ptr(self.dW2), _ptr(self.dprob),
                                 _ptr(self.ws_bwd), self.ws_bwd_bytes, self._stream())
         return self.dX, self.dW1, self.dW2, self.dprob
@@ -252,7 +272,7 @@ class GroupedMLP:
         out = self.forward()
         if dY is None:
             return out
-        return (out,) + tuple(self.backward(dY))
+        return (out,) + tuple(self.backward(dY, x))
 
     def device_status(self) -> int:
         return lib.moe_get_device_status(self._stream())

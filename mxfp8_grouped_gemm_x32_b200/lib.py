@@ -73,17 +73,17 @@ _decl("moe_mlp_quantize_weights", _I32, _P, _P, _I32, _I32, _I32, _P, _P, _P, _P
 _decl("moe_permute", _I32, _P, _P, _P, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
       _P, _P, _SZ, _P)
 _decl("moe_grouped_mlp_fwd", _I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P,
-      _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
+      _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
 _decl("moe_combine", _I32, _P, _I32, _I32, _I32, _P, _P)
 _decl("moe_router_topk", _I32, _P, _I32, _I32, _I32, _I32, _P, _P, _P)
 _decl("moe_grouped_mlp_bwd", _I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P,
-      _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
+      _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
 _decl("moe_mx_scales_to_blocked", _I32, _P, _I32, _I64, _I64, _I64, _P, _P)
 _decl("moe_mx_scales_from_blocked", _I32, _P, _I32, _I64, _I64, _P, _I64, _P)
 _decl("moe_route_permute", _I32, _P, _I32, _P, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
       _P, _P, _P, _P, _SZ, _P)
 _decl("moe_grouped_mlp_fwd_bf16", _I32, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P, _P,
-      _SZ, _P)
+      _P, _SZ, _P)
 _decl("moe_get_device_status", _I32, _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
 _decl("moe_launch_count", _I64, _I32)
@@ -143,11 +143,11 @@ def moe_permute_noalloc(x, topk_idx, topk_prob, T, H, k, E, rows_cap, split_size
 
 
 def moe_grouped_mlp_fwd(w1q, w1sf, w2q, w2sf, T, H, I, E, k, rows_cap, split_sizes, group_offsets,
-                        row_to_slot, prob_perm, xq, xq_sf, out, saved_a, hq, hq_sf, workspace,
+                        row_to_slot, slot_to_row, prob_perm, xq, xq_sf, out, saved_a, hq, hq_sf, workspace,
                         workspace_bytes, stream=0):
     _check("moe_grouped_mlp_fwd", _lib.moe_grouped_mlp_fwd(
-        w1q, w1sf, w2q, w2sf, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot, prob_perm,
-        xq, xq_sf, out, saved_a, hq, hq_sf, workspace, workspace_bytes, stream))
+        w1q, w1sf, w2q, w2sf, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot, slot_to_row,
+        prob_perm, xq, xq_sf, out, saved_a, hq, hq_sf, workspace, workspace_bytes, stream))
 
 
 def moe_mx_scales_to_blocked(plain, groups, rows, k, ld, blocked, stream=0):
@@ -159,10 +159,10 @@ def moe_mx_scales_from_blocked(blocked, groups, rows, k, plain, ld, stream=0):
 
 
 def moe_grouped_mlp_fwd_bf16(w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot,
-                             prob_perm, x, out, workspace, workspace_bytes, stream=0):
+                             slot_to_row, prob_perm, x, out, workspace, workspace_bytes, stream=0):
     _check("moe_grouped_mlp_fwd_bf16", _lib.moe_grouped_mlp_fwd_bf16(
-        w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot, prob_perm, x, out,
-        workspace, workspace_bytes, stream))
+        w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot, slot_to_row, prob_perm,
+        x, out, workspace, workspace_bytes, stream))
 
 
 def moe_combine(y, T, k, H, out, stream=0):
@@ -182,11 +182,11 @@ def moe_route_permute(logits, logits_dtype, x, T, H, k, E, rows_cap, topk_idx, t
 
 
 def moe_grouped_mlp_bwd(w2tq, w2tsf, w1tq, w1tsf, T, H, I, E, k, rows_cap, split_sizes, group_offsets,
-                        row_to_slot, slot_to_row, prob_perm, dY, saved_a, xq_col, xq_col_sf, dX, dW1,
+                        row_to_slot, slot_to_row, prob_perm, dY, saved_a, x, dX, dW1,
                         dW2, dprob, workspace, workspace_bytes, stream=0):
     _check("moe_grouped_mlp_bwd", _lib.moe_grouped_mlp_bwd(
         w2tq, w2tsf, w1tq, w1tsf, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot,
-        slot_to_row, prob_perm, dY, saved_a, xq_col, xq_col_sf, dX, dW1, dW2, dprob, workspace,
+        slot_to_row, prob_perm, dY, saved_a, x, dX, dW1, dW2, dprob, workspace,
         workspace_bytes, stream))
 
 

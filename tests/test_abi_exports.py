@@ -109,7 +109,7 @@ def _fwd_args(T=64, H=256, I=512, E=4, k=2, rows_cap=None, w1q=P, out=P, hq=P, h
     from mxfp8_grouped_gemm_x32_b200 import lib
     if rows_cap is None:
         rows_cap = lib.moe_padded_rows(T, k, E)
-    return (w1q, P, P, P, T, H, I, E, k, rows_cap, P, P, P, P, P, P, out, P, hq, hq_sf, ws, ws_bytes, None)
+    return (w1q, P, P, P, T, H, I, E, k, rows_cap, P, P, P, P, P, P, P, out, P, hq, hq_sf, ws, ws_bytes, None)
 
 
 def test_forward_argument_errors():
@@ -131,7 +131,7 @@ def test_forward_argument_errors():
 def _bwd_args(T=64, H=256, I=512, E=4, k=2, saved=P, dW1=P, ws_bytes=1 << 40):
     from mxfp8_grouped_gemm_x32_b200 import lib
     rows_cap = lib.moe_padded_rows(T, k, E)
-    return (P, P, P, P, T, H, I, E, k, rows_cap, P, P, P, P, P, P, saved, P, P, P, dW1, P, P, P, ws_bytes, None)
+    return (P, P, P, P, T, H, I, E, k, rows_cap, P, P, P, P, P, P, saved, P, P, dW1, P, P, P, ws_bytes, None)
 
 
 def test_backward_argument_errors():

@@ -42,21 +42,22 @@ def _rel_rms(g, r):
 
 
 def _slot_buffers(L, cfg):
-    """fp32 per-slot rows kept by the library in the caller's workspaces:
-    the forward's y (first piece when hq is caller-provided, [T*k][H] in slot
-    order) and the backward's dx (the piece after the MX operands, [rows_cap][H]
-    in permuted order), both returned in slot order."""
+    """fp32 rows kept by the library in the caller's workspaces: the
+    forward's y (first piece when hq is caller-provided) and the backward's
+    dx (the piece after the MX operands), both [rows_cap][H] in permuted
+    order, returned in slot order."""
     import torch
     from mxfp8_grouped_gemm_x32_b200 import lib
-    rc, H, I, n = L.rows_cap, cfg.H, cfg.I, cfg.T * cfg.k * cfg.H
+    rc, H, I = L.rows_cap, cfg.H, cfg.I
     a256 = lambda v: (v + 255) // 256 * 256
     sb = lib.moe_mx_scale_bytes
     pieces = [rc * H, sb(1, rc, H), H * rc, sb(1, H, rc), rc * 2 * I, sb(1, rc, 2 * I),
               2 * I * rc, sb(1, 2 * I, rc), I * rc, sb(1, I, rc)]
     off = sum(a256(p) for p in pieces)
-    y = L.ws_fwd[: n * 4].view(torch.float32)
+    y = L.ws_fwd[: rc * H * 4].view(torch.float32).view(rc, H)
     dx = L.ws_bwd[off: off + rc * H * 4].view(torch.float32).view(rc, H)
-    return y.view(cfg.T * cfg.k, H), dx[L.slot_to_row.long()]
+    s2r = L.slot_to_row.long()
+    return y[s2r], dx[s2r]
 
 
 @pytest.mark.parametrize("name", ["mixtral_8x7b", "qwen3_30b_ragged", "gpt_oss_20b"])

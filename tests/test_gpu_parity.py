@@ -119,6 +119,9 @@ class Layer:
                      torch.from_numpy(inp["topk_prob"]).cuda(), _bf(torch, inp["w1"]),
                      _bf(torch, inp["w2"]), _bf(torch, inp["dy"]))
         self.res = self.L.step(*self.args)
+        # the permutation once more with the optional column form of x (the
+        # backward makes its own): checked in test_permute_bitexact
+        self.L.permute(self.args[0], self.args[1], self.args[2], with_cols=True)
         torch.cuda.synchronize()
         from mxfp8_grouped_gemm_x32_b200 import lib
         self.status = lib.moe_get_device_status(0)
@@ -197,8 +200,11 @@ def test_permute_bitexact(run):
     s2r = L.slot_to_row.cpu().numpy()
     pp = L.prob_perm.cpu().numpy()
     offs = f["offsets"]
-    xq = L.xq.cpu().numpy()[: L.rows_cap * cfg.H].reshape(L.rows_cap, cfg.H)
-    xsf = sf_unblock(L.xq_sf.cpu().numpy(), 1, L.rows_cap, cfg.H)[0]
+    xq = L.xq.cpu().numpy()[: cfg.T * cfg.H].reshape(cfg.T, cfg.H)      # token order
+    xsf = sf_unblock(L.xq_sf.cpu().numpy(), 1, cfg.T, cfg.H)[0]
+    cq, sq = omx.quantize_rows(_f64(inp["x"]))
+    assert np.array_equal(xq, cq) and np.array_equal(xsf, sq)
+    assert np.all(L.xq_sf.cpu().numpy()[sf_padding_offsets(1, cfg.T, cfg.H)] == 0)
     xcol = L.xq_col.cpu().numpy()[: cfg.H * L.rows_cap].reshape(cfg.H, L.rows_cap)
     xcsf = sf_unblock(L.xq_col_sf.cpu().numpy(), 1, cfg.H, L.rows_cap)[0]
     x = _f64(inp["x"])
@@ -208,8 +214,10 @@ def test_permute_bitexact(run):
         rows = slice(g0, g0 + n)
         used[rows] = True
         assert np.array_equal(r2s[rows], f["perm"][offs[e]:offs[e + 1]])
-        assert np.array_equal(xq[rows], f["xq_codes"][offs[e]:offs[e + 1]])
-        assert np.array_equal(xsf[rows], f["xq_scales"][offs[e]:offs[e + 1]])
+        # the rows the GEMM gathers for this group are the oracle's permuted codes
+        tk = r2s[rows] // cfg.k
+        assert np.array_equal(xq[tk], f["xq_codes"][offs[e]:offs[e + 1]])
+        assert np.array_equal(xsf[tk], f["xq_scales"][offs[e]:offs[e + 1]])
         assert np.array_equal(pp[rows], inp["topk_prob"].reshape(-1)[f["perm"][offs[e]:offs[e + 1]]])
         # along tokens, blocks restart at the group start
         c, s = omx.quantize_cols_grouped(x[f["tok"][offs[e]:offs[e + 1]]], [n])[0]
@@ -218,8 +226,7 @@ def test_permute_bitexact(run):
         assert np.array_equal(xcsf[:, g0 // 32:(g0 + mp) // 32], s)
         assert np.all(xcol[:, g0 + mp:go[e + 1]] == 0)
     assert np.all(r2s[~used] == -1)
-    pad = ~used[: go[cfg.E]]        # padding rows inside the groups (rows past the last group are not written)
-    assert np.all(xq[: go[cfg.E]][pad] == 0) and np.all(xsf[: go[cfg.E]][pad] == 0)
+
     assert np.array_equal(s2r[r2s[used]], np.flatnonzero(used))
     assert np.all(pp[~used] == 0)
 
@@ -400,6 +407,7 @@ def test_forward_only_equals_training_forward(torch_cuda, name, over):
     without the saved activation) writes exactly the bytes of the training
     path's permutation and forward."""
     torch = torch_cuda
+    from mxfp8_grouped_gemm_x32_b200 import lib
     from mxfp8_grouped_gemm_x32_b200.layer import GroupedMLP
     cfg = get_config(name, **over)
     inp = make_inputs(cfg, seed=4, grad=False)
@@ -414,11 +422,10 @@ def test_forward_only_equals_training_forward(torch_cuda, name, over):
         torch.cuda.synchronize()
         routed = L.row_to_slot.cpu().numpy() >= 0    # h is written for routed rows only
         rc = L.rows_cap
-        used = int(L.group_offsets[cfg.E])           # rows past the last group are not written
         h = L.hq.cpu().numpy()[: rc * cfg.I].reshape(rc, cfg.I)[routed]
         hs = sf_unblock(L.hq_sf.cpu().numpy(), 1, rc, cfg.I)[0][routed]
-        xq = L.xq.cpu().numpy()[: used * cfg.H]
-        xs = sf_unblock(L.xq_sf.cpu().numpy(), 1, rc, cfg.H)[0][:used]
+        xq = L.xq.cpu().numpy()[: cfg.T * cfg.H]
+        xs = L.xq_sf.cpu().numpy()[: lib.moe_mx_scale_bytes(1, cfg.T, cfg.H)]
         outs.append([xq, xs, h, hs, out.view(torch.uint8).cpu().numpy()])
     for a, b in zip(*outs):
         assert np.array_equal(a, b)
