@@ -180,16 +180,16 @@ moe_status_t moe_mlp_quantize_weights(const void* w_gate_up, const void* w_down,
  *   row_to_slot    int32 [rows_cap]  slot of each padded row, -1 = padding.
  *   slot_to_row    int32 [T*k]       padded row of each slot.
  *   prob_perm      float [rows_cap]  routing probability per padded row (0 pad).
- *   xq, xq_sf      MX tensor (1, T, H): x quantised along H, in token order
- *                  (each token once; the forward's gate_up GEMM gathers the
- *                  rows of every group itself).  Both NULL (then xq_col
- *                  too): only the routing outputs above are produced, as the
- *                  BF16 forward needs.
+ *   xq, xq_sf      MX tensor (1, rows_cap, H): gathered x, quantised along H
+ *                  (rows from group_offsets[E] on are left unwritten).  Both
+ *                  NULL (then xq_col too): only the routing outputs above
+ *                  are produced, as the BF16 forward needs.
  *   xq_col, xq_col_sf  optional (both NULL or both set): MX tensor
  *                  (1, H, rows_cap) = gathered x^T quantised along tokens
  *                  (32-token blocks inside each 128-aligned group; padding
  *                  tokens are zero; columns from group_offsets[E] on are
- *                  left unwritten) -- the weight-gradient operand.
+ *                  left unwritten) -- the weight-gradient operand, which
+ *                  moe_grouped_mlp_bwd also makes for itself from x.
  *   workspace  >= moe_workspace_size(MOE_OP_PERMUTE, T, k, E, H, 0) bytes.
  * Limits: 1 <= k <= E, H % 32 == 0 (else MOE_ERR_INVALID / MOE_ERR_UNSUPPORTED
  * as for the other calls); E <= MOE_MAX_EXPERTS and T*k < 2^30
@@ -237,8 +237,7 @@ moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_idx, const f
  *   routing    split_sizes, group_offsets, row_to_slot, slot_to_row, prob_perm
  *              from moe_permute (the combine gathers each token's k rows
  *              through slot_to_row).
- *   xq, xq_sf  MX tensor (1, T, H) from moe_permute (x in token order; the
- *              gate_up GEMM gathers row r's token, row_to_slot[r] / k).
+ *   xq, xq_sf  MX tensor (1, rows_cap, H) from moe_permute.
  *   out        bf16 [T][H]: out[t] = sum_j y[t*k+j], y = down(h),
  *              h = prob * silu(gate) * up, gate = A[:, :I], up = A[:, I:],
  *              A = x W_gate_up^T (fp32 accumulation).

@@ -147,20 +147,16 @@ bool device_ok() {
 
 }  // namespace
 
-// x quantised along H once per token (token order, the gate_up GEMM gathers
-// the rows it needs) and, for training, the gathered rows quantised along
-// tokens in permuted order (the weight-gradient operand).
+// x rows gathered to permuted order and quantised along H and, optionally,
+// along tokens (the wgrad operand; the backward makes its own from x) -- one
+// read of the gathered rows for both forms.
 moe_status_t quantize_x(const void* x, int32_t T, int32_t H, int32_t k, int32_t E, int64_t rows_cap,
                         const int32_t* row_to_slot, const int32_t* group_offsets, uint8_t* xq, uint8_t* xq_sf,
                         uint8_t* xq_col, uint8_t* xq_col_sf, cudaStream_t st) {
-  QuantRowsArgs qr{static_cast<const uint8_t*>(x), H, nullptr, 1, 1, T, H, xq, xq_sf};
-  if (launch_quant_rows(qr, st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (xq_col) {
-    QuantBothArgs qb{static_cast<const uint8_t*>(x), 1, rows_cap, H, rows_cap, nullptr, nullptr, xq_col, xq_col_sf,
-                     row_to_slot, k, group_offsets + E};
-    if (launch_quant_both(qb, st) != cudaSuccess) return MOE_ERR_CUDA;
-  }
-  return MOE_OK;
+  (void)T;
+  QuantBothArgs qb{static_cast<const uint8_t*>(x), 1, rows_cap, H, rows_cap, xq, xq_sf, xq_col, xq_col_sf,
+                   row_to_slot, k, group_offsets + E};
+  return launch_quant_both(qb, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 namespace {
@@ -323,11 +319,10 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (T == 0) return MOE_OK;
 
-  // gate_up grouped GEMM + ScaledSwiGLU + requantisation of h; the A rows
-  // are gathered from x's codes in token order inside the GEMM
-  GemmMaps m1{};
+  // gate_up grouped GEMM + ScaledSwiGLU + requantisation of h
+  GemmMaps m1;
   cudaError_t e;
-  if ((e = make_map_2d(&m1.a, xq, H, T, 1)) != cudaSuccess) return MOE_ERR_CUDA;  // one-row box: gathers
+  if ((e = make_map_2d(&m1.a, xq, H, rows_cap, 128)) != cudaSuccess) return MOE_ERR_CUDA;
   if ((e = make_map_3d(&m1.b, w1q, H, I, 2 * int64_t(E), 128)) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs g1{};
   g1.mode = 0; g1.E = E; g1.N = I; g1.num_kt = int32_t(cdiv(H, 128)); g1.n_tiles = int32_t(cdiv(I, 128));
@@ -337,7 +332,6 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   g1.prob = prob_perm; g1.row_to_slot = row_to_slot;
   g1.out2 = static_cast<uint8_t*>(saved_a);
   g1.q_out = w.hq; g1.sf_out = w.hq_sf; g1.q_KT = int32_t(cdiv(I, 128));
-  g1.gather_sf = xq_sf; g1.gather_k = k; g1.gather_rows = T;
   {
     TimeScope ts(st, "gemm_gate_up_swiglu");
     if ((e = launch_grouped_gemm(EPI_SWIGLU, 256, m1, g1, st)) != cudaSuccess) return MOE_ERR_CUDA;
@@ -459,9 +453,9 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   // h along tokens, and sums dprob per 64-column chunk
   GemmMaps m;
   if (make_map_2d(&m.a, w.dyq, H, rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
-  if (make_map_3d(&m.b, w2tq, H, I, E, 192) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m.b, w2tq, H, I, E, 128) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs g{};
-  g.mode = 0; g.E = E; g.N = I; g.num_kt = int32_t(cdiv(H, 128)); g.n_tiles = int32_t(cdiv(I, 192));
+  g.mode = 0; g.E = E; g.N = I; g.num_kt = int32_t(cdiv(H, 128)); g.n_tiles = int32_t(cdiv(I, 128));
   g.group_offsets = group_offsets; g.split_sizes = split_sizes;
   g.sfa = w.dyq_sf; g.a_KT = int32_t(cdiv(H, 128));
   g.sfb = w2tsf; g.b_RT = int32_t(cdiv(I, 128)); g.b_KT = int32_t(cdiv(H, 128));
@@ -470,7 +464,7 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   g.dprob_part = reinterpret_cast<float*>(w.dpp);
   {
     TimeScope ts(st, "gemm_dgrad_down_swiglu");
-    if (launch_grouped_gemm(EPI_SWIGLU_BWD, 192, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_grouped_gemm(EPI_SWIGLU_BWD, 128, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
   {
     TimeScope ts(st, "dprob_reduce");

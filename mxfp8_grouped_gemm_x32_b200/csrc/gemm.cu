@@ -54,12 +54,13 @@ constexpr int STAGE_PITCH_W = 20;                  // words per staged 64-byte r
 // (two accumulators, 12 epilogue warps of 64 columns each).
 template <int BN>
 struct Cfg {
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = BN == 128 ? 5 : 4;
   static constexpr int ACC = BN == 256 ? 1 : 2;   // TMEM accumulators
-  static constexpr int EPI_WARPS = BN == 256 ? 8 : 12;
+  static constexpr int EPI_WARPS = BN == 192 ? 12 : 8;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int NC = BN / (EPI_WARPS / 4);  // accumulator columns per epilogue warp
-  static constexpr uint32_t SFA_COL = ACC * BN, SFB_COL = ACC * BN + 4;  // scale factors after the accumulators
+  static constexpr uint32_t ACC_STRIDE = BN;        // TMEM columns between the accumulators
+  static constexpr uint32_t SFA_COL = ACC * ACC_STRIDE, SFB_COL = SFA_COL + 4;  // scale factors after them
   static constexpr int SMEM_A = BM * BK;
   static constexpr int SMEM_B = BN * BK;
   static constexpr int SMEM_SFA = 512;
@@ -446,6 +447,38 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
   a.dprob_part[int64_t(cb >> 6) * a.rows_cap + r] = dps;
 }
 
+// The B operand of one K tile (and, for MXFP8, its scale atoms) into a stage:
+// gate_up pairs gate rows n0.. with the matching up rows (two boxes of BN/2
+// rows from groups 2e and 2e+1); the others load BN rows of expert e (mode 0)
+// or of the token-major operand (mode 1).
+template <int EPI, int BN, bool MX>
+__device__ __forceinline__ void load_b_stage(const GemmArgs& a, const CUtensorMap* tmB, const Tile& ti, int kg,
+                                             uint8_t* sb, uint8_t* ssfb, uint64_t* bar) {
+  using C = Cfg<BN>;
+  if constexpr (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16) {
+    tma_load_3d(sb, tmB, bar, kg * BK, ti.n0, 2 * ti.e);
+    tma_load_3d(sb + C::SMEM_B / 2, tmB, bar, kg * BK, ti.n0, 2 * ti.e + 1);
+    if constexpr (MX) {
+      const int rb = ti.n0 >> 7;
+      bulk_load(ssfb, a.sfb + ((int64_t(2 * ti.e) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
+      bulk_load(ssfb + 512, a.sfb + ((int64_t(2 * ti.e + 1) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
+    }
+  } else {
+    if (a.mode == 0)
+      tma_load_3d(sb, tmB, bar, kg * BK, ti.n0, ti.e);
+    else
+      tma_load_2d(sb, tmB, bar, kg * BK, ti.n0);
+    if constexpr (MX) {
+      const int64_t gb = a.mode == 0 ? int64_t(ti.e) * a.b_RT : 0;
+#pragma unroll
+      for (int h = 0; h < C::SFB_ATOMS; ++h) {
+        const int rb = min((ti.n0 >> 7) + h, a.b_RT - 1);  // rows past N: any finite atom
+        bulk_load(ssfb + 512 * h, a.sfb + ((gb + rb) * a.b_KT + kg) * 512, 512, bar);
+      }
+    }
+  }
+}
+
 template <int EPI, int BN, int KIND>
 __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
     grouped_mxf8_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -455,9 +488,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
   constexpr bool MX = KIND == KIND_MXF8;
   constexpr bool GATE_UP = EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16;  // B tile = gate rows + up rows
   constexpr uint32_t TX = MX ? C::STAGE_TX : uint32_t(C::SMEM_A + C::SMEM_B);
-  // EPI_SWIGLU gathers the A rows (x in token order) with four-row TMA
-  // gathers issued by all of warp 0; the other launches load A with TMA
-  constexpr bool GATHER = EPI == EPI_SWIGLU;
+
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -473,7 +504,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], GATHER ? 33 : 1);  // gather: + one arrival per producer lane
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < ACC; ++b) {
@@ -496,67 +527,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
   const int ntiles = total_tiles(a, go);
 
   if (warp == 0) {
-    if constexpr (GATHER) {
-      // ---------------- gathering producer (whole warp) ----------------
-      // lane 0 arms the stage and loads B and its scales with TMA / bulk
-      // copies; lane l gathers the A rows 4l..4l+3 with one four-row TMA
-      // gather from x's codes in token order (padding rows read past the
-      // tensor: zeros) and copies their four scale bytes of the K tile
-      prefetch_tmap(&tmA);
-      prefetch_tmap(&tmB);
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile ti = decode_tile<EPI, BN>(a, go, t);
-        int tok[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = ti.m0 + 4 * lane + i;
-          const int sl = r < ti.row_end ? __ldg(a.row_to_slot + r) : -1;
-          tok[i] = sl >= 0 ? sl / a.gather_k : a.gather_rows;  // a row past the tensor: zero fill
-        }
-        for (int kt = 0; kt < ti.nkt; ++kt) {
-          // every lane waits for the MMAs that read the stage, then all agree
-          const bool okl = mbar_wait(&empty[stage], phase ^ 1u, abort_flag);
-          if (!__all_sync(0xFFFFFFFFu, okl)) { ok = false; break; }
-          uint64_t* bar = &full[stage];
-          const int kg = ti.kt0 + kt;
-          uint8_t* sa = smem + C::OFF_A + stage * C::SMEM_A;
-          uint8_t* sb = smem + C::OFF_B + stage * C::SMEM_B;
-          uint8_t* ssfa = smem + C::OFF_SFA + stage * C::SMEM_SFA;
-          uint8_t* ssfb = smem + C::OFF_SFB + stage * C::SMEM_SFB;
-          if (lane == 0) {
-            ++issued;
-            mbar_arrive_expect_tx(bar, C::SMEM_A + C::SMEM_B + C::SMEM_SFB);
-            tma_load_3d(sb, &tmB, bar, kg * BK, ti.n0, 2 * ti.e);
-            tma_load_3d(sb + C::SMEM_B / 2, &tmB, bar, kg * BK, ti.n0, 2 * ti.e + 1);
-            const int rb = ti.n0 >> 7;
-            bulk_load(ssfb, a.sfb + ((int64_t(2 * ti.e) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
-            bulk_load(ssfb + 512, a.sfb + ((int64_t(2 * ti.e + 1) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
-          }
-          __syncwarp();  // the stage's byte count is armed before any gather lands
-          tma_gather4(sa + 512 * lane, &tmA, bar, kg * BK, tok[0], tok[1], tok[2], tok[3]);
-          const uint32_t sfa_u = smem_u32(ssfa);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int row = 4 * lane + i;
-            const bool val = tok[i] < a.gather_rows;
-            cp_async_4_zfill(sfa_u + (row & 31) * 16 + (row >> 5) * 4,
-                             val ? a.gather_sf + sf_offset(0, tok[i], 4 * kg, 0, a.a_KT) : a.gather_sf,
-                             val ? 4u : 0u);
-          }
-          cp_async_mbar_arrive_noinc(bar);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-      }
-      if (lane == 0 && *abort_flag) {
-        const uint32_t first = issued > uint32_t(STAGES) ? issued - STAGES : 0u;
-        for (uint32_t i = first; i < issued; ++i)
-          mbar_wait_drain(&full[i % STAGES], (i / STAGES) & 1u);
-      }
-    } else if (lane == 0) {
+    if (lane == 0) {
       // ---------------- TMA producer ----------------
       prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
@@ -578,29 +549,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
           uint8_t* ssfb = smem + C::OFF_SFB + stage * C::SMEM_SFB;
           tma_load_2d(sa, &tmA, bar, kg * BK, ti.m0);
           if constexpr (MX) bulk_load(ssfa, a.sfa + (int64_t(ti.m0 >> 7) * a.a_KT + kg) * 512, 512, bar);
-          if constexpr (GATE_UP) {
-            tma_load_3d(sb, &tmB, bar, kg * BK, ti.n0, 2 * ti.e);
-            tma_load_3d(sb + C::SMEM_B / 2, &tmB, bar, kg * BK, ti.n0, 2 * ti.e + 1);
-            if constexpr (MX) {
-              const int rb = ti.n0 >> 7;
-              bulk_load(ssfb, a.sfb + ((int64_t(2 * ti.e) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
-              bulk_load(ssfb + 512, a.sfb + ((int64_t(2 * ti.e + 1) * a.b_RT + rb) * a.b_KT + kg) * 512,
-                        512, bar);
-            }
-          } else {
-            if (a.mode == 0)
-              tma_load_3d(sb, &tmB, bar, kg * BK, ti.n0, ti.e);
-            else
-              tma_load_2d(sb, &tmB, bar, kg * BK, ti.n0);
-            if constexpr (MX) {
-              const int64_t gb = a.mode == 0 ? int64_t(ti.e) * a.b_RT : 0;
-#pragma unroll
-              for (int h = 0; h < C::SFB_ATOMS; ++h) {
-                const int rb = min((ti.n0 >> 7) + h, a.b_RT - 1);  // rows past N: any finite atom
-                bulk_load(ssfb + 512 * h, a.sfb + ((gb + rb) * a.b_KT + kg) * 512, 512, bar);
-              }
-            }
-          }
+          load_b_stage<EPI, BN, MX>(a, &tmB, ti, kg, sb, ssfb, bar);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -625,11 +574,10 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
         const uint32_t buf = acc_it % ACC, use = acc_it / ACC;
         if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, abort_flag)) break;
         tc_fence_after();
-        const uint32_t acc = tmem + buf * BN;
+        const uint32_t acc = tmem + buf * C::ACC_STRIDE;
         for (int kt = 0; kt < ti.nkt; ++kt) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          if constexpr (GATHER) fence_proxy_async_smem();  // A arrived through cp.async (generic proxy)
           const uint32_t sa = smem_u32(smem + C::OFF_A + stage * C::SMEM_A);
           const uint32_t sb = smem_u32(smem + C::OFF_B + stage * C::SMEM_B);
           const uint32_t ssfa = smem_u32(smem + C::OFF_SFA + stage * C::SMEM_SFA);
@@ -689,7 +637,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
       const uint32_t buf = acc_it % ACC, use = acc_it / ACC;
       if (!mbar_wait(&acc_full[buf], use & 1u, abort_flag)) break;
       tc_fence_after();
-      const uint32_t tl = tmem + (uint32_t(32 * q) << 16) + buf * BN;
+      const uint32_t tl = tmem + (uint32_t(32 * q) << 16) + buf * C::ACC_STRIDE;
       if constexpr (EPI == EPI_SWIGLU_BWD) {
         // reads TMEM chunk by chunk; the other accumulator keeps the MMAs busy
         epilogue_swiglu_bwd(a, ti, tl, q, half, lane, stage);
@@ -788,8 +736,8 @@ cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const Gem
       case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256>(maps, a, st);
       case EPI_WGRAD: return launch_epi<EPI_WGRAD, 256>(maps, a, st);
     }
-  } else if (bn == 192) {
-    if (epi == EPI_SWIGLU_BWD) return launch_epi<EPI_SWIGLU_BWD, 192>(maps, a, st);
+  } else if (bn == 128) {
+    if (epi == EPI_SWIGLU_BWD) return launch_epi<EPI_SWIGLU_BWD, 128>(maps, a, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -62,17 +62,9 @@ struct GemmArgs {
   uint8_t* hcol;
   uint8_t* hcol_sf;
   float* dprob_part;
-  // EPI_SWIGLU: A is gathered row by row from the MX tensor of x in token
-  // order (codes [T][K] through tensor map A with a one-row box, blocked
-  // scales (1, T, K)): row r of the permuted space reads token
-  // row_to_slot[r] / gather_k
-  const uint8_t* gather_sf;  // blocked scales (1, T, K) of x in token order (codes: tensor map A)
-  int32_t gather_k;
-  int32_t gather_rows;       // T
 };
 
-// Tensor maps: A 2-D {K, rows} with a 128 x 128 box (EPI_SWIGLU: x's codes
-// {K, T} with a 128 x 1 box, for four-row gathers); B either 3-D
+// Tensor maps: A 2-D {K, rows} with a 128 x 128 box; B either 3-D
 // {K, rows, groups} or 2-D {K, rows} with a 128 x bn box (EPI_SWIGLU: two
 // boxes of bn/2 rows); all uint8 with 128-byte swizzle.
 struct GemmMaps {

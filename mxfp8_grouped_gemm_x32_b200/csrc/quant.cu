@@ -288,7 +288,7 @@ __device__ __forceinline__ void qb_compute(const QuantBothArgs& a, const QbTile&
     const int64_t c = c0 + 2 * cp;
     const int64_t rbeg = r0 + 32 * rb;
     uint32_t sb2[2] = {0u, 0u};
-    if (c < a.cols && rbeg < a.rows) {
+    if (a.q_col && c < a.cols && rbeg < a.rows) {
       uint32_t wv[32];  // bf16 pairs: column c in the low half, c + 1 in the high half
 #pragma unroll
       for (int j = 0; j < 32; ++j)
@@ -334,7 +334,7 @@ __device__ __forceinline__ void qb_store(const QuantBothArgs& a, const QbTile& q
     if (a.q_row && q.r0 + rr < a.rows && 16 * chunk < vrow_bytes)
       *reinterpret_cast<uint4*>(qr + int64_t(rr) * a.cols) =
           *reinterpret_cast<const uint4*>(out_row + rr * QB_OUT_PITCH + 16 * chunk);
-    if (q.c0 + rr < a.cols && 16 * chunk < vcol_bytes)
+    if (a.q_col && q.c0 + rr < a.cols && 16 * chunk < vcol_bytes)
       *reinterpret_cast<uint4*>(qc + int64_t(rr) * a.rows) =
           *reinterpret_cast<const uint4*>(out_col + rr * QB_OUT_PITCH + 16 * chunk);
   }
@@ -346,7 +346,7 @@ __device__ __forceinline__ void qb_store(const QuantBothArgs& a, const QbTile& q
       reinterpret_cast<uint4*>(a.sf_row + sf_offset(rg, rr, q.c0 / 32, cdiv(a.row_split, 128),
                                                     cdiv(a.cols, 128)))[tid] = reinterpret_cast<const uint4*>(atoms)[tid];
     }
-  } else if (tid < 64) {
+  } else if (tid < 64 && a.q_col) {
     reinterpret_cast<uint4*>(a.sf_col + sf_offset(q.g, q.c0, q.r0 / 32, cdiv(a.cols, QC_TILE), cdiv(a.rows, QC_TILE)))[tid - 32] =
         reinterpret_cast<const uint4*>(atoms + 512)[tid - 32];
   }

@@ -49,8 +49,8 @@ namespace moe {
 //    rows / row_split row-groups of row_split rows (W_gate_up: gate and up
 //    halves) -- q_row [groups*rows][cols], sf_row blocked
 //    (groups*rows/row_split, row_split, cols);
-//  column mode output: q_col [groups][cols][rows], sf_col blocked
-//    (groups, cols, rows).
+//  column mode output (skipped when q_col is null): q_col [groups][cols][rows],
+//    sf_col blocked (groups, cols, rows).
 struct QuantBothArgs {
   const uint8_t* src;
   int32_t groups;
@@ -79,8 +79,8 @@ cudaError_t launch_quant_both(const QuantBothArgs& a, cudaStream_t st);
 namespace moe {
 
 // The permutation's quantisation of x (defined with the C entry points):
-// xq, xq_sf = MX tensor (1, T, H) of x in token order; with xq_col, the
-// gathered rows quantised along tokens, MX tensor (1, H, rows_cap).
+// xq, xq_sf = MX tensor (1, rows_cap, H) of the gathered rows; with xq_col,
+// the gathered rows quantised along tokens, MX tensor (1, H, rows_cap).
 moe_status_t quantize_x(const void* x, int32_t T, int32_t H, int32_t k, int32_t E, int64_t rows_cap,
                         const int32_t* row_to_slot, const int32_t* group_offsets, uint8_t* xq, uint8_t* xq_sf,
                         uint8_t* xq_col, uint8_t* xq_col_sf, cudaStream_t st);

@@ -102,8 +102,8 @@ class GroupedMLP:
         self.topk_idx = al.typed((T, k), torch.int32, "topk_idx")        # router outputs
         self.topk_prob = al.typed((T, k), torch.float32, "topk_prob")
         self.prob_perm = al.typed((rc,), torch.float32, "prob_perm")
-        self.xq = u8(T * H, "xq")                # x quantised along H, token order
-        self.xq_sf = u8(sb(1, T, H), "xq_sf")
+        self.xq = u8(rc * H, "xq")
+        self.xq_sf = u8(sb(1, rc, H), "xq_sf")
         self.hq = u8(rc * I, "hq")
         self.hq_sf = u8(sb(1, rc, I), "hq_sf")
         self.out = al.typed((T, H), torch.bfloat16, "out")

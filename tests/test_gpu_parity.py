@@ -200,11 +200,8 @@ def test_permute_bitexact(run):
     s2r = L.slot_to_row.cpu().numpy()
     pp = L.prob_perm.cpu().numpy()
     offs = f["offsets"]
-    xq = L.xq.cpu().numpy()[: cfg.T * cfg.H].reshape(cfg.T, cfg.H)      # token order
-    xsf = sf_unblock(L.xq_sf.cpu().numpy(), 1, cfg.T, cfg.H)[0]
-    cq, sq = omx.quantize_rows(_f64(inp["x"]))
-    assert np.array_equal(xq, cq) and np.array_equal(xsf, sq)
-    assert np.all(L.xq_sf.cpu().numpy()[sf_padding_offsets(1, cfg.T, cfg.H)] == 0)
+    xq = L.xq.cpu().numpy()[: L.rows_cap * cfg.H].reshape(L.rows_cap, cfg.H)
+    xsf = sf_unblock(L.xq_sf.cpu().numpy(), 1, L.rows_cap, cfg.H)[0]
     xcol = L.xq_col.cpu().numpy()[: cfg.H * L.rows_cap].reshape(cfg.H, L.rows_cap)
     xcsf = sf_unblock(L.xq_col_sf.cpu().numpy(), 1, cfg.H, L.rows_cap)[0]
     x = _f64(inp["x"])
@@ -214,10 +211,8 @@ def test_permute_bitexact(run):
         rows = slice(g0, g0 + n)
         used[rows] = True
         assert np.array_equal(r2s[rows], f["perm"][offs[e]:offs[e + 1]])
-        # the rows the GEMM gathers for this group are the oracle's permuted codes
-        tk = r2s[rows] // cfg.k
-        assert np.array_equal(xq[tk], f["xq_codes"][offs[e]:offs[e + 1]])
-        assert np.array_equal(xsf[tk], f["xq_scales"][offs[e]:offs[e + 1]])
+        assert np.array_equal(xq[rows], f["xq_codes"][offs[e]:offs[e + 1]])
+        assert np.array_equal(xsf[rows], f["xq_scales"][offs[e]:offs[e + 1]])
         assert np.array_equal(pp[rows], inp["topk_prob"].reshape(-1)[f["perm"][offs[e]:offs[e + 1]]])
         # along tokens, blocks restart at the group start
         c, s = omx.quantize_cols_grouped(x[f["tok"][offs[e]:offs[e + 1]]], [n])[0]
@@ -226,6 +221,8 @@ def test_permute_bitexact(run):
         assert np.array_equal(xcsf[:, g0 // 32:(g0 + mp) // 32], s)
         assert np.all(xcol[:, g0 + mp:go[e + 1]] == 0)
     assert np.all(r2s[~used] == -1)
+    pad = ~used[: go[cfg.E]]        # padding rows inside the groups (rows past the last group are not written)
+    assert np.all(xq[: go[cfg.E]][pad] == 0) and np.all(xsf[: go[cfg.E]][pad] == 0)
 
     assert np.array_equal(s2r[r2s[used]], np.flatnonzero(used))
     assert np.all(pp[~used] == 0)
@@ -424,8 +421,9 @@ def test_forward_only_equals_training_forward(torch_cuda, name, over):
         rc = L.rows_cap
         h = L.hq.cpu().numpy()[: rc * cfg.I].reshape(rc, cfg.I)[routed]
         hs = sf_unblock(L.hq_sf.cpu().numpy(), 1, rc, cfg.I)[0][routed]
-        xq = L.xq.cpu().numpy()[: cfg.T * cfg.H]
-        xs = L.xq_sf.cpu().numpy()[: lib.moe_mx_scale_bytes(1, cfg.T, cfg.H)]
+        used = int(L.group_offsets[cfg.E])           # rows past the last group are not written
+        xq = L.xq.cpu().numpy()[: used * cfg.H]
+        xs = L.xq_sf.cpu().numpy()[: lib.moe_mx_scale_bytes(1, used, cfg.H)]
         outs.append([xq, xs, h, hs, out.view(torch.uint8).cpu().numpy()])
     for a, b in zip(*outs):
         assert np.array_equal(a, b)

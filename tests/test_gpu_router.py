@@ -111,8 +111,8 @@ def test_route_permute_equals_router_then_permute(cuda, name, T, training):
     names = ["topk_idx", "topk_prob", "split_sizes", "group_offsets", "row_to_slot", "slot_to_row", "prob_perm"]
     for n in names:
         assert torch.equal(getattr(a, n), getattr(b, n)), n
-    assert torch.equal(a.xq[: cfg.T * cfg.H], b.xq[: cfg.T * cfg.H])          # x in token order
-    nsf = lib.moe_mx_scale_bytes(1, cfg.T, cfg.H)
+    assert torch.equal(a.xq[: go * cfg.H], b.xq[: go * cfg.H])        # rows past the last group: unwritten
+    nsf = lib.moe_mx_scale_bytes(1, go, cfg.H)
     assert torch.equal(a.xq_sf[:nsf], b.xq_sf[:nsf])
     if training:
         xa = a.xq_col[: cfg.H * a.rows_cap].view(cfg.H, a.rows_cap)[:, :go]
