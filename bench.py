@@ -160,7 +160,7 @@ def attainable_fwd(cfg, split, p_tflops: float, bw_gbs: float, rows_cap: int) ->
     plus the permutation's and the combine's bytes at BW.  Bytes per GEMM:
     MX weights (+1/32 scales) and the expert's activation rows in and out
     (gate_up: x codes in, bf16 saved A and h codes out; down: h codes in,
-    fp32 per-slot rows out)."""
+    f24 rows out, 3 bytes per value)."""
     H, I, T, k = cfg.H, cfg.I, cfg.T, cfg.k
     P, BW = p_tflops * 1e12, bw_gbs * 1e9
     t = 0.0
@@ -168,10 +168,10 @@ def attainable_fwd(cfg, split, p_tflops: float, bw_gbs: float, rows_cap: int) ->
         m = float(m)
         f1, f2 = 2 * m * H * 2 * I, 2 * m * I * H
         b1 = 2 * I * H * (1 + 1 / 32) + m * H + m * 2 * I * 2 + m * I
-        b2 = H * I * (1 + 1 / 32) + m * I + m * H * 4
+        b2 = H * I * (1 + 1 / 32) + m * I + m * H * 3
         t += max(f1 / P, b1 / BW) + max(f2 / P, b2 / BW)
     permute_bytes = T * H * 2 + 2 * rows_cap * H * (1 + 1 / 32)
-    combine_bytes = T * k * H * 4 + T * H * 2
+    combine_bytes = T * k * H * 3 + T * H * 2
     t += (permute_bytes + combine_bytes) / BW
     return {"ms": t * 1e3, "peak_tflops": p_tflops, "hbm_gbs": bw_gbs,
             "what": "sum over experts of max(FLOP/P, bytes/BW) for both GEMMs + permutation and combine bytes / BW"}

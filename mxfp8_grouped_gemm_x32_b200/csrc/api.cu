@@ -83,7 +83,7 @@ FwdWs carve_fwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t r
     w.hq = c.take(rows_cap * I);
     w.hq_sf = c.take(mx_scale_bytes(1, rows_cap, I));
   }
-  w.y = c.take(rows_cap * H * 4);  // fp32 down-projection rows in permuted order
+  w.y = c.take(rows_cap * H * 3);  // f24 down-projection rows in permuted order
   return w;
 }
 
@@ -126,7 +126,7 @@ BwdWs carve_bwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t r
   w.dac_sf = c.take(mx_scale_bytes(1, 2 * I, rows_cap));
   w.hc = c.take(I * rows_cap);
   w.hc_sf = c.take(mx_scale_bytes(1, I, rows_cap));
-  w.dx = c.take(rows_cap * H * 4);  // fp32 dgrad rows in permuted order
+  w.dx = c.take(rows_cap * H * 3);  // f24 dgrad rows in permuted order
   w.dpp = c.take(I / 64 * rows_cap * 4);  // dprob partial sums per 64-column chunk
   w.xc = c.take(H * rows_cap);             // gathered x quantised along tokens (wgrad1 operand)
   w.xc_sf = c.take(mx_scale_bytes(1, H, rows_cap));
@@ -291,7 +291,7 @@ moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* o
   if (!device_ok()) return MOE_ERR_NO_DEVICE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   TimeScope ts(st, "combine");
-  return cuda_status(launch_combine(y, false, nullptr, T, k, H, out, st));
+  return cuda_status(launch_combine(y, COMBINE_BF16, nullptr, T, k, H, out, st));
 }
 
 moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const uint8_t* w2q,
@@ -346,16 +346,16 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   g2.group_offsets = group_offsets; g2.split_sizes = split_sizes;
   g2.sfa = w.hq_sf; g2.a_KT = int32_t(cdiv(I, 128));
   g2.sfb = w2sf; g2.b_RT = int32_t(cdiv(H, 128)); g2.b_KT = int32_t(cdiv(I, 128));
-  g2.out = w.y; g2.ld_out = H;
+  g2.out = w.y; g2.ld_out = 3 * int64_t(H);
   {
     TimeScope ts(st, "gemm_down");
-    if ((e = launch_grouped_gemm(EPI_F32_ROWS, 256, m2, g2, st)) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((e = launch_grouped_gemm(EPI_F24_ROWS, 256, m2, g2, st)) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // top-k combine back to token order: a token's k rows gathered through
-  // slot_to_row and summed in ascending j
+  // slot_to_row and summed in fp32 in ascending j
   TimeScope ts(st, "combine");
-  return cuda_status(launch_combine(w.y, true, slot_to_row, T, k, H, out, st));
+  return cuda_status(launch_combine(w.y, COMBINE_F24, slot_to_row, T, k, H, out, st));
 }
 
 moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down, int32_t T, int32_t H, int32_t I,
@@ -412,7 +412,7 @@ moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down,
     if (launch_grouped_gemm_bf16(EPI_F32_ROWS, m2, g2, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
   TimeScope ts(st, "combine");
-  return cuda_status(launch_combine(w.y, true, slot_to_row, T, k, H, out, st));
+  return cuda_status(launch_combine(w.y, COMBINE_F32, slot_to_row, T, k, H, out, st));
 }
 
 moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, const uint8_t* w1tq,
@@ -498,14 +498,14 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   g.group_offsets = group_offsets; g.split_sizes = split_sizes;
   g.sfa = w.daq_sf; g.a_KT = int32_t(cdiv(2 * int64_t(I), 128));
   g.sfb = w1tsf; g.b_RT = int32_t(cdiv(H, 128)); g.b_KT = int32_t(cdiv(2 * int64_t(I), 128));
-  g.out = w.dx; g.ld_out = H;
+  g.out = w.dx; g.ld_out = 3 * int64_t(H);
   {
     TimeScope ts(st, "gemm_dgrad_gate_up");
-    if (launch_grouped_gemm(EPI_F32_ROWS, 256, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_grouped_gemm(EPI_F24_ROWS, 256, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
   {
     TimeScope ts(st, "combine_dx");
-    if (launch_combine(w.dx, true, slot_to_row, T, k, H, dX, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_combine(w.dx, COMBINE_F24, slot_to_row, T, k, H, dX, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // x gathered and quantised along tokens (the operand of wgrad1), right

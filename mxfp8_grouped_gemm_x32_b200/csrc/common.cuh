@@ -164,6 +164,29 @@ __device__ __forceinline__ uint32_t fastdiv(uint32_t m, const FastDiv& f) {
 }
 
 // ----------------------------------------------------------------------------
+// f24: the top 24 bits of an fp32 value (sign, 8 exponent bits, 15 mantissa
+// bits; the low 8 bits are dropped, a relative error below 2^-15 -- 64
+// times finer than bf16's rounding).  Four values pack into three 32-bit
+// words, little-endian: value 0 in bytes 0-2, value 1 in bytes 3-5, ...
+// Infinities stay infinite; a NaN whose top 15 mantissa bits are zero would
+// read back as an infinity (fp32 results of the GEMMs are finite unless an
+// input is not).
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void f24_pack4(uint32_t u0, uint32_t u1, uint32_t u2, uint32_t u3, uint32_t& w0,
+                                          uint32_t& w1, uint32_t& w2) {
+  w0 = __byte_perm(u0, u1, 0x5321);  // u0 bytes 1-3, u1 byte 1
+  w1 = __byte_perm(u1, u2, 0x6532);  // u1 bytes 2-3, u2 bytes 1-2
+  w2 = __byte_perm(u2, u3, 0x7653);  // u2 byte 3, u3 bytes 1-3
+}
+// fp32 values (as bits, low byte zero) of the four f24 values packed in w0..w2
+__device__ __forceinline__ void f24_unpack4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t* f) {
+  f[0] = w0 << 8;
+  f[1] = __byte_perm(w0, w1, 0x5430) & 0xFFFFFF00u;  // w0 byte 3, w1 bytes 0-1
+  f[2] = __byte_perm(w1, w2, 0x4320) & 0xFFFFFF00u;  // w1 bytes 2-3, w2 byte 0
+  f[3] = w2 & 0xFFFFFF00u;
+}
+
+// ----------------------------------------------------------------------------
 // small vector helpers
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -291,7 +291,16 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
     const int nb = ti.n0 + NC * half;
     if (nb >= a.N) return;  // uniform across the warp
     const int ncols = min(NC, a.N - nb);
-    if constexpr (EPI == EPI_F32_SCATTER || EPI == EPI_F32_ROWS) {
+    if constexpr (EPI == EPI_F24_ROWS) {
+      // keep the top 24 bits of each value, four values in three words, in place
+#pragma unroll
+      for (int i = 0; i < NC / 4; ++i) {
+        const uint32_t u0 = v[4 * i], u1 = v[4 * i + 1], u2 = v[4 * i + 2], u3 = v[4 * i + 3];
+        f24_pack4(u0, u1, u2, u3, v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+      }
+      uint8_t* dst = rv ? a.out + int64_t(r) * a.ld_out + int64_t(nb) * 3 : nullptr;
+      warp_store_rows<NC * 3 / 4>(stage, dst, v, ncols * 3, lane);
+    } else if constexpr (EPI == EPI_F32_SCATTER || EPI == EPI_F32_ROWS) {
       uint8_t* dst = nullptr;
       if (rv) {
         int64_t orow = r;
@@ -734,6 +743,7 @@ cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const Gem
       case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, 256>(maps, a, st);
       case EPI_F32_SCATTER: return launch_epi<EPI_F32_SCATTER, 256>(maps, a, st);
       case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256>(maps, a, st);
+      case EPI_F24_ROWS: return launch_epi<EPI_F24_ROWS, 256>(maps, a, st);
       case EPI_WGRAD: return launch_epi<EPI_WGRAD, 256>(maps, a, st);
     }
   } else if (bn == 128) {

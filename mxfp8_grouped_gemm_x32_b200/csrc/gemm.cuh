@@ -11,7 +11,8 @@ enum EpiKind : int {
   EPI_F32_ROWS = 2,      // dgrad2: fp32 rows in permuted order (feeds the requantising SwiGLU backward)
   EPI_WGRAD = 3,         // weight gradients: one bf16 matrix per expert
   EPI_SWIGLU_BWD = 4,    // dgrad2 + ScaledSwiGLU backward: da (along 2I and tokens), h (tokens), dprob partials
-  EPI_SWIGLU_BF16 = 5    // BF16 path gate_up: h = p * silu(gate) * up written in bf16 (q_out)
+  EPI_SWIGLU_BF16 = 5,   // BF16 path gate_up: h = p * silu(gate) * up written in bf16 (q_out)
+  EPI_F24_ROWS = 6       // down / dgrad1: the top 24 bits of each fp32 value (f24, see common.cuh), rows in permuted order
 };
 
 // Operand kind of the tensor-core MMA.
@@ -43,8 +44,8 @@ struct GemmArgs {
   int32_t b_RT, b_KT;  // row tiles per group and K tiles in B's scale layout
   const float* prob;
   const int32_t* row_to_slot;
-  uint8_t* out;       // output: fp32 rows (EPI_F32_*), bf16 per-expert matrices (EPI_WGRAD)
-  int64_t ld_out;     // elements between output rows
+  uint8_t* out;       // output: fp32 rows (EPI_F32_*), f24 rows (EPI_F24_ROWS), bf16 per-expert matrices (EPI_WGRAD)
+  int64_t ld_out;     // elements between output rows (EPI_F24_ROWS: bytes)
   int64_t out_group_stride;  // mode 1: elements between experts' matrices
   uint8_t* out2;      // EPI_SWIGLU: saved A, bf16 [rows][2N] (nullable)
   uint8_t* q_out;     // EPI_SWIGLU: h codes [rows][N]; EPI_SWIGLU_BF16: h bf16 [rows][N]

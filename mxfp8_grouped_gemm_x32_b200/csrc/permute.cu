@@ -112,9 +112,10 @@ __global__ void __launch_bounds__(PB) perm_scatter_kernel(const int32_t* __restr
 
 // out[t] = sum_j y[row(t, j)], fp32 sum in ascending j, 8 columns per thread;
 // row(t, j) = t*k + j (rows in slot order) or slot_to_row[t*k + j] (rows in
-// permuted order).  F32_IN: y holds fp32 rows (a grouped GEMM's output),
-// else bf16.
-template <bool F32_IN>
+// permuted order).  FMT: y holds bf16 rows (COMBINE_BF16), fp32 rows
+// (COMBINE_F32) or f24 rows (COMBINE_F24: the top 3 bytes of each fp32
+// value, see common.cuh).
+template <int FMT>
 __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ yv, const int32_t* __restrict__ slot_to_row,
                                                       int64_t T, int32_t k, int64_t H8, uint4* __restrict__ out) {
   const int64_t n = T * H8;
@@ -125,11 +126,19 @@ __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y
     for (int j = 0; j < k; ++j) {
       const int64_t row = slot_to_row ? int64_t(__ldg(slot_to_row + t * k + j)) : t * k + j;
       if (row < 0) continue;  // a slot whose expert id was rejected
-      if constexpr (F32_IN) {
+      if constexpr (FMT == COMBINE_F32) {
         const float4* y = static_cast<const float4*>(yv) + (row * H8 + c) * 2;
         const float4 v0 = __ldg(y), v1 = __ldg(y + 1);
         acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
         acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
+      } else if constexpr (FMT == COMBINE_F24) {
+        const uint2* y = static_cast<const uint2*>(yv) + (row * H8 + c) * 3;  // 24 bytes: 8 values
+        const uint2 a = __ldg(y), b = __ldg(y + 1), d = __ldg(y + 2);
+        uint32_t f[8];
+        f24_unpack4(a.x, a.y, b.x, f);
+        f24_unpack4(b.y, d.x, d.y, f + 4);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += __uint_as_float(f[e]);
       } else {
         const uint4 v = __ldg(static_cast<const uint4*>(yv) + row * H8 + c);
         acc[0] += bf16lo(v.x); acc[1] += bf16hi(v.x);
@@ -179,16 +188,19 @@ cudaError_t launch_permute_index(const int32_t* idx, const float* prob, int64_t 
   return launch_permute_scan_scatter(idx, prob, R, E, split, offs, row_to_slot, slot_to_row, prob_perm, ws, st);
 }
 
-cudaError_t launch_combine(const void* y, bool f32_in, const int32_t* slot_to_row, int64_t T, int32_t k, int64_t H,
+cudaError_t launch_combine(const void* y, int fmt, const int32_t* slot_to_row, int64_t T, int32_t k, int64_t H,
                            void* out, cudaStream_t st) {
   const int64_t n = T * (H / 8);
   if (n == 0) return cudaSuccess;
   int64_t blocks = cdiv(n, 256);
   if (blocks > 148 * 32) blocks = 148 * 32;
-  if (f32_in)
-    combine_kernel<true><<<unsigned(blocks), 256, 0, st>>>(y, slot_to_row, T, k, H / 8, static_cast<uint4*>(out));
+  uint4* o = static_cast<uint4*>(out);
+  if (fmt == COMBINE_F32)
+    combine_kernel<COMBINE_F32><<<unsigned(blocks), 256, 0, st>>>(y, slot_to_row, T, k, H / 8, o);
+  else if (fmt == COMBINE_F24)
+    combine_kernel<COMBINE_F24><<<unsigned(blocks), 256, 0, st>>>(y, slot_to_row, T, k, H / 8, o);
   else
-    combine_kernel<false><<<unsigned(blocks), 256, 0, st>>>(y, slot_to_row, T, k, H / 8, static_cast<uint4*>(out));
+    combine_kernel<COMBINE_BF16><<<unsigned(blocks), 256, 0, st>>>(y, slot_to_row, T, k, H / 8, o);
   count_launch();
   return cudaGetLastError();
 }

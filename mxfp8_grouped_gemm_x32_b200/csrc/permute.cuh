@@ -23,10 +23,13 @@ cudaError_t launch_permute_index(const int32_t* idx, const float* prob, int64_t 
                                  int32_t* row_to_slot, int32_t* slot_to_row, float* prob_perm,
                                  void* ws, cudaStream_t st);
 
-// out[t] = sum_{j<k} y[row(t,j)]  (fp32 or bf16 in, fp32 sum in ascending j,
-// bf16 out), H % 8 == 0; row(t,j) = t*k+j, or slot_to_row[t*k+j] when
-// slot_to_row is given (negative entries are skipped).
-cudaError_t launch_combine(const void* y, bool f32_in, const int32_t* slot_to_row, int64_t T, int32_t k, int64_t H,
+// Row formats the combine reads.
+enum CombineFmt : int { COMBINE_BF16 = 0, COMBINE_F32 = 1, COMBINE_F24 = 2 };
+
+// out[t] = sum_{j<k} y[row(t,j)]  (bf16, fp32 or f24 rows in, fp32 sum in
+// ascending j, bf16 out), H % 8 == 0; row(t,j) = t*k+j, or
+// slot_to_row[t*k+j] when slot_to_row is given (negative entries are skipped).
+cudaError_t launch_combine(const void* y, int fmt, const int32_t* slot_to_row, int64_t T, int32_t k, int64_t H,
                            void* out, cudaStream_t st);
 
 }  // namespace moe

@@ -15,8 +15,9 @@ gradients depend only on that channel over the expert's rows, with the same
   fp32 before the combine, and dprob), and two 32-channel blocks of the
   expert's weight gradients, one of them the last (dW_gate_up rows, gate and
   up, and dW_down columns) over every routed row of the expert;
-* at every token: out = bf16(sum_j y) and dX = bf16(sum_j dx), bit-exact (the
-  combine, a property that holds at any size).
+* at every token: out = bf16(sum_j y) and dX = bf16(sum_j dx), bit-exact, with
+  y and dx the f24 rows the library keeps (the combine, a property that holds
+  at any size).
 Bars as in test_gpu_parity.py (with the allowance of tests/ambiguity.py).
 """
 import numpy as np
@@ -42,10 +43,10 @@ def _rel_rms(g, r):
 
 
 def _slot_buffers(L, cfg):
-    """fp32 rows kept by the library in the caller's workspaces: the
-    forward's y (first piece when hq is caller-provided) and the backward's
-    dx (the piece after the MX operands), both [rows_cap][H] in permuted
-    order, returned in slot order."""
+    """Rows kept by the library in the caller's workspaces: the forward's y
+    (first piece when hq is caller-provided) and the backward's dx (the piece
+    after the MX operands), both [rows_cap][H] f24 rows in permuted order,
+    returned as float32 in slot order."""
     import torch
     from mxfp8_grouped_gemm_x32_b200 import lib
     rc, H, I = L.rows_cap, cfg.H, cfg.I
@@ -54,10 +55,18 @@ def _slot_buffers(L, cfg):
     pieces = [rc * H, sb(1, rc, H), H * rc, sb(1, H, rc), rc * 2 * I, sb(1, rc, 2 * I),
               2 * I * rc, sb(1, 2 * I, rc), I * rc, sb(1, I, rc)]
     off = sum(a256(p) for p in pieces)
-    y = L.ws_fwd[: rc * H * 4].view(torch.float32).view(rc, H)
-    dx = L.ws_bwd[off: off + rc * H * 4].view(torch.float32).view(rc, H)
-    s2r = L.slot_to_row.long()
-    return y[s2r], dx[s2r]
+    s2r = L.slot_to_row.cpu().numpy().astype(np.int64)
+    y = _f24_rows(L.ws_fwd[: rc * H * 3], rc, H)
+    dx = _f24_rows(L.ws_bwd[off: off + rc * H * 3], rc, H)
+    return torch.from_numpy(y[s2r]).cuda(), torch.from_numpy(dx[s2r]).cuda()
+
+
+def _f24_rows(buf, rows, H):
+    """Rows stored as f24 (the top 24 bits of each fp32 value, 3 bytes per
+    value, little-endian) -> float32 [rows, H]."""
+    b = buf.cpu().numpy().reshape(rows, H, 3).astype(np.uint32)
+    bits = (b[..., 0] << np.uint32(8)) | (b[..., 1] << np.uint32(16)) | (b[..., 2] << np.uint32(24))
+    return bits.view(np.float32)
 
 
 @pytest.mark.parametrize("name", ["mixtral_8x7b", "qwen3_30b_ragged", "gpt_oss_20b"])
