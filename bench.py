@@ -72,6 +72,36 @@ def gate_up_flops(cfg) -> float:
     return 4.0 * cfg.R * cfg.H * cfg.I
 
 
+def bandwidth_bytes(cfg) -> dict:
+    """Algorithmic HBM bytes per step of the bandwidth-bound kernels (reads
+    + writes; MX codes count 1 byte and their scales 1/32 byte per value;
+    x and dY are counted once per token however often they are gathered):
+      quant_weights  bf16 W_gate_up and W_down in, both MX forms out;
+      permute_quant  x in, R = T*k MX rows along H out;
+      dy_quant       dY in, R rows along H and along tokens out;
+      x_quant_cols   x in, R rows along tokens out;
+      combine(_dx)   R f24 rows in (3 bytes per value), T bf16 rows out."""
+    T, H, I, E, R = cfg.T, cfg.H, cfg.I, cfg.E, cfg.R
+    mx = 1 + 1 / 32
+    return {"quant_weights": 3.0 * E * H * I * (2 + 2 * mx),
+            "permute_quant": T * H * 2 + R * H * mx,
+            "dy_quant": T * H * 2 + 2 * R * H * mx,
+            "x_quant_cols": T * H * 2 + R * H * mx,
+            "combine": R * H * 3 + T * H * 2,
+            "combine_dx": R * H * 3 + T * H * 2}
+
+
+def annotate_bandwidth(kernels: dict, cfg, hbm_gbs: float) -> dict:
+    """Adds algorithmic bytes per step, GB/s and the fraction of the HBM copy
+    bandwidth to the bandwidth-bound kernels' entries."""
+    for name, b in bandwidth_bytes(cfg).items():
+        k = kernels.get(name)
+        if k and k.get("ms_per_step"):
+            gbs = b / (k["ms_per_step"] * 1e-3) / 1e9
+            k.update({"bytes_per_step": b, "gbs": gbs, "frac_of_hbm": gbs / hbm_gbs})
+    return kernels
+
+
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -170,7 +200,7 @@ def attainable_fwd(cfg, split, p_tflops: float, bw_gbs: float, rows_cap: int) ->
         b1 = 2 * I * H * (1 + 1 / 32) + m * H + m * 2 * I * 2 + m * I
         b2 = H * I * (1 + 1 / 32) + m * I + m * H * 3
         t += max(f1 / P, b1 / BW) + max(f2 / P, b2 / BW)
-    permute_bytes = T * H * 2 + 2 * rows_cap * H * (1 + 1 / 32)
+    permute_bytes = T * H * 2 + T * k * H * (1 + 1 / 32)
     combine_bytes = T * k * H * 3 + T * H * 2
     t += (permute_bytes + combine_bytes) / BW
     return {"ms": t * 1e3, "peak_tflops": p_tflops, "hbm_gbs": bw_gbs,
@@ -498,8 +528,8 @@ def measure_workload(torch, lib, name: str, seed: int, dev, steps: int, warmup: 
            "layer": phase_rates(cfg, fwd, bwd, peaks["mxfp8_sustained"], clk_peak),
            "peak_tflops": peaks["mxfp8_sustained"], "clock_peak_tflops": clk_peak,
            "rows_per_expert": split_histogram(layer.split_sizes.cpu().tolist()),
-           "kernels": {k: {"ms_per_step": v[0] / steps, "launches_per_step": v[1] / steps}
-                       for k, v in per_kernel.items()},
+           "kernels": annotate_bandwidth({k: {"ms_per_step": v[0] / steps, "launches_per_step": v[1] / steps}
+                                          for k, v in per_kernel.items()}, cfg, peaks["hbm_gbs"]),
            "clocks": clocks}
     del layer, flush
     torch.cuda.empty_cache()
@@ -682,8 +712,8 @@ def run_ours(args):
     peaks = load_peaks()
     peak = peaks["mxfp8_sustained"]
     clk_peak = clock_peak_tflops(clocks["sm_mhz"]) if clocks else None
-    kernels = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
-               for k, v in per_kernel.items()}
+    kernels = annotate_bandwidth({k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
+                                  for k, v in per_kernel.items()}, cfg, peaks["hbm_gbs"])
     g1 = per_kernel.get("gemm_gate_up_swiglu")
     roofline = None
     if g1 and g1[1]:

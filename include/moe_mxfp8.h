@@ -20,6 +20,9 @@
  *           (moe_workspace_size).  Calls are asynchronous on `stream`.
  *           For an empty batch (T == 0) arrays with a token dimension (x,
  *           dY, out, dX, routing, logits, slot maps, dprob) may be null.
+ *           Pointers are 16-byte aligned; moe_grouped_mlp_bwd also needs a
+ *           256-byte aligned workspace and a 32-byte aligned saved_a (it
+ *           reads and writes them with 256-bit accesses).
  * Errors.   Argument errors (null pointer, bad size, misalignment, an
  *           unsupported shape) are detected on the host before any launch
  *           and return MOE_ERR_INVALID / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE

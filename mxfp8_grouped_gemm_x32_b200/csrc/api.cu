@@ -55,6 +55,8 @@ void timing_end(cudaStream_t st) {
 namespace {
 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool al32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+inline bool al256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 inline int64_t align256(int64_t v) { return (v + 255) / 256 * 256; }
 
 inline moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
@@ -151,9 +153,15 @@ bool device_ok() {
 // along tokens (the wgrad operand; the backward makes its own from x) -- one
 // read of the gathered rows for both forms.
 moe_status_t quantize_x(const void* x, int32_t T, int32_t H, int32_t k, int32_t E, int64_t rows_cap,
-                        const int32_t* row_to_slot, const int32_t* group_offsets, uint8_t* xq, uint8_t* xq_sf,
-                        uint8_t* xq_col, uint8_t* xq_col_sf, cudaStream_t st) {
-  (void)T;
+                        const int32_t* row_to_slot, const int32_t* slot_to_row, const int32_t* group_offsets,
+                        uint8_t* xq, uint8_t* xq_sf, uint8_t* xq_col, uint8_t* xq_col_sf, cudaStream_t st) {
+  if (!xq_col) {
+    // row form only: each token quantised once, its codes copied to its k rows
+    ScatterRowsArgs sa{static_cast<const uint8_t*>(x), T, H, k, slot_to_row, row_to_slot, group_offsets + E, xq,
+                       xq_sf};
+    if (int64_t(T) * (H / 8) < (int64_t(1) << 31) - (int64_t(1) << 24))
+      return launch_quant_rows_scatter(sa, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
   QuantBothArgs qb{static_cast<const uint8_t*>(x), 1, rows_cap, H, rows_cap, xq, xq_sf, xq_col, xq_col_sf,
                    row_to_slot, k, group_offsets + E};
   return launch_quant_both(qb, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -282,7 +290,8 @@ moe_status_t moe_permute(const void* x, const int32_t* topk_idx, const float* to
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (!xq) return MOE_OK;
   TimeScope ts(st, "permute_quant");
-  return quantize_x(x, T, H, k, E, rows_cap, row_to_slot, group_offsets, xq, xq_sf, xq_col, xq_col_sf, st);
+  return quantize_x(x, T, H, k, E, rows_cap, row_to_slot, slot_to_row, group_offsets, xq, xq_sf, xq_col, xq_col_sf,
+                    st);
 }
 
 moe_status_t moe_combine(const void* y, int32_t T, int32_t k, int32_t H, void* out, moe_stream_t stream) {
@@ -326,7 +335,7 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   if ((e = make_map_3d(&m1.b, w1q, H, I, 2 * int64_t(E), 128)) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs g1{};
   g1.mode = 0; g1.E = E; g1.N = I; g1.num_kt = int32_t(cdiv(H, 128)); g1.n_tiles = int32_t(cdiv(I, 128));
-  g1.group_offsets = group_offsets; g1.split_sizes = split_sizes;
+  g1.group_offsets = group_offsets; g1.split_sizes = split_sizes; g1.rows_cap = rows_cap;
   g1.sfa = xq_sf; g1.a_KT = int32_t(cdiv(H, 128));
   g1.sfb = w1sf; g1.b_RT = int32_t(cdiv(I, 128)); g1.b_KT = int32_t(cdiv(H, 128));
   g1.prob = prob_perm; g1.row_to_slot = row_to_slot;
@@ -340,10 +349,10 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
   // down grouped GEMM, fp32 rows in permuted order
   GemmMaps m2;
   if ((e = make_map_2d(&m2.a, w.hq, I, rows_cap, 128)) != cudaSuccess) return MOE_ERR_CUDA;
-  if ((e = make_map_3d(&m2.b, w2q, I, H, E, 256)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((e = make_map_3d(&m2.b, w2q, I, H, E, gemm_b_box(256))) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs g2{};
   g2.mode = 0; g2.E = E; g2.N = H; g2.num_kt = int32_t(cdiv(I, 128)); g2.n_tiles = int32_t(cdiv(H, 256));
-  g2.group_offsets = group_offsets; g2.split_sizes = split_sizes;
+  g2.group_offsets = group_offsets; g2.split_sizes = split_sizes; g2.rows_cap = rows_cap;
   g2.sfa = w.hq_sf; g2.a_KT = int32_t(cdiv(I, 128));
   g2.sfb = w2sf; g2.b_RT = int32_t(cdiv(H, 128)); g2.b_KT = int32_t(cdiv(I, 128));
   g2.out = w.y; g2.ld_out = 3 * int64_t(H);
@@ -402,7 +411,7 @@ moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down,
   // down grouped GEMM (bf16), fp32 rows in permuted order
   GemmMaps m2;
   if (make_map_2d(&m2.a, w.h, 2 * int64_t(I), rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
-  if (make_map_3d(&m2.b, w_down, 2 * int64_t(I), H, E, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m2.b, w_down, 2 * int64_t(I), H, E, gemm_b_box(256)) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs g2{};
   g2.mode = 0; g2.E = E; g2.N = H; g2.num_kt = int32_t(cdiv(2 * int64_t(I), 128)); g2.n_tiles = int32_t(cdiv(H, 256));
   g2.group_offsets = group_offsets; g2.split_sizes = split_sizes;
@@ -433,6 +442,7 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
                         dY, saved_a, x, (const void*)dX,
                         (const void*)dW1, (const void*)dW2})
     if (!al16(p)) return MOE_ERR_INVALID;
+  if (!al32(saved_a) || !al256(workspace)) return MOE_ERR_INVALID;  // 256-bit loads and stores
   Carver c{static_cast<uint8_t*>(workspace)};
   BwdWs w = carve_bwd(c, T, k, H, I, rows_cap);
   if (!workspace || int64_t(workspace_bytes) < c.off) return MOE_ERR_WORKSPACE;
@@ -453,7 +463,7 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   // h along tokens, and sums dprob per 64-column chunk
   GemmMaps m;
   if (make_map_2d(&m.a, w.dyq, H, rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
-  if (make_map_3d(&m.b, w2tq, H, I, E, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m.b, w2tq, H, I, E, gemm_b_box(128)) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs g{};
   g.mode = 0; g.E = E; g.N = I; g.num_kt = int32_t(cdiv(H, 128)); g.n_tiles = int32_t(cdiv(I, 128));
   g.group_offsets = group_offsets; g.split_sizes = split_sizes;
@@ -475,7 +485,7 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
 
   // wgrad2: dW_down_e = dy_e^T h_e (contraction over the group's tokens)
   if (make_map_2d(&m.a, w.dyc, rows_cap, H, 128) != cudaSuccess) return MOE_ERR_CUDA;
-  if (make_map_2d(&m.b, w.hc, rows_cap, I, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_2d(&m.b, w.hc, rows_cap, I, gemm_b_box(256)) != cudaSuccess) return MOE_ERR_CUDA;
   g = GemmArgs{};
   g.mode = 1; g.E = E; g.N = I; g.n_tiles = int32_t(cdiv(I, 256));
   g.m_tiles = int32_t(cdiv(H, 128)); g.M_out = H;
@@ -491,11 +501,11 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   // dgrad1: dx = da W_gate_up (contraction over 2I), fp32 rows in permuted
   // order; the combine gathers a token's k rows through slot_to_row
   if (make_map_2d(&m.a, w.daq, 2 * int64_t(I), rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
-  if (make_map_3d(&m.b, w1tq, 2 * int64_t(I), H, E, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m.b, w1tq, 2 * int64_t(I), H, E, gemm_b_box(256)) != cudaSuccess) return MOE_ERR_CUDA;
   g = GemmArgs{};
   g.mode = 0; g.E = E; g.N = H; g.num_kt = int32_t(cdiv(2 * int64_t(I), 128));
   g.n_tiles = int32_t(cdiv(H, 256));
-  g.group_offsets = group_offsets; g.split_sizes = split_sizes;
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes; g.rows_cap = rows_cap;
   g.sfa = w.daq_sf; g.a_KT = int32_t(cdiv(2 * int64_t(I), 128));
   g.sfb = w1tsf; g.b_RT = int32_t(cdiv(H, 128)); g.b_KT = int32_t(cdiv(2 * int64_t(I), 128));
   g.out = w.dx; g.ld_out = 3 * int64_t(H);
@@ -519,7 +529,7 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
 
   // wgrad1: dW_gate_up_e = da_e^T x_e (contraction over the group's tokens)
   if (make_map_2d(&m.a, w.dac, rows_cap, 2 * int64_t(I), 128) != cudaSuccess) return MOE_ERR_CUDA;
-  if (make_map_2d(&m.b, w.xc, rows_cap, H, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_2d(&m.b, w.xc, rows_cap, H, gemm_b_box(256)) != cudaSuccess) return MOE_ERR_CUDA;
   g = GemmArgs{};
   g.mode = 1; g.E = E; g.N = H; g.n_tiles = int32_t(cdiv(H, 256));
   g.m_tiles = int32_t(cdiv(2 * int64_t(I), 128)); g.M_out = 2 * I;
@@ -580,7 +590,8 @@ moe_status_t moe_route_permute(const void* logits, int32_t logits_dtype, const v
       return MOE_ERR_CUDA;
   }
   TimeScope ts(st, "permute_quant");
-  return quantize_x(x, T, H, k, E, rows_cap, row_to_slot, group_offsets, xq, xq_sf, xq_col, xq_col_sf, st);
+  return quantize_x(x, T, H, k, E, rows_cap, row_to_slot, slot_to_row, group_offsets, xq, xq_sf, xq_col, xq_col_sf,
+                    st);
 }
 
 moe_status_t moe_get_device_status(moe_stream_t stream) {

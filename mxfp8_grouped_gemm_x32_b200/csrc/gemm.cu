@@ -12,15 +12,14 @@
 //                   ScaledSwiGLU backward into the epilogue of the GEMM that
 //                   produces dh, so dh is never written either.
 //
-// Design (one CTA per SM), two tile widths BN:
+// Design (one CTA per SM, 8 epilogue warps, 320 threads), two tile widths BN:
 //   BN = 256: 128 x 256 tiles, one fp32 accumulator of 256 TMEM columns,
-//             8 epilogue warps (320 threads);
-//   BN = 192: 128 x 192 tiles, two accumulators of 192 columns (the MMAs of
-//             the next tile run while the epilogue drains the previous one,
-//             so the epilogue may read TMEM lazily and hold it longer),
-//             12 epilogue warps of 64 columns (448 threads) -- the fused
-//             ScaledSwiGLU backward, whose epilogue does the most work;
-//   both with a 4-stage shared-memory ring.
+//             4-stage shared-memory ring;
+//   BN = 128: 128 x 128 tiles, two accumulators of 128 columns (the MMAs of
+//             the next tile run while the epilogue works on the previous
+//             one, so the epilogue may read TMEM lazily and hold it longer),
+//             5-stage ring -- the fused ScaledSwiGLU backward, whose
+//             epilogue does the most work.
 //   warp 0      TMA producer: A tile 128x128 B, B tile BNx128 B (2-D or
 //               3-D tensor maps, 128-byte swizzle), the scale atoms by bulk
 //               copy, into the shared-memory ring (mbarrier pipeline).
@@ -50,23 +49,26 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int STAGE_PITCH_W = 20;                  // words per staged 64-byte row (16 used): conflict-free v4
 
 // Shared-memory plan, pipeline depth, TMEM plan and warp count of the two
-// tile widths: BN = 256 (one accumulator, 8 epilogue warps) and BN = 192
-// (two accumulators, 12 epilogue warps of 64 columns each).
-template <int BN>
+// tile widths: BN = 256 (one accumulator) and BN = 128 (two accumulators),
+// for a CTA on its own (M = 128 tiles) or one of a CTA pair (PAIR: M = 256
+// tiles, each CTA stages its 128 rows of A and half of the BN rows of B, so
+// a K tile takes less shared memory and the ring gets deeper).
+template <int BN, bool PAIR = false>
 struct Cfg {
-  static constexpr int STAGES = BN == 128 ? 5 : 4;
+  static constexpr int STAGES = PAIR ? (BN == 128 ? 7 : 6) : (BN == 128 ? 5 : 4);
   static constexpr int ACC = BN == 256 ? 1 : 2;   // TMEM accumulators
-  static constexpr int EPI_WARPS = BN == 192 ? 12 : 8;
+  static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int NC = BN / (EPI_WARPS / 4);  // accumulator columns per epilogue warp
   static constexpr uint32_t ACC_STRIDE = BN;        // TMEM columns between the accumulators
   static constexpr uint32_t SFA_COL = ACC * ACC_STRIDE, SFB_COL = SFA_COL + 4;  // scale factors after them
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // rows of B this CTA stages per K tile
   static constexpr int SMEM_A = BM * BK;
-  static constexpr int SMEM_B = BN * BK;
+  static constexpr int SMEM_B = B_ROWS * BK;
   static constexpr int SMEM_SFA = 512;
   static constexpr int SFB_ATOMS = (BN + 127) / 128;
-  static constexpr int SMEM_SFB = SFB_ATOMS * 512;  // one 512-byte atom per 128 rows of B
-  static constexpr uint32_t STAGE_TX = SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB;
+  static constexpr int SMEM_SFB = SFB_ATOMS * 512;  // one 512-byte atom per 128 rows of B (all BN rows)
+  static constexpr uint32_t STAGE_TX = SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB;  // bytes one CTA copies
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * SMEM_A;
   static constexpr int OFF_SFA = OFF_B + STAGES * SMEM_B;
@@ -75,10 +77,11 @@ struct Cfg {
   static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;   // tmem address, abort flag
   static constexpr int OFF_GO = OFF_MISC + 16;              // group offsets [E+1]
+  static constexpr int OFF_PC = OFF_GO + (MOE_MAX_EXPERTS + 1) * 4;  // PAIR: first tile of each expert [E+1]
   // per-warp staging: 32 rows x 20 words (64-byte rows) or 16 rows x 36 words
-  // (128-byte rows); BN = 192 transposes 32 x 32 fp32 values (pitch 36)
+  // (128-byte rows); BN = 128 transposes 32 x 32 fp32 values (pitch 36)
   static constexpr int STAGE_WARP_BYTES = BN == 256 ? 2560 : 32 * 36 * 4;
-  static constexpr int OFF_STAGE = (OFF_GO + (MOE_MAX_EXPERTS + 1) * 4 + 127) / 128 * 128;
+  static constexpr int OFF_STAGE = (OFF_PC + (PAIR ? (MOE_MAX_EXPERTS + 1) * 4 : 0) + 127) / 128 * 128;
   static constexpr int SMEM_TOTAL = OFF_STAGE + EPI_WARPS * STAGE_WARP_BYTES;
   static constexpr int SMEM_LAUNCH = SMEM_TOTAL + 1024;     // slack for 1 KB alignment
   static_assert(SMEM_LAUNCH <= 232448, "shared memory plan exceeds 227 KB");
@@ -87,44 +90,56 @@ struct Cfg {
 
 struct Tile {
   int e, m0, n0, kt0, nkt, row_end;
+  int row_lim;  // mode 0: end of the expert's (padded) rows; rows from there on belong to no tile of it
 };
 
-__device__ __forceinline__ int total_tiles(const GemmArgs& a, const int* go) {
-  if (a.mode == 0) return (go[a.E] >> 7) * a.n_tiles;
-  return a.E * a.m_tiles * a.n_tiles;
+// Tiles of the schedule.  Mode 0 walks each expert's 128-row tiles (PAIR:
+// 256-row tiles, the last one of an odd count half past the group) times the
+// N tiles; pc[e] holds the first PAIR tile of expert e.  Mode 1 walks experts
+// x output tiles.
+template <bool PAIR>
+__device__ __forceinline__ int total_tiles(const GemmArgs& a, const int* go, const int* pc) {
+  if (a.mode == 0) return PAIR ? pc[a.E] : (go[a.E] >> 7) * a.n_tiles;
+  return a.E * (PAIR ? (a.m_tiles + 1) >> 1 : a.m_tiles) * a.n_tiles;
 }
 
-template <int EPI, int BN>
-__device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, int t) {
+template <int EPI, int BN, bool PAIR>
+__device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, const int* pc, int t) {
+  constexpr int MSHIFT = PAIR ? 8 : 7;  // log2 of the tile's rows
   Tile ti;
   if (a.mode == 0) {
     const int nt = a.n_tiles;
     int lo = 0, hi = a.E - 1;  // last expert whose first tile is <= t
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if ((go[mid] >> 7) * nt <= t) lo = mid; else hi = mid - 1;
+      const int first = PAIR ? pc[mid] : (go[mid] >> 7) * nt;
+      if (first <= t) lo = mid; else hi = mid - 1;
     }
     const int e = lo;
-    const int mt = (go[e + 1] - go[e]) >> 7;
-    const int local = t - (go[e] >> 7) * nt;
+    const int mt128 = (go[e + 1] - go[e]) >> 7;
+    const int mt = PAIR ? (mt128 + 1) >> 1 : mt128;
+    const int local = t - (PAIR ? pc[e] : (go[e] >> 7) * nt);
     const int n_idx = local / mt, m_idx = local - n_idx * mt;  // rows fastest: B panel reuse
     ti.e = e;
-    ti.m0 = go[e] + (m_idx << 7);
+    ti.m0 = go[e] + (m_idx << MSHIFT);
     ti.n0 = n_idx * ((EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16) ? BN / 2 : BN);
     ti.kt0 = 0;
     ti.nkt = a.num_kt;
     ti.row_end = go[e] + a.split_sizes[e];
+    ti.row_lim = go[e + 1];
   } else {
-    const int per = a.m_tiles * a.n_tiles;
+    const int mt = PAIR ? (a.m_tiles + 1) >> 1 : a.m_tiles;
+    const int per = mt * a.n_tiles;
     const int e = t / per;
     const int local = t - e * per;
-    const int n_idx = local / a.m_tiles, m_idx = local - n_idx * a.m_tiles;
+    const int n_idx = local / mt, m_idx = local - n_idx * mt;
     ti.e = e;
-    ti.m0 = m_idx << 7;
+    ti.m0 = m_idx << MSHIFT;
     ti.n0 = n_idx * BN;
     ti.kt0 = go[e] >> 7;
     ti.nkt = (go[e + 1] - go[e]) >> 7;
     ti.row_end = a.M_out;
+    ti.row_lim = 0x7FFFFFFF;
   }
   return ti;
 }
@@ -317,7 +332,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
 }
 
 // ---------------------------------------------------------------------------
-// EPI_SWIGLU_BWD (BN = 192): the ScaledSwiGLU backward on the dh tile.
+// EPI_SWIGLU_BWD (BN = 128): the ScaledSwiGLU backward on the dh tile.
 // The warp owns rows rb..rb+31 (one 32-row block along tokens: groups start
 // on multiples of 128) and dh columns cb..cb+63, read from TMEM in two
 // chunks of 32.  Per element, with g, u from the saved bf16 A and p the row's
@@ -329,23 +344,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
 // staging buffer and lane c quantises column c over the warp's 32 rows.
 // Rows past the group's last token hold zeros in every output.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float bf16_elem(const uint4* v, int e) {
-  const uint4 w4 = v[e >> 3];
-  const int i = (e >> 1) & 3;
-  const uint32_t w = i == 0 ? w4.x : (i == 1 ? w4.y : (i == 2 ? w4.z : w4.w));
-  return (e & 1) ? bf16hi(w) : bf16lo(w);
-}
-
-// 32 values -> E4M3 codes + E8M0 scale byte; codes stored at dst (32 bytes).
+// 32 values -> E4M3 codes + E8M0 scale byte; codes stored at dst (32 bytes,
+// one 256-bit store: dst is 32-byte aligned).
 __device__ __forceinline__ uint32_t encode32_store(const float* o, uint8_t* dst) {
   const uint32_t sb = e8m0_from_amax_bits(__float_as_uint(abs_max_n<32>(o)));
   const float inv = inv_scale_from_e8m0(sb);
   uint32_t w[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) w[j] = pack4_e4m3(o[4 * j] * inv, o[4 * j + 1] * inv, o[4 * j + 2] * inv, o[4 * j + 3] * inv);
-  uint4* d = reinterpret_cast<uint4*>(dst);
-  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  stg256(dst, w);
   return sb;
 }
 
@@ -367,6 +374,35 @@ __device__ __forceinline__ void quant_cols32(const float* o, uint32_t* stage, in
   const int64_t col = col0 + lane;
   const uint32_t sb = encode32_store(f, q + col * ld + rb);
   sf[sf_offset(0, col, rb >> 5, 0, KT)] = uint8_t(sb);
+}
+
+// Gate and up values (bf16 pairs) of one 32-column chunk of a lane's row of
+// the saved A; zeros for rows past the group's last token.
+struct GuChunk {
+  uint32_t g[16], u[16];
+};
+
+// Chunk j (columns n0 + 64*half + 32*j ..) of tile ti for this lane's row:
+// four 256-bit loads (the saved A is 32-byte aligned and its rows are
+// 4*I bytes long, a multiple of 256).
+__device__ __forceinline__ void load_gu(const GemmArgs& a, const Tile& ti, int q, int half, int lane, int j,
+                                        GuChunk& x) {
+  const int cb = ti.n0 + 64 * half;
+  const int64_t r = ti.m0 + 32 * q + lane;
+  if (cb < a.N && r < ti.row_end) {
+    const uint8_t* gp = a.saved + (r * 2 * a.N + cb + 32 * j) * 2;
+    ldg256(gp, x.g);
+    ldg256(gp + 32, x.g + 8);
+    ldg256(gp + int64_t(a.N) * 2, x.u);
+    ldg256(gp + int64_t(a.N) * 2 + 32, x.u + 8);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x.g[i] = x.u[i] = 0u;
+  }
+}
+
+__device__ __forceinline__ float gu_elem(const uint32_t* w, int e) {
+  return (e & 1) ? bf16hi(w[e >> 1]) : bf16lo(w[e >> 1]);
 }
 
 // dh columns [col, col + 32) of the warp's 32 rows from TMEM (zero for rows
@@ -392,32 +428,32 @@ __device__ __forceinline__ void prefetch_saved(const GemmArgs& a, const Tile& ti
   asm volatile("prefetch.global.L2 [%0];" ::"l"(g + int64_t(a.N) * 2));
 }
 
-__device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Tile& ti, uint32_t tl, int q, int half,
-                                                    int lane, uint32_t* stage) {
+// `cur` holds g/u of chunk 0 of this tile on entry; the loads of the next
+// chunk (chunk 1, then chunk 0 of the warp's next tile `tn`, if any) are
+// issued once a chunk's dh has been read for the last time, so they land
+// while its last pass runs.  On return `cur` holds chunk 0 of `tn`.
+__device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Tile& ti, const Tile* tn, uint32_t tl,
+                                                    int q, int half, int lane, uint32_t* stage, GuChunk& cur) {
   const int I = a.N;
   const int cb = ti.n0 + 64 * half;
-  if (cb >= I) return;  // uniform across the warp
+  if (cb >= I) {  // no columns for this warp in this tile (uniform across the warp)
+    if (tn) load_gu(a, *tn, q, half, lane, 0, cur);
+    return;
+  }
   const int64_t rb = ti.m0 + 32 * q;
   const int64_t r = rb + lane;
   const bool rv = r < ti.row_end;
   const int64_t I2 = 2 * int64_t(I);
   const int64_t KT2 = I2 / 128, KTt = a.rows_cap / 128;
   const float p = rv ? a.prob[r] : 0.0f;
-  const uint8_t* grow = a.saved + (r * I2 + cb) * 2;
   float dps = 0.0f;
   uint32_t sb_dg = 0, sb_du = 0;
-  // dh is read from TMEM once per output quantity rather than held in
-  // registers across all three (the accumulator stays ours until released)
+  // dh is read from TMEM once per pass rather than held in registers (the
+  // accumulator stays ours until released)
 #pragma unroll 1
   for (int j = 0; j < 2; ++j) {
     const int cc = cb + 32 * j;
     const uint32_t tc = tl + 64 * half + 32 * j;
-    uint4 gv[4], uv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      gv[i] = rv ? __ldg(reinterpret_cast<const uint4*>(grow + 64 * j) + i) : make_uint4(0u, 0u, 0u, 0u);
-      uv[i] = rv ? __ldg(reinterpret_cast<const uint4*>(grow + int64_t(I) * 2 + 64 * j) + i) : make_uint4(0u, 0u, 0u, 0u);
-    }
     float sv[32], o[32];  // sv: s = g * sigmoid(g), kept across the three passes
     uint32_t d[32];
     // dg = dh*p*u*sig*(1+g*(1-sig)), quantised along 2I (columns cc..cc+31)
@@ -425,29 +461,36 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
     load_dh32(tc, rv, d);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-      const float g = bf16_elem(gv, e), u = bf16_elem(uv, e);
+      const float g = gu_elem(cur.g, e), u = gu_elem(cur.u, e);
       const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
       o[e] = (__uint_as_float(d[e]) * p) * (u * sg) * fmaf(g, 1.0f - sg, 1.0f);
       sv[e] = g * sg;
     }
     sb_dg |= encode32_store(o, a.daq + r * I2 + cc) << (8 * j);
     quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, cc, a.rows_cap, rb, KTt);
-    // du = dh*p*s, quantised along 2I (columns I+cc..) and along tokens
-    load_dh32(tc, rv, d);
-#pragma unroll
-    for (int e = 0; e < 32; ++e) o[e] = (__uint_as_float(d[e]) * p) * sv[e];
-    sb_du |= encode32_store(o, a.daq + r * I2 + I + cc) << (8 * j);
-    quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, int64_t(I) + cc, a.rows_cap, rb, KTt);
-    // h = p*s*u along tokens (operand of the down projection's weight
-    // gradient); dprob partial sum
+    // du = dh*p*s, quantised along 2I (columns I+cc..) and along tokens;
+    // dprob partial sum dh*s*u
     load_dh32(tc, rv, d);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-      const float su = sv[e] * bf16_elem(uv, e);
-      o[e] = p * su;
-      dps = fmaf(__uint_as_float(d[e]), su, dps);
+      o[e] = (__uint_as_float(d[e]) * p) * sv[e];
+      dps = fmaf(__uint_as_float(d[e]), sv[e] * gu_elem(cur.u, e), dps);
     }
+    sb_du |= encode32_store(o, a.daq + r * I2 + I + cc) << (8 * j);
+    quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, int64_t(I) + cc, a.rows_cap, rb, KTt);
+    // dh is used up: load the next chunk's g/u now (it lands during the
+    // last pass and the start of the next chunk)
+    GuChunk nxt;
+    if (j == 0)
+      load_gu(a, ti, q, half, lane, 1, nxt);
+    else if (tn)
+      load_gu(a, *tn, q, half, lane, 0, nxt);
+    // h = p*s*u along tokens (operand of the down projection's weight
+    // gradient)
+#pragma unroll
+    for (int e = 0; e < 32; ++e) o[e] = p * (sv[e] * gu_elem(cur.u, e));
     quant_cols32(o, stage, lane, a.hcol, a.hcol_sf, cc, a.rows_cap, rb, KTt);
+    cur = nxt;
   }
   // scale bytes of dg and du along 2I: blocks cb/32, cb/32+1 (cb % 64 == 0,
   // so the pair shares a 4-byte group of the atom)
@@ -459,44 +502,81 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
 // The B operand of one K tile (and, for MXFP8, its scale atoms) into a stage:
 // gate_up pairs gate rows n0.. with the matching up rows (two boxes of BN/2
 // rows from groups 2e and 2e+1); the others load BN rows of expert e (mode 0)
-// or of the token-major operand (mode 1).
-template <int EPI, int BN, bool MX>
-__device__ __forceinline__ void load_b_stage(const GemmArgs& a, const CUtensorMap* tmB, const Tile& ti, int kg,
-                                             uint8_t* sb, uint8_t* ssfb, uint64_t* bar) {
-  using C = Cfg<BN>;
+// or of the token-major operand (mode 1).  PAIR: this CTA (rank 0 or 1)
+// copies half of the rows -- gate_up: rank 0 the gate rows, rank 1 the up
+// rows -- but every scale atom of the tile (each CTA's TMEM needs all of
+// them), reporting the bytes to the pair's stage barrier `barp`.
+template <int EPI, int BN, bool MX, bool PAIR>
+__device__ __forceinline__ void load_b_stage(const GemmArgs& a, const CUtensorMap* tmB, const CUtensorMap* tmSFB,
+                                             const Tile& ti, int kg, uint8_t* sb, uint8_t* ssfb, uint64_t* bar,
+                                             uint32_t barp, uint32_t rank) {
+  using C = Cfg<BN, PAIR>;
   if constexpr (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16) {
-    tma_load_3d(sb, tmB, bar, kg * BK, ti.n0, 2 * ti.e);
-    tma_load_3d(sb + C::SMEM_B / 2, tmB, bar, kg * BK, ti.n0, 2 * ti.e + 1);
-    if constexpr (MX) {
-      const int rb = ti.n0 >> 7;
-      bulk_load(ssfb, a.sfb + ((int64_t(2 * ti.e) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
-      bulk_load(ssfb + 512, a.sfb + ((int64_t(2 * ti.e + 1) * a.b_RT + rb) * a.b_KT + kg) * 512, 512, bar);
+    const int rb = ti.n0 >> 7;
+    const int64_t atom_g = (int64_t(2 * ti.e) * a.b_RT + rb) * a.b_KT + kg;
+    const int64_t atom_u = (int64_t(2 * ti.e + 1) * a.b_RT + rb) * a.b_KT + kg;
+    if constexpr (PAIR) {
+      tma_load_3d_pair(sb, tmB, barp, kg * BK, ti.n0, 2 * ti.e + int(rank));
+      if constexpr (MX) {
+        tma_load_2d_pair(ssfb, tmSFB, barp, 0, int(2 * atom_g));
+        tma_load_2d_pair(ssfb + 512, tmSFB, barp, 0, int(2 * atom_u));
+      }
+    } else {
+      tma_load_3d(sb, tmB, bar, kg * BK, ti.n0, 2 * ti.e);
+      tma_load_3d(sb + C::SMEM_B / 2, tmB, bar, kg * BK, ti.n0, 2 * ti.e + 1);
+      if constexpr (MX) {
+        bulk_load(ssfb, a.sfb + atom_g * 512, 512, bar);
+        bulk_load(ssfb + 512, a.sfb + atom_u * 512, 512, bar);
+      }
     }
   } else {
-    if (a.mode == 0)
-      tma_load_3d(sb, tmB, bar, kg * BK, ti.n0, ti.e);
-    else
-      tma_load_2d(sb, tmB, bar, kg * BK, ti.n0);
+    const int nb = ti.n0 + (PAIR ? C::B_ROWS * int(rank) : 0);
+    if constexpr (PAIR) {
+      if (a.mode == 0)
+        tma_load_3d_pair(sb, tmB, barp, kg * BK, nb, ti.e);
+      else
+        tma_load_2d_pair(sb, tmB, barp, kg * BK, nb);
+    } else {
+      if (a.mode == 0)
+        tma_load_3d(sb, tmB, bar, kg * BK, nb, ti.e);
+      else
+        tma_load_2d(sb, tmB, bar, kg * BK, nb);
+    }
     if constexpr (MX) {
       const int64_t gb = a.mode == 0 ? int64_t(ti.e) * a.b_RT : 0;
 #pragma unroll
       for (int h = 0; h < C::SFB_ATOMS; ++h) {
         const int rb = min((ti.n0 >> 7) + h, a.b_RT - 1);  // rows past N: any finite atom
-        bulk_load(ssfb + 512 * h, a.sfb + ((gb + rb) * a.b_KT + kg) * 512, 512, bar);
+        const int64_t atom = (gb + rb) * a.b_KT + kg;
+        if constexpr (PAIR)
+          tma_load_2d_pair(ssfb + 512 * h, tmSFB, barp, 0, int(2 * atom));
+        else
+          bulk_load(ssfb + 512 * h, a.sfb + atom * 512, 512, bar);
       }
     }
   }
 }
 
-template <int EPI, int BN, int KIND>
-__global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
+// The persistent GEMM.  PAIR: launched as clusters of two CTAs; tile t of
+// the schedule is a 256-row tile of which CTA `rank` owns rows
+// m0 + 128*rank .. (its epilogue, its TMEM, its A rows); CTA 0 issues the
+// M = 256 MMAs and the commits that free both CTAs' stages and signal both
+// epilogues; both epilogues release the accumulator to CTA 0.  A CTA whose
+// 128 rows lie past its expert's group (odd tile counts) loads zeros (an
+// out-of-range TMA box) and writes nothing.
+// (320 threads: ten warps, three of them on two of the SM's four
+// sub-partitions, whose 16K registers each cap a thread at 168)
+template <int EPI, int BN, int KIND, bool PAIR>
+__global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
     grouped_mxf8_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                             const __grid_constant__ CUtensorMap tmB, const GemmArgs a) {
-  using C = Cfg<BN>;
+                             const __grid_constant__ CUtensorMap tmB,
+                             const __grid_constant__ CUtensorMap tmSFA,
+                             const __grid_constant__ CUtensorMap tmSFB, const GemmArgs a) {
+  using C = Cfg<BN, PAIR>;
   constexpr int STAGES = C::STAGES, ACC = C::ACC, NUM_THREADS = C::THREADS;
   constexpr bool MX = KIND == KIND_MXF8;
-  constexpr bool GATE_UP = EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16;  // B tile = gate rows + up rows
   constexpr uint32_t TX = MX ? C::STAGE_TX : uint32_t(C::SMEM_A + C::SMEM_B);
+  constexpr int OOB_ROW = 1 << 30;  // a TMA row coordinate past every tensor: the box is zero filled
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -508,8 +588,14 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* go = reinterpret_cast<int*>(smem + C::OFF_GO);
+  int* pc = reinterpret_cast<int*>(smem + C::OFF_PC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int cid = PAIR ? int(blockIdx.x >> 1) : int(blockIdx.x);   // pair (cluster) index
+  const int ncl = PAIR ? int(gridDim.x >> 1) : int(gridDim.x);
+  const int row_off = PAIR ? 128 * int(rank) : 0;                   // this CTA's rows within a tile
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -518,67 +604,122 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
     }
     for (int b = 0; b < ACC; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], C::EPI_WARPS);
+      mbar_init(&acc_empty[b], C::EPI_WARPS * (PAIR ? 2 : 1));
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   for (int i = threadIdx.x; i <= a.E; i += NUM_THREADS) go[i] = a.group_offsets[i];
+  if constexpr (PAIR) {
+    __syncthreads();
+    if (warp == 2 && a.mode == 0) {
+      // pc[e] = sum over e' < e of ceil(tiles128(e') / 2) * n_tiles: each lane
+      // sums a run of up to 8 experts, then a warp-wide inclusive scan
+      const int per = (a.E + 31) / 32;
+      const int e0 = lane * per, e1 = min(e0 + per, a.E);
+      int run = 0;
+      for (int e = e0; e < e1; ++e) run += ((((go[e + 1] - go[e]) >> 7) + 1) >> 1) * a.n_tiles;
+      int incl = run;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += v;
+      }
+      int acc = incl - run;
+      for (int e = e0; e < e1; ++e) {
+        pc[e] = acc;
+        acc += ((((go[e + 1] - go[e]) >> 7) + 1) >> 1) * a.n_tiles;
+      }
+      if (lane == 31) pc[a.E] = incl;
+    }
+  }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated in both
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int ntiles = total_tiles(a, go);
+  const int ntiles = total_tiles<PAIR>(a, go, pc);
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
+      if constexpr (PAIR && MX) {
+        prefetch_tmap(&tmSFA);
+        prefetch_tmap(&tmSFB);
+      }
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0;  // stages armed so far
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile ti = decode_tile<EPI, BN>(a, go, t);
+      for (int t = cid; t < ntiles && ok; t += ncl) {
+        const Tile ti = decode_tile<EPI, BN, PAIR>(a, go, pc, t);
+        const int my_m0 = ti.m0 + row_off;
+        const bool a_oob = PAIR && a.mode == 0 && my_m0 >= ti.row_lim;  // rows of another expert: load zeros
         for (int kt = 0; kt < ti.nkt; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           ++issued;
           uint64_t* bar = &full[stage];
-          mbar_arrive_expect_tx(bar, TX);
+          if (leader) mbar_arrive_expect_tx(bar, PAIR ? 2 * TX : TX);
           const int kg = ti.kt0 + kt;
           uint8_t* sa = smem + C::OFF_A + stage * C::SMEM_A;
           uint8_t* sb = smem + C::OFF_B + stage * C::SMEM_B;
           uint8_t* ssfa = smem + C::OFF_SFA + stage * C::SMEM_SFA;
           uint8_t* ssfb = smem + C::OFF_SFB + stage * C::SMEM_SFB;
-          tma_load_2d(sa, &tmA, bar, kg * BK, ti.m0);
-          if constexpr (MX) bulk_load(ssfa, a.sfa + (int64_t(ti.m0 >> 7) * a.a_KT + kg) * 512, 512, bar);
-          load_b_stage<EPI, BN, MX>(a, &tmB, ti, kg, sb, ssfb, bar);
+          uint32_t barp = 0;
+          if constexpr (PAIR) {
+            barp = smem_in_cta(bar, 0);
+            tma_load_2d_pair(sa, &tmA, barp, kg * BK, a_oob ? OOB_ROW : my_m0);
+            if constexpr (MX)
+              tma_load_2d_pair(ssfa, &tmSFA, barp, 0,
+                               a_oob ? OOB_ROW : int(2 * (int64_t(my_m0 >> 7) * a.a_KT + kg)));
+          } else {
+            tma_load_2d(sa, &tmA, bar, kg * BK, my_m0);
+            if constexpr (MX) bulk_load(ssfa, a.sfa + (int64_t(my_m0 >> 7) * a.a_KT + kg) * 512, 512, bar);
+          }
+          load_b_stage<EPI, BN, MX, PAIR>(a, &tmB, &tmSFB, ti, kg, sb, ssfb, bar, barp, rank);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       if (*abort_flag) {
-        // shutting down early: let the copies of the last armed stages land
-        // before the shared memory they write is released
-        const uint32_t first = issued > uint32_t(STAGES) ? issued - STAGES : 0u;
-        for (uint32_t i = first; i < issued; ++i)
-          mbar_wait_drain(&full[i % STAGES], (i / STAGES) & 1u);
+        if (leader) {
+          // shutting down early: let the copies of the last armed stages land
+          // before the shared memory they write is released (in a pair the
+          // stage barriers count both CTAs' copies)
+          const uint32_t first = issued > uint32_t(STAGES) ? issued - STAGES : 0u;
+          for (uint32_t i = first; i < issued; ++i)
+            mbar_wait_drain(&full[i % STAGES], (i / STAGES) & 1u);
+        } else {
+          // the peer's copies report to CTA 0's barriers: give them time to land
+          const long long t0 = clock64();
+          while (clock64() - t0 < 2000000ll) {
+          }
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ---------------- MMA issuer ----------------
       int stage = 0;
       uint32_t phase = 0, acc_it = 0;
       bool ok = true;
       const uint32_t sfa_t = tmem + C::SFA_COL, sfb_t = tmem + C::SFB_COL;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile ti = decode_tile<EPI, BN>(a, go, t);
+      constexpr int MMA_M = PAIR ? 2 * BM : BM;
+      for (int t = cid; t < ntiles && ok; t += ncl) {
+        const Tile ti = decode_tile<EPI, BN, PAIR>(a, go, pc, t);
         if (ti.nkt == 0) continue;
         const uint32_t buf = acc_it % ACC, use = acc_it / ACC;
         if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, abort_flag)) break;
@@ -592,33 +733,58 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
           const uint32_t ssfa = smem_u32(smem + C::OFF_SFA + stage * C::SMEM_SFA);
           const uint32_t ssfb = smem_u32(smem + C::OFF_SFB + stage * C::SMEM_SFB);
           if constexpr (MX) {
-            tc_cp_32x128b_warpx4(sfa_t, make_smem_desc(ssfa, 0, 128, 0));
+            if constexpr (PAIR) {
+              tc_cp_32x128b_warpx4_pair(sfa_t, make_smem_desc(ssfa, 0, 128, 0));
 #pragma unroll
-            for (int h = 0; h < C::SFB_ATOMS; ++h)
-              tc_cp_32x128b_warpx4(sfb_t + 4 * h, make_smem_desc(ssfb + 512 * h, 0, 128, 0));
+              for (int h = 0; h < C::SFB_ATOMS; ++h)
+                tc_cp_32x128b_warpx4_pair(sfb_t + 4 * h, make_smem_desc(ssfb + 512 * h, 0, 128, 0));
+            } else {
+              tc_cp_32x128b_warpx4(sfa_t, make_smem_desc(ssfa, 0, 128, 0));
+#pragma unroll
+              for (int h = 0; h < C::SFB_ATOMS; ++h)
+                tc_cp_32x128b_warpx4(sfb_t + 4 * h, make_smem_desc(ssfb + 512 * h, 0, 128, 0));
+            }
           }
           // four MMAs of 32 bytes of K each (32 E4M3 values, or 16 bf16)
 #pragma unroll
           for (uint32_t kk = 0; kk < 4; ++kk) {
             const uint64_t ad = make_smem_desc(sa + 32 * kk, 16, 1024, 2);
             const uint64_t bd = make_smem_desc(sb + 32 * kk, 16, 1024, 2);
-            if constexpr (MX)
-              tc_mma_mxf8(acc, ad, bd, make_idesc_mxf8(BM, BN, kk, kk), sfa_t | (kk << 30),
-                          sfb_t | (kk << 30), (kt | kk) != 0 ? 1u : 0u);
-            else
-              tc_mma_bf16(acc, ad, bd, make_idesc_bf16(BM, BN), (kt | kk) != 0 ? 1u : 0u);
+            const uint32_t accum = (kt | kk) != 0 ? 1u : 0u;
+            if constexpr (MX) {
+              if constexpr (PAIR)
+                tc_mma_mxf8_pair(acc, ad, bd, make_idesc_mxf8(MMA_M, BN, kk, kk), sfa_t | (kk << 30),
+                                 sfb_t | (kk << 30), accum);
+              else
+                tc_mma_mxf8(acc, ad, bd, make_idesc_mxf8(MMA_M, BN, kk, kk), sfa_t | (kk << 30),
+                            sfb_t | (kk << 30), accum);
+            } else {
+              if constexpr (PAIR)
+                tc_mma_bf16_pair(acc, ad, bd, make_idesc_bf16(MMA_M, BN), accum);
+              else
+                tc_mma_bf16(acc, ad, bd, make_idesc_bf16(MMA_M, BN), accum);
+            }
           }
-          tc_commit(&empty[stage]);
+          if constexpr (PAIR)
+            tc_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
+          else
+            tc_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc_commit(&acc_full[buf]);
+        if constexpr (PAIR)
+          tc_commit_pair(&acc_full[buf], 0x3);  // both CTAs' epilogues
+        else
+          tc_commit(&acc_full[buf]);
         ++acc_it;
       }
       if (*abort_flag) {
         // shutting down early: wait until every MMA issued so far has
         // finished writing TMEM before it is freed
-        tc_commit(drain);
+        if constexpr (PAIR)
+          tc_commit_pair(drain, 0x1);
+        else
+          tc_commit(drain);
         mbar_wait_drain(drain, 0);
       }
     }
@@ -629,12 +795,37 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
     uint32_t* stage = reinterpret_cast<uint32_t*>(smem + C::OFF_STAGE + (warp - 2) * C::STAGE_WARP_BYTES);
     uint32_t acc_it = 0;
     uint32_t v[C::NC];
+    // this CTA's part of tile t (and whether it has any rows of the expert)
+    auto my_tile = [&](int t, bool* none) {
+      Tile ti = decode_tile<EPI, BN, PAIR>(a, go, pc, t);
+      ti.m0 += row_off;
+      *none = PAIR && a.mode == 0 && ti.m0 >= ti.row_lim;
+      return ti;
+    };
+    const uint32_t release_bar = PAIR ? smem_in_cta(&acc_empty[0], 0) : 0u;
+    auto release = [&](uint32_t buf) {
+      if (lane == 0) {
+        if (PAIR && !leader)
+          mbar_arrive_cluster(release_bar + 8 * buf);
+        else
+          mbar_arrive(&acc_empty[buf]);
+      }
+    };
+    GuChunk gu;  // EPI_SWIGLU_BWD: g/u of the next chunk to process
     if constexpr (EPI == EPI_SWIGLU_BWD)
-      if (int(blockIdx.x) < ntiles) prefetch_saved(a, decode_tile<EPI, BN>(a, go, blockIdx.x), q, half, lane);
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      const Tile ti = decode_tile<EPI, BN>(a, go, t);
+      if (cid < ntiles) {
+        bool none;
+        load_gu(a, my_tile(cid, &none), q, half, lane, 0, gu);
+      }
+    for (int t = cid; t < ntiles; t += ncl) {
+      bool none;
+      const Tile ti = my_tile(t, &none);
+      const bool has_next = t + ncl < ntiles;
       if constexpr (EPI == EPI_SWIGLU_BWD)  // one tile ahead
-        if (t + int(gridDim.x) < ntiles) prefetch_saved(a, decode_tile<EPI, BN>(a, go, t + gridDim.x), q, half, lane);
+        if (has_next) {
+          bool nn;
+          prefetch_saved(a, my_tile(t + ncl, &nn), q, half, lane);
+        }
       if (ti.nkt == 0) {
         if constexpr (EPI == EPI_WGRAD) {
 #pragma unroll
@@ -647,14 +838,26 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
       if (!mbar_wait(&acc_full[buf], use & 1u, abort_flag)) break;
       tc_fence_after();
       const uint32_t tl = tmem + (uint32_t(32 * q) << 16) + buf * C::ACC_STRIDE;
-      if constexpr (EPI == EPI_SWIGLU_BWD) {
-        // reads TMEM chunk by chunk; the other accumulator keeps the MMAs busy
-        epilogue_swiglu_bwd(a, ti, tl, q, half, lane, stage);
+      if (none) {
+        // rows of another expert: nothing to read or write
+        if constexpr (EPI == EPI_SWIGLU_BWD)
+          if (has_next) {
+            bool nn;
+            load_gu(a, my_tile(t + ncl, &nn), q, half, lane, 0, gu);
+          }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        release(buf);
+      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+        // reads TMEM chunk by chunk; the other accumulator keeps the MMAs busy
+        bool nn;
+        const Tile tn = my_tile(has_next ? t + ncl : t, &nn);
+        epilogue_swiglu_bwd(a, ti, has_next ? &tn : nullptr, tl, q, half, lane, stage, gu);
+        tc_fence_before();
+        __syncwarp();
+        release(buf);
       } else {
-        if constexpr (GATE_UP) {  // gate columns 64*half.., up columns 128 + 64*half..
+        if constexpr (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16) {  // gate columns 64*half.., up columns 128 + 64*half..
           tmem_ld64(tl + 64 * half, v);
           tmem_ld64(tl + 128 + 64 * half, v + 64);
         } else if constexpr (C::NC == 128) {
@@ -665,7 +868,7 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        release(buf);
         epilogue_tile<EPI, BN>(a, ti, v, q, half, lane, stage);
       }
       ++acc_it;
@@ -673,10 +876,16 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync_all();  // no MMA of the pair writes either CTA's TMEM any more
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem, TMEM_COLS);
+    else
+      tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -697,15 +906,80 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <int EPI, int BN, int KIND = KIND_MXF8>
+// Clusters of two CTAs that can be resident at once (one per SM pair), per
+// device and kernel.
+template <typename Kernel>
+int pair_clusters(Kernel kern, cudaLaunchConfig_t cfg, std::atomic<int>* cache) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    const int cap = device_sm_count() / 2;
+    cfg.gridDim = dim3(2 * cap);
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = cap;
+    }
+    n = n < cap ? n : cap;
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+template <int EPI, int BN, int KIND, bool PAIR>
 cudaError_t launch_epi(const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
+  using C = Cfg<BN, PAIR>;
   static std::atomic<uint64_t> configured{0};
-  constexpr int smem = Cfg<BN>::SMEM_LAUNCH;
-  cudaError_t e = ensure_smem_limit(grouped_mxf8_gemm_kernel<EPI, BN, KIND>, smem, configured);
+  auto kern = grouped_mxf8_gemm_kernel<EPI, BN, KIND, PAIR>;
+  cudaError_t e = ensure_smem_limit(kern, C::SMEM_LAUNCH, configured);
   if (e != cudaSuccess) return e;
-  grouped_mxf8_gemm_kernel<EPI, BN, KIND><<<device_sm_count(), Cfg<BN>::THREADS, smem, st>>>(maps.a, maps.b, a);
+  if constexpr (!PAIR) {
+    kern<<<device_sm_count(), C::THREADS, C::SMEM_LAUNCH, st>>>(maps.a, maps.b, maps.sfa, maps.sfb, a);
+  } else {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_LAUNCH;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    static std::atomic<int> clusters[64];
+    cfg.gridDim = dim3(2 * pair_clusters(kern, cfg, clusters));
+    e = cudaLaunchKernelEx(&cfg, kern, maps.a, maps.b, maps.sfa, maps.sfb, a);
+    if (e != cudaSuccess) return e;
+  }
   count_launch();
   return cudaGetLastError();
+}
+
+// Scale atoms as a 2-D uint8 tensor [bytes / 256][256]: one 512-byte atom is
+// a {256, 2} box at row 2 * atom (CTA pairs load scales with tensor copies).
+cudaError_t make_map_sf(CUtensorMap* m, const void* base, int64_t bytes) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  if (bytes <= 0 || bytes % 512) return cudaErrorInvalidValue;
+  cuuint64_t dims[2] = {256, cuuint64_t(bytes / 256)};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {256, 2};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Scale maps of a pair launch: A (a_RT x a_KT atoms: mode 0 the permuted
+// rows, mode 1 the output rows) and B (its groups x b_RT x b_KT atoms).
+cudaError_t pair_scale_maps(GemmMaps& m, const GemmArgs& a, bool gate_up) {
+  const int64_t a_rt = a.mode == 0 ? a.rows_cap / 128 : a.m_tiles;
+  const int64_t b_groups = a.mode == 0 ? (gate_up ? 2 * int64_t(a.E) : a.E) : 1;
+  cudaError_t e = make_map_sf(&m.sfa, a.sfa, a_rt * a.a_KT * 512);
+  if (e != cudaSuccess) return e;
+  return make_map_sf(&m.sfb, a.sfb, b_groups * a.b_RT * a.b_KT * 512);
 }
 
 }  // namespace
@@ -737,25 +1011,61 @@ cudaError_t make_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
+// CTA pairs are opt-in (MOE_GEMM_PAIR=1): on the layer shapes benchmarked
+// here they were measured no faster than single CTAs (the M = 128 kernel is
+// not bound by its L2 operand traffic), and slower on ragged groups, whose
+// odd 128-row tile counts leave half of a 256-row tile empty.
+bool gemm_pair() {
+  static const bool on = [] {
+    const char* v = std::getenv("MOE_GEMM_PAIR");
+    return v && v[0] == '1';
+  }();
+  return on;
+}
+
+uint32_t gemm_b_box(uint32_t bn) { return gemm_pair() ? bn / 2 : bn; }
+
+cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps_in, const GemmArgs& a, cudaStream_t st) {
+  if (gemm_pair()) {
+    GemmMaps maps = maps_in;
+    cudaError_t e = pair_scale_maps(maps, a, epi == EPI_SWIGLU);
+    if (e != cudaSuccess) return e;
+    if (bn == 256) {
+      switch (epi) {
+        case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, 256, KIND_MXF8, true>(maps, a, st);
+        case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256, KIND_MXF8, true>(maps, a, st);
+        case EPI_F24_ROWS: return launch_epi<EPI_F24_ROWS, 256, KIND_MXF8, true>(maps, a, st);
+        case EPI_WGRAD: return launch_epi<EPI_WGRAD, 256, KIND_MXF8, true>(maps, a, st);
+      }
+    } else if (bn == 128) {
+      if (epi == EPI_SWIGLU_BWD) return launch_epi<EPI_SWIGLU_BWD, 128, KIND_MXF8, true>(maps, a, st);
+    }
+    return cudaErrorInvalidValue;
+  }
   if (bn == 256) {
     switch (epi) {
-      case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, 256>(maps, a, st);
-      case EPI_F32_SCATTER: return launch_epi<EPI_F32_SCATTER, 256>(maps, a, st);
-      case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256>(maps, a, st);
-      case EPI_F24_ROWS: return launch_epi<EPI_F24_ROWS, 256>(maps, a, st);
-      case EPI_WGRAD: return launch_epi<EPI_WGRAD, 256>(maps, a, st);
+      case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, 256, KIND_MXF8, false>(maps_in, a, st);
+      case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256, KIND_MXF8, false>(maps_in, a, st);
+      case EPI_F24_ROWS: return launch_epi<EPI_F24_ROWS, 256, KIND_MXF8, false>(maps_in, a, st);
+      case EPI_WGRAD: return launch_epi<EPI_WGRAD, 256, KIND_MXF8, false>(maps_in, a, st);
     }
   } else if (bn == 128) {
-    if (epi == EPI_SWIGLU_BWD) return launch_epi<EPI_SWIGLU_BWD, 128>(maps, a, st);
+    if (epi == EPI_SWIGLU_BWD) return launch_epi<EPI_SWIGLU_BWD, 128, KIND_MXF8, false>(maps_in, a, st);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_grouped_gemm_bf16(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
+  if (gemm_pair()) {
+    switch (epi) {
+      case EPI_SWIGLU_BF16: return launch_epi<EPI_SWIGLU_BF16, 256, KIND_BF16, true>(maps, a, st);
+      case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256, KIND_BF16, true>(maps, a, st);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (epi) {
-    case EPI_SWIGLU_BF16: return launch_epi<EPI_SWIGLU_BF16, 256, KIND_BF16>(maps, a, st);
-    case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256, KIND_BF16>(maps, a, st);
+    case EPI_SWIGLU_BF16: return launch_epi<EPI_SWIGLU_BF16, 256, KIND_BF16, false>(maps, a, st);
+    case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256, KIND_BF16, false>(maps, a, st);
   }
   return cudaErrorInvalidValue;
 }

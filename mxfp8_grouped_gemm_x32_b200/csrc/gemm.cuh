@@ -70,6 +70,7 @@ struct GemmArgs {
 // boxes of bn/2 rows); all uint8 with 128-byte swizzle.
 struct GemmMaps {
   CUtensorMap a, b;
+  CUtensorMap sfa, sfb;  // CTA-pair launches: scale atoms (set by launch_grouped_gemm)
 };
 
 cudaError_t make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
@@ -77,8 +78,15 @@ cudaError_t make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64
 cudaError_t make_map_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                         uint64_t groups, uint32_t box_rows);
 
+// CTA pairs (M = 256 tiles on two SMs; only with MOE_GEMM_PAIR=1): the B
+// tensor maps then carry boxes of half the tile's rows -- gemm_b_box(bn)
+// gives the box rows for a B operand of bn rows per tile.  Mode 0 launches
+// must set rows_cap (the rows of A's scale layout).
+bool gemm_pair();
+uint32_t gemm_b_box(uint32_t bn);
+
 // bn: tile width, 256 (one accumulator; every epilogue but EPI_SWIGLU_BWD)
-// or 192 (two accumulators, 12 epilogue warps; EPI_SWIGLU_BWD).
+// or 128 (two accumulators; EPI_SWIGLU_BWD).
 cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);
 
 // BF16 operands (kind::f16), bn = 256: EPI_SWIGLU_BF16 and EPI_F32_ROWS.

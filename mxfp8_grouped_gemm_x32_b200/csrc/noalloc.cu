@@ -74,5 +74,6 @@ extern "C" moe_status_t moe_permute_noalloc(const void* x, const int32_t* topk_i
   if (launch_permute_index(topk_idx, topk_prob, R, E, rows_cap, split_sizes, group_offsets, row_to_slot,
                            slot_to_row, prob_perm, scratch, st) != cudaSuccess)
     return MOE_ERR_CUDA;
-  return quantize_x(x, T, H, k, E, rows_cap, row_to_slot, group_offsets, xq, xq_sf, xq_col, xq_col_sf, st);
+  return quantize_x(x, T, H, k, E, rows_cap, row_to_slot, slot_to_row, group_offsets, xq, xq_sf, xq_col, xq_col_sf,
+                    st);
 }

@@ -379,6 +379,83 @@ __global__ void __launch_bounds__(256, 3) quant_both_kernel(QuantBothArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Row form of the permuted x without a gather.  Token t is read once and
+// quantised once (blocks of 32 along H); its codes and scale bytes are
+// written to each of its k rows slot_to_row[t*k + j].  One thread per 8
+// values and four lanes per block (the block's |max| by two shuffles), so a
+// warp reads 512 contiguous bytes and writes 256 contiguous code bytes per
+// destination row; many small threads keep enough loads in flight.  The
+// padding rows inside the expert groups (row_to_slot < 0 below
+// group_offsets[E]) then get zero codes and zero scale bytes.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256, 6) quant_rows_scatter_kernel(ScatterRowsArgs a) {
+  const uint32_t H8 = a.h8_div.d;                // 8-value units per row (a multiple of 4)
+  const uint32_t n = uint32_t(a.T) * H8;         // < 2^31 (checked by the launcher)
+  const uint32_t KB = H8 / 4;
+  const int k = a.k;
+  const uint32_t lane = threadIdx.x & 31;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  // the loop bound is tested on the warp's first index, so whole warps
+  // iterate together (the shuffles need all 32 lanes)
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i - lane < n; i += stride) {
+    const bool in = i < n;
+    const uint32_t t = fastdiv(in ? i : 0u, a.h8_div);
+    const uint32_t u = (in ? i : 0u) - t * H8;
+    const uint4 v = in ? __ldg(reinterpret_cast<const uint4*>(a.src + (int64_t(t) * a.H + u * 8) * 2))
+                       : make_uint4(0u, 0u, 0u, 0u);
+    float f[8];
+    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+    float m = abs_max_n<8>(f);
+    m = abs_max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));  // lanes 4b..4b+3 hold one block
+    m = abs_max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    if (!in) continue;
+    const uint32_t sb = e8m0_from_amax_bits(__float_as_uint(m));
+    const float inv = inv_scale_from_e8m0(sb);
+    const uint2 w = make_uint2(pack4_e4m3(f[0] * inv, f[1] * inv, f[2] * inv, f[3] * inv),
+                               pack4_e4m3(f[4] * inv, f[5] * inv, f[6] * inv, f[7] * inv));
+    const uint32_t kb = u >> 2;
+    const bool lead = (u & 3) == 0;                  // writes the block's scale byte
+    const bool last = lead && kb + 1 == KB;          // also clears the padding blocks of the last K tile
+    const int32_t* rows = a.slot_to_row + int64_t(t) * k;
+    for (int j0 = 0; j0 < k; j0 += 4) {
+      int32_t rw[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) rw[j] = j0 + j < k ? __ldg(rows + j0 + j) : -1;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (rw[j] < 0) continue;
+        const int64_t r = rw[j];
+        *reinterpret_cast<uint2*>(a.q + r * a.H + u * 8) = w;
+        if (lead) {
+          a.sf[sf_offset(0, r, kb, 0, a.KT)] = uint8_t(sb);
+          if (last)
+            for (int64_t p = KB; p < 4 * a.KT; ++p) a.sf[sf_offset(0, r, p, 0, a.KT)] = 0;
+        }
+      }
+    }
+  }
+  // padding rows inside the groups, 32 rows per warp at a time
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = stride >> 5;
+  const int64_t used = max(*a.rows_used, 0);
+  for (int64_t r0 = int64_t(warp) * 32; r0 < used; r0 += int64_t(nwarps) * 32) {
+    const int64_t r = r0 + lane;
+    const bool pad = r < used && __ldg(a.row_to_slot + r) < 0;
+    uint32_t mask = __ballot_sync(0xFFFFFFFFu, pad);
+    while (mask) {
+      const int l = __ffs(mask) - 1;
+      mask &= mask - 1;
+      const int64_t pr = r0 + l;
+      for (int64_t c = int64_t(lane) * 16; c < a.H; c += 512)
+        *reinterpret_cast<uint4*>(a.q + pr * a.H + c) = make_uint4(0u, 0u, 0u, 0u);
+      for (int64_t kt = lane; kt < a.KT; kt += 32)
+        *reinterpret_cast<uint32_t*>(a.sf + sf_offset(0, pr, 4 * kt, 0, a.KT)) = 0u;
+    }
+  }
+}
+
 cudaError_t launch_quant_rows(const QuantRowsArgs& args, cudaStream_t st) {
   const int64_t total = int64_t(args.groups) * cdiv(args.rows, 128) * 128 * cdiv(args.K, 128);
   if (total == 0) return cudaSuccess;
@@ -424,6 +501,21 @@ cudaError_t launch_quant_both(const QuantBothArgs& args, cudaStream_t st) {
   int64_t grid = int64_t(device_sm_count()) * 3;
   if (grid > tiles) grid = tiles;
   quant_both_kernel<<<unsigned(grid), 256, smem, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows_scatter(const ScatterRowsArgs& args, cudaStream_t st) {
+  if (args.T == 0) return cudaSuccess;
+  const int64_t n = args.T * (args.H / 8);
+  if (n >= (int64_t(1) << 31) - (int64_t(1) << 24) || args.H % 32) return cudaErrorInvalidValue;
+  ScatterRowsArgs a = args;
+  a.h8_div = make_fastdiv(uint32_t(a.H / 8));
+  a.KT = cdiv(a.H, 128);
+  int64_t blocks = cdiv(n, 256);
+  const int64_t cap = int64_t(device_sm_count()) * 6;  // one wave (six CTAs per SM)
+  if (blocks > cap) blocks = cap;
+  quant_rows_scatter_kernel<<<unsigned(blocks), 256, 0, st>>>(a);
   count_launch();
   return cudaGetLastError();
 }

@@ -74,6 +74,24 @@ struct QuantBothArgs {
 
 cudaError_t launch_quant_both(const QuantBothArgs& a, cudaStream_t st);
 
+// Row mode of the permuted x without a gather: token t is quantised once
+// and written to each of its rows slot_to_row[t*k + j]; padding rows inside
+// the groups (row_to_slot < 0 below *rows_used) get zero codes and scales.
+struct ScatterRowsArgs {
+  const uint8_t* src;           // x [T][H] bf16
+  int64_t T, H;
+  int32_t k;
+  const int32_t* slot_to_row;   // [T*k]
+  const int32_t* row_to_slot;   // [rows_cap]
+  const int32_t* rows_used;     // group_offsets + E (device)
+  uint8_t* q;                   // [rows_cap][H]
+  uint8_t* sf;                  // blocked (1, rows_cap, H)
+  int64_t KT = 0;               // set by the launcher
+  FastDiv h8_div;               // H / 8 (set by the launcher)
+};
+
+cudaError_t launch_quant_rows_scatter(const ScatterRowsArgs& a, cudaStream_t st);
+
 }  // namespace moe
 
 namespace moe {
@@ -82,7 +100,7 @@ namespace moe {
 // xq, xq_sf = MX tensor (1, rows_cap, H) of the gathered rows; with xq_col,
 // the gathered rows quantised along tokens, MX tensor (1, H, rows_cap).
 moe_status_t quantize_x(const void* x, int32_t T, int32_t H, int32_t k, int32_t E, int64_t rows_cap,
-                        const int32_t* row_to_slot, const int32_t* group_offsets, uint8_t* xq, uint8_t* xq_sf,
-                        uint8_t* xq_col, uint8_t* xq_col_sf, cudaStream_t st);
+                        const int32_t* row_to_slot, const int32_t* slot_to_row, const int32_t* group_offsets,
+                        uint8_t* xq, uint8_t* xq_sf, uint8_t* xq_col, uint8_t* xq_col_sf, cudaStream_t st);
 
 }  // namespace moe

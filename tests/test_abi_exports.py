@@ -128,10 +128,10 @@ def test_forward_argument_errors():
     assert f(*_fwd_args(hq=None, hq_sf=None, ws_bytes=need - 1)) == WORKSPACE   # h in the workspace
 
 
-def _bwd_args(T=64, H=256, I=512, E=4, k=2, saved=P, dW1=P, ws_bytes=1 << 40):
+def _bwd_args(T=64, H=256, I=512, E=4, k=2, saved=P, dW1=P, ws=P, ws_bytes=1 << 40):
     from mxfp8_grouped_gemm_x32_b200 import lib
     rows_cap = lib.moe_padded_rows(T, k, E)
-    return (P, P, P, P, T, H, I, E, k, rows_cap, P, P, P, P, P, P, saved, P, P, dW1, P, P, P, ws_bytes, None)
+    return (P, P, P, P, T, H, I, E, k, rows_cap, P, P, P, P, P, P, saved, P, P, dW1, P, P, ws, ws_bytes, None)
 
 
 def test_backward_argument_errors():
@@ -141,6 +141,8 @@ def test_backward_argument_errors():
     assert f(*_bwd_args(H=48)) == UNSUPPORTED
     assert f(*_bwd_args(E=300, k=2)) == UNSUPPORTED
     assert f(*_bwd_args(dW1=M)) == INVALID
+    assert f(*_bwd_args(saved=P + 16)) == INVALID                   # saved_a needs 32-byte alignment
+    assert f(*_bwd_args(ws=P + 128)) == INVALID                     # workspace needs 256-byte alignment
     need = lib.moe_workspace_size(lib.MOE_OP_BWD, 64, 2, 4, 256, 512)
     assert f(*_bwd_args(ws_bytes=need - 1)) == WORKSPACE
 

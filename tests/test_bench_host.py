@@ -98,7 +98,7 @@ def test_attainable_fwd_limits():
     split = [256, 256, 256, 256]
     big_bw = bench.attainable_fwd(cfg, split, 1000.0, 1e12, 1536)["ms"]
     flops = sum(6.0 * m * H * I for m in split)
-    pc_bytes = T * H * 2 + 2 * 1536 * H * (1 + 1 / 32) + T * k * H * 4 + T * H * 2
+    pc_bytes = T * H * 2 + T * k * H * (1 + 1 / 32) + T * k * H * 3 + T * H * 2
     assert big_bw == pytest.approx((flops / 1e15 + pc_bytes / 1e21) * 1e3, rel=1e-12)  # GEMM bytes take no time
     empty = bench.attainable_fwd(cfg, [0, 0, 0, 1024], 1e9, 1000.0, 1536)["ms"]
     w_bytes = 3 * (1 + 1 / 32) * H * I                               # MX W_gate_up + W_down of one expert
@@ -106,6 +106,22 @@ def test_attainable_fwd_limits():
     a = bench.attainable_fwd(cfg, [100, 200, 300, 424], 2000.0, 6000.0, 1536)["ms"]
     b = bench.attainable_fwd(cfg, [200, 200, 300, 424], 2000.0, 6000.0, 1536)["ms"]
     assert b >= a
+
+
+def test_bandwidth_annotation():
+    """Bandwidth kernels get algorithmic bytes, GB/s and the HBM fraction;
+    other kernels are left as they are."""
+    cfg = get_config("mixtral_8x7b")                  # T8192 H4096 I14336 E8 k2
+    b = bench.bandwidth_bytes(cfg)
+    mx = 1 + 1 / 32
+    assert b["quant_weights"] == pytest.approx(3 * 8 * 4096 * 14336 * (2 + 2 * mx))   # 5.71 GB
+    assert b["permute_quant"] == pytest.approx(8192 * 4096 * 2 + 16384 * 4096 * mx)
+    assert b["dy_quant"] == pytest.approx(8192 * 4096 * 2 + 2 * 16384 * 4096 * mx)
+    assert b["combine"] == pytest.approx(16384 * 4096 * 3 + 8192 * 4096 * 2)
+    k = bench.annotate_bandwidth({"combine": {"ms_per_step": 0.05}, "gemm_down": {"ms_per_step": 0.9}}, cfg, 6650.0)
+    assert k["combine"]["gbs"] == pytest.approx(b["combine"] / 0.05e-3 / 1e9)
+    assert k["combine"]["frac_of_hbm"] == pytest.approx(k["combine"]["gbs"] / 6650.0)
+    assert "gbs" not in k["gemm_down"]
 
 
 def test_l2_note_states_the_weight_bytes():
