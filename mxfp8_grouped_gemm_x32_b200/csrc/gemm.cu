@@ -58,7 +58,16 @@ struct Cfg {
   static constexpr int STAGES = PAIR ? (BN == 128 ? 7 : 6) : (BN == 128 ? 5 : 4);
   static constexpr int ACC = BN == 256 ? 1 : 2;   // TMEM accumulators
   static constexpr int EPI_WARPS = 8;
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  // warps before the epilogue warps: producer, MMA issuer and, for BN = 128,
+  // two idle warps that complete warpgroup 0, so that the three warpgroups
+  // can trade registers (setmaxnreg): warpgroup 0 drops to REGS_LEAD, the
+  // two epilogue warpgroups rise to REGS_EPI
+  static constexpr int LEAD_WARPS = BN == 128 ? 4 : 2;
+  static constexpr int THREADS = 32 * (LEAD_WARPS + EPI_WARPS);
+  static constexpr int REGS_LAUNCH = 168, REGS_LEAD = 40, REGS_EPI = 232;
+  static_assert(LEAD_WARPS != 4 || (4 * REGS_LEAD + 8 * REGS_EPI == 12 * REGS_LAUNCH &&
+                                    REGS_LEAD + 2 * REGS_EPI <= 512),
+                "register split must equal the launch allocation and fit each SM sub-partition");
   static constexpr int NC = BN / (EPI_WARPS / 4);  // accumulator columns per epilogue warp
   static constexpr uint32_t ACC_STRIDE = BN;        // TMEM columns between the accumulators
   static constexpr uint32_t SFA_COL = ACC * ACC_STRIDE, SFB_COL = SFA_COL + 4;  // scale factors after them
@@ -448,14 +457,14 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
   const float p = rv ? a.prob[r] : 0.0f;
   float dps = 0.0f;
   uint32_t sb_dg = 0, sb_du = 0;
-  // dh is read from TMEM once per pass rather than held in registers (the
-  // accumulator stays ours until released)
+  // (the accumulator stays ours until released; the other one keeps the
+  // MMAs busy)
 #pragma unroll 1
   for (int j = 0; j < 2; ++j) {
     const int cc = cb + 32 * j;
     const uint32_t tc = tl + 64 * half + 32 * j;
     float sv[32], o[32];  // sv: s = g * sigmoid(g), kept across the three passes
-    uint32_t d[32];
+    uint32_t d[32];       // dh, read from TMEM once per chunk
     // dg = dh*p*u*sig*(1+g*(1-sig)), quantised along 2I (columns cc..cc+31)
     // and along tokens
     load_dh32(tc, rv, d);
@@ -470,7 +479,6 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
     quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, cc, a.rows_cap, rb, KTt);
     // du = dh*p*s, quantised along 2I (columns I+cc..) and along tokens;
     // dprob partial sum dh*s*u
-    load_dh32(tc, rv, d);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       o[e] = (__uint_as_float(d[e]) * p) * sv[e];
@@ -478,8 +486,8 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
     }
     sb_du |= encode32_store(o, a.daq + r * I2 + I + cc) << (8 * j);
     quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, int64_t(I) + cc, a.rows_cap, rb, KTt);
-    // dh is used up: load the next chunk's g/u now (it lands during the
-    // last pass and the start of the next chunk)
+    // dh and g are used up: load the next chunk's g/u now (it lands during
+    // the last pass and the start of the next chunk)
     GuChunk nxt;
     if (j == 0)
       load_gu(a, ti, q, half, lane, 1, nxt);
@@ -652,7 +660,10 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const int ntiles = total_tiles<PAIR>(a, go, pc);
 
+  // (BN = 128: the launch gave every thread REGS_LAUNCH registers, checked on
+  // the host; each role's branch starts by resizing its warpgroup's share)
   if (warp == 0) {
+    if constexpr (C::LEAD_WARPS == 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_LEAD));
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       prefetch_tmap(&tmA);
@@ -711,6 +722,7 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
       }
     }
   } else if (warp == 1) {
+    if constexpr (C::LEAD_WARPS == 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_LEAD));
     if (lane == 0 && leader) {
       // ---------------- MMA issuer ----------------
       int stage = 0;
@@ -788,11 +800,16 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
         mbar_wait_drain(drain, 0);
       }
     }
+  } else if (warp < C::LEAD_WARPS) {
+    // idle warps completing warpgroup 0
+    if constexpr (C::LEAD_WARPS == 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_LEAD));
   } else {
     // ---------------- epilogue warps ----------------
+    if constexpr (C::LEAD_WARPS == 4) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_EPI));
     const int q = warp & 3;            // TMEM sub-partition this warp may read
-    const int half = (warp - 2) >> 2;  // which NC-column part of the tile's columns
-    uint32_t* stage = reinterpret_cast<uint32_t*>(smem + C::OFF_STAGE + (warp - 2) * C::STAGE_WARP_BYTES);
+    const int half = (warp - C::LEAD_WARPS) >> 2;  // which NC-column part of the tile's columns
+    uint32_t* stage =
+        reinterpret_cast<uint32_t*>(smem + C::OFF_STAGE + (warp - C::LEAD_WARPS) * C::STAGE_WARP_BYTES);
     uint32_t acc_it = 0;
     uint32_t v[C::NC];
     // this CTA's part of tile t (and whether it has any rows of the expert)
@@ -933,6 +950,18 @@ cudaError_t launch_epi(const GemmMaps& maps, const GemmArgs& a, cudaStream_t st)
   auto kern = grouped_mxf8_gemm_kernel<EPI, BN, KIND, PAIR>;
   cudaError_t e = ensure_smem_limit(kern, C::SMEM_LAUNCH, configured);
   if (e != cudaSuccess) return e;
+  if constexpr (C::LEAD_WARPS == 4) {
+    // the warpgroups' register split assumes exactly REGS_LAUNCH registers
+    // per thread at launch; anything else could leave setmaxnreg.inc waiting
+    static std::atomic<int> regs{0};
+    if (regs.load(std::memory_order_relaxed) == 0) {
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, kern);
+      if (e != cudaSuccess) return e;
+      regs.store(fa.numRegs, std::memory_order_relaxed);
+    }
+    if (regs.load(std::memory_order_relaxed) != C::REGS_LAUNCH) return cudaErrorLaunchOutOfResources;
+  }
   if constexpr (!PAIR) {
     kern<<<device_sm_count(), C::THREADS, C::SMEM_LAUNCH, st>>>(maps.a, maps.b, maps.sfa, maps.sfb, a);
   } else {
