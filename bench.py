@@ -703,6 +703,21 @@ def run_ours(args):
     st = layer.device_status()
     if st != 0:
         raise SystemExit(f"device status after the BF16 forward: {lib.status_string(st)}")
+    # the per-tensor FP8 recipe's forward (one factor per tensor, quantised
+    # from the bf16 weights and x every call): routing + forward
+    for _ in range(3):
+        layer.permute_index(idx, prob)
+        layer.forward_fp8_tensor(x, w1, w2)
+    e0.record(stream)
+    for _ in range(10):
+        layer.permute_index(idx, prob)
+        layer.forward_fp8_tensor(x, w1, w2)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_f8t = max_over_ranks(e0.elapsed_time(e1) / 10, world, dev)
+    st = layer.device_status()
+    if st != 0:
+        raise SystemExit(f"device status after the per-tensor FP8 forward: {lib.status_string(st)}")
 
     if world > 1:
         dist.destroy_process_group()
@@ -760,6 +775,11 @@ def run_ours(args):
                      "frac_of_bf16_peak": cfg.fwd_flops() / (ms_bf16 * 1e-3) / 1e12 / peaks["bf16_sustained"],
                      "what": "BF16 recipe layer forward (moe_permute without x + moe_grouped_mlp_fwd_bf16): "
                              "bf16 operands, no MXFP8"},
+        "fp8_tensor_fwd": {"value": world * cfg.fwd_flops() / (ms_f8t * 1e-3) / 1e12, "unit": "TFLOP/s",
+                           "ms_per_call": ms_f8t,
+                           "what": "per-tensor FP8 recipe layer forward (moe_permute without x + "
+                                   "moe_grouped_mlp_fwd_fp8_tensor): factors from the current |max| of x, of every "
+                                   "expert's weights and of h, weights quantised in the call"},
         "router": {"ms_per_call": router_ms, "in_step": False,
                    "what": "moe_router_topk on fp32 logits [T, E] (softmax, top-k, renormalise)"},
         "roofline": roofline,

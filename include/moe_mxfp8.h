@@ -93,6 +93,7 @@ typedef enum {
 #define MOE_OP_FWD 2
 #define MOE_OP_BWD 3
 #define MOE_OP_FWD_BF16 4
+#define MOE_OP_FWD_FP8_TENSOR 5
 
 /* Limits checked on the host. */
 #define MOE_MAX_EXPERTS 256
@@ -286,6 +287,35 @@ moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down,
                                       const int32_t* group_offsets, const int32_t* row_to_slot,
                                       const int32_t* slot_to_row, const float* prob_perm, const void* x,
                                       void* out, void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* Per-tensor FP8 grouped MLP forward: the FP8 recipe Challenge 2 contrasts
+ * with MXFP8 -- one float32 factor for a whole tensor instead of one per 32
+ * values.  Every call takes each tensor's current |max| and quantises:
+ *   scale = 448 / amax (IEEE float32 division; the largest finite float32
+ *   where that overflows; 1 for amax 0 or non-finite), code = E4M3(float32
+ *   (v * scale)), value = code / scale;
+ * tensors: x (one factor), each expert's W_gate_up [2I][H] and W_down [H][I]
+ * (one factor per expert matrix), and h over all routed rows.  A = x
+ * W_gate_up^T and y = h W_down^T run on the kind::f8f6f4 tensor cores (fp32
+ * accumulation, dequantised by 1 / (scale_a scale_b) per expert); h = prob *
+ * silu(gate) * up is held in bf16 between the GEMMs (as in the BF16 recipe)
+ * and its factor comes from that bf16 tensor; out[t] = sum_j y[t*k+j] (fp32,
+ * ascending j, one bf16 rounding).
+ *   w_gate_up  bf16 [E][2I][H] (gate rows first); w_down bf16 [E][H][I].
+ *   routing    from moe_permute (xq may be NULL there).
+ *   x          bf16 [T][H];  out bf16 [T][H].
+ *   scales     NULL, or float [2 + 2E] receiving the factors: x, h,
+ *              W_gate_up[0..E), W_down[0..E).
+ *   workspace  >= moe_workspace_size(MOE_OP_FWD_FP8_TENSOR, T, k, E, H, I),
+ *              256-byte aligned.
+ * Limits as moe_grouped_mlp_fwd.  The pages describe no kernel for this
+ * recipe; the factor rule above is this library's reading. */
+moe_status_t moe_grouped_mlp_fwd_fp8_tensor(const void* w_gate_up, const void* w_down, int32_t T, int32_t H,
+                                            int32_t I, int32_t E, int32_t k, int64_t rows_cap,
+                                            const int32_t* split_sizes, const int32_t* group_offsets,
+                                            const int32_t* row_to_slot, const int32_t* slot_to_row,
+                                            const float* prob_perm, const void* x, void* out, float* scales,
+                                            void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* Top-k combine (Challenge 1, index_add back to token order):
  *   y  bf16 [T*k][H] in slot order -> out bf16 [T][H], out[t] = sum_j y[t*k+j]

@@ -100,6 +100,30 @@ FwdBf16Ws carve_fwd_bf16(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, 
   return w;
 }
 
+// Per-tensor FP8 forward workspace: E4M3 codes of x (permuted rows), of the
+// weights and of h, h in bf16, f24 rows, and the factors: |max| bits
+// [2 + 2E] (x, h, W_gate_up[E], W_down[E]), scales [2 + 2E] and
+// dequantisation factors [2E].
+struct FwdF8tWs {
+  uint8_t *xq, *w1q, *w2q, *h, *hq, *y;
+  uint32_t* amax;
+  float *scale, *deq;
+};
+FwdF8tWs carve_fwd_f8t(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t E, int64_t rows_cap) {
+  (void)T; (void)k;
+  FwdF8tWs w{};
+  w.xq = c.take(rows_cap * H);
+  w.w1q = c.take(E * 2 * I * H);
+  w.w2q = c.take(E * H * I);
+  w.h = c.take(rows_cap * I * 2);
+  w.hq = c.take(rows_cap * I);
+  w.y = c.take(rows_cap * H * 3);
+  w.amax = reinterpret_cast<uint32_t*>(c.take((2 + 2 * E) * 4));
+  w.scale = reinterpret_cast<float*>(c.take((2 + 2 * E) * 4));
+  w.deq = reinterpret_cast<float*>(c.take(2 * E * 4));
+  return w;
+}
+
 // xp[r] = x[row_to_slot[r] / k] (bf16 rows, 16 bytes per thread) for the
 // rows of the groups; padding rows inside a group are zero.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ row_to_slot,
@@ -217,6 +241,10 @@ int64_t moe_workspace_size(int32_t op, int32_t T, int32_t k, int32_t E, int32_t 
     case MOE_OP_FWD_BF16:
       if (H <= 0 || I <= 0) return -1;
       carve_fwd_bf16(c, T, k, H, I, rows_cap);
+      return c.off;
+    case MOE_OP_FWD_FP8_TENSOR:
+      if (H <= 0 || I <= 0) return -1;
+      carve_fwd_f8t(c, T, k, H, I, E, rows_cap);
       return c.off;
   }
   return -1;
@@ -422,6 +450,86 @@ moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down,
   }
   TimeScope ts(st, "combine");
   return cuda_status(launch_combine(w.y, COMBINE_F32, slot_to_row, T, k, H, out, st));
+}
+
+moe_status_t moe_grouped_mlp_fwd_fp8_tensor(const void* w_gate_up, const void* w_down, int32_t T, int32_t H,
+                                            int32_t I, int32_t E, int32_t k, int64_t rows_cap,
+                                            const int32_t* split_sizes, const int32_t* group_offsets,
+                                            const int32_t* row_to_slot, const int32_t* slot_to_row,
+                                            const float* prob_perm, const void* x, void* out, float* scales,
+                                            void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  if (!w_gate_up || !w_down || !split_sizes || !group_offsets || !row_to_slot || !prob_perm ||
+      (T > 0 && (!x || !out || !slot_to_row)))
+    return MOE_ERR_INVALID;
+  if (!layer_dims_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
+  for (const void* p : {w_gate_up, w_down, x, (const void*)out})
+    if (!al16(p)) return MOE_ERR_INVALID;
+  if (scales && (reinterpret_cast<uintptr_t>(scales) & 3u)) return MOE_ERR_INVALID;
+  Carver c{static_cast<uint8_t*>(workspace)};
+  FwdF8tWs w = carve_fwd_f8t(c, T, k, H, I, E, rows_cap);
+  if (!workspace || int64_t(workspace_bytes) < c.off || !al256(workspace)) return MOE_ERR_WORKSPACE;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const uint8_t* w1 = static_cast<const uint8_t*>(w_gate_up);
+  const uint8_t* w2 = static_cast<const uint8_t*>(w_down);
+  const int64_t nw1 = 2 * int64_t(I) * H, nw2 = int64_t(H) * I;
+  {
+    // factors of x and of every expert's weights from their current |max|
+    TimeScope ts(st, "fp8t_quant_inputs");
+    if (cudaMemsetAsync(w.amax, 0, (2 + 2 * size_t(E)) * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (T > 0 && launch_f8t_amax(static_cast<const uint8_t*>(x), 1, int64_t(T) * H, w.amax, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (launch_f8t_amax(w1, E, nw1, w.amax + 2, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_f8t_amax(w2, E, nw2, w.amax + 2 + E, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_f8t_scales(w.amax, E, 0, w.scale, w.deq, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_f8t_quant(w1, E * nw1, nw1, w.scale + 2, nullptr, 0, w.w1q, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_f8t_quant(w2, E * nw2, nw2, w.scale + 2 + E, nullptr, 0, w.w2q, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_f8t_quant_scatter(static_cast<const uint8_t*>(x), T, H, k, slot_to_row, row_to_slot, group_offsets + E,
+                                 w.scale, w.xq, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  if (T > 0) {
+    // gate_up grouped GEMM, dequantised, + ScaledSwiGLU: h in bf16 and its |max|
+    GemmMaps m1;
+    if (make_map_2d(&m1.a, w.xq, H, rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
+    if (make_map_3d(&m1.b, w.w1q, H, I, 2 * int64_t(E), 128) != cudaSuccess) return MOE_ERR_CUDA;
+    GemmArgs g1{};
+    g1.mode = 0; g1.E = E; g1.N = I; g1.num_kt = int32_t(cdiv(H, 128)); g1.n_tiles = int32_t(cdiv(I, 128));
+    g1.group_offsets = group_offsets; g1.split_sizes = split_sizes; g1.rows_cap = rows_cap;
+    g1.prob = prob_perm; g1.row_to_slot = row_to_slot; g1.q_out = w.h;
+    g1.deq = w.deq; g1.amax_out = w.amax + 1;
+    {
+      TimeScope ts(st, "gemm_gate_up_swiglu_fp8t");
+      if (launch_grouped_gemm_f8t(EPI_SWIGLU_F8T, m1, g1, st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    // h's factor, then its codes (rows of the groups)
+    {
+      TimeScope ts(st, "fp8t_quant_h");
+      if (launch_f8t_scales(w.amax, E, 1, w.scale, w.deq, st) != cudaSuccess) return MOE_ERR_CUDA;
+      if (launch_f8t_quant(w.h, rows_cap * I, rows_cap * I, w.scale + 1, group_offsets + E, I, w.hq, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    // down grouped GEMM, dequantised, f24 rows in permuted order
+    GemmMaps m2;
+    if (make_map_2d(&m2.a, w.hq, I, rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
+    if (make_map_3d(&m2.b, w.w2q, I, H, E, 256) != cudaSuccess) return MOE_ERR_CUDA;
+    GemmArgs g2{};
+    g2.mode = 0; g2.E = E; g2.N = H; g2.num_kt = int32_t(cdiv(I, 128)); g2.n_tiles = int32_t(cdiv(H, 256));
+    g2.group_offsets = group_offsets; g2.split_sizes = split_sizes; g2.rows_cap = rows_cap;
+    g2.out = w.y; g2.ld_out = 3 * int64_t(H); g2.deq = w.deq + E;
+    {
+      TimeScope ts(st, "gemm_down_fp8t");
+      if (launch_grouped_gemm_f8t(EPI_F24_ROWS, m2, g2, st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    {
+      TimeScope ts(st, "combine");
+      if (launch_combine(w.y, COMBINE_F24, slot_to_row, T, k, H, out, st) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+  }
+  if (scales && cudaMemcpyAsync(scales, w.scale, (2 + 2 * size_t(E)) * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, const uint8_t* w1tq,

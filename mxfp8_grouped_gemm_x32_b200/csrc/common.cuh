@@ -473,6 +473,29 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// D[tmem] (+)= A x B^T, E4M3 operands from shared memory without block
+// scales (kind::f8f6f4), fp32 accumulators in TMEM.
+__device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor of kind::f8f6f4 MMA without block scales: E4M3 x
+// E4M3 -> fp32, both K-major, M x N.
+__host__ __device__ constexpr uint32_t make_idesc_f8(int M, int N) {
+  return 1u << 4                  // D format F32
+         | 0u << 7                // A format E4M3
+         | 0u << 10               // B format E4M3
+         | 0u << 15 | 0u << 16    // both K-major
+         | uint32_t(N >> 3) << 17 // N / 8
+         | uint32_t(M >> 4) << 24;// M / 16
+}
+
 // Instruction descriptor of kind::f16 MMA: bf16 x bf16 -> fp32, both
 // K-major, M x N.
 __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N) {

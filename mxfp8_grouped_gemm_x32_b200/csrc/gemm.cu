@@ -131,7 +131,7 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, co
     const int n_idx = local / mt, m_idx = local - n_idx * mt;  // rows fastest: B panel reuse
     ti.e = e;
     ti.m0 = go[e] + (m_idx << MSHIFT);
-    ti.n0 = n_idx * ((EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16) ? BN / 2 : BN);
+    ti.n0 = n_idx * ((EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16 || EPI == EPI_SWIGLU_F8T) ? BN / 2 : BN);
     ti.kt0 = 0;
     ti.nkt = a.num_kt;
     ti.row_end = go[e] + a.split_sizes[e];
@@ -240,26 +240,43 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
   constexpr int NC = Cfg<BN>::NC;  // accumulator columns per warp
   const int r = ti.m0 + 32 * q + lane;
   const bool rv = r < ti.row_end;
-  if constexpr (EPI == EPI_SWIGLU_BF16) {
+  if constexpr (EPI == EPI_SWIGLU_BF16 || EPI == EPI_SWIGLU_F8T) {
     static_assert(BN == 256, "the gate_up epilogue pairs 128 gate with 128 up columns");
     // v[0:64] gate columns nb..nb+63, v[64:128] the matching up columns;
-    // h = p * silu(g) * u leaves in bf16 (the BF16 path keeps h in 16 bits)
+    // h = p * silu(g) * u leaves in bf16 (the BF16 and per-tensor FP8
+    // recipes hold h in 16 bits between the GEMMs).  Per-tensor FP8: the
+    // accumulator is first dequantised by deq[e], and the |max| of the
+    // rounded h of the group's rows is folded into amax_out.
     const int nb = ti.n0 + 64 * half;
     if (nb >= a.N) return;  // uniform across the warp
     const float p = rv ? a.prob[r] : 0.0f;
+    const float dq = EPI == EPI_SWIGLU_F8T ? a.deq[ti.e] : 1.0f;
     uint32_t hw[32];
+    uint32_t hmax = 0;  // |h| as bf16 bits (both halves), max over this lane's values
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       float h2[2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const float g = __uint_as_float(v[2 * j + i]);
-        const float u = __uint_as_float(v[64 + 2 * j + i]);
+        float g = __uint_as_float(v[2 * j + i]);
+        float u = __uint_as_float(v[64 + 2 * j + i]);
+        if constexpr (EPI == EPI_SWIGLU_F8T) {
+          g *= dq;
+          u *= dq;
+        }
         h2[i] = p * __fdividef(g, 1.0f + __expf(-g)) * u;
       }
       hw[j] = pack_bf16x2(h2[0], h2[1]);
+      if constexpr (EPI == EPI_SWIGLU_F8T) {
+        const uint32_t m = hw[j] & 0x7FFF7FFFu;  // non-negative bf16 compare as integers
+        hmax = max(hmax, max(m & 0xFFFFu, m >> 16));
+      }
     }
     warp_store_rows<32>(stage, rv ? a.q_out + (int64_t(r) * a.N + nb) * 2 : nullptr, hw, 128, lane);
+    if constexpr (EPI == EPI_SWIGLU_F8T) {
+      hmax = __reduce_max_sync(0xFFFFFFFFu, rv ? hmax : 0u);
+      if (lane == 0 && hmax) atomicMax(a.amax_out, hmax << 16);  // as float bits
+    }
   } else if constexpr (EPI == EPI_SWIGLU) {
     static_assert(BN == 256, "the gate_up epilogue pairs 128 gate with 128 up columns");
     // v[0:64] gate columns nb..nb+63, v[64:128] the matching up columns
@@ -316,6 +333,11 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
     if (nb >= a.N) return;  // uniform across the warp
     const int ncols = min(NC, a.N - nb);
     if constexpr (EPI == EPI_F24_ROWS) {
+      if (a.deq) {  // per-tensor FP8: dequantise first
+        const float dq = a.deq[ti.e];
+#pragma unroll
+        for (int i = 0; i < NC; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * dq);
+      }
       // keep the top 24 bits of each value, four values in three words, in place
 #pragma unroll
       for (int i = 0; i < NC / 4; ++i) {
@@ -519,7 +541,7 @@ __device__ __forceinline__ void load_b_stage(const GemmArgs& a, const CUtensorMa
                                              const Tile& ti, int kg, uint8_t* sb, uint8_t* ssfb, uint64_t* bar,
                                              uint32_t barp, uint32_t rank) {
   using C = Cfg<BN, PAIR>;
-  if constexpr (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16) {
+  if constexpr (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16 || EPI == EPI_SWIGLU_F8T) {
     const int rb = ti.n0 >> 7;
     const int64_t atom_g = (int64_t(2 * ti.e) * a.b_RT + rb) * a.b_KT + kg;
     const int64_t atom_u = (int64_t(2 * ti.e + 1) * a.b_RT + rb) * a.b_KT + kg;
@@ -770,11 +792,14 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
               else
                 tc_mma_mxf8(acc, ad, bd, make_idesc_mxf8(MMA_M, BN, kk, kk), sfa_t | (kk << 30),
                             sfb_t | (kk << 30), accum);
-            } else {
+            } else if constexpr (KIND == KIND_BF16) {
               if constexpr (PAIR)
                 tc_mma_bf16_pair(acc, ad, bd, make_idesc_bf16(MMA_M, BN), accum);
               else
                 tc_mma_bf16(acc, ad, bd, make_idesc_bf16(MMA_M, BN), accum);
+            } else {
+              static_assert(!PAIR, "per-tensor FP8 GEMMs are single-CTA");
+              tc_mma_f8(acc, ad, bd, make_idesc_f8(MMA_M, BN), accum);
             }
           }
           if constexpr (PAIR)
@@ -874,7 +899,7 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
         __syncwarp();
         release(buf);
       } else {
-        if constexpr (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16) {  // gate columns 64*half.., up columns 128 + 64*half..
+        if constexpr (EPI == EPI_SWIGLU || EPI == EPI_SWIGLU_BF16 || EPI == EPI_SWIGLU_F8T) {  // gate columns 64*half.., up columns 128 + 64*half..
           tmem_ld64(tl + 64 * half, v);
           tmem_ld64(tl + 128 + 64 * half, v + 64);
         } else if constexpr (C::NC == 128) {
@@ -1080,6 +1105,14 @@ cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps_in, const 
     }
   } else if (bn == 128) {
     if (epi == EPI_SWIGLU_BWD) return launch_epi<EPI_SWIGLU_BWD, 128, KIND_MXF8, false>(maps_in, a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_grouped_gemm_f8t(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st) {
+  switch (epi) {
+    case EPI_SWIGLU_F8T: return launch_epi<EPI_SWIGLU_F8T, 256, KIND_F8T, false>(maps, a, st);
+    case EPI_F24_ROWS: return launch_epi<EPI_F24_ROWS, 256, KIND_F8T, false>(maps, a, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -12,13 +12,15 @@ enum EpiKind : int {
   EPI_WGRAD = 3,         // weight gradients: one bf16 matrix per expert
   EPI_SWIGLU_BWD = 4,    // dgrad2 + ScaledSwiGLU backward: da (along 2I and tokens), h (tokens), dprob partials
   EPI_SWIGLU_BF16 = 5,   // BF16 path gate_up: h = p * silu(gate) * up written in bf16 (q_out)
-  EPI_F24_ROWS = 6       // down / dgrad1: the top 24 bits of each fp32 value (f24, see common.cuh), rows in permuted order
+  EPI_F24_ROWS = 6,      // down / dgrad1: the top 24 bits of each fp32 value (f24, see common.cuh), rows in permuted order
+  EPI_SWIGLU_F8T = 7     // per-tensor FP8 gate_up: dequantised by deq[e], h in bf16 (q_out) and its |max| (amax_out)
 };
 
 // Operand kind of the tensor-core MMA.
 enum MmaKind : int {
   KIND_MXF8 = 0,  // E4M3 x E4M3 with E8M0 block scales (kind::mxf8f6f4.block_scale)
-  KIND_BF16 = 1   // bf16 x bf16, no scales (kind::f16); operands are addressed as bytes, 64 values per K tile
+  KIND_BF16 = 1,  // bf16 x bf16, no scales (kind::f16); operands are addressed as bytes, 64 values per K tile
+  KIND_F8T = 2    // E4M3 x E4M3 without block scales (kind::f8f6f4): per-tensor FP8, dequantised in the epilogue
 };
 
 // One grouped GEMM  D = (A * SFA) (B * SFB)^T  over ragged expert groups.
@@ -63,6 +65,11 @@ struct GemmArgs {
   uint8_t* hcol;
   uint8_t* hcol_sf;
   float* dprob_part;
+  // per-tensor FP8 (KIND_F8T): per-expert dequantisation factor applied to
+  // the accumulator (EPI_SWIGLU_F8T and EPI_F24_ROWS; null: none), and the
+  // running |max| of h as float bits (EPI_SWIGLU_F8T)
+  const float* deq;
+  uint32_t* amax_out;
 };
 
 // Tensor maps: A 2-D {K, rows} with a 128 x 128 box; B either 3-D
@@ -93,5 +100,9 @@ cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const Gem
 // The tensor maps describe the bf16 matrices as bytes (inner extent 2K), and
 // num_kt / a_KT count 128-byte K tiles.
 cudaError_t launch_grouped_gemm_bf16(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);
+
+// Per-tensor FP8 operands (kind::f8f6f4, no block scales), bn = 256:
+// EPI_SWIGLU_F8T and EPI_F24_ROWS (with deq).
+cudaError_t launch_grouped_gemm_f8t(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);
 
 }  // namespace moe

@@ -456,6 +456,158 @@ __global__ void __launch_bounds__(256, 6) quant_rows_scatter_kernel(ScatterRowsA
   }
 }
 
+// ---------------------------------------------------------------------------
+// Per-tensor FP8 (the recipe Challenge 2 contrasts with MXFP8): one float32
+// factor per tensor, scale = 448 / amax of the whole tensor, codes
+// E4M3(float32(v * scale)).
+// ---------------------------------------------------------------------------
+
+// |max| of each group's bf16 values as float bits (atomicMax into amax[g],
+// zeroed by the caller): blockIdx.y = group, 8 values per thread and load.
+__global__ void __launch_bounds__(256) amax_bf16_kernel(const uint8_t* __restrict__ src, int64_t group_elems,
+                                                        uint32_t* amax) {
+  const int64_t g = blockIdx.y;
+  const uint4* p = reinterpret_cast<const uint4*>(src + g * group_elems * 2);
+  const int64_t n8 = group_elems / 8;
+  uint32_t m = 0;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
+    const uint4 v = __ldg(p + i);
+    // each 16-bit half with its sign cleared: non-negative bf16 values
+    // compare as integers (NaN above Inf above every finite value)
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+  }
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t wm[8];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t r = 0;
+    for (int w = 0; w < int(blockDim.x >> 5); ++w) r = max(r, wm[w]);
+    if (r) atomicMax(amax + g, r << 16);
+  }
+}
+
+// float32 factor from a tensor's |max| bits: 448 / amax (IEEE division),
+// the largest finite float32 where that overflows, 1 for 0 or non-finite.
+__device__ __forceinline__ float f8t_scale(uint32_t amax_bits) {
+  const float a = __uint_as_float(amax_bits);
+  if (a == 0.0f || !isfinite(a)) return 1.0f;
+  const float s = __fdiv_rn(448.0f, a);
+  return isfinite(s) ? s : 3.402823466e38f;
+}
+
+// phase 0: scale[0] (x), scale[2..2+2E) (W_gate_up, W_down per expert) and
+// deq[e] = 1 / (scale_x * scale_w1[e]); phase 1: scale[1] (h) and
+// deq[E + e] = 1 / (scale_h * scale_w2[e]).
+__global__ void f8t_scales_kernel(const uint32_t* amax, int E, int phase, float* scale, float* deq) {
+  const int i = threadIdx.x;
+  if (phase == 0) {
+    const float sx = f8t_scale(amax[0]);
+    if (i == 0) scale[0] = sx;
+    for (int j = i; j < 2 * E; j += blockDim.x) scale[2 + j] = f8t_scale(amax[2 + j]);
+    for (int e = i; e < E; e += blockDim.x) deq[e] = __frcp_rn(__fmul_rn(sx, f8t_scale(amax[2 + e])));
+  } else {
+    const float sh = f8t_scale(amax[1]);
+    if (i == 0) scale[1] = sh;
+    for (int e = i; e < E; e += blockDim.x) deq[E + e] = __frcp_rn(__fmul_rn(sh, f8t_scale(amax[2 + E + e])));
+  }
+}
+
+// Codes of bf16 values with one factor per group of group_elems values
+// (scale[g]); with rows_used, only the first *rows_used * row_elems values.
+__global__ void __launch_bounds__(256) f8t_quant_kernel(const uint8_t* __restrict__ src, int64_t n_elems,
+                                                        int64_t group_elems, const float* scale,
+                                                        const int32_t* rows_used, int64_t row_elems,
+                                                        uint8_t* q) {
+  int64_t n = n_elems;
+  if (rows_used) n = min(n, int64_t(max(*rows_used, 0)) * row_elems);
+  const int64_t n8 = n / 8;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
+    const float s = scale[(i * 8) / group_elems];
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i);
+    *reinterpret_cast<uint2*>(q + i * 8) =
+        make_uint2(pack4_e4m3(__fmul_rn(bf16lo(v.x), s), __fmul_rn(bf16hi(v.x), s), __fmul_rn(bf16lo(v.y), s),
+                              __fmul_rn(bf16hi(v.y), s)),
+                   pack4_e4m3(__fmul_rn(bf16lo(v.z), s), __fmul_rn(bf16hi(v.z), s), __fmul_rn(bf16lo(v.w), s),
+                              __fmul_rn(bf16hi(v.w), s)));
+  }
+}
+
+// x [T][H] -> codes of its k permuted rows slot_to_row[t*k + j] (factor
+// scale[0]); padding rows below *rows_used (row_to_slot < 0) get zeros.
+__global__ void __launch_bounds__(256) f8t_quant_scatter_kernel(const uint8_t* __restrict__ src, int64_t T,
+                                                                int64_t H, int32_t k,
+                                                                const int32_t* slot_to_row,
+                                                                const int32_t* row_to_slot,
+                                                                const int32_t* rows_used, const float* scale,
+                                                                uint8_t* q) {
+  const float s = scale[0];
+  const int64_t h8 = H / 8, n = T * h8;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += stride) {
+    const int64_t t = i / h8, c = (i - t * h8) * 8;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (t * H + c) * 2));
+    const uint2 w =
+        make_uint2(pack4_e4m3(__fmul_rn(bf16lo(v.x), s), __fmul_rn(bf16hi(v.x), s), __fmul_rn(bf16lo(v.y), s),
+                              __fmul_rn(bf16hi(v.y), s)),
+                   pack4_e4m3(__fmul_rn(bf16lo(v.z), s), __fmul_rn(bf16hi(v.z), s), __fmul_rn(bf16lo(v.w), s),
+                              __fmul_rn(bf16hi(v.w), s)));
+    for (int j = 0; j < k; ++j) {
+      const int32_t r = __ldg(slot_to_row + t * k + j);
+      if (r >= 0) *reinterpret_cast<uint2*>(q + int64_t(r) * H + c) = w;
+    }
+  }
+  const int64_t used = max(*rows_used, 0);
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < used * h8; i += stride) {
+    const int64_t r = i / h8;
+    if (__ldg(row_to_slot + r) < 0) *reinterpret_cast<uint2*>(q + r * H + (i - r * h8) * 8) = make_uint2(0u, 0u);
+  }
+}
+
+cudaError_t launch_f8t_amax(const uint8_t* src, int groups, int64_t group_elems, uint32_t* amax, cudaStream_t st) {
+  if (groups <= 0 || group_elems <= 0) return cudaSuccess;
+  if (group_elems % 8) return cudaErrorInvalidValue;
+  int64_t bx = cdiv(group_elems / 8, 256);
+  const int64_t cap = cdiv(int64_t(device_sm_count()) * 8, groups);
+  bx = bx > cap ? cap : bx;
+  amax_bf16_kernel<<<dim3(unsigned(bx > 0 ? bx : 1), unsigned(groups)), 256, 0, st>>>(src, group_elems, amax);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f8t_scales(const uint32_t* amax, int E, int phase, float* scale, float* deq, cudaStream_t st) {
+  f8t_scales_kernel<<<1, 256, 0, st>>>(amax, E, phase, scale, deq);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f8t_quant(const uint8_t* src, int64_t n_elems, int64_t group_elems, const float* scale,
+                             const int32_t* rows_used, int64_t row_elems, uint8_t* q, cudaStream_t st) {
+  if (n_elems <= 0) return cudaSuccess;
+  if (n_elems % 8 || group_elems % 8) return cudaErrorInvalidValue;
+  int64_t blocks = cdiv(n_elems / 8, 256);
+  const int64_t cap = int64_t(device_sm_count()) * 8;
+  blocks = blocks > cap ? cap : blocks;
+  f8t_quant_kernel<<<unsigned(blocks), 256, 0, st>>>(src, n_elems, group_elems, scale, rows_used, row_elems, q);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f8t_quant_scatter(const uint8_t* x, int64_t T, int64_t H, int32_t k, const int32_t* slot_to_row,
+                                     const int32_t* row_to_slot, const int32_t* rows_used, const float* scale,
+                                     uint8_t* q, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (H % 8) return cudaErrorInvalidValue;
+  int64_t blocks = cdiv(T * (H / 8), 256);
+  const int64_t cap = int64_t(device_sm_count()) * 8;
+  blocks = blocks > cap ? cap : blocks;
+  f8t_quant_scatter_kernel<<<unsigned(blocks), 256, 0, st>>>(x, T, H, k, slot_to_row, row_to_slot, rows_used, scale, q);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quant_rows(const QuantRowsArgs& args, cudaStream_t st) {
   const int64_t total = int64_t(args.groups) * cdiv(args.rows, 128) * 128 * cdiv(args.K, 128);
   if (total == 0) return cudaSuccess;

@@ -92,6 +92,24 @@ struct ScatterRowsArgs {
 
 cudaError_t launch_quant_rows_scatter(const ScatterRowsArgs& a, cudaStream_t st);
 
+// Per-tensor FP8 (one float32 factor 448 / amax per tensor):
+//  amax: |max| of each of `groups` bf16 groups as float bits (atomicMax into
+//        amax[g]; the caller zeroes it);
+//  scales: phase 0 -> scale[0] (x), scale[2..2+2E) (W_gate_up[e], W_down[e])
+//        and deq[e] = 1/(scale_x scale_w1[e]); phase 1 -> scale[1] (h) and
+//        deq[E+e] = 1/(scale_h scale_w2[e]), from amax[0..2+2E);
+//  quant: codes E4M3(float32(v * scale[g])) of bf16 values, groups of
+//        group_elems (optional device row count x row_elems bounds the work);
+//  quant_scatter: x [T][H] (factor scale[0]) to its k permuted rows, padding
+//        rows zero.
+cudaError_t launch_f8t_amax(const uint8_t* src, int groups, int64_t group_elems, uint32_t* amax, cudaStream_t st);
+cudaError_t launch_f8t_scales(const uint32_t* amax, int E, int phase, float* scale, float* deq, cudaStream_t st);
+cudaError_t launch_f8t_quant(const uint8_t* src, int64_t n_elems, int64_t group_elems, const float* scale,
+                             const int32_t* rows_used, int64_t row_elems, uint8_t* q, cudaStream_t st);
+cudaError_t launch_f8t_quant_scatter(const uint8_t* x, int64_t T, int64_t H, int32_t k, const int32_t* slot_to_row,
+                                     const int32_t* row_to_slot, const int32_t* rows_used, const float* scale,
+                                     uint8_t* q, cudaStream_t st);
+
 }  // namespace moe
 
 namespace moe {

@@ -168,6 +168,26 @@ class GroupedMLP:
                                      self.ws_bf16_bytes, self._stream())
         return self.out
 
+    def forward_fp8_tensor(self, x: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor) -> torch.Tensor:
+        """Per-tensor FP8 recipe forward (moe_grouped_mlp_fwd_fp8_tensor) on
+        the routing of the last permute / permute_index: x bf16 [T, H], w1
+        bf16 [E, 2I, H], w2 bf16 [E, H, I] -> out; the factors land in
+        self.fp8_scales (x, h, W_gate_up[E], W_down[E])."""
+        E, H, I = self.E, self.H, self.I
+        check_tensor(x, "x", torch.bfloat16, (self.T, H), self.dev)
+        check_tensor(w1, "w_gate_up", torch.bfloat16, (E, 2 * I, H), self.dev)
+        check_tensor(w2, "w_down", torch.bfloat16, (E, H, I), self.dev)
+        if getattr(self, "ws_f8t", None) is None:
+            self.ws_f8t_bytes = lib.moe_workspace_size(lib.MOE_OP_FWD_FP8_TENSOR, self.T, self.k, E, H, I)
+            self.ws_f8t = self._alloc.raw(self.ws_f8t_bytes, "ws_f8t")
+            self.fp8_scales = self._alloc.typed((2 + 2 * E,), torch.float32, "fp8_scales")
+        lib.moe_grouped_mlp_fwd_fp8_tensor(w1.data_ptr(), w2.data_ptr(), self.T, H, I, E, self.k, self.rows_cap,
+                                           _ptr(self.split_sizes), _ptr(self.group_offsets), _ptr(self.row_to_slot),
+                                           _ptr(self.slot_to_row), _ptr(self.prob_perm), x.data_ptr(),
+                                           _ptr(self.out), _ptr(self.fp8_scales), _ptr(self.ws_f8t),
+                                           self.ws_f8t_bytes, self._stream())
+        return self.out
+
     def check_guards(self):
         """Names of the buffers written past their end (layers built with
         guard > 0; always empty otherwise)."""

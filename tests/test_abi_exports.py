@@ -147,6 +147,22 @@ def test_backward_argument_errors():
     assert f(*_bwd_args(ws_bytes=need - 1)) == WORKSPACE
 
 
+def test_fp8_tensor_forward_argument_errors():
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    f = lib._lib.moe_grouped_mlp_fwd_fp8_tensor
+    rc = lib.moe_padded_rows(64, 2, 4)
+    args = lambda H=256, ws=P, wsb=1 << 40, x=P, sc=None: (P, P, 64, H, 512, 4, 2, rc, P, P, P, P, P, x, P, sc, ws,
+                                                          wsb, None)
+    assert f(*args(x=None)) == INVALID                                      # x missing with T > 0
+    assert f(*args(x=M)) == INVALID                                         # misaligned x
+    assert f(*args(sc=P + 2)) == INVALID                                    # misaligned factor output
+    assert f(*args(H=48)) == UNSUPPORTED
+    need = lib.moe_workspace_size(lib.MOE_OP_FWD_FP8_TENSOR, 64, 2, 4, 256, 512)
+    assert need > 0
+    assert f(*args(wsb=need - 1)) == WORKSPACE
+    assert f(*args(ws=P + 128)) == WORKSPACE                                # 256-byte aligned workspace
+
+
 def test_quantise_and_combine_argument_errors():
     from mxfp8_grouped_gemm_x32_b200 import lib
     q = lib._lib.moe_mlp_quantize_mxfp8
