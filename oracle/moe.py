@@ -191,13 +191,16 @@ def forward(x, w1, w2, topk_idx, topk_prob, *, quantize=True, round_saved=True,
 # ----------------------------------------------------------------------------
 
 
-def backward(fwd, x, w1, w2, topk_prob, dy, *, quantize=True, experts=None):
+def backward(fwd, x, w1, w2, topk_prob, dy, *, quantize=True, experts=None, bf16_held=False):
     """Backward pass given the forward's dict.
 
     dy [T, H] is the gradient of the combined output.  Returns dX [T, H],
     dW1 [E, 2I, H], dW2 [E, H, I] (float64 and bf16 bits) and dprob
     float32 [T, k] in slot order, plus the intermediates dh, da and h_b
     (per permuted row) for kernel-level checks.
+    ``bf16_held=True`` (with ``quantize=False``: the BF16 recipe, whose
+    tensors between the GEMMs are bf16) rounds da = [dg, du] and the
+    recomputed h to bf16 before the GEMMs that consume them.
     """
     x = np.asarray(x, dtype=np.float64)
     dy = np.asarray(dy, dtype=np.float64)
@@ -237,6 +240,8 @@ def backward(fwd, x, w1, w2, topk_prob, dy, *, quantize=True, experts=None):
         dp_rows[r0:r1] = np.sum(dh * s * u, axis=1)
         hb = pe * s * u
         da = np.concatenate([dg, du], axis=1)
+        if bf16_held:
+            hb, da = bf16_round(hb), bf16_round(da)
         # wgrad2: dW2_e = dy^T h, contraction over the group's tokens
         if quantize:
             dyc = mxfp8.roundtrip_cols_grouped(dyg, [r1 - r0])[0]

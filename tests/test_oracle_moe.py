@@ -140,6 +140,52 @@ def test_identity_expert_bf16_path():
     assert np.allclose(out2[:, :I], h, rtol=1e-15, atol=0)
 
 
+def _is_rne_bf16_of(v, exact):
+    """v holds the bf16 values nearest to `exact` (ties to even), checked by
+    brute force over the neighbouring bf16 values."""
+    bits = v.astype(np.float32).view(np.uint32)
+    if not (np.all(v.astype(np.float32).astype(np.float64) == v) and np.all(bits & 0xFFFF == 0)):
+        return False
+    nb = bits >> 16
+    for step in (-1, 1):
+        w = ((nb.astype(np.int64) + step).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        dv, dw = np.abs(v - exact), np.abs(w - exact)
+        if not np.all((dv < dw) | ((dv == dw) & (nb % 2 == 0))):
+            return False
+    return True
+
+
+def test_identity_expert_bf16_backward():
+    """BF16 recipe backward (da and the recomputed h held in bf16): with the
+    identity expert (W_gate_up = I, W_down = [I; 0], p = 1, k = 1) dX is
+    da = [dg, du] rounded to bf16 and dW_down's top block is dy1^T bf16(h),
+    with dg, du, h written out here from the ScaledSwiGLU backward's
+    definition (the saved activation A = x in bf16)."""
+    I, T = 32, 24
+    H = 2 * I
+    rng = np.random.default_rng(9)
+    x = moe.bf16_round(rng.standard_normal((T, H)))
+    dy = moe.bf16_round(rng.standard_normal((T, H)))
+    w1 = np.eye(2 * I)[None]
+    w2 = np.concatenate([np.eye(I), np.zeros((H - I, I))], axis=0)[None]
+    idx = np.zeros((T, 1), np.int32)
+    prob = np.ones((T, 1), np.float32)
+    fwd = moe.forward(x, w1, w2, idx, prob, quantize=False, h_bf16=True)
+    b = moe.backward(fwd, x, w1, w2, prob, dy, quantize=False, bf16_held=True)
+    g, u, dh = x[:, :I], x[:, I:], dy[:, :I]
+    sig = 1.0 / (1.0 + np.exp(-g))
+    dg = dh * u * sig * (1.0 + g * (1.0 - sig))
+    du = dh * g * sig
+    h = g * sig * u
+    assert _is_rne_bf16_of(b["dX"][:, :I], dg) and _is_rne_bf16_of(b["dX"][:, I:], du)
+    assert _is_rne_bf16_of(b["h_b"], h)
+    assert np.allclose(b["dW2"][0][:I], dy[:, :I].T @ b["h_b"], rtol=1e-12, atol=0)
+    assert np.all(b["dW2"][0][I:] == dy[:, I:].T @ b["h_b"])
+    # without the bf16 step da passes through unrounded
+    b2 = moe.backward(fwd, x, w1, w2, prob, dy, quantize=False)
+    assert np.allclose(b2["dX"][:, :I], dg, rtol=1e-13, atol=0)
+
+
 def test_permutation_invariants(tiny):
     cfg, inp = tiny
     perm, split = moe.permute(inp["topk_idx"], cfg.E)
