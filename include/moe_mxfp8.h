@@ -94,6 +94,7 @@ typedef enum {
 #define MOE_OP_BWD 3
 #define MOE_OP_FWD_BF16 4
 #define MOE_OP_FWD_FP8_TENSOR 5
+#define MOE_OP_BWD_BF16 6
 
 /* Limits checked on the host. */
 #define MOE_MAX_EXPERTS 256
@@ -109,7 +110,8 @@ int64_t moe_mx_scale_bytes(int32_t groups, int64_t rows, int64_t k);
  * for every routing (= roundup(T*k + 127*E, 128)). -1 on invalid sizes. */
 int64_t moe_padded_rows(int32_t T, int32_t k, int32_t E);
 
-/* Workspace bytes for op MOE_OP_PERMUTE / MOE_OP_FWD / MOE_OP_BWD of a layer
+/* Workspace bytes for op MOE_OP_PERMUTE / MOE_OP_FWD / MOE_OP_BWD /
+ * MOE_OP_FWD_BF16 / MOE_OP_FWD_FP8_TENSOR / MOE_OP_BWD_BF16 of a layer
  * (T tokens, top-k, E experts, hidden H, intermediate I).  -1 if invalid. */
 int64_t moe_workspace_size(int32_t op, int32_t T, int32_t k, int32_t E, int32_t H, int32_t I);
 
@@ -280,13 +282,17 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
  *   routing    split_sizes, group_offsets, row_to_slot, slot_to_row,
  *              prob_perm from moe_permute (xq may be NULL there).
  *   x          bf16 [T][H];  out bf16 [T][H].
+ *   saved_a    bf16 [rows_cap][2I] or NULL: A rounded to bf16, kept for
+ *              moe_grouped_mlp_bwd_bf16 (rows of the groups, padding rows
+ *              included, are written; 16-byte aligned).
  *   workspace  >= moe_workspace_size(MOE_OP_FWD_BF16, T, k, E, H, I).
  * Limits as moe_grouped_mlp_fwd. */
 moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down, int32_t T, int32_t H, int32_t I,
                                       int32_t E, int32_t k, int64_t rows_cap, const int32_t* split_sizes,
                                       const int32_t* group_offsets, const int32_t* row_to_slot,
                                       const int32_t* slot_to_row, const float* prob_perm, const void* x,
-                                      void* out, void* workspace, size_t workspace_bytes, moe_stream_t stream);
+                                      void* out, void* saved_a, void* workspace, size_t workspace_bytes,
+                                      moe_stream_t stream);
 
 /* Per-tensor FP8 grouped MLP forward: the FP8 recipe Challenge 2 contrasts
  * with MXFP8 -- one float32 factor for a whole tensor instead of one per 32
@@ -393,6 +399,34 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
                                  void* dW2,
                                  float* dprob, void* workspace, size_t workspace_bytes,
                                  moe_stream_t stream);
+
+/* BF16 recipe backward: the same gradients as moe_grouped_mlp_bwd with BF16
+ * operands and no quantisation (Challenge 2: both recipes run the layer; the
+ * BF16 one keeps every tensor between the GEMMs in 16 bits).  dh = dy W_down
+ * runs on the bf16 tensor cores (fp32 accumulation) and its epilogue computes
+ * the ScaledSwiGLU backward from saved_a, writing da = [dg, du] and the
+ * recomputed h = p*s*u in bf16 (da along 2I and along tokens, h along
+ * tokens); dW_down_e = dy_e^T h_e, dx = da W_gate_up (fp32 rows),
+ * dW_gate_up_e = da_e^T x_e; dX[t] = sum_j dx[row(t,j)] (fp32, ascending j,
+ * one bf16 rounding); dprob as moe_grouped_mlp_bwd.  The weights are taken in
+ * the forward's layout and transposed in the workspace on every call.
+ *   w_gate_up  bf16 [E][2I][H]; w_down bf16 [E][H][I] (as the forward).
+ *   routing    as the forward, slot_to_row included.
+ *   dY         bf16 [T][H].  saved_a bf16 [rows_cap][2I] from
+ *              moe_grouped_mlp_fwd_bf16 (32-byte aligned).
+ *   x          bf16 [T][H], the forward's input.
+ * Outputs: dX bf16 [T][H]; dW1 bf16 [E][2I][H]; dW2 bf16 [E][H][I];
+ *   dprob float [T][k] (slot order).
+ *   workspace  >= moe_workspace_size(MOE_OP_BWD_BF16, T, k, E, H, I),
+ *              256-byte aligned.
+ * Pointers 16-byte aligned (MOE_ERR_INVALID otherwise); limits as
+ * moe_grouped_mlp_bwd. */
+moe_status_t moe_grouped_mlp_bwd_bf16(const void* w_gate_up, const void* w_down, int32_t T, int32_t H, int32_t I,
+                                      int32_t E, int32_t k, int64_t rows_cap, const int32_t* split_sizes,
+                                      const int32_t* group_offsets, const int32_t* row_to_slot,
+                                      const int32_t* slot_to_row, const float* prob_perm, const void* dY,
+                                      const void* saved_a, const void* x, void* dX, void* dW1, void* dW2,
+                                      float* dprob, void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /* ------------------------------------------------------------- status --- */
 

@@ -12,8 +12,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmoe_mxfp8.so")
-SOURCES = ["moe_mxfp8_all.cu", "api.cu", "gemm.cu", "permute.cu", "quant.cu", "swiglu_bwd.cu", "noalloc.cu", "router.cu", "scales.cu",
-           "common.cuh", "gemm.cuh", "permute.cuh", "quant.cuh", "swiglu_bwd.cuh"]
+SOURCES = ["moe_mxfp8_all.cu", "api.cu", "gemm.cu", "permute.cu", "quant.cu", "swiglu_bwd.cu", "noalloc.cu", "router.cu",
+           "scales.cu", "transpose.cu", "common.cuh", "gemm.cuh", "permute.cuh", "quant.cuh", "swiglu_bwd.cuh",
+           "router.cuh", "scales.cuh", "transpose.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared", "-diag-suppress", "550"]
 

@@ -10,6 +10,7 @@
 #include "permute.cuh"
 #include "quant.cuh"
 #include "swiglu_bwd.cuh"
+#include "transpose.cuh"
 #include "router.cuh"
 
 namespace moe {
@@ -159,6 +160,30 @@ BwdWs carve_bwd(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t r
   return w;
 }
 
+// BF16 recipe backward workspace: the weights transposed (the dgrad GEMMs
+// contract them over their other dimension), dy gathered to permuted rows and
+// transposed, da along 2I and along tokens, h along tokens, x gathered and
+// transposed, fp32 dgrad rows and the dprob partial sums -- all bf16 but the
+// last two.
+struct BwdBf16Ws {
+  uint8_t *w2t, *w1t, *dyp, *dyc, *da, *dac, *hc, *xc, *dx, *dpp;
+};
+BwdBf16Ws carve_bwd_bf16(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t E, int64_t rows_cap) {
+  (void)T; (void)k;
+  BwdBf16Ws w{};
+  w.w2t = c.take(E * I * H * 2);
+  w.w1t = c.take(E * H * 2 * I * 2);
+  w.dyp = c.take(rows_cap * H * 2);
+  w.dyc = c.take(H * rows_cap * 2);
+  w.da = c.take(rows_cap * 2 * I * 2);
+  w.dac = c.take(2 * I * rows_cap * 2);
+  w.hc = c.take(I * rows_cap * 2);
+  w.xc = c.take(H * rows_cap * 2);
+  w.dx = c.take(rows_cap * H * 4);
+  w.dpp = c.take(I / 64 * rows_cap * 4);
+  return w;
+}
+
 bool layer_dims_ok(int32_t T, int32_t H, int32_t I, int32_t E, int32_t k) {
   return T >= 0 && H > 0 && I > 0 && E > 0 && k > 0 && k <= E && E <= MOE_MAX_EXPERTS &&
          H % 32 == 0 && I % 64 == 0 && int64_t(T) * k < (int64_t(1) << 30);
@@ -245,6 +270,10 @@ int64_t moe_workspace_size(int32_t op, int32_t T, int32_t k, int32_t E, int32_t 
     case MOE_OP_FWD_FP8_TENSOR:
       if (H <= 0 || I <= 0) return -1;
       carve_fwd_f8t(c, T, k, H, I, E, rows_cap);
+      return c.off;
+    case MOE_OP_BWD_BF16:
+      if (H <= 0 || I <= 0) return -1;
+      carve_bwd_bf16(c, T, k, H, I, E, rows_cap);
       return c.off;
   }
   return -1;
@@ -399,7 +428,8 @@ moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down,
                                       int32_t E, int32_t k, int64_t rows_cap, const int32_t* split_sizes,
                                       const int32_t* group_offsets, const int32_t* row_to_slot,
                                       const int32_t* slot_to_row, const float* prob_perm, const void* x,
-                                      void* out, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+                                      void* out, void* saved_a, void* workspace, size_t workspace_bytes,
+                                      moe_stream_t stream) {
   if (!w_gate_up || !w_down || !split_sizes || !group_offsets || !row_to_slot || !prob_perm ||
       (T > 0 && (!x || !out || !slot_to_row)))
     return MOE_ERR_INVALID;
@@ -407,6 +437,7 @@ moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down,
   if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
   for (const void* p : {w_gate_up, w_down, x, (const void*)out})
     if (!al16(p)) return MOE_ERR_INVALID;
+  if (saved_a && !al16(saved_a)) return MOE_ERR_INVALID;
   Carver c{static_cast<uint8_t*>(workspace)};
   FwdBf16Ws w = carve_fwd_bf16(c, T, k, H, I, rows_cap);
   if (!workspace || int64_t(workspace_bytes) < c.off) return MOE_ERR_WORKSPACE;
@@ -432,6 +463,7 @@ moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down,
   g1.mode = 0; g1.E = E; g1.N = I; g1.num_kt = int32_t(cdiv(2 * int64_t(H), 128)); g1.n_tiles = int32_t(cdiv(I, 128));
   g1.group_offsets = group_offsets; g1.split_sizes = split_sizes;
   g1.prob = prob_perm; g1.row_to_slot = row_to_slot; g1.q_out = w.h;
+  g1.out2 = static_cast<uint8_t*>(saved_a);
   {
     TimeScope ts(st, "gemm_gate_up_swiglu_bf16");
     if (launch_grouped_gemm_bf16(EPI_SWIGLU_BF16, m1, g1, st) != cudaSuccess) return MOE_ERR_CUDA;
@@ -648,6 +680,122 @@ moe_status_t moe_grouped_mlp_bwd(const uint8_t* w2tq, const uint8_t* w2tsf, cons
   {
     TimeScope ts(st, "gemm_wgrad_gate_up");
     if (launch_grouped_gemm(EPI_WGRAD, 256, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_grouped_mlp_bwd_bf16(const void* w_gate_up, const void* w_down, int32_t T, int32_t H, int32_t I,
+                                      int32_t E, int32_t k, int64_t rows_cap, const int32_t* split_sizes,
+                                      const int32_t* group_offsets, const int32_t* row_to_slot,
+                                      const int32_t* slot_to_row, const float* prob_perm, const void* dY,
+                                      const void* saved_a, const void* x, void* dX, void* dW1, void* dW2,
+                                      float* dprob, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  if (!w_gate_up || !w_down || !split_sizes || !group_offsets || !row_to_slot || !prob_perm || !saved_a ||
+      !dW1 || !dW2 || (T > 0 && (!slot_to_row || !dY || !dX || !dprob || !x)))
+    return MOE_ERR_INVALID;
+  if (!layer_dims_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
+  for (const void* p : {w_gate_up, w_down, dY, x, (const void*)dX, (const void*)dW1, (const void*)dW2})
+    if (!al16(p)) return MOE_ERR_INVALID;
+  if (!al32(saved_a) || !al256(workspace)) return MOE_ERR_INVALID;  // 256-bit loads and stores
+  Carver c{static_cast<uint8_t*>(workspace)};
+  BwdBf16Ws w = carve_bwd_bf16(c, T, k, H, I, E, rows_cap);
+  if (!workspace || int64_t(workspace_bytes) < c.off) return MOE_ERR_WORKSPACE;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t I2 = 2 * int64_t(I);
+
+  // the weights transposed: W_down^T [E][I][H], W_gate_up^T [E][H][2I]
+  {
+    TimeScope ts(st, "weights_transpose_bf16");
+    TransposeArgs t2{static_cast<const uint16_t*>(w_down), reinterpret_cast<uint16_t*>(w.w2t), E, H, I, H,
+                     nullptr, k, nullptr, nullptr};
+    TransposeArgs t1{static_cast<const uint16_t*>(w_gate_up), reinterpret_cast<uint16_t*>(w.w1t), E, I2, H, I2,
+                     nullptr, k, nullptr, nullptr};
+    if (launch_transpose_bf16(t2, st) != cudaSuccess || launch_transpose_bf16(t1, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  // dy gathered to permuted rows, in both orientations (one read of dY)
+  {
+    TimeScope ts(st, "dy_gather_bf16");
+    TransposeArgs td{static_cast<const uint16_t*>(dY), reinterpret_cast<uint16_t*>(w.dyc), 1, rows_cap, H, rows_cap,
+                     row_to_slot, k, group_offsets + E, reinterpret_cast<uint16_t*>(w.dyp)};
+    if (launch_transpose_bf16(td, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
+  // dgrad2 + ScaledSwiGLU backward: dh = dy W_down (contraction over H) in
+  // TMEM; the epilogue writes da = [dg | du] along 2I and along tokens and h
+  // along tokens (bf16), and dprob partial sums per 64-column chunk
+  GemmMaps m;
+  if (make_map_2d(&m.a, w.dyp, 2 * int64_t(H), rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m.b, w.w2t, 2 * int64_t(H), I, E, gemm_b_box(128)) != cudaSuccess) return MOE_ERR_CUDA;
+  GemmArgs g{};
+  g.mode = 0; g.E = E; g.N = I; g.num_kt = int32_t(cdiv(2 * int64_t(H), 128)); g.n_tiles = int32_t(cdiv(I, 128));
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes;
+  g.prob = prob_perm; g.saved = static_cast<const uint8_t*>(saved_a); g.rows_cap = rows_cap;
+  g.daq = w.da; g.dacol = w.dac; g.hcol = w.hc;
+  g.dprob_part = reinterpret_cast<float*>(w.dpp);
+  {
+    TimeScope ts(st, "gemm_dgrad_down_swiglu_bf16");
+    if (launch_grouped_gemm_bf16(EPI_SWIGLU_BWD_BF16, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  {
+    TimeScope ts(st, "dprob_reduce");
+    if (launch_dprob_reduce(group_offsets, E, row_to_slot, rows_cap, reinterpret_cast<const float*>(w.dpp),
+                            I / 64, dprob, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+
+  // wgrad2: dW_down_e = dy_e^T h_e (contraction over the group's tokens,
+  // 64 per 128-byte K tile)
+  if (make_map_2d(&m.a, w.dyc, 2 * rows_cap, H, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_2d(&m.b, w.hc, 2 * rows_cap, I, gemm_b_box(256)) != cudaSuccess) return MOE_ERR_CUDA;
+  g = GemmArgs{};
+  g.mode = 1; g.k_shift = 6; g.E = E; g.N = I; g.n_tiles = int32_t(cdiv(I, 256));
+  g.m_tiles = int32_t(cdiv(H, 128)); g.M_out = H;
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes;
+  g.out = static_cast<uint8_t*>(dW2); g.ld_out = I; g.out_group_stride = int64_t(H) * I;
+  {
+    TimeScope ts(st, "gemm_wgrad_down_bf16");
+    if (launch_grouped_gemm_bf16(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
+  // dgrad1: dx = da W_gate_up (contraction over 2I), fp32 rows in permuted
+  // order; the combine gathers a token's k rows through slot_to_row
+  if (make_map_2d(&m.a, w.da, 2 * I2, rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m.b, w.w1t, 2 * I2, H, E, gemm_b_box(256)) != cudaSuccess) return MOE_ERR_CUDA;
+  g = GemmArgs{};
+  g.mode = 0; g.E = E; g.N = H; g.num_kt = int32_t(cdiv(2 * I2, 128)); g.n_tiles = int32_t(cdiv(H, 256));
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes; g.rows_cap = rows_cap;
+  g.out = w.dx; g.ld_out = H;
+  {
+    TimeScope ts(st, "gemm_dgrad_gate_up_bf16");
+    if (launch_grouped_gemm_bf16(EPI_F32_ROWS, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  {
+    TimeScope ts(st, "combine_dx");
+    if (launch_combine(w.dx, COMBINE_F32, slot_to_row, T, k, H, dX, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
+  // x gathered to permuted rows and transposed (the operand of wgrad1)
+  {
+    TimeScope ts(st, "x_gather_cols_bf16");
+    TransposeArgs tx{static_cast<const uint16_t*>(x), reinterpret_cast<uint16_t*>(w.xc), 1, rows_cap, H, rows_cap,
+                     row_to_slot, k, group_offsets + E, nullptr};
+    if (launch_transpose_bf16(tx, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
+  // wgrad1: dW_gate_up_e = da_e^T x_e (contraction over the group's tokens)
+  if (make_map_2d(&m.a, w.dac, 2 * rows_cap, I2, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_2d(&m.b, w.xc, 2 * rows_cap, H, gemm_b_box(256)) != cudaSuccess) return MOE_ERR_CUDA;
+  g = GemmArgs{};
+  g.mode = 1; g.k_shift = 6; g.E = E; g.N = H; g.n_tiles = int32_t(cdiv(H, 256));
+  g.m_tiles = int32_t(cdiv(I2, 128)); g.M_out = int32_t(I2);
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes;
+  g.out = static_cast<uint8_t*>(dW1); g.ld_out = H; g.out_group_stride = I2 * H;
+  {
+    TimeScope ts(st, "gemm_wgrad_gate_up_bf16");
+    if (launch_grouped_gemm_bf16(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
   return MOE_OK;
 }

@@ -145,8 +145,11 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, co
     ti.e = e;
     ti.m0 = m_idx << MSHIFT;
     ti.n0 = n_idx * BN;
-    ti.kt0 = go[e] >> 7;
-    ti.nkt = (go[e + 1] - go[e]) >> 7;
+    // log2 of the tokens in a 128-byte K tile: 7 (8-bit operands) or 6 (bf16;
+    // only the weight gradients run in mode 1)
+    const int ks = (EPI == EPI_WGRAD && a.k_shift) ? a.k_shift : 7;
+    ti.kt0 = go[e] >> ks;
+    ti.nkt = (go[e + 1] - go[e]) >> ks;
     ti.row_end = a.M_out;
     ti.row_lim = 0x7FFFFFFF;
   }
@@ -249,6 +252,18 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
     // rounded h of the group's rows is folded into amax_out.
     const int nb = ti.n0 + 64 * half;
     if (nb >= a.N) return;  // uniform across the warp
+    if (EPI == EPI_SWIGLU_BF16 && a.out2) {
+      // saved A in bf16 (the BF16 recipe's backward recomputes g, u, h from it)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t t[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          t[j] = pack_bf16x2(__uint_as_float(v[32 * c + 2 * j]), __uint_as_float(v[32 * c + 2 * j + 1]));
+        const int64_t col = (c < 2 ? 0 : a.N) + nb + 32 * (c & 1);
+        warp_store_rows<16>(stage, rv ? a.out2 + (int64_t(r) * 2 * a.N + col) * 2 : nullptr, t, 64, lane);
+      }
+    }
     const float p = rv ? a.prob[r] : 0.0f;
     const float dq = EPI == EPI_SWIGLU_F8T ? a.deq[ti.e] : 1.0f;
     uint32_t hw[32];
@@ -459,10 +474,40 @@ __device__ __forceinline__ void prefetch_saved(const GemmArgs& a, const Tile& ti
   asm volatile("prefetch.global.L2 [%0];" ::"l"(g + int64_t(a.N) * 2));
 }
 
+// 32 fp32 values -> 16 bf16x2 words (round to nearest even), stored as 64
+// bytes with two 256-bit stores (dst 32-byte aligned).
+__device__ __forceinline__ void bf16_store32(const float* o, uint8_t* dst) {
+  uint32_t w[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(o[2 * j], o[2 * j + 1]);
+  stg256(dst, w);
+  stg256(dst + 32, w + 8);
+}
+
+// Columns of a 32 x 32 chunk held one row per lane, in bf16: lane c writes
+// the 32 values of column col0 + c over the warp's rows to
+// dst + ((col0 + c) * ld + rb) * 2.
+__device__ __forceinline__ void bf16_cols32(const float* o, uint32_t* stage, int lane, uint8_t* dst, int64_t col0,
+                                            int64_t ld, int64_t rb) {
+  __syncwarp();
+  float4* srow = reinterpret_cast<float4*>(stage + lane * TP_W);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) srow[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+  __syncwarp();
+  float f[32];
+#pragma unroll
+  for (int rr = 0; rr < 32; ++rr) f[rr] = __uint_as_float(stage[rr * TP_W + lane]);
+  bf16_store32(f, dst + ((col0 + lane) * ld + rb) * 2);
+}
+
 // `cur` holds g/u of chunk 0 of this tile on entry; the loads of the next
 // chunk (chunk 1, then chunk 0 of the warp's next tile `tn`, if any) are
 // issued once a chunk's dh has been read for the last time, so they land
 // while its last pass runs.  On return `cur` holds chunk 0 of `tn`.
+// MXF: the MXFP8 outputs (codes and block scales of da along 2I and along
+// tokens, of h along tokens); otherwise the BF16 recipe's (da along 2I,
+// da and h along tokens, all bf16).
+template <bool MXF>
 __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Tile& ti, const Tile* tn, uint32_t tl,
                                                     int q, int half, int lane, uint32_t* stage, GuChunk& cur) {
   const int I = a.N;
@@ -497,8 +542,13 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
       o[e] = (__uint_as_float(d[e]) * p) * (u * sg) * fmaf(g, 1.0f - sg, 1.0f);
       sv[e] = g * sg;
     }
-    sb_dg |= encode32_store(o, a.daq + r * I2 + cc) << (8 * j);
-    quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, cc, a.rows_cap, rb, KTt);
+    if constexpr (MXF) {
+      sb_dg |= encode32_store(o, a.daq + r * I2 + cc) << (8 * j);
+      quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, cc, a.rows_cap, rb, KTt);
+    } else {
+      bf16_store32(o, a.daq + (r * I2 + cc) * 2);
+      bf16_cols32(o, stage, lane, a.dacol, cc, a.rows_cap, rb);
+    }
     // du = dh*p*s, quantised along 2I (columns I+cc..) and along tokens;
     // dprob partial sum dh*s*u
 #pragma unroll
@@ -506,8 +556,13 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
       o[e] = (__uint_as_float(d[e]) * p) * sv[e];
       dps = fmaf(__uint_as_float(d[e]), sv[e] * gu_elem(cur.u, e), dps);
     }
-    sb_du |= encode32_store(o, a.daq + r * I2 + I + cc) << (8 * j);
-    quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, int64_t(I) + cc, a.rows_cap, rb, KTt);
+    if constexpr (MXF) {
+      sb_du |= encode32_store(o, a.daq + r * I2 + I + cc) << (8 * j);
+      quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, int64_t(I) + cc, a.rows_cap, rb, KTt);
+    } else {
+      bf16_store32(o, a.daq + (r * I2 + I + cc) * 2);
+      bf16_cols32(o, stage, lane, a.dacol, int64_t(I) + cc, a.rows_cap, rb);
+    }
     // dh and g are used up: load the next chunk's g/u now (it lands during
     // the last pass and the start of the next chunk)
     GuChunk nxt;
@@ -519,13 +574,18 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
     // gradient)
 #pragma unroll
     for (int e = 0; e < 32; ++e) o[e] = p * (sv[e] * gu_elem(cur.u, e));
-    quant_cols32(o, stage, lane, a.hcol, a.hcol_sf, cc, a.rows_cap, rb, KTt);
+    if constexpr (MXF)
+      quant_cols32(o, stage, lane, a.hcol, a.hcol_sf, cc, a.rows_cap, rb, KTt);
+    else
+      bf16_cols32(o, stage, lane, a.hcol, cc, a.rows_cap, rb);
     cur = nxt;
   }
-  // scale bytes of dg and du along 2I: blocks cb/32, cb/32+1 (cb % 64 == 0,
-  // so the pair shares a 4-byte group of the atom)
-  *reinterpret_cast<uint16_t*>(a.daq_sf + sf_offset(0, r, cb >> 5, 0, KT2)) = uint16_t(sb_dg);
-  *reinterpret_cast<uint16_t*>(a.daq_sf + sf_offset(0, r, (int64_t(I) + cb) >> 5, 0, KT2)) = uint16_t(sb_du);
+  if constexpr (MXF) {
+    // scale bytes of dg and du along 2I: blocks cb/32, cb/32+1 (cb % 64 == 0,
+    // so the pair shares a 4-byte group of the atom)
+    *reinterpret_cast<uint16_t*>(a.daq_sf + sf_offset(0, r, cb >> 5, 0, KT2)) = uint16_t(sb_dg);
+    *reinterpret_cast<uint16_t*>(a.daq_sf + sf_offset(0, r, (int64_t(I) + cb) >> 5, 0, KT2)) = uint16_t(sb_du);
+  }
   a.dprob_part[int64_t(cb >> 6) * a.rows_cap + r] = dps;
 }
 
@@ -853,8 +913,9 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
           mbar_arrive(&acc_empty[buf]);
       }
     };
-    GuChunk gu;  // EPI_SWIGLU_BWD: g/u of the next chunk to process
-    if constexpr (EPI == EPI_SWIGLU_BWD)
+    constexpr bool SWB = EPI == EPI_SWIGLU_BWD || EPI == EPI_SWIGLU_BWD_BF16;
+    GuChunk gu;  // fused ScaledSwiGLU backward: g/u of the next chunk to process
+    if constexpr (SWB)
       if (cid < ntiles) {
         bool none;
         load_gu(a, my_tile(cid, &none), q, half, lane, 0, gu);
@@ -863,7 +924,7 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
       bool none;
       const Tile ti = my_tile(t, &none);
       const bool has_next = t + ncl < ntiles;
-      if constexpr (EPI == EPI_SWIGLU_BWD)  // one tile ahead
+      if constexpr (SWB)  // one tile ahead
         if (has_next) {
           bool nn;
           prefetch_saved(a, my_tile(t + ncl, &nn), q, half, lane);
@@ -882,7 +943,7 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
       const uint32_t tl = tmem + (uint32_t(32 * q) << 16) + buf * C::ACC_STRIDE;
       if (none) {
         // rows of another expert: nothing to read or write
-        if constexpr (EPI == EPI_SWIGLU_BWD)
+        if constexpr (SWB)
           if (has_next) {
             bool nn;
             load_gu(a, my_tile(t + ncl, &nn), q, half, lane, 0, gu);
@@ -890,11 +951,11 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         release(buf);
-      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+      } else if constexpr (SWB) {
         // reads TMEM chunk by chunk; the other accumulator keeps the MMAs busy
         bool nn;
         const Tile tn = my_tile(has_next ? t + ncl : t, &nn);
-        epilogue_swiglu_bwd(a, ti, has_next ? &tn : nullptr, tl, q, half, lane, stage, gu);
+        epilogue_swiglu_bwd<EPI == EPI_SWIGLU_BWD>(a, ti, has_next ? &tn : nullptr, tl, q, half, lane, stage, gu);
         tc_fence_before();
         __syncwarp();
         release(buf);
@@ -1122,12 +1183,17 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const GemmMaps& maps, const GemmAr
     switch (epi) {
       case EPI_SWIGLU_BF16: return launch_epi<EPI_SWIGLU_BF16, 256, KIND_BF16, true>(maps, a, st);
       case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256, KIND_BF16, true>(maps, a, st);
+      case EPI_WGRAD: return launch_epi<EPI_WGRAD, 256, KIND_BF16, true>(maps, a, st);
+      case EPI_SWIGLU_BWD_BF16: return launch_epi<EPI_SWIGLU_BWD_BF16, 128, KIND_BF16, true>(maps, a, st);
     }
     return cudaErrorInvalidValue;
   }
   switch (epi) {
     case EPI_SWIGLU_BF16: return launch_epi<EPI_SWIGLU_BF16, 256, KIND_BF16, false>(maps, a, st);
     case EPI_F32_ROWS: return launch_epi<EPI_F32_ROWS, 256, KIND_BF16, false>(maps, a, st);
+    case EPI_F24_ROWS: return launch_epi<EPI_F24_ROWS, 256, KIND_BF16, false>(maps, a, st);
+    case EPI_WGRAD: return launch_epi<EPI_WGRAD, 256, KIND_BF16, false>(maps, a, st);
+    case EPI_SWIGLU_BWD_BF16: return launch_epi<EPI_SWIGLU_BWD_BF16, 128, KIND_BF16, false>(maps, a, st);
   }
   return cudaErrorInvalidValue;
 }

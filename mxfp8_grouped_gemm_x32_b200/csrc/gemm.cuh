@@ -13,7 +13,8 @@ enum EpiKind : int {
   EPI_SWIGLU_BWD = 4,    // dgrad2 + ScaledSwiGLU backward: da (along 2I and tokens), h (tokens), dprob partials
   EPI_SWIGLU_BF16 = 5,   // BF16 path gate_up: h = p * silu(gate) * up written in bf16 (q_out)
   EPI_F24_ROWS = 6,      // down / dgrad1: the top 24 bits of each fp32 value (f24, see common.cuh), rows in permuted order
-  EPI_SWIGLU_F8T = 7     // per-tensor FP8 gate_up: dequantised by deq[e], h in bf16 (q_out) and its |max| (amax_out)
+  EPI_SWIGLU_F8T = 7,    // per-tensor FP8 gate_up: dequantised by deq[e], h in bf16 (q_out) and its |max| (amax_out)
+  EPI_SWIGLU_BWD_BF16 = 8  // BF16 recipe dgrad2 + ScaledSwiGLU backward: da rows and columns, h columns in bf16
 };
 
 // Operand kind of the tensor-core MMA.
@@ -49,7 +50,7 @@ struct GemmArgs {
   uint8_t* out;       // output: fp32 rows (EPI_F32_*), f24 rows (EPI_F24_ROWS), bf16 per-expert matrices (EPI_WGRAD)
   int64_t ld_out;     // elements between output rows (EPI_F24_ROWS: bytes)
   int64_t out_group_stride;  // mode 1: elements between experts' matrices
-  uint8_t* out2;      // EPI_SWIGLU: saved A, bf16 [rows][2N] (nullable)
+  uint8_t* out2;      // EPI_SWIGLU(_BF16): saved A, bf16 [rows][2N] (nullable)
   uint8_t* q_out;     // EPI_SWIGLU: h codes [rows][N]; EPI_SWIGLU_BF16: h bf16 [rows][N]
   uint8_t* sf_out;    // EPI_SWIGLU: h scales, blocked (1, rows, N)
   int32_t q_KT;
@@ -70,6 +71,9 @@ struct GemmArgs {
   // running |max| of h as float bits (EPI_SWIGLU_F8T)
   const float* deq;
   uint32_t* amax_out;
+  // mode 1: log2 of the tokens in a 128-byte K tile (0: 7, 8-bit operands;
+  // 6 for bf16 operands)
+  int32_t k_shift;
 };
 
 // Tensor maps: A 2-D {K, rows} with a 128 x 128 box; B either 3-D
@@ -96,7 +100,8 @@ uint32_t gemm_b_box(uint32_t bn);
 // or 128 (two accumulators; EPI_SWIGLU_BWD).
 cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);
 
-// BF16 operands (kind::f16), bn = 256: EPI_SWIGLU_BF16 and EPI_F32_ROWS.
+// BF16 operands (kind::f16): EPI_SWIGLU_BF16, EPI_F32_ROWS, EPI_F24_ROWS and
+// EPI_WGRAD (bn = 256), EPI_SWIGLU_BWD_BF16 (bn = 128).
 // The tensor maps describe the bf16 matrices as bytes (inner extent 2K), and
 // num_kt / a_KT count 128-byte K tiles.
 cudaError_t launch_grouped_gemm_bf16(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);

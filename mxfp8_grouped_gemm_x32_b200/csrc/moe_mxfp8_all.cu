@@ -5,6 +5,7 @@
 #include "permute.cu"
 #include "quant.cu"
 #include "swiglu_bwd.cu"
+#include "transpose.cu"
 #include "noalloc.cu"
 #include "router.cu"
 #include "scales.cu"

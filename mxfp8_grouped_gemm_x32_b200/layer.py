@@ -12,6 +12,7 @@ Steps (names of the C entry points):
                     down GEMM, top-k combine
   forward_bf16      moe_grouped_mlp_fwd_bf16: the same layer with bf16 operands
                     (routing from permute_index, moe_permute without x)
+  backward_bf16     moe_grouped_mlp_bwd_bf16: its backward
   backward          moe_grouped_mlp_bwd: dgrad/wgrad of both projections,
                     ScaledSwiGLU backward, d(prob)
 """
@@ -164,9 +165,30 @@ class GroupedMLP:
         lib.moe_grouped_mlp_fwd_bf16(w1.data_ptr(), w2.data_ptr(), self.T, H, I, E, self.k, self.rows_cap,
                                      _ptr(self.split_sizes), _ptr(self.group_offsets), _ptr(self.row_to_slot),
                                      _ptr(self.slot_to_row), _ptr(self.prob_perm), x.data_ptr(), _ptr(self.out),
-                                     _ptr(self.ws_bf16),
-                                     self.ws_bf16_bytes, self._stream())
+                                     _ptr(self.saved_a), _ptr(self.ws_bf16), self.ws_bf16_bytes, self._stream())
         return self.out
+
+    def backward_bf16(self, dY: torch.Tensor, x: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor):
+        """BF16 recipe backward (moe_grouped_mlp_bwd_bf16) after forward_bf16
+        on the same routing: dY, x bf16 [T, H], w1 bf16 [E, 2I, H], w2 bf16
+        [E, H, I] -> (dX, dW1, dW2, dprob)."""
+        if not self.backward_enabled:
+            raise RuntimeError("this layer was built with backward=False")
+        E, H, I = self.E, self.H, self.I
+        check_tensor(dY, "dY", torch.bfloat16, (self.T, H), self.dev)
+        check_tensor(x, "x", torch.bfloat16, (self.T, H), self.dev)
+        check_tensor(w1, "w_gate_up", torch.bfloat16, (E, 2 * I, H), self.dev)
+        check_tensor(w2, "w_down", torch.bfloat16, (E, H, I), self.dev)
+        if getattr(self, "ws_bwd_bf16", None) is None:
+            self.ws_bwd_bf16_bytes = lib.moe_workspace_size(lib.MOE_OP_BWD_BF16, self.T, self.k, E, H, I)
+            self.ws_bwd_bf16 = self._alloc.raw(self.ws_bwd_bf16_bytes, "ws_bwd_bf16")
+        lib.moe_grouped_mlp_bwd_bf16(w1.data_ptr(), w2.data_ptr(), self.T, H, I, E, self.k, self.rows_cap,
+                                     _ptr(self.split_sizes), _ptr(self.group_offsets), _ptr(self.row_to_slot),
+                                     _ptr(self.slot_to_row), _ptr(self.prob_perm), dY.data_ptr(),
+                                     _ptr(self.saved_a), x.data_ptr(), _ptr(self.dX), _ptr(self.dW1),
+                                     _ptr(self.dW2), _ptr(self.dprob), _ptr(self.ws_bwd_bf16),
+                                     self.ws_bwd_bf16_bytes, self._stream())
+        return self.dX, self.dW1, self.dW2, self.dprob
 
     def forward_fp8_tensor(self, x: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor) -> torch.Tensor:
         """Per-tensor FP8 recipe forward (moe_grouped_mlp_fwd_fp8_tensor) on

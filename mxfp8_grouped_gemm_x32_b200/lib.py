@@ -22,6 +22,7 @@ MOE_OP_FWD = 2
 MOE_OP_BWD = 3
 MOE_OP_FWD_BF16 = 4
 MOE_OP_FWD_FP8_TENSOR = 5
+MOE_OP_BWD_BF16 = 6
 MOE_MAX_EXPERTS = 256
 
 STATUS = {
@@ -37,7 +38,7 @@ EXPORTED = [
     "moe_get_device_status", "moe_status_string", "moe_launch_count", "moe_selftest_wait_timeout",
     "moe_timing_enable", "moe_timing_read", "moe_permute_noalloc", "moe_mlp_quantize_weights",
     "moe_router_topk", "moe_mx_scales_to_blocked", "moe_mx_scales_from_blocked", "moe_route_permute",
-    "moe_grouped_mlp_fwd_bf16", "moe_grouped_mlp_fwd_fp8_tensor",
+    "moe_grouped_mlp_fwd_bf16", "moe_grouped_mlp_fwd_fp8_tensor", "moe_grouped_mlp_bwd_bf16",
 ]
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 
@@ -84,7 +85,9 @@ _decl("moe_mx_scales_from_blocked", _I32, _P, _I32, _I64, _I64, _P, _I64, _P)
 _decl("moe_route_permute", _I32, _P, _I32, _P, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P,
       _P, _P, _P, _P, _SZ, _P)
 _decl("moe_grouped_mlp_fwd_bf16", _I32, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P, _P,
-      _P, _SZ, _P)
+      _P, _P, _SZ, _P)
+_decl("moe_grouped_mlp_bwd_bf16", _I32, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P,
+      _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
 _decl("moe_grouped_mlp_fwd_fp8_tensor", _I32, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P,
       _P, _P, _P, _SZ, _P)
 _decl("moe_get_device_status", _I32, _P)
@@ -162,10 +165,18 @@ def moe_mx_scales_from_blocked(blocked, groups, rows, k, plain, ld, stream=0):
 
 
 def moe_grouped_mlp_fwd_bf16(w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot,
-                             slot_to_row, prob_perm, x, out, workspace, workspace_bytes, stream=0):
+                             slot_to_row, prob_perm, x, out, saved_a, workspace, workspace_bytes, stream=0):
     _check("moe_grouped_mlp_fwd_bf16", _lib.moe_grouped_mlp_fwd_bf16(
         w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot, slot_to_row, prob_perm,
-        x, out, workspace, workspace_bytes, stream))
+        x, out, saved_a, workspace, workspace_bytes, stream))
+
+
+def moe_grouped_mlp_bwd_bf16(w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot,
+                             slot_to_row, prob_perm, dY, saved_a, x, dX, dW1, dW2, dprob, workspace,
+                             workspace_bytes, stream=0):
+    _check("moe_grouped_mlp_bwd_bf16", _lib.moe_grouped_mlp_bwd_bf16(
+        w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot, slot_to_row, prob_perm,
+        dY, saved_a, x, dX, dW1, dW2, dprob, workspace, workspace_bytes, stream))
 
 
 def moe_grouped_mlp_fwd_fp8_tensor(w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets,

@@ -182,6 +182,70 @@ def backward_allowance(f, b, x, w1, w2, dy, topk_idx):
     return {"dX": aX, "dW1": aW1, "dW2": aW2, "dprob": dprob.reshape(T, k)}
 
 
+def bf16_ambiguity(v: np.ndarray, band: np.ndarray) -> np.ndarray:
+    """max |bf16(any value in [v-band, v+band]) - bf16(v)| (rounding is
+    monotone, so the ends of the band give it)."""
+    ref = omoe.bf16_round(v)
+    lo, hi = bf16_alternatives(v, band)
+    return np.maximum(np.abs(lo - ref), np.abs(hi - ref))
+
+
+def backward_allowance_bf16(f, b, x, w1, w2, dy, topk_idx):
+    """Element-wise allowances for dX, dW1, dW2 and dprob of the BF16
+    recipe's backward: the operands are exact bf16 values, and the tensors
+    held in bf16 between the GEMMs (the saved A, da = [dg | du] and h) may
+    round either way where their value is ambiguous."""
+    E, I2, H = w1.shape
+    I = I2 // 2
+    T, k = topk_idx.shape
+    R = f["perm"].size
+    allow_dx = np.zeros((R, H))
+    allow_dp = np.zeros(R)
+    aW1 = np.zeros(w1.shape)
+    aW2 = np.zeros(w2.shape)
+    for e, sl in enumerate(_rows_by_expert(f["offsets"], E)):
+        m = sl.stop - sl.start
+        if m == 0:
+            continue
+        tok = f["tok"][sl]
+        p = f["p"][sl][:, None]
+        xg, dyg = x[tok], dy[tok]
+        lo, hi = bf16_alternatives(f["A"][sl], acc_band(xg, w1[e]))
+        a = f["saved"][sl]
+        g, u = a[:, :I], a[:, I:]
+        dh = b["dh"][sl]
+        bdh = acc_band(dyg, w2[e].T)
+
+        def parts(gg, uu, dd):
+            sg = omoe.sigmoid(gg)
+            s = gg * sg
+            return dd * p * uu * sg * (1 + gg * (1 - sg)), dd * p * s, p * s * uu, dd * s * uu
+
+        base = parts(g, u, dh)
+        band = [np.zeros_like(t) for t in base]
+        for gg in (lo[:, :I], hi[:, :I], g):
+            for uu in (lo[:, I:], hi[:, I:], u):
+                alt = parts(gg, uu, dh)
+                for i in range(4):
+                    band[i] = np.maximum(band[i], np.abs(alt[i] - base[i]))
+        sg = omoe.sigmoid(g)
+        band[0] += np.abs(p * u * sg * (1 + g * (1 - sg))) * bdh + ACT * np.abs(base[0])
+        band[1] += np.abs(p * g * sg) * bdh + ACT * np.abs(base[1])
+        band[2] += ACT * np.abs(base[2])
+        band[3] += np.abs(g * sg * u) * bdh + ACT * np.abs(base[3])
+        allow_dp[sl] = band[3].sum(axis=1)
+        Dda = bf16_ambiguity(np.concatenate([base[0], base[1]], axis=1),
+                             np.concatenate([band[0], band[1]], axis=1))
+        Dh = bf16_ambiguity(base[2], band[2])
+        allow_dx[sl] = Dda @ np.abs(w1[e])          # dgrad1: da W_gate_up
+        aW2[e] = np.abs(dyg).T @ Dh                  # wgrad2: dy^T h
+        aW1[e] = Dda.T @ np.abs(xg)                  # wgrad1: da^T x
+    aX = allow_dx[f["slot_row"]].reshape(T, k, -1).sum(axis=1)
+    dprob = np.zeros(R)
+    dprob[f["perm"]] = allow_dp
+    return {"dX": aX, "dW1": aW1, "dW2": aW2, "dprob": dprob.reshape(T, k)}
+
+
 def within(gpu, ref, tol, allow, bf16_out=True):
     """max over elements of (|gpu - ref| - allow) / rms(ref), to compare
     with tol.  For bf16 outputs the allowance also holds the output's own

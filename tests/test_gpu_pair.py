@@ -16,3 +16,14 @@ def test_pair_gemm_smoke():
     r = subprocess.run([sys.executable, "-c", "import __graft_entry__ as g; g.smoke()"], cwd=ROOT, env=env,
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+
+
+@pytest.mark.gpu
+def test_pair_gemm_bf16_recipe():
+    """The BF16 recipe's forward and backward GEMMs on CTA pairs (kind::f16,
+    mode-1 weight gradients over 64-token K tiles included)."""
+    env = dict(os.environ, MOE_GEMM_PAIR="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                        "tests/test_gpu_bf16.py", "tests/test_gpu_bf16_bwd.py"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
