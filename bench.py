@@ -703,6 +703,22 @@ def run_ours(args):
     st = layer.device_status()
     if st != 0:
         raise SystemExit(f"device status after the BF16 forward: {lib.status_string(st)}")
+    # the BF16 recipe's training step: routing + forward (saving A) + backward
+    for _ in range(3):
+        layer.permute_index(idx, prob)
+        layer.forward_bf16(x, w1, w2)
+        layer.backward_bf16(dy, x, w1, w2)
+    e0.record(stream)
+    for _ in range(10):
+        layer.permute_index(idx, prob)
+        layer.forward_bf16(x, w1, w2)
+        layer.backward_bf16(dy, x, w1, w2)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_bf16_step = max_over_ranks(e0.elapsed_time(e1) / 10, world, dev)
+    st = layer.device_status()
+    if st != 0:
+        raise SystemExit(f"device status after the BF16 backward: {lib.status_string(st)}")
     # the per-tensor FP8 recipe's forward (one factor per tensor, quantised
     # from the bf16 weights and x every call): routing + forward
     for _ in range(3):
@@ -775,6 +791,14 @@ def run_ours(args):
                      "frac_of_bf16_peak": cfg.fwd_flops() / (ms_bf16 * 1e-3) / 1e12 / peaks["bf16_sustained"],
                      "what": "BF16 recipe layer forward (moe_permute without x + moe_grouped_mlp_fwd_bf16): "
                              "bf16 operands, no MXFP8"},
+        "bf16_step": {"value": world * flops / (ms_bf16_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "ms_per_call": ms_bf16_step, "bwd_ms": ms_bf16_step - ms_bf16,
+                      "bwd_tflops": cfg.bwd_flops() / ((ms_bf16_step - ms_bf16) * 1e-3) / 1e12,
+                      "peak_bf16_tflops": peaks["bf16_sustained"],
+                      "frac_of_bf16_peak": flops / (ms_bf16_step * 1e-3) / 1e12 / peaks["bf16_sustained"],
+                      "what": "BF16 recipe layer step: moe_permute without x + moe_grouped_mlp_fwd_bf16 (saving A) "
+                              "+ moe_grouped_mlp_bwd_bf16 (weights transposed in the call); bwd_ms = step - "
+                              "bf16_fwd"},
         "fp8_tensor_fwd": {"value": world * cfg.fwd_flops() / (ms_f8t * 1e-3) / 1e12, "unit": "TFLOP/s",
                            "ms_per_call": ms_f8t,
                            "what": "per-tensor FP8 recipe layer forward (moe_permute without x + "

@@ -532,6 +532,13 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
     const uint32_t tc = tl + 64 * half + 32 * j;
     float sv[32], o[32];  // sv: s = g * sigmoid(g), kept across the three passes
     uint32_t d[32];       // dh, read from TMEM once per chunk
+    // g/u of the next chunk (chunk 1, then chunk 0 of the warp's next tile):
+    // issued before this chunk's three passes, which cover their latency
+    GuChunk nxt;
+    if (j == 0)
+      load_gu(a, ti, q, half, lane, 1, nxt);
+    else if (tn)
+      load_gu(a, *tn, q, half, lane, 0, nxt);
     // dg = dh*p*u*sig*(1+g*(1-sig)), quantised along 2I (columns cc..cc+31)
     // and along tokens
     load_dh32(tc, rv, d);
@@ -563,13 +570,6 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
       bf16_store32(o, a.daq + (r * I2 + I + cc) * 2);
       bf16_cols32(o, stage, lane, a.dacol, int64_t(I) + cc, a.rows_cap, rb);
     }
-    // dh and g are used up: load the next chunk's g/u now (it lands during
-    // the last pass and the start of the next chunk)
-    GuChunk nxt;
-    if (j == 0)
-      load_gu(a, ti, q, half, lane, 1, nxt);
-    else if (tn)
-      load_gu(a, *tn, q, half, lane, 0, nxt);
     // h = p*s*u along tokens (operand of the down projection's weight
     // gradient)
 #pragma unroll
