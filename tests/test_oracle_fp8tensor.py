@@ -139,3 +139,85 @@ def test_close_to_the_unquantised_layer():
     rms = np.sqrt(np.mean(ref ** 2))
     assert np.sqrt(np.mean((q - ref) ** 2)) <= 0.1 * rms
     assert np.max(np.abs(q - ref)) <= rms
+
+
+# ---------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------
+
+def _q_brute(v: np.ndarray) -> np.ndarray:
+    """Per-tensor round trip written out from the definitions: factor = the
+    float32 nearest to 448 / amax (exact rational), code = nearest E4M3 of
+    the float32 product, value = code / factor."""
+    amax = float(np.max(np.abs(v)))
+    s = _f32(float(Fraction(448) / Fraction(amax)))
+    flat = [E4M3_TABLE[_nearest_e4m3(_f32(float(Fraction(x) * Fraction(s))))]    # code carries the sign
+            for x in np.asarray(v, np.float64).reshape(-1)]
+    return np.array(flat).reshape(np.shape(v)) / s
+
+
+def test_backward_identity_expert_closed_form():
+    """W_gate_up = identity, W_down = [I; 0], p = 1, x and dY of E4M3 values
+    with |max| 448: x, the weights and dY quantise exactly, so dh = dY[:, :I]
+    and dX = Q(da), dW_gate_up = Q(da)^T x, dW_down = dY^T Q(h), dprob =
+    sum dh*silu(g)*u, with da = bf16([dg, du]), h = bf16(silu(g)*u) and Q the
+    round trip through each tensor's factor -- all written out here from the
+    definitions (brute-force E4M3, exact-rational factors)."""
+    I = 32
+    H = 2 * I
+    T = 16
+    rng = np.random.default_rng(11)
+    sign = lambda shape: np.where(rng.random(shape) < 0.5, -1.0, 1.0)
+    x = E4M3_TABLE[rng.integers(0, 0x7F, size=(T, H))] * sign((T, H)) / 64.0
+    x[0, 0] = 448.0 / 64.0                                       # amax 7 -> factor 64, still exact
+    dy = E4M3_TABLE[rng.integers(0, 0x7F, size=(T, H))] * sign((T, H))
+    dy[1, 3] = -448.0
+    w1 = np.eye(2 * I)[None]
+    w2 = np.concatenate([np.eye(I), np.zeros((I, I))])[None]
+    idx = np.zeros((T, 1), np.int32)
+    prob = np.ones((T, 1), np.float32)
+    f = ft.forward(x, w1, w2, idx, prob)
+    assert f["s_x"] == np.float32(64.0)
+    b = ft.backward(f, dy, prob)
+    assert b["s_dy"] == np.float32(1.0)
+    g, u = omoe.bf16_round(x[:, :I]), omoe.bf16_round(x[:, I:])
+    sg = 1.0 / (1.0 + np.exp(-g))
+    dh = dy[:, :I]
+    da = omoe.bf16_round(np.concatenate([dh * u * sg * (1.0 + g * (1.0 - sg)), dh * g * sg], axis=1))
+    hb = omoe.bf16_round(g * sg * u)
+    qda, qh = _q_brute(da), _q_brute(hb)
+    assert np.array_equal(b["dX"], qda)
+    assert np.allclose(b["dW1"][0], qda.T @ x, rtol=1e-12, atol=1e-12)
+    assert np.allclose(b["dW2"][0], dy.T @ qh, rtol=1e-12, atol=1e-12)
+    assert np.allclose(b["dprob_f64"][:, 0], np.sum(dh * g * sg * u, axis=1), rtol=1e-12, atol=1e-12)
+
+
+def test_backward_scales_exactly_with_dy():
+    """dY -> 2^5 dY: its factor divides by exactly 2^5 and every gradient is
+    multiplied by exactly 2^5 (dh, da and their codes scale through; h does
+    not depend on dY) -- a dropped, doubled or misplaced factor breaks this."""
+    x, w1, w2, idx, p = _case(seed=7)
+    rng = np.random.default_rng(8)
+    dy = bf16_bits_to_f32(omoe.bf16_bits(rng.standard_normal(x.shape))).astype(np.float64)
+    f = ft.forward(x, w1, w2, idx, p)
+    a = ft.backward(f, dy, p)
+    b = ft.backward(f, dy * 32.0, p)
+    assert b["s_dy"] * np.float32(32.0) == a["s_dy"] and b["s_da"] * np.float32(32.0) == a["s_da"]
+    assert b["s_hb"] == a["s_hb"]
+    for key in ("dX", "dW1", "dW2", "dprob_f64"):
+        assert np.array_equal(b[key], 32.0 * a[key]), key
+
+
+def test_backward_close_to_the_unquantised_layer():
+    """FP8 rounding error only: every gradient within 12 % of the rms of the
+    exact layer's gradient in rms (a transposed operand, a wrong row or a
+    dropped term gives errors of the order of the rms itself)."""
+    x, w1, w2, idx, p = _case(seed=9)
+    rng = np.random.default_rng(10)
+    dy = bf16_bits_to_f32(omoe.bf16_bits(rng.standard_normal(x.shape))).astype(np.float64)
+    q = ft.backward(ft.forward(x, w1, w2, idx, p), dy, p)
+    fe = omoe.forward(x, w1, w2, idx, p, quantize=False, round_saved=False)
+    ref = omoe.backward(fe, x, w1, w2, p, dy, quantize=False)
+    for key, rk in (("dX", "dX"), ("dW1", "dW1"), ("dW2", "dW2"), ("dprob_f64", "dprob_f64")):
+        rms = np.sqrt(np.mean(ref[rk] ** 2))
+        assert np.sqrt(np.mean((q[key] - ref[rk]) ** 2)) <= 0.12 * rms, key
