@@ -95,6 +95,7 @@ typedef enum {
 #define MOE_OP_FWD_BF16 4
 #define MOE_OP_FWD_FP8_TENSOR 5
 #define MOE_OP_BWD_BF16 6
+#define MOE_OP_BWD_FP8_TENSOR 7
 
 /* Limits checked on the host. */
 #define MOE_MAX_EXPERTS 256
@@ -111,7 +112,7 @@ int64_t moe_mx_scale_bytes(int32_t groups, int64_t rows, int64_t k);
 int64_t moe_padded_rows(int32_t T, int32_t k, int32_t E);
 
 /* Workspace bytes for op MOE_OP_PERMUTE / MOE_OP_FWD / MOE_OP_BWD /
- * MOE_OP_FWD_BF16 / MOE_OP_FWD_FP8_TENSOR / MOE_OP_BWD_BF16 of a layer
+ * MOE_OP_FWD_BF16 / MOE_OP_FWD_FP8_TENSOR / MOE_OP_BWD_BF16 / MOE_OP_BWD_FP8_TENSOR of a layer
  * (T tokens, top-k, E experts, hidden H, intermediate I).  -1 if invalid. */
 int64_t moe_workspace_size(int32_t op, int32_t T, int32_t k, int32_t E, int32_t H, int32_t I);
 
@@ -310,8 +311,10 @@ moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down,
  *   w_gate_up  bf16 [E][2I][H] (gate rows first); w_down bf16 [E][H][I].
  *   routing    from moe_permute (xq may be NULL there).
  *   x          bf16 [T][H];  out bf16 [T][H].
+ *   saved_a    bf16 [rows_cap][2I] or NULL: A (dequantised) rounded to bf16,
+ *              kept for moe_grouped_mlp_bwd_fp8_tensor (16-byte aligned).
  *   scales     NULL, or float [2 + 2E] receiving the factors: x, h,
- *              W_gate_up[0..E), W_down[0..E).
+ *              W_gate_up[0..E), W_down[0..E) (the backward's fwd_scales).
  *   workspace  >= moe_workspace_size(MOE_OP_FWD_FP8_TENSOR, T, k, E, H, I),
  *              256-byte aligned.
  * Limits as moe_grouped_mlp_fwd.  The pages describe no kernel for this
@@ -320,8 +323,42 @@ moe_status_t moe_grouped_mlp_fwd_fp8_tensor(const void* w_gate_up, const void* w
                                             int32_t I, int32_t E, int32_t k, int64_t rows_cap,
                                             const int32_t* split_sizes, const int32_t* group_offsets,
                                             const int32_t* row_to_slot, const int32_t* slot_to_row,
-                                            const float* prob_perm, const void* x, void* out, float* scales,
-                                            void* workspace, size_t workspace_bytes, moe_stream_t stream);
+                                            const float* prob_perm, const void* x, void* out, void* saved_a,
+                                            float* scales, void* workspace, size_t workspace_bytes,
+                                            moe_stream_t stream);
+
+/* Per-tensor FP8 recipe backward, after moe_grouped_mlp_fwd_fp8_tensor on the
+ * same routing, weights and x.  The pages give no formula; the readings:
+ * the forward's factors of x and of each expert's weights are reused (under
+ * one factor per tensor a code does not depend on the layout, so W^T carries
+ * the forward's codes); dY gets its own factor; dh = dy W_down (dequantised
+ * per expert), the ScaledSwiGLU backward and dprob as moe_grouped_mlp_bwd,
+ * from saved_a; da = [dg, du] and the recomputed h = p*s*u are held in bf16
+ * and each gets one factor (448 / |max| over all routed rows, as the
+ * forward's rule); dW_down_e = dy_e^T h_e, dx = da W_gate_up (f24 rows,
+ * combined per token in fp32, one bf16 rounding), dW_gate_up_e = da_e^T x_e,
+ * every GEMM on kind::f8f6f4 with fp32 accumulation dequantised by
+ * 1 / (scale_a scale_b).
+ *   w_gate_up, w_down, x   bf16, as the forward.
+ *   routing    as the forward, slot_to_row included.
+ *   dY         bf16 [T][H].  saved_a bf16 [rows_cap][2I] from the forward
+ *              (32-byte aligned).
+ *   fwd_scales device float [2 + 2E], the forward's `scales` output.
+ * Outputs: dX bf16 [T][H]; dW1 bf16 [E][2I][H]; dW2 bf16 [E][H][I];
+ *   dprob float [T][k] (slot order); scales NULL or float [3] receiving the
+ *   factors of dY, da and h.
+ *   workspace  >= moe_workspace_size(MOE_OP_BWD_FP8_TENSOR, T, k, E, H, I),
+ *              256-byte aligned.
+ * Pointers 16-byte aligned, factor arrays 4-byte aligned (MOE_ERR_INVALID
+ * otherwise); limits as moe_grouped_mlp_bwd. */
+moe_status_t moe_grouped_mlp_bwd_fp8_tensor(const void* w_gate_up, const void* w_down, int32_t T, int32_t H,
+                                            int32_t I, int32_t E, int32_t k, int64_t rows_cap,
+                                            const int32_t* split_sizes, const int32_t* group_offsets,
+                                            const int32_t* row_to_slot, const int32_t* slot_to_row,
+                                            const float* prob_perm, const void* dY, const void* saved_a,
+                                            const void* x, const float* fwd_scales, void* dX, void* dW1, void* dW2,
+                                            float* dprob, float* scales, void* workspace, size_t workspace_bytes,
+                                            moe_stream_t stream);
 
 /* Top-k combine (Challenge 1, index_add back to token order):
  *   y  bf16 [T*k][H] in slot order -> out bf16 [T][H], out[t] = sum_j y[t*k+j]

@@ -184,6 +184,42 @@ BwdBf16Ws carve_bwd_bf16(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, 
   return w;
 }
 
+// Per-tensor FP8 backward workspace: bf16 staging (the transposed weights,
+// one at a time; dy gathered in both orientations; da and h from the dgrad2
+// epilogue; x gathered and transposed), their E4M3 codes, f24 dgrad rows,
+// dprob partials, |max| bits (dY, da, h), factors (dY, da, h) and the
+// dequantisation factors of the four GEMMs [4E].
+struct BwdF8tWs {
+  uint8_t *wt, *w2tq, *w1tq, *dyp, *dyc, *dyq, *dycq, *da, *dac, *hc, *daq, *dacq, *hcq, *xc, *xcq, *dx, *dpp;
+  uint32_t* amax;
+  float *scale, *deq;
+};
+BwdF8tWs carve_bwd_f8t(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t E, int64_t rows_cap) {
+  (void)T; (void)k;
+  BwdF8tWs w{};
+  w.wt = c.take(E * 2 * I * H * 2);
+  w.w2tq = c.take(E * I * H);
+  w.w1tq = c.take(E * H * 2 * I);
+  w.dyp = c.take(rows_cap * H * 2);
+  w.dyc = c.take(H * rows_cap * 2);
+  w.dyq = c.take(rows_cap * H);
+  w.dycq = c.take(H * rows_cap);
+  w.da = c.take(rows_cap * 2 * I * 2);
+  w.dac = c.take(2 * I * rows_cap * 2);
+  w.hc = c.take(I * rows_cap * 2);
+  w.daq = c.take(rows_cap * 2 * I);
+  w.dacq = c.take(2 * I * rows_cap);
+  w.hcq = c.take(I * rows_cap);
+  w.xc = c.take(H * rows_cap * 2);
+  w.xcq = c.take(H * rows_cap);
+  w.dx = c.take(rows_cap * H * 3);
+  w.dpp = c.take(I / 64 * rows_cap * 4);
+  w.amax = reinterpret_cast<uint32_t*>(c.take(3 * 4));
+  w.scale = reinterpret_cast<float*>(c.take(3 * 4));
+  w.deq = reinterpret_cast<float*>(c.take(4 * E * 4));
+  return w;
+}
+
 bool layer_dims_ok(int32_t T, int32_t H, int32_t I, int32_t E, int32_t k) {
   return T >= 0 && H > 0 && I > 0 && E > 0 && k > 0 && k <= E && E <= MOE_MAX_EXPERTS &&
          H % 32 == 0 && I % 64 == 0 && int64_t(T) * k < (int64_t(1) << 30);
@@ -274,6 +310,10 @@ int64_t moe_workspace_size(int32_t op, int32_t T, int32_t k, int32_t E, int32_t 
     case MOE_OP_BWD_BF16:
       if (H <= 0 || I <= 0) return -1;
       carve_bwd_bf16(c, T, k, H, I, E, rows_cap);
+      return c.off;
+    case MOE_OP_BWD_FP8_TENSOR:
+      if (H <= 0 || I <= 0) return -1;
+      carve_bwd_f8t(c, T, k, H, I, E, rows_cap);
       return c.off;
   }
   return -1;
@@ -488,8 +528,9 @@ moe_status_t moe_grouped_mlp_fwd_fp8_tensor(const void* w_gate_up, const void* w
                                             int32_t I, int32_t E, int32_t k, int64_t rows_cap,
                                             const int32_t* split_sizes, const int32_t* group_offsets,
                                             const int32_t* row_to_slot, const int32_t* slot_to_row,
-                                            const float* prob_perm, const void* x, void* out, float* scales,
-                                            void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+                                            const float* prob_perm, const void* x, void* out, void* saved_a,
+                                            float* scales, void* workspace, size_t workspace_bytes,
+                                            moe_stream_t stream) {
   if (!w_gate_up || !w_down || !split_sizes || !group_offsets || !row_to_slot || !prob_perm ||
       (T > 0 && (!x || !out || !slot_to_row)))
     return MOE_ERR_INVALID;
@@ -497,6 +538,7 @@ moe_status_t moe_grouped_mlp_fwd_fp8_tensor(const void* w_gate_up, const void* w
   if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
   for (const void* p : {w_gate_up, w_down, x, (const void*)out})
     if (!al16(p)) return MOE_ERR_INVALID;
+  if (saved_a && !al16(saved_a)) return MOE_ERR_INVALID;
   if (scales && (reinterpret_cast<uintptr_t>(scales) & 3u)) return MOE_ERR_INVALID;
   Carver c{static_cast<uint8_t*>(workspace)};
   FwdF8tWs w = carve_fwd_f8t(c, T, k, H, I, E, rows_cap);
@@ -530,7 +572,7 @@ moe_status_t moe_grouped_mlp_fwd_fp8_tensor(const void* w_gate_up, const void* w
     g1.mode = 0; g1.E = E; g1.N = I; g1.num_kt = int32_t(cdiv(H, 128)); g1.n_tiles = int32_t(cdiv(I, 128));
     g1.group_offsets = group_offsets; g1.split_sizes = split_sizes; g1.rows_cap = rows_cap;
     g1.prob = prob_perm; g1.row_to_slot = row_to_slot; g1.q_out = w.h;
-    g1.deq = w.deq; g1.amax_out = w.amax + 1;
+    g1.deq = w.deq; g1.amax_out = w.amax + 1; g1.out2 = static_cast<uint8_t*>(saved_a);
     {
       TimeScope ts(st, "gemm_gate_up_swiglu_fp8t");
       if (launch_grouped_gemm_f8t(EPI_SWIGLU_F8T, m1, g1, st) != cudaSuccess) return MOE_ERR_CUDA;
@@ -797,6 +839,151 @@ moe_status_t moe_grouped_mlp_bwd_bf16(const void* w_gate_up, const void* w_down,
     TimeScope ts(st, "gemm_wgrad_gate_up_bf16");
     if (launch_grouped_gemm_bf16(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
+  return MOE_OK;
+}
+
+moe_status_t moe_grouped_mlp_bwd_fp8_tensor(const void* w_gate_up, const void* w_down, int32_t T, int32_t H,
+                                            int32_t I, int32_t E, int32_t k, int64_t rows_cap,
+                                            const int32_t* split_sizes, const int32_t* group_offsets,
+                                            const int32_t* row_to_slot, const int32_t* slot_to_row,
+                                            const float* prob_perm, const void* dY, const void* saved_a,
+                                            const void* x, const float* fwd_scales, void* dX, void* dW1, void* dW2,
+                                            float* dprob, float* scales, void* workspace, size_t workspace_bytes,
+                                            moe_stream_t stream) {
+  if (!w_gate_up || !w_down || !split_sizes || !group_offsets || !row_to_slot || !prob_perm || !saved_a ||
+      !fwd_scales || !dW1 || !dW2 || (T > 0 && (!slot_to_row || !dY || !dX || !dprob || !x)))
+    return MOE_ERR_INVALID;
+  if (!layer_dims_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap < moe_padded_rows(T, k, E) || rows_cap % 128) return MOE_ERR_INVALID;
+  for (const void* p : {w_gate_up, w_down, dY, x, (const void*)dX, (const void*)dW1, (const void*)dW2})
+    if (!al16(p)) return MOE_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(fwd_scales) & 3u) || (scales && (reinterpret_cast<uintptr_t>(scales) & 3u)))
+    return MOE_ERR_INVALID;
+  if (!al32(saved_a) || !al256(workspace)) return MOE_ERR_INVALID;  // 256-bit loads and stores
+  Carver c{static_cast<uint8_t*>(workspace)};
+  BwdF8tWs w = carve_bwd_f8t(c, T, k, H, I, E, rows_cap);
+  if (!workspace || int64_t(workspace_bytes) < c.off) return MOE_ERR_WORKSPACE;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t I2 = 2 * int64_t(I);
+  const int32_t* rows_used = group_offsets + E;
+  auto quant = [&](const uint8_t* src, int64_t n, int64_t group, const float* sc, const int32_t* ru, int64_t row,
+                   uint8_t* q) { return launch_f8t_quant(src, n, group, sc, ru, row, q, st) == cudaSuccess; };
+
+  // dY's factor; dy gathered to permuted rows in both orientations, then its codes
+  {
+    TimeScope ts(st, "fp8t_dy");
+    if (cudaMemsetAsync(w.amax, 0, 3 * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (T > 0 && launch_f8t_amax(static_cast<const uint8_t*>(dY), 1, int64_t(T) * H, w.amax, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (launch_f8t_bwd_scales(w.amax, fwd_scales, E, 0, w.scale, w.deq, st) != cudaSuccess) return MOE_ERR_CUDA;
+    TransposeArgs td{static_cast<const uint16_t*>(dY), reinterpret_cast<uint16_t*>(w.dyc), 1, rows_cap, H, rows_cap,
+                     row_to_slot, k, rows_used, reinterpret_cast<uint16_t*>(w.dyp)};
+    if (launch_transpose_bf16(td, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!quant(w.dyp, rows_cap * H, rows_cap * H, w.scale, rows_used, H, w.dyq) ||
+        !quant(w.dyc, H * rows_cap, H * rows_cap, w.scale, nullptr, 0, w.dycq))
+      return MOE_ERR_CUDA;
+  }
+  // W_down^T codes with the forward's per-expert factors
+  {
+    TimeScope ts(st, "fp8t_w_down_t");
+    TransposeArgs t2{static_cast<const uint16_t*>(w_down), reinterpret_cast<uint16_t*>(w.wt), E, H, I, H, nullptr, k,
+                     nullptr, nullptr};
+    if (launch_transpose_bf16(t2, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!quant(w.wt, E * I * H, int64_t(I) * H, fwd_scales + 2 + E, nullptr, 0, w.w2tq)) return MOE_ERR_CUDA;
+  }
+
+  // dgrad2 + ScaledSwiGLU backward: dh = dy W_down dequantised per expert;
+  // the epilogue writes da (rows, tokens) and h (tokens) in bf16 with their
+  // |max|, and the dprob partial sums
+  GemmMaps m;
+  if (make_map_2d(&m.a, w.dyq, H, rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m.b, w.w2tq, H, I, E, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  GemmArgs g{};
+  g.mode = 0; g.E = E; g.N = I; g.num_kt = int32_t(cdiv(H, 128)); g.n_tiles = int32_t(cdiv(I, 128));
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes;
+  g.prob = prob_perm; g.saved = static_cast<const uint8_t*>(saved_a); g.rows_cap = rows_cap;
+  g.daq = w.da; g.dacol = w.dac; g.hcol = w.hc;
+  g.dprob_part = reinterpret_cast<float*>(w.dpp);
+  g.deq = w.deq; g.amax_out = w.amax + 1;
+  {
+    TimeScope ts(st, "gemm_dgrad_down_swiglu_fp8t");
+    if (launch_grouped_gemm_f8t(EPI_SWIGLU_BWD_F8T, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  {
+    TimeScope ts(st, "dprob_reduce");
+    if (launch_dprob_reduce(group_offsets, E, row_to_slot, rows_cap, reinterpret_cast<const float*>(w.dpp),
+                            I / 64, dprob, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  // da's and h's factors, then their codes
+  {
+    TimeScope ts(st, "fp8t_quant_da_h");
+    if (launch_f8t_bwd_scales(w.amax, fwd_scales, E, 1, w.scale, w.deq, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!quant(w.da, rows_cap * I2, rows_cap * I2, w.scale + 1, rows_used, I2, w.daq) ||
+        !quant(w.dac, I2 * rows_cap, I2 * rows_cap, w.scale + 1, nullptr, 0, w.dacq) ||
+        !quant(w.hc, int64_t(I) * rows_cap, int64_t(I) * rows_cap, w.scale + 2, nullptr, 0, w.hcq))
+      return MOE_ERR_CUDA;
+  }
+
+  // wgrad2: dW_down_e = dy_e^T h_e (contraction over the group's tokens)
+  if (make_map_2d(&m.a, w.dycq, rows_cap, H, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_2d(&m.b, w.hcq, rows_cap, I, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  g = GemmArgs{};
+  g.mode = 1; g.E = E; g.N = I; g.n_tiles = int32_t(cdiv(I, 256));
+  g.m_tiles = int32_t(cdiv(H, 128)); g.M_out = H;
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes;
+  g.out = static_cast<uint8_t*>(dW2); g.ld_out = I; g.out_group_stride = int64_t(H) * I; g.deq = w.deq + E;
+  {
+    TimeScope ts(st, "gemm_wgrad_down_fp8t");
+    if (launch_grouped_gemm_f8t(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
+  // W_gate_up^T codes; dgrad1: dx = da W_gate_up, f24 rows; dX combine
+  {
+    TimeScope ts(st, "fp8t_w_gate_up_t");
+    TransposeArgs t1{static_cast<const uint16_t*>(w_gate_up), reinterpret_cast<uint16_t*>(w.wt), E, I2, H, I2,
+                     nullptr, k, nullptr, nullptr};
+    if (launch_transpose_bf16(t1, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!quant(w.wt, E * H * I2, int64_t(H) * I2, fwd_scales + 2, nullptr, 0, w.w1tq)) return MOE_ERR_CUDA;
+  }
+  if (make_map_2d(&m.a, w.daq, I2, rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_3d(&m.b, w.w1tq, I2, H, E, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  g = GemmArgs{};
+  g.mode = 0; g.E = E; g.N = H; g.num_kt = int32_t(cdiv(I2, 128)); g.n_tiles = int32_t(cdiv(H, 256));
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes; g.rows_cap = rows_cap;
+  g.out = w.dx; g.ld_out = 3 * int64_t(H); g.deq = w.deq + 2 * E;
+  {
+    TimeScope ts(st, "gemm_dgrad_gate_up_fp8t");
+    if (launch_grouped_gemm_f8t(EPI_F24_ROWS, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  {
+    TimeScope ts(st, "combine_dx");
+    if (launch_combine(w.dx, COMBINE_F24, slot_to_row, T, k, H, dX, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
+  // x gathered and transposed, with the forward's factor; wgrad1:
+  // dW_gate_up_e = da_e^T x_e (contraction over the group's tokens)
+  {
+    TimeScope ts(st, "fp8t_x_cols");
+    TransposeArgs tx{static_cast<const uint16_t*>(x), reinterpret_cast<uint16_t*>(w.xc), 1, rows_cap, H, rows_cap,
+                     row_to_slot, k, rows_used, nullptr};
+    if (launch_transpose_bf16(tx, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!quant(w.xc, H * rows_cap, H * rows_cap, fwd_scales, nullptr, 0, w.xcq)) return MOE_ERR_CUDA;
+  }
+  if (make_map_2d(&m.a, w.dacq, rows_cap, I2, 128) != cudaSuccess) return MOE_ERR_CUDA;
+  if (make_map_2d(&m.b, w.xcq, rows_cap, H, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  g = GemmArgs{};
+  g.mode = 1; g.E = E; g.N = H; g.n_tiles = int32_t(cdiv(H, 256));
+  g.m_tiles = int32_t(cdiv(I2, 128)); g.M_out = int32_t(I2);
+  g.group_offsets = group_offsets; g.split_sizes = split_sizes;
+  g.out = static_cast<uint8_t*>(dW1); g.ld_out = H; g.out_group_stride = I2 * H; g.deq = w.deq + 3 * E;
+  {
+    TimeScope ts(st, "gemm_wgrad_gate_up_fp8t");
+    if (launch_grouped_gemm_f8t(EPI_WGRAD, m, g, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if (scales && cudaMemcpyAsync(scales, w.scale, 3 * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

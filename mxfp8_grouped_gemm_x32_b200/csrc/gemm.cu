@@ -252,8 +252,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
     // rounded h of the group's rows is folded into amax_out.
     const int nb = ti.n0 + 64 * half;
     if (nb >= a.N) return;  // uniform across the warp
-    if (EPI == EPI_SWIGLU_BF16 && a.out2) {
-      // saved A in bf16 (the BF16 recipe's backward recomputes g, u, h from it)
+    const float dq = EPI == EPI_SWIGLU_F8T ? a.deq[ti.e] : 1.0f;
+    if constexpr (EPI == EPI_SWIGLU_F8T) {
+#pragma unroll
+      for (int i = 0; i < 128; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * dq);
+    }
+    if (a.out2) {
+      // saved A in bf16 (the backward recomputes g, u, h from it)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t t[16];
@@ -265,7 +270,6 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
       }
     }
     const float p = rv ? a.prob[r] : 0.0f;
-    const float dq = EPI == EPI_SWIGLU_F8T ? a.deq[ti.e] : 1.0f;
     uint32_t hw[32];
     uint32_t hmax = 0;  // |h| as bf16 bits (both halves), max over this lane's values
 #pragma unroll
@@ -273,12 +277,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
       float h2[2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        float g = __uint_as_float(v[2 * j + i]);
-        float u = __uint_as_float(v[64 + 2 * j + i]);
-        if constexpr (EPI == EPI_SWIGLU_F8T) {
-          g *= dq;
-          u *= dq;
-        }
+        const float g = __uint_as_float(v[2 * j + i]);
+        const float u = __uint_as_float(v[64 + 2 * j + i]);
         h2[i] = p * __fdividef(g, 1.0f + __expf(-g)) * u;
       }
       hw[j] = pack_bf16x2(h2[0], h2[1]);
@@ -370,6 +370,11 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, const Tile& ti,
       }
       warp_store_rows<NC>(stage, dst, v, ncols * 4, lane);
     } else {
+      if (a.deq) {  // per-tensor FP8: dequantise first
+        const float dq = a.deq[ti.e];
+#pragma unroll
+        for (int i = 0; i < NC; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * dq);
+      }
       pack_bf16_inplace<NC / 2>(v);
       uint8_t* dst = rv ? a.out + (int64_t(ti.e) * a.out_group_stride + int64_t(r) * a.ld_out + nb) * 2 : nullptr;
       warp_store_rows<NC / 2>(stage, dst, v, ncols * 2, lane);
@@ -504,12 +509,19 @@ __device__ __forceinline__ void bf16_cols32(const float* o, uint32_t* stage, int
 // chunk (chunk 1, then chunk 0 of the warp's next tile `tn`, if any) are
 // issued once a chunk's dh has been read for the last time, so they land
 // while its last pass runs.  On return `cur` holds chunk 0 of `tn`.
-// MXF: the MXFP8 outputs (codes and block scales of da along 2I and along
-// tokens, of h along tokens); otherwise the BF16 recipe's (da along 2I,
-// da and h along tokens, all bf16).
-template <bool MXF>
+// OUT: BWD_MX writes the MXFP8 outputs (codes and block scales of da along
+// 2I and along tokens, of h along tokens); BWD_BF16 the BF16 recipe's (da
+// along 2I, da and h along tokens, all bf16); BWD_F8T the per-tensor FP8
+// recipe's: dh first multiplied by the expert's dequantisation factor
+// deq[e], the BF16 outputs, and the |max| of the bf16 da and of the bf16 h
+// (the bf16 rounding of the fp32 |max|: rounding is monotone) folded into
+// amax_out[0] and amax_out[1] as float bits.
+enum BwdOut : int { BWD_MX = 0, BWD_BF16 = 1, BWD_F8T = 2 };
+
+template <int OUT>
 __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Tile& ti, const Tile* tn, uint32_t tl,
                                                     int q, int half, int lane, uint32_t* stage, GuChunk& cur) {
+  constexpr bool MXF = OUT == BWD_MX;
   const int I = a.N;
   const int cb = ti.n0 + 64 * half;
   if (cb >= I) {  // no columns for this warp in this tile (uniform across the warp)
@@ -522,7 +534,9 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
   const int64_t I2 = 2 * int64_t(I);
   const int64_t KT2 = I2 / 128, KTt = a.rows_cap / 128;
   const float p = rv ? a.prob[r] : 0.0f;
+  const float dq = OUT == BWD_F8T ? a.deq[ti.e] : 1.0f;
   float dps = 0.0f;
+  float mda = 0.0f, mh = 0.0f;  // BWD_F8T: |max| of da and of h over this lane's values
   uint32_t sb_dg = 0, sb_du = 0;
   // (the accumulator stays ours until released; the other one keeps the
   // MMAs busy)
@@ -542,6 +556,10 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
     // dg = dh*p*u*sig*(1+g*(1-sig)), quantised along 2I (columns cc..cc+31)
     // and along tokens
     load_dh32(tc, rv, d);
+    if constexpr (OUT == BWD_F8T) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) d[e] = __float_as_uint(__uint_as_float(d[e]) * dq);
+    }
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const float g = gu_elem(cur.g, e), u = gu_elem(cur.u, e);
@@ -549,6 +567,7 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
       o[e] = (__uint_as_float(d[e]) * p) * (u * sg) * fmaf(g, 1.0f - sg, 1.0f);
       sv[e] = g * sg;
     }
+    if constexpr (OUT == BWD_F8T) mda = abs_max(mda, abs_max_n<32>(o));
     if constexpr (MXF) {
       sb_dg |= encode32_store(o, a.daq + r * I2 + cc) << (8 * j);
       quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, cc, a.rows_cap, rb, KTt);
@@ -563,6 +582,7 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
       o[e] = (__uint_as_float(d[e]) * p) * sv[e];
       dps = fmaf(__uint_as_float(d[e]), sv[e] * gu_elem(cur.u, e), dps);
     }
+    if constexpr (OUT == BWD_F8T) mda = abs_max(mda, abs_max_n<32>(o));
     if constexpr (MXF) {
       sb_du |= encode32_store(o, a.daq + r * I2 + I + cc) << (8 * j);
       quant_cols32(o, stage, lane, a.dacol, a.dacol_sf, int64_t(I) + cc, a.rows_cap, rb, KTt);
@@ -574,6 +594,7 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
     // gradient)
 #pragma unroll
     for (int e = 0; e < 32; ++e) o[e] = p * (sv[e] * gu_elem(cur.u, e));
+    if constexpr (OUT == BWD_F8T) mh = abs_max(mh, abs_max_n<32>(o));
     if constexpr (MXF)
       quant_cols32(o, stage, lane, a.hcol, a.hcol_sf, cc, a.rows_cap, rb, KTt);
     else
@@ -587,6 +608,16 @@ __device__ __forceinline__ void epilogue_swiglu_bwd(const GemmArgs& a, const Til
     *reinterpret_cast<uint16_t*>(a.daq_sf + sf_offset(0, r, (int64_t(I) + cb) >> 5, 0, KT2)) = uint16_t(sb_du);
   }
   a.dprob_part[int64_t(cb >> 6) * a.rows_cap + r] = dps;
+  if constexpr (OUT == BWD_F8T) {
+    // non-negative bf16 bits compare as integers (NaN above every number)
+    uint32_t bda = pack_bf16x2(mda, 0.0f) & 0x7FFFu, bh = pack_bf16x2(mh, 0.0f) & 0x7FFFu;
+    bda = __reduce_max_sync(0xFFFFFFFFu, bda);
+    bh = __reduce_max_sync(0xFFFFFFFFu, bh);
+    if (lane == 0) {
+      if (bda) atomicMax(a.amax_out, bda << 16);
+      if (bh) atomicMax(a.amax_out + 1, bh << 16);
+    }
+  }
 }
 
 // The B operand of one K tile (and, for MXFP8, its scale atoms) into a stage:
@@ -913,7 +944,7 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
           mbar_arrive(&acc_empty[buf]);
       }
     };
-    constexpr bool SWB = EPI == EPI_SWIGLU_BWD || EPI == EPI_SWIGLU_BWD_BF16;
+    constexpr bool SWB = EPI == EPI_SWIGLU_BWD || EPI == EPI_SWIGLU_BWD_BF16 || EPI == EPI_SWIGLU_BWD_F8T;
     GuChunk gu;  // fused ScaledSwiGLU backward: g/u of the next chunk to process
     if constexpr (SWB)
       if (cid < ntiles) {
@@ -955,7 +986,8 @@ __global__ void __launch_bounds__(Cfg<BN, PAIR>::THREADS, 1)
         // reads TMEM chunk by chunk; the other accumulator keeps the MMAs busy
         bool nn;
         const Tile tn = my_tile(has_next ? t + ncl : t, &nn);
-        epilogue_swiglu_bwd<EPI == EPI_SWIGLU_BWD>(a, ti, has_next ? &tn : nullptr, tl, q, half, lane, stage, gu);
+        constexpr int OUT = EPI == EPI_SWIGLU_BWD ? BWD_MX : (EPI == EPI_SWIGLU_BWD_BF16 ? BWD_BF16 : BWD_F8T);
+        epilogue_swiglu_bwd<OUT>(a, ti, has_next ? &tn : nullptr, tl, q, half, lane, stage, gu);
         tc_fence_before();
         __syncwarp();
         release(buf);
@@ -1174,6 +1206,8 @@ cudaError_t launch_grouped_gemm_f8t(int epi, const GemmMaps& maps, const GemmArg
   switch (epi) {
     case EPI_SWIGLU_F8T: return launch_epi<EPI_SWIGLU_F8T, 256, KIND_F8T, false>(maps, a, st);
     case EPI_F24_ROWS: return launch_epi<EPI_F24_ROWS, 256, KIND_F8T, false>(maps, a, st);
+    case EPI_WGRAD: return launch_epi<EPI_WGRAD, 256, KIND_F8T, false>(maps, a, st);
+    case EPI_SWIGLU_BWD_F8T: return launch_epi<EPI_SWIGLU_BWD_F8T, 128, KIND_F8T, false>(maps, a, st);
   }
   return cudaErrorInvalidValue;
 }

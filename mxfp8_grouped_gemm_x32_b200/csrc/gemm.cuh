@@ -14,7 +14,9 @@ enum EpiKind : int {
   EPI_SWIGLU_BF16 = 5,   // BF16 path gate_up: h = p * silu(gate) * up written in bf16 (q_out)
   EPI_F24_ROWS = 6,      // down / dgrad1: the top 24 bits of each fp32 value (f24, see common.cuh), rows in permuted order
   EPI_SWIGLU_F8T = 7,    // per-tensor FP8 gate_up: dequantised by deq[e], h in bf16 (q_out) and its |max| (amax_out)
-  EPI_SWIGLU_BWD_BF16 = 8  // BF16 recipe dgrad2 + ScaledSwiGLU backward: da rows and columns, h columns in bf16
+  EPI_SWIGLU_BWD_BF16 = 8,  // BF16 recipe dgrad2 + ScaledSwiGLU backward: da rows and columns, h columns in bf16
+  EPI_SWIGLU_BWD_F8T = 9    // per-tensor FP8 dgrad2 + ScaledSwiGLU backward: as BF16, dh dequantised by deq[e],
+                            // |max| of da and h into amax_out[0..1]
 };
 
 // Operand kind of the tensor-core MMA.
@@ -67,8 +69,9 @@ struct GemmArgs {
   uint8_t* hcol_sf;
   float* dprob_part;
   // per-tensor FP8 (KIND_F8T): per-expert dequantisation factor applied to
-  // the accumulator (EPI_SWIGLU_F8T and EPI_F24_ROWS; null: none), and the
-  // running |max| of h as float bits (EPI_SWIGLU_F8T)
+  // the accumulator (EPI_SWIGLU_F8T, EPI_F24_ROWS, EPI_WGRAD and
+  // EPI_SWIGLU_BWD_F8T; null: none), and the running |max| as float bits of
+  // h (EPI_SWIGLU_F8T) or of da and h (EPI_SWIGLU_BWD_F8T, two words)
   const float* deq;
   uint32_t* amax_out;
   // mode 1: log2 of the tokens in a 128-byte K tile (0: 7, 8-bit operands;
@@ -106,8 +109,9 @@ cudaError_t launch_grouped_gemm(int epi, int bn, const GemmMaps& maps, const Gem
 // num_kt / a_KT count 128-byte K tiles.
 cudaError_t launch_grouped_gemm_bf16(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);
 
-// Per-tensor FP8 operands (kind::f8f6f4, no block scales), bn = 256:
-// EPI_SWIGLU_F8T and EPI_F24_ROWS (with deq).
+// Per-tensor FP8 operands (kind::f8f6f4, no block scales): EPI_SWIGLU_F8T,
+// EPI_F24_ROWS and EPI_WGRAD (bn = 256, dequantised by deq), and
+// EPI_SWIGLU_BWD_F8T (bn = 128).
 cudaError_t launch_grouped_gemm_f8t(int epi, const GemmMaps& maps, const GemmArgs& a, cudaStream_t st);
 
 }  // namespace moe

@@ -515,6 +515,34 @@ __global__ void f8t_scales_kernel(const uint32_t* amax, int E, int phase, float*
   }
 }
 
+// Factors of the backward (amax: dY, da, h; fwd: the forward's factors x,
+// h, W_gate_up[E], W_down[E]).  phase 0: scale[0] = s_dy and
+// deq[e] = 1 / (s_dy * s_w2[e]) (dgrad2); phase 1: scale[1] = s_da,
+// scale[2] = s_h, deq[E + e] = 1 / (s_dy * s_h) (wgrad2),
+// deq[2E + e] = 1 / (s_da * s_w1[e]) (dgrad1), deq[3E + e] = 1 / (s_da * s_x)
+// (wgrad1).
+__global__ void f8t_bwd_scales_kernel(const uint32_t* amax, const float* fwd, int E, int phase, float* scale,
+                                      float* deq) {
+  const int i = threadIdx.x;
+  const float sdy = f8t_scale(amax[0]);
+  if (phase == 0) {
+    if (i == 0) scale[0] = sdy;
+    for (int e = i; e < E; e += blockDim.x) deq[e] = __frcp_rn(__fmul_rn(sdy, fwd[2 + E + e]));
+  } else {
+    const float sda = f8t_scale(amax[1]), sh = f8t_scale(amax[2]);
+    if (i == 0) {
+      scale[1] = sda;
+      scale[2] = sh;
+    }
+    const float w2 = __frcp_rn(__fmul_rn(sdy, sh)), w1 = __frcp_rn(__fmul_rn(sda, fwd[0]));
+    for (int e = i; e < E; e += blockDim.x) {
+      deq[E + e] = w2;
+      deq[2 * E + e] = __frcp_rn(__fmul_rn(sda, fwd[2 + e]));
+      deq[3 * E + e] = w1;
+    }
+  }
+}
+
 // Codes of bf16 values with one factor per group of group_elems values
 // (scale[g]); with rows_used, only the first *rows_used * row_elems values.
 __global__ void __launch_bounds__(256) f8t_quant_kernel(const uint8_t* __restrict__ src, int64_t n_elems,
@@ -579,6 +607,13 @@ cudaError_t launch_f8t_amax(const uint8_t* src, int groups, int64_t group_elems,
 
 cudaError_t launch_f8t_scales(const uint32_t* amax, int E, int phase, float* scale, float* deq, cudaStream_t st) {
   f8t_scales_kernel<<<1, 256, 0, st>>>(amax, E, phase, scale, deq);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f8t_bwd_scales(const uint32_t* amax, const float* fwd_scales, int E, int phase, float* scale,
+                                  float* deq, cudaStream_t st) {
+  f8t_bwd_scales_kernel<<<1, 256, 0, st>>>(amax, fwd_scales, E, phase, scale, deq);
   count_launch();
   return cudaGetLastError();
 }

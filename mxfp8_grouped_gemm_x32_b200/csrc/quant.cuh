@@ -104,6 +104,10 @@ cudaError_t launch_quant_rows_scatter(const ScatterRowsArgs& a, cudaStream_t st)
 //        rows zero.
 cudaError_t launch_f8t_amax(const uint8_t* src, int groups, int64_t group_elems, uint32_t* amax, cudaStream_t st);
 cudaError_t launch_f8t_scales(const uint32_t* amax, int E, int phase, float* scale, float* deq, cudaStream_t st);
+// Backward factors from amax (dY, da, h) and the forward's factors (phase 0
+// after dY's |max|, phase 1 after da's and h's); scale [3], deq [4E].
+cudaError_t launch_f8t_bwd_scales(const uint32_t* amax, const float* fwd_scales, int E, int phase, float* scale,
+                                  float* deq, cudaStream_t st);
 cudaError_t launch_f8t_quant(const uint8_t* src, int64_t n_elems, int64_t group_elems, const float* scale,
                              const int32_t* rows_used, int64_t row_elems, uint8_t* q, cudaStream_t st);
 cudaError_t launch_f8t_quant_scatter(const uint8_t* x, int64_t T, int64_t H, int32_t k, const int32_t* slot_to_row,

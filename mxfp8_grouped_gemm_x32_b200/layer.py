@@ -13,6 +13,8 @@ Steps (names of the C entry points):
   forward_bf16      moe_grouped_mlp_fwd_bf16: the same layer with bf16 operands
                     (routing from permute_index, moe_permute without x)
   backward_bf16     moe_grouped_mlp_bwd_bf16: its backward
+  forward_fp8_tensor / backward_fp8_tensor
+                    moe_grouped_mlp_fwd/bwd_fp8_tensor: the per-tensor FP8 recipe
   backward          moe_grouped_mlp_bwd: dgrad/wgrad of both projections,
                     ScaledSwiGLU backward, d(prob)
 """
@@ -206,9 +208,36 @@ class GroupedMLP:
         lib.moe_grouped_mlp_fwd_fp8_tensor(w1.data_ptr(), w2.data_ptr(), self.T, H, I, E, self.k, self.rows_cap,
                                            _ptr(self.split_sizes), _ptr(self.group_offsets), _ptr(self.row_to_slot),
                                            _ptr(self.slot_to_row), _ptr(self.prob_perm), x.data_ptr(),
-                                           _ptr(self.out), _ptr(self.fp8_scales), _ptr(self.ws_f8t),
-                                           self.ws_f8t_bytes, self._stream())
+                                           _ptr(self.out), _ptr(self.saved_a), _ptr(self.fp8_scales),
+                                           _ptr(self.ws_f8t), self.ws_f8t_bytes, self._stream())
         return self.out
+
+    def backward_fp8_tensor(self, dY: torch.Tensor, x: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor):
+        """Per-tensor FP8 recipe backward (moe_grouped_mlp_bwd_fp8_tensor)
+        after forward_fp8_tensor on the same routing, x and weights -> (dX,
+        dW1, dW2, dprob); the factors of dY, da and h land in
+        self.fp8_bwd_scales."""
+        if not self.backward_enabled:
+            raise RuntimeError("this layer was built with backward=False")
+        if getattr(self, "fp8_scales", None) is None:
+            raise RuntimeError("backward_fp8_tensor needs forward_fp8_tensor first")
+        E, H, I = self.E, self.H, self.I
+        check_tensor(dY, "dY", torch.bfloat16, (self.T, H), self.dev)
+        check_tensor(x, "x", torch.bfloat16, (self.T, H), self.dev)
+        check_tensor(w1, "w_gate_up", torch.bfloat16, (E, 2 * I, H), self.dev)
+        check_tensor(w2, "w_down", torch.bfloat16, (E, H, I), self.dev)
+        if getattr(self, "ws_bwd_f8t", None) is None:
+            self.ws_bwd_f8t_bytes = lib.moe_workspace_size(lib.MOE_OP_BWD_FP8_TENSOR, self.T, self.k, E, H, I)
+            self.ws_bwd_f8t = self._alloc.raw(self.ws_bwd_f8t_bytes, "ws_bwd_f8t")
+            self.fp8_bwd_scales = self._alloc.typed((3,), torch.float32, "fp8_bwd_scales")
+        lib.moe_grouped_mlp_bwd_fp8_tensor(w1.data_ptr(), w2.data_ptr(), self.T, H, I, E, self.k, self.rows_cap,
+                                           _ptr(self.split_sizes), _ptr(self.group_offsets), _ptr(self.row_to_slot),
+                                           _ptr(self.slot_to_row), _ptr(self.prob_perm), dY.data_ptr(),
+                                           _ptr(self.saved_a), x.data_ptr(), _ptr(self.fp8_scales), _ptr(self.dX),
+                                           _ptr(self.dW1), _ptr(self.dW2), _ptr(self.dprob),
+                                           _ptr(self.fp8_bwd_scales), _ptr(self.ws_bwd_f8t), self.ws_bwd_f8t_bytes,
+                                           self._stream())
+        return self.dX, self.dW1, self.dW2, self.dprob
 
     def check_guards(self):
         """Names of the buffers written past their end (layers built with

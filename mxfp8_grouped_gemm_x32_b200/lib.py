@@ -23,6 +23,7 @@ MOE_OP_BWD = 3
 MOE_OP_FWD_BF16 = 4
 MOE_OP_FWD_FP8_TENSOR = 5
 MOE_OP_BWD_BF16 = 6
+MOE_OP_BWD_FP8_TENSOR = 7
 MOE_MAX_EXPERTS = 256
 
 STATUS = {
@@ -39,6 +40,7 @@ EXPORTED = [
     "moe_timing_enable", "moe_timing_read", "moe_permute_noalloc", "moe_mlp_quantize_weights",
     "moe_router_topk", "moe_mx_scales_to_blocked", "moe_mx_scales_from_blocked", "moe_route_permute",
     "moe_grouped_mlp_fwd_bf16", "moe_grouped_mlp_fwd_fp8_tensor", "moe_grouped_mlp_bwd_bf16",
+    "moe_grouped_mlp_bwd_fp8_tensor",
 ]
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 
@@ -89,7 +91,9 @@ _decl("moe_grouped_mlp_fwd_bf16", _I32, _P, _P, _I32, _I32, _I32, _I32, _I32, _I
 _decl("moe_grouped_mlp_bwd_bf16", _I32, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P,
       _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
 _decl("moe_grouped_mlp_fwd_fp8_tensor", _I32, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P,
-      _P, _P, _P, _SZ, _P)
+      _P, _P, _P, _P, _SZ, _P)
+_decl("moe_grouped_mlp_bwd_fp8_tensor", _I32, _P, _P, _I32, _I32, _I32, _I32, _I32, _I64, _P, _P, _P, _P, _P, _P,
+      _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P)
 _decl("moe_get_device_status", _I32, _P)
 _decl("moe_status_string", ctypes.c_char_p, _I32)
 _decl("moe_launch_count", _I64, _I32)
@@ -180,11 +184,19 @@ def moe_grouped_mlp_bwd_bf16(w_gate_up, w_down, T, H, I, E, k, rows_cap, split_s
 
 
 def moe_grouped_mlp_fwd_fp8_tensor(w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets,
-                                   row_to_slot, slot_to_row, prob_perm, x, out, scales, workspace, workspace_bytes,
-                                   stream=0):
+                                   row_to_slot, slot_to_row, prob_perm, x, out, saved_a, scales, workspace,
+                                   workspace_bytes, stream=0):
     _check("moe_grouped_mlp_fwd_fp8_tensor", _lib.moe_grouped_mlp_fwd_fp8_tensor(
         w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot, slot_to_row, prob_perm,
-        x, out, scales, workspace, workspace_bytes, stream))
+        x, out, saved_a, scales, workspace, workspace_bytes, stream))
+
+
+def moe_grouped_mlp_bwd_fp8_tensor(w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets,
+                                   row_to_slot, slot_to_row, prob_perm, dY, saved_a, x, fwd_scales, dX, dW1, dW2,
+                                   dprob, scales, workspace, workspace_bytes, stream=0):
+    _check("moe_grouped_mlp_bwd_fp8_tensor", _lib.moe_grouped_mlp_bwd_fp8_tensor(
+        w_gate_up, w_down, T, H, I, E, k, rows_cap, split_sizes, group_offsets, row_to_slot, slot_to_row, prob_perm,
+        dY, saved_a, x, fwd_scales, dX, dW1, dW2, dprob, scales, workspace, workspace_bytes, stream))
 
 
 def moe_combine(y, T, k, H, out, stream=0):

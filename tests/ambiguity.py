@@ -246,6 +246,74 @@ def backward_allowance_bf16(f, b, x, w1, w2, dy, topk_idx):
     return {"dX": aX, "dW1": aW1, "dW2": aW2, "dprob": dprob.reshape(T, k)}
 
 
+def backward_allowance_f8t(f, b, dy, topk_idx):
+    """Element-wise allowances for dX, dW1, dW2 and dprob of the per-tensor
+    FP8 recipe's backward (oracle/fp8tensor.py): as the BF16 recipe's, with
+    the operands dequantised through their factors and, for da and h, the
+    change of the per-tensor round trip (at the oracle's factors) over the
+    bf16 values an ambiguous element may take."""
+    from oracle import fp8tensor as ft
+    E, I2, H = f["w1q"].shape
+    I = I2 // 2
+    T, k = topk_idx.shape
+    R = f["perm"].size
+    xd = ft.dequantize_tensor(f["xq"], f["s_x"])
+    dyd = ft.dequantize_tensor(ft.quantize_tensor(dy, b["s_dy"]), b["s_dy"])
+    s_da, s_hb = b["s_da"], b["s_hb"]
+
+    def code_amb(v, band, s):
+        q = lambda t: ft.dequantize_tensor(ft.quantize_tensor(t, s), s)
+        ref = q(omoe.bf16_round(v))
+        lo, hi = bf16_alternatives(v, band)
+        return np.maximum(np.abs(q(lo) - ref), np.abs(q(hi) - ref))
+
+    allow_dx = np.zeros((R, H))
+    allow_dp = np.zeros(R)
+    aW1 = np.zeros((E, I2, H))
+    aW2 = np.zeros((E, H, I))
+    for e, sl in enumerate(_rows_by_expert(f["offsets"], E)):
+        if sl.stop == sl.start:
+            continue
+        tok = f["tok"][sl]
+        p = f["p"][sl][:, None]
+        w1d = ft.dequantize_tensor(f["w1q"][e], f["s_w1"][e])
+        w2d = ft.dequantize_tensor(f["w2q"][e], f["s_w2"][e])
+        xg, dyg = xd[tok], dyd[tok]
+        lo, hi = bf16_alternatives(f["A"][sl], acc_band(xg, w1d))
+        a = f["saved"][sl]
+        g, u = a[:, :I], a[:, I:]
+        dh = b["dh"][sl]
+        bdh = acc_band(dyg, w2d.T)
+
+        def parts(gg, uu, dd):
+            sg = omoe.sigmoid(gg)
+            s = gg * sg
+            return dd * p * uu * sg * (1 + gg * (1 - sg)), dd * p * s, p * s * uu, dd * s * uu
+
+        base = parts(g, u, dh)
+        band = [np.zeros_like(t) for t in base]
+        for gg in (lo[:, :I], hi[:, :I], g):
+            for uu in (lo[:, I:], hi[:, I:], u):
+                alt = parts(gg, uu, dh)
+                for i in range(4):
+                    band[i] = np.maximum(band[i], np.abs(alt[i] - base[i]))
+        sg = omoe.sigmoid(g)
+        band[0] += np.abs(p * u * sg * (1 + g * (1 - sg))) * bdh + ACT * np.abs(base[0])
+        band[1] += np.abs(p * g * sg) * bdh + ACT * np.abs(base[1])
+        band[2] += ACT * np.abs(base[2])
+        band[3] += np.abs(g * sg * u) * bdh + ACT * np.abs(base[3])
+        allow_dp[sl] = band[3].sum(axis=1)
+        Dda = code_amb(np.concatenate([base[0], base[1]], axis=1), np.concatenate([band[0], band[1]], axis=1), s_da)
+        Dh = code_amb(base[2], band[2], s_hb)
+        allow_dx[sl] = Dda @ np.abs(w1d)             # dgrad1: da W_gate_up
+        aW2[e] = np.abs(dyg).T @ Dh                   # wgrad2: dy^T h
+        aW1[e] = Dda.T @ np.abs(xg)                   # wgrad1: da^T x
+    aX = allow_dx[f["slot_row"]].reshape(T, k, -1).sum(axis=1)
+    dprob = np.zeros(R)
+    dprob[f["perm"]] = allow_dp
+    return {"dX": aX, "dW1": aW1, "dW2": aW2, "dprob": dprob.reshape(T, k)}
+
+
 def within(gpu, ref, tol, allow, bf16_out=True):
     """max over elements of (|gpu - ref| - allow) / rms(ref), to compare
     with tol.  For bf16 outputs the allowance also holds the output's own

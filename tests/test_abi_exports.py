@@ -151,11 +151,12 @@ def test_fp8_tensor_forward_argument_errors():
     from mxfp8_grouped_gemm_x32_b200 import lib
     f = lib._lib.moe_grouped_mlp_fwd_fp8_tensor
     rc = lib.moe_padded_rows(64, 2, 4)
-    args = lambda H=256, ws=P, wsb=1 << 40, x=P, sc=None: (P, P, 64, H, 512, 4, 2, rc, P, P, P, P, P, x, P, sc, ws,
-                                                          wsb, None)
+    args = lambda H=256, ws=P, wsb=1 << 40, x=P, sc=None, sa=None: (P, P, 64, H, 512, 4, 2, rc, P, P, P, P, P, x, P,
+                                                                    sa, sc, ws, wsb, None)
     assert f(*args(x=None)) == INVALID                                      # x missing with T > 0
     assert f(*args(x=M)) == INVALID                                         # misaligned x
     assert f(*args(sc=P + 2)) == INVALID                                    # misaligned factor output
+    assert f(*args(sa=M)) == INVALID                                        # misaligned saved A
     assert f(*args(H=48)) == UNSUPPORTED
     need = lib.moe_workspace_size(lib.MOE_OP_FWD_FP8_TENSOR, 64, 2, 4, 256, 512)
     assert need > 0
@@ -212,3 +213,38 @@ def test_route_permute_argument_errors():
     assert f(*args(H=48)) == UNSUPPORTED
     assert f(*args(x=M)) == INVALID
     assert f(*args(ws_bytes=16)) == WORKSPACE
+
+
+def _recipe_bwd_args(fp8, T=64, H=256, I=512, E=4, k=2, saved=P, x=P, dW1=P, fs=P, sc=None, ws=P, ws_bytes=1 << 40):
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    rc = lib.moe_padded_rows(T, k, E)
+    head = (P, P, T, H, I, E, k, rc, P, P, P, P, P, P, saved, x)
+    tail = (P, dW1, P, P)
+    if fp8:
+        return head + (fs,) + tail + (sc, ws, ws_bytes, None)
+    return head + tail + (ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_recipe_backward_argument_errors(fp8):
+    """moe_grouped_mlp_bwd_bf16 / moe_grouped_mlp_bwd_fp8_tensor reject bad
+    arguments with their documented codes before looking for a device."""
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    f = lib._lib.moe_grouped_mlp_bwd_fp8_tensor if fp8 else lib._lib.moe_grouped_mlp_bwd_bf16
+    a = lambda **kw: _recipe_bwd_args(fp8, **kw)
+    assert f(*a(saved=None)) == INVALID                                     # no saved A
+    assert f(*a(x=None)) == INVALID
+    assert f(*a(H=48)) == UNSUPPORTED
+    assert f(*a(I=96)) == UNSUPPORTED
+    assert f(*a(E=300, k=2)) == UNSUPPORTED
+    assert f(*a(dW1=M)) == INVALID                                          # misaligned output
+    assert f(*a(saved=P + 16)) == INVALID                                   # saved A needs 32-byte alignment
+    assert f(*a(ws=P + 128)) == INVALID                                     # workspace needs 256-byte alignment
+    op = lib.MOE_OP_BWD_FP8_TENSOR if fp8 else lib.MOE_OP_BWD_BF16
+    need = lib.moe_workspace_size(op, 64, 2, 4, 256, 512)
+    assert need > 0
+    assert f(*a(ws_bytes=need - 1)) == WORKSPACE
+    if fp8:
+        assert f(*a(fs=None)) == INVALID                                    # the forward's factors are needed
+        assert f(*a(fs=P + 2)) == INVALID
+        assert f(*a(sc=P + 2)) == INVALID

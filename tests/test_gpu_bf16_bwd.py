@@ -61,7 +61,8 @@ def _run(case):
                       bf16_held=True)
     g = lambda t: t.float().cpu().numpy().astype(np.float64)
     res = dict(cfg=cfg, inp=inp, f=f, b=b, dX=g(dX), dW1=g(dW1), dW2=g(dW2), dprob=g(dprob),
-               saved=g(L.saved_a), go=L.group_offsets.cpu().numpy(), split=L.split_sizes.cpu().numpy())
+               saved=g(L.saved_a[: int(L.group_offsets[cfg.E])]), go=L.group_offsets.cpu().numpy(),
+               split=L.split_sizes.cpu().numpy())
     _RUNS[case] = res
     return res
 
