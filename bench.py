@@ -734,6 +734,23 @@ def run_ours(args):
     st = layer.device_status()
     if st != 0:
         raise SystemExit(f"device status after the per-tensor FP8 forward: {lib.status_string(st)}")
+    # the per-tensor FP8 recipe's training step: routing + forward (saving A)
+    # + backward
+    for _ in range(3):
+        layer.permute_index(idx, prob)
+        layer.forward_fp8_tensor(x, w1, w2)
+        layer.backward_fp8_tensor(dy, x, w1, w2)
+    e0.record(stream)
+    for _ in range(10):
+        layer.permute_index(idx, prob)
+        layer.forward_fp8_tensor(x, w1, w2)
+        layer.backward_fp8_tensor(dy, x, w1, w2)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_f8t_step = max_over_ranks(e0.elapsed_time(e1) / 10, world, dev)
+    st = layer.device_status()
+    if st != 0:
+        raise SystemExit(f"device status after the per-tensor FP8 backward: {lib.status_string(st)}")
 
     if world > 1:
         dist.destroy_process_group()
@@ -804,6 +821,13 @@ def run_ours(args):
                            "what": "per-tensor FP8 recipe layer forward (moe_permute without x + "
                                    "moe_grouped_mlp_fwd_fp8_tensor): factors from the current |max| of x, of every "
                                    "expert's weights and of h, weights quantised in the call"},
+        "fp8_tensor_step": {"value": world * flops / (ms_f8t_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+                            "ms_per_call": ms_f8t_step, "bwd_ms": ms_f8t_step - ms_f8t,
+                            "bwd_tflops": cfg.bwd_flops() / ((ms_f8t_step - ms_f8t) * 1e-3) / 1e12,
+                            "what": "per-tensor FP8 recipe layer step: moe_permute without x + "
+                                    "moe_grouped_mlp_fwd_fp8_tensor (saving A) + moe_grouped_mlp_bwd_fp8_tensor "
+                                    "(dY, da, h factored in the call, weights transposed and coded in the call); "
+                                    "bwd_ms = step - fp8_tensor_fwd"},
         "router": {"ms_per_call": router_ms, "in_step": False,
                    "what": "moe_router_topk on fp32 logits [T, E] (softmax, top-k, renormalise)"},
         "roofline": roofline,
