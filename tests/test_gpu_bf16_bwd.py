@@ -59,7 +59,10 @@ def _run(case):
                      h_bf16=True)
     b = omoe.backward(f, f64("x"), f64("w1"), f64("w2"), inp["topk_prob"], f64("dy"), quantize=False,
                       bf16_held=True)
-    g = lambda t: t.float().cpu().numpy().astype(np.float64)
+    def g(t):
+        with np.errstate(invalid="ignore"):   # padding rows of the saved A are never written (any bits)
+            return t.float().cpu().numpy().astype(np.float64)
+
     res = dict(cfg=cfg, inp=inp, f=f, b=b, dX=g(dX), dW1=g(dW1), dW2=g(dW2), dprob=g(dprob),
                saved=g(L.saved_a[: int(L.group_offsets[cfg.E])]), go=L.group_offsets.cpu().numpy(),
                split=L.split_sizes.cpu().numpy())
