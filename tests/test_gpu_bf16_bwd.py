@@ -29,6 +29,7 @@ CASES = {
     "tiny": dict(),
     "gptoss_k2880": dict(name="gpt_oss_20b", T=160, E=4, k=2),
     "ragged_128e": dict(name="qwen3_30b_ragged", T=96, H=256, I=256, E=128, k=8),
+    "one_token": dict(T=1),
 }
 
 _RUNS = {}

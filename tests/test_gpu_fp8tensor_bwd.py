@@ -25,6 +25,7 @@ CASES = {
     "tiny": dict(),
     "gptoss_k2880": dict(name="gpt_oss_20b", T=160, E=4, k=2),
     "ragged_128e": dict(name="qwen3_30b_ragged", T=96, H=256, I=256, E=128, k=8),
+    "one_token": dict(T=1),
 }
 
 _RUNS = {}
@@ -87,3 +88,27 @@ def test_empty_experts_have_zero_weight_gradients(case):
     r = _run(case)
     empty = np.flatnonzero(r["split"] == 0)
     assert np.all(r["dW1"][empty] == 0.0) and np.all(r["dW2"][empty] == 0.0)
+
+
+@pytest.mark.parametrize("recipe", ["bf16", "fp8_tensor"])
+def test_zero_tokens(recipe):
+    """A batch with no tokens runs every launch of both recipes' forward and
+    backward and leaves zero weight gradients."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    from mxfp8_grouped_gemm_x32_b200.layer import GroupedMLP
+    cfg = get_config("tiny", T=0)
+    inp = make_inputs(cfg, seed=31)
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    L = GroupedMLP(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, backward=True, guard=4096)
+    x, w1, w2, dy = bf(inp["x"]), bf(inp["w1"]), bf(inp["w2"]), bf(inp["dy"])
+    L.permute_index(torch.from_numpy(inp["topk_idx"]).cuda(), torch.from_numpy(inp["topk_prob"]).cuda())
+    getattr(L, "forward_" + recipe)(x, w1, w2)
+    dX, dW1, dW2, dprob = getattr(L, "backward_" + recipe)(dy, x, w1, w2)
+    torch.cuda.synchronize()
+    assert lib.moe_get_device_status(0) == 0
+    assert L.check_guards() == []
+    assert dX.shape == (0, cfg.H) and dprob.shape == (0, cfg.k)
+    assert float(dW1.float().abs().max()) == 0.0 and float(dW2.float().abs().max()) == 0.0
