@@ -184,24 +184,21 @@ BwdBf16Ws carve_bwd_bf16(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, 
   return w;
 }
 
-// Per-tensor FP8 backward workspace: bf16 staging (the transposed weights,
-// one at a time; dy gathered in both orientations; da and h from the dgrad2
-// epilogue; x gathered and transposed), their E4M3 codes, f24 dgrad rows,
-// dprob partials, |max| bits (dY, da, h), factors (dY, da, h) and the
-// dequantisation factors of the four GEMMs [4E].
+// Per-tensor FP8 backward workspace: E4M3 codes of the transposed weights,
+// of dy gathered (rows and transposed) and of x gathered and transposed (each
+// coded as it is transposed); da and h in bf16 from the dgrad2 epilogue and
+// their codes; f24 dgrad rows, dprob partials, |max| bits (dY, da, h),
+// factors (dY, da, h) and the dequantisation factors of the four GEMMs [4E].
 struct BwdF8tWs {
-  uint8_t *wt, *w2tq, *w1tq, *dyp, *dyc, *dyq, *dycq, *da, *dac, *hc, *daq, *dacq, *hcq, *xc, *xcq, *dx, *dpp;
+  uint8_t *w2tq, *w1tq, *dyq, *dycq, *da, *dac, *hc, *daq, *dacq, *hcq, *xcq, *dx, *dpp;
   uint32_t* amax;
   float *scale, *deq;
 };
 BwdF8tWs carve_bwd_f8t(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, int64_t E, int64_t rows_cap) {
   (void)T; (void)k;
   BwdF8tWs w{};
-  w.wt = c.take(E * 2 * I * H * 2);
   w.w2tq = c.take(E * I * H);
   w.w1tq = c.take(E * H * 2 * I);
-  w.dyp = c.take(rows_cap * H * 2);
-  w.dyc = c.take(H * rows_cap * 2);
   w.dyq = c.take(rows_cap * H);
   w.dycq = c.take(H * rows_cap);
   w.da = c.take(rows_cap * 2 * I * 2);
@@ -210,7 +207,6 @@ BwdF8tWs carve_bwd_f8t(Carver& c, int64_t T, int64_t k, int64_t H, int64_t I, in
   w.daq = c.take(rows_cap * 2 * I);
   w.dacq = c.take(2 * I * rows_cap);
   w.hcq = c.take(I * rows_cap);
-  w.xc = c.take(H * rows_cap * 2);
   w.xcq = c.take(H * rows_cap);
   w.dx = c.take(rows_cap * H * 3);
   w.dpp = c.take(I / 64 * rows_cap * 4);
@@ -754,7 +750,7 @@ moe_status_t moe_grouped_mlp_bwd_bf16(const void* w_gate_up, const void* w_down,
                      nullptr, k, nullptr, nullptr};
     TransposeArgs t1{static_cast<const uint16_t*>(w_gate_up), reinterpret_cast<uint16_t*>(w.w1t), E, I2, H, I2,
                      nullptr, k, nullptr, nullptr};
-    if (launch_transpose_bf16(t2, st) != cudaSuccess || launch_transpose_bf16(t1, st) != cudaSuccess)
+    if (launch_transpose(t2, st) != cudaSuccess || launch_transpose(t1, st) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
   // dy gathered to permuted rows, in both orientations (one read of dY)
@@ -762,7 +758,7 @@ moe_status_t moe_grouped_mlp_bwd_bf16(const void* w_gate_up, const void* w_down,
     TimeScope ts(st, "dy_gather_bf16");
     TransposeArgs td{static_cast<const uint16_t*>(dY), reinterpret_cast<uint16_t*>(w.dyc), 1, rows_cap, H, rows_cap,
                      row_to_slot, k, group_offsets + E, reinterpret_cast<uint16_t*>(w.dyp)};
-    if (launch_transpose_bf16(td, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_transpose(td, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // dgrad2 + ScaledSwiGLU backward: dh = dy W_down (contraction over H) in
@@ -824,7 +820,7 @@ moe_status_t moe_grouped_mlp_bwd_bf16(const void* w_gate_up, const void* w_down,
     TimeScope ts(st, "x_gather_cols_bf16");
     TransposeArgs tx{static_cast<const uint16_t*>(x), reinterpret_cast<uint16_t*>(w.xc), 1, rows_cap, H, rows_cap,
                      row_to_slot, k, group_offsets + E, nullptr};
-    if (launch_transpose_bf16(tx, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_transpose(tx, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // wgrad1: dW_gate_up_e = da_e^T x_e (contraction over the group's tokens)
@@ -870,27 +866,23 @@ moe_status_t moe_grouped_mlp_bwd_fp8_tensor(const void* w_gate_up, const void* w
   auto quant = [&](const uint8_t* src, int64_t n, int64_t group, const float* sc, const int32_t* ru, int64_t row,
                    uint8_t* q) { return launch_f8t_quant(src, n, group, sc, ru, row, q, st) == cudaSuccess; };
 
-  // dY's factor; dy gathered to permuted rows in both orientations, then its codes
+  // dY's factor; dy gathered to permuted rows in both orientations and coded in the same pass
   {
     TimeScope ts(st, "fp8t_dy");
     if (cudaMemsetAsync(w.amax, 0, 3 * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
     if (T > 0 && launch_f8t_amax(static_cast<const uint8_t*>(dY), 1, int64_t(T) * H, w.amax, st) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (launch_f8t_bwd_scales(w.amax, fwd_scales, E, 0, w.scale, w.deq, st) != cudaSuccess) return MOE_ERR_CUDA;
-    TransposeArgs td{static_cast<const uint16_t*>(dY), reinterpret_cast<uint16_t*>(w.dyc), 1, rows_cap, H, rows_cap,
-                     row_to_slot, k, rows_used, reinterpret_cast<uint16_t*>(w.dyp)};
-    if (launch_transpose_bf16(td, st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (!quant(w.dyp, rows_cap * H, rows_cap * H, w.scale, rows_used, H, w.dyq) ||
-        !quant(w.dyc, H * rows_cap, H * rows_cap, w.scale, nullptr, 0, w.dycq))
-      return MOE_ERR_CUDA;
+    TransposeArgs td{static_cast<const uint16_t*>(dY), w.dycq, 1, rows_cap, H, rows_cap, row_to_slot, k, rows_used,
+                     w.dyq, w.scale};
+    if (launch_transpose(td, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
-  // W_down^T codes with the forward's per-expert factors
+  // W_down^T codes with the forward's per-expert factors (transposed and coded in one pass)
   {
     TimeScope ts(st, "fp8t_w_down_t");
-    TransposeArgs t2{static_cast<const uint16_t*>(w_down), reinterpret_cast<uint16_t*>(w.wt), E, H, I, H, nullptr, k,
-                     nullptr, nullptr};
-    if (launch_transpose_bf16(t2, st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (!quant(w.wt, E * I * H, int64_t(I) * H, fwd_scales + 2 + E, nullptr, 0, w.w2tq)) return MOE_ERR_CUDA;
+    TransposeArgs t2{static_cast<const uint16_t*>(w_down), w.w2tq, E, H, I, H, nullptr, k, nullptr, nullptr,
+                     fwd_scales + 2 + E};
+    if (launch_transpose(t2, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // dgrad2 + ScaledSwiGLU backward: dh = dy W_down dequantised per expert;
@@ -942,10 +934,9 @@ moe_status_t moe_grouped_mlp_bwd_fp8_tensor(const void* w_gate_up, const void* w
   // W_gate_up^T codes; dgrad1: dx = da W_gate_up, f24 rows; dX combine
   {
     TimeScope ts(st, "fp8t_w_gate_up_t");
-    TransposeArgs t1{static_cast<const uint16_t*>(w_gate_up), reinterpret_cast<uint16_t*>(w.wt), E, I2, H, I2,
-                     nullptr, k, nullptr, nullptr};
-    if (launch_transpose_bf16(t1, st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (!quant(w.wt, E * H * I2, int64_t(H) * I2, fwd_scales + 2, nullptr, 0, w.w1tq)) return MOE_ERR_CUDA;
+    TransposeArgs t1{static_cast<const uint16_t*>(w_gate_up), w.w1tq, E, I2, H, I2, nullptr, k, nullptr, nullptr,
+                     fwd_scales + 2};
+    if (launch_transpose(t1, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
   if (make_map_2d(&m.a, w.daq, I2, rows_cap, 128) != cudaSuccess) return MOE_ERR_CUDA;
   if (make_map_3d(&m.b, w.w1tq, I2, H, E, 256) != cudaSuccess) return MOE_ERR_CUDA;
@@ -966,10 +957,9 @@ moe_status_t moe_grouped_mlp_bwd_fp8_tensor(const void* w_gate_up, const void* w
   // dW_gate_up_e = da_e^T x_e (contraction over the group's tokens)
   {
     TimeScope ts(st, "fp8t_x_cols");
-    TransposeArgs tx{static_cast<const uint16_t*>(x), reinterpret_cast<uint16_t*>(w.xc), 1, rows_cap, H, rows_cap,
-                     row_to_slot, k, rows_used, nullptr};
-    if (launch_transpose_bf16(tx, st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (!quant(w.xc, H * rows_cap, H * rows_cap, fwd_scales, nullptr, 0, w.xcq)) return MOE_ERR_CUDA;
+    TransposeArgs tx{static_cast<const uint16_t*>(x), w.xcq, 1, rows_cap, H, rows_cap, row_to_slot, k, rows_used,
+                     nullptr, fwd_scales};
+    if (launch_transpose(tx, st) != cudaSuccess) return MOE_ERR_CUDA;
   }
   if (make_map_2d(&m.a, w.dacq, rows_cap, I2, 128) != cudaSuccess) return MOE_ERR_CUDA;
   if (make_map_2d(&m.b, w.xcq, rows_cap, H, 256) != cudaSuccess) return MOE_ERR_CUDA;
