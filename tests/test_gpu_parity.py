@@ -311,6 +311,39 @@ def test_backward_requant_da(run):
     assert bad == 0
 
 
+def test_backward_dy_codes_bitexact(run):
+    """dY gathered to permuted rows and quantised along H and along tokens (the
+    backward workspace's first four pieces: see carve_bwd) equals the oracle's
+    codec on the gathered rows, bit for bit; padding rows are zero."""
+    cfg, inp, layer, f, b = run
+    L = layer.L
+    rc, H = L.rows_cap, cfg.H
+    from mxfp8_grouped_gemm_x32_b200 import lib
+    a256 = lambda n: (n + 255) // 256 * 256
+    ws = L.ws_bwd.cpu().numpy()
+    o_sf = a256(rc * H)
+    o_c = o_sf + a256(lib.moe_mx_scale_bytes(1, rc, H))
+    o_csf = o_c + a256(H * rc)
+    dyq = ws[:rc * H].reshape(rc, H)
+    dysf = sf_unblock(ws[o_sf:o_sf + lib.moe_mx_scale_bytes(1, rc, H)], 1, rc, H)[0]
+    dyc = ws[o_c:o_c + H * rc].reshape(H, rc)
+    dycsf = sf_unblock(ws[o_csf:o_csf + lib.moe_mx_scale_bytes(1, H, rc)], 1, H, rc)[0]
+    dy = _f64(inp["dy"])
+    go = L.group_offsets.cpu().numpy()
+    offs = f["offsets"]
+    for e in range(cfg.E):
+        g0, n = go[e], f["split_sizes"][e]
+        tok = f["tok"][offs[e]:offs[e + 1]]
+        c, s = omx.quantize_rows(dy[tok])
+        assert np.array_equal(dyq[g0:g0 + n], c) and np.array_equal(dysf[g0:g0 + n], s)
+        assert np.all(dyq[g0 + n:go[e + 1]] == 0) and np.all(dysf[g0 + n:go[e + 1]] == 0)
+        c, s = omx.quantize_cols_grouped(dy[tok], [n])[0]
+        mp = c.shape[1]
+        assert np.array_equal(dyc[:, g0:g0 + mp], c)
+        assert np.array_equal(dycsf[:, g0 // 32:(g0 + mp) // 32], s)
+        assert np.all(dyc[:, g0 + mp:go[e + 1]] == 0)
+
+
 def test_wait_timeout_selftest(torch_cuda):
     from mxfp8_grouped_gemm_x32_b200 import lib
     st = lib.moe_selftest_wait_timeout(20, 0)
