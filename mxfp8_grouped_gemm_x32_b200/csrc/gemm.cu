@@ -166,7 +166,10 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int* go, co
 //    the layer shapes benchmarked here);
 //  NW == 16: 16 words of all 32 rows, 8 rows x 64 bytes per instruction.
 // The staged pitch (144 bytes, or 80 for 64-byte rows) keeps the 16-byte
-// shared stores and loads free of bank conflicts.
+// shared stores and loads free of bank conflicts.  The global stores are
+// streaming (evict-first in L2): the GEMM's outputs are not re-read by it, and
+// lines it writes should not displace the operand panels that its later
+// tiles re-read from L2.
 constexpr int STAGE128_PITCH_W = 36;
 static_assert(16 * STAGE128_PITCH_W * 4 <= Cfg<256>::STAGE_WARP_BYTES, "staging buffer too small");
 static_assert(32 * STAGE_PITCH_W * 4 <= Cfg<256>::STAGE_WARP_BYTES, "staging buffer too small");
@@ -197,8 +200,8 @@ __device__ __forceinline__ void warp_store_rows(uint32_t* stage, uint8_t* row, c
           const uint64_t dst = __shfl_sync(0xFFFFFFFFu, rp, 16 * hh + rr);
           const int off = 128 * c + 16 * piece;
           if (dst != 0 && off < bytes)
-            *reinterpret_cast<uint4*>(dst + off) =
-                *reinterpret_cast<const uint4*>(stage + rr * STAGE128_PITCH_W + 4 * piece);
+            __stcs(reinterpret_cast<uint4*>(dst + off),
+                   *reinterpret_cast<const uint4*>(stage + rr * STAGE128_PITCH_W + 4 * piece));
         }
       }
     }
@@ -218,8 +221,8 @@ __device__ __forceinline__ void warp_store_rows(uint32_t* stage, uint8_t* row, c
         const uint64_t dst = __shfl_sync(0xFFFFFFFFu, rp, rr);
         const int off = 64 * c + 16 * piece;
         if (dst != 0 && off < bytes)
-          *reinterpret_cast<uint4*>(dst + off) =
-              *reinterpret_cast<const uint4*>(stage + rr * STAGE_PITCH_W + 4 * piece);
+          __stcs(reinterpret_cast<uint4*>(dst + off),
+                 *reinterpret_cast<const uint4*>(stage + rr * STAGE_PITCH_W + 4 * piece));
       }
     }
   }
