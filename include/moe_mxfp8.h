@@ -284,8 +284,9 @@ moe_status_t moe_grouped_mlp_fwd(const uint8_t* w1q, const uint8_t* w1sf, const 
  *              prob_perm from moe_permute (xq may be NULL there).
  *   x          bf16 [T][H];  out bf16 [T][H].
  *   saved_a    bf16 [rows_cap][2I] or NULL: A rounded to bf16, kept for
- *              moe_grouped_mlp_bwd_bf16 (rows of the groups, padding rows
- *              included, are written; 16-byte aligned).
+ *              moe_grouped_mlp_bwd_bf16 (routed rows only: padding rows are
+ *              not written, and the backward never reads them; 16-byte
+ *              aligned).
  *   workspace  >= moe_workspace_size(MOE_OP_FWD_BF16, T, k, E, H, I).
  * Limits as moe_grouped_mlp_fwd. */
 moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down, int32_t T, int32_t H, int32_t I,
@@ -312,7 +313,8 @@ moe_status_t moe_grouped_mlp_fwd_bf16(const void* w_gate_up, const void* w_down,
  *   routing    from moe_permute (xq may be NULL there).
  *   x          bf16 [T][H];  out bf16 [T][H].
  *   saved_a    bf16 [rows_cap][2I] or NULL: A (dequantised) rounded to bf16,
- *              kept for moe_grouped_mlp_bwd_fp8_tensor (16-byte aligned).
+ *              kept for moe_grouped_mlp_bwd_fp8_tensor (routed rows only;
+ *              16-byte aligned).
  *   scales     NULL, or float [2 + 2E] receiving the factors: x, h,
  *              W_gate_up[0..E), W_down[0..E) (the backward's fwd_scales).
  *   workspace  >= moe_workspace_size(MOE_OP_FWD_FP8_TENSOR, T, k, E, H, I),
