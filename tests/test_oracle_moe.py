@@ -186,6 +186,38 @@ def test_identity_expert_bf16_backward():
     assert np.allclose(b2["dX"][:, :I], dg, rtol=1e-13, atol=0)
 
 
+def test_bf16_backward_scales_exactly_with_dy():
+    """BF16 recipe backward: dY -> 2^5 dY multiplies every gradient by exactly
+    2^5 (bf16 rounding commutes with a power-of-two scale; h does not depend
+    on dY) -- a dropped or doubled term of the dY path breaks this."""
+    x, w1, w2, idx, prob, _ = _small_layer(seed=21)
+    rng = np.random.default_rng(22)
+    dy = moe.bf16_round(rng.standard_normal(x.shape))
+    fwd = moe.forward(x, w1, w2, idx, prob, quantize=False, h_bf16=True)
+    a = moe.backward(fwd, x, w1, w2, prob, dy, quantize=False, bf16_held=True)
+    b = moe.backward(fwd, x, w1, w2, prob, 32.0 * dy, quantize=False, bf16_held=True)
+    for key in ("dX", "dW1", "dW2", "dprob_f64", "da"):
+        assert np.array_equal(b[key], 32.0 * a[key]), key
+    assert np.array_equal(b["h_b"], a["h_b"])
+
+
+def test_bf16_backward_close_to_the_exact_gradient():
+    """The bf16 roundings of da and h change each gradient by at most a few
+    bf16 steps: within 2 % of the rms of the unrounded backward, element by
+    element (an index or sign mistake in the rounded path gives errors of the
+    order of the rms)."""
+    x, w1, w2, idx, prob, _ = _small_layer(seed=23, T=40)
+    rng = np.random.default_rng(24)
+    dy = moe.bf16_round(rng.standard_normal(x.shape))
+    fwd = moe.forward(x, w1, w2, idx, prob, quantize=False, h_bf16=True)
+    held = moe.backward(fwd, x, w1, w2, prob, dy, quantize=False, bf16_held=True)
+    exact = moe.backward(fwd, x, w1, w2, prob, dy, quantize=False)
+    for key in ("dX", "dW1", "dW2"):
+        rms = np.sqrt(np.mean(exact[key] ** 2))
+        assert np.max(np.abs(held[key] - exact[key])) <= 2e-2 * rms, key
+    assert np.array_equal(held["dprob_f64"], exact["dprob_f64"])       # dprob does not use da or h
+
+
 def test_permutation_invariants(tiny):
     cfg, inp = tiny
     perm, split = moe.permute(inp["topk_idx"], cfg.E)
